@@ -1,0 +1,271 @@
+"""Seeded synthetic batches for paged-KV attention (inputs only, no attention arithmetic).
+
+This module is the single source of inputs for both sides of every parity check: the
+float64 CPU oracle (``oracle/``) and the CUDA path (``paged_kv_attention_verify_b200``).
+It holds no part of the attention computation itself: it draws lengths, draft-tree
+parent arrays, Q/K/V values and a page permutation, then lays K/V out twice — once
+contiguous per sequence (what the oracle reads) and once scattered into a pool of
+fixed-size pages addressed through a block table (what the kernels read).
+
+Workload shapes follow the five batches the pages' problem is benchmarked on
+(decode on a Llama-3-8B-shaped cache, chunked prefill on a Llama-3.3-70B-shaped
+cache, a unified prefill/decode/verify batch on a Qwen2-7B-shaped cache, and a
+long-context decode with outlier keys). XY-Serve (arXiv 2412.18106, verdict page,
+``core_discovery``) names the mixed prefill / decode / verify batch over a
+PagedAttention-style block cache; the sizes are those of the benchmark configs.
+
+Randomness recipe (stated once, used everywhere):
+  * sequence lengths and draft trees come from a CPU ``torch.Generator`` seeded with
+    the config seed (the config's index, 0..4);
+  * the page permutation comes from a CPU generator seeded with ``seed + 1000``, so
+    structure is identical whatever device the values are drawn on;
+  * bulk values (Q, K, V, outlier flags, page-tail filler) come from a generator on
+    the target device seeded with ``seed + 1001``; values are N(0,1) rounded to bf16
+    (a CPU draw and a CUDA draw of the same seed differ; each test feeds both sides
+    from one draw);
+  * page slots past a sequence's length are filled with finite values of large
+    magnitude (N(0,1) x 50) so that any failure to mask them shows up in parity.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import List, Optional, Sequence
+
+import torch
+
+CAUSAL = 0
+TREE = 1
+
+
+@dataclasses.dataclass
+class SeqSpec:
+    seq_len: int          # total KV length including the new tokens
+    query_len: int        # number of new query tokens (their K/V are already cached)
+    mask_kind: int        # CAUSAL or TREE
+    parents: List[int]    # TREE only: parents[i] in {-1} U [0, i)
+
+
+@dataclasses.dataclass
+class Batch:
+    name: str
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    page_size: int
+    seqs: List[SeqSpec]
+    q: torch.Tensor                  # [sum T, Hq, d] bf16
+    k: Optional[torch.Tensor]        # [sum L, Hkv, d] bf16, contiguous per sequence
+    v: Optional[torch.Tensor]
+    k_cache: torch.Tensor            # [num_pages, Hkv, page_size, d] bf16
+    v_cache: torch.Tensor
+    block_table: torch.Tensor        # [B, max_pages] int32, -1 = unused slot
+    page_perm: torch.Tensor          # [num_pages] int64 (CPU): logical page -> physical page
+    seed: int = 0
+    outlier_frac: float = 0.0
+
+    # -- convenience views (layout only) ---------------------------------------------
+    @property
+    def seq_lens(self) -> List[int]:
+        return [s.seq_len for s in self.seqs]
+
+    @property
+    def query_lens(self) -> List[int]:
+        return [s.query_len for s in self.seqs]
+
+    @property
+    def mask_kinds(self) -> List[int]:
+        return [s.mask_kind for s in self.seqs]
+
+    @property
+    def parents_flat(self) -> List[int]:
+        out: List[int] = []
+        for s in self.seqs:
+            if s.mask_kind == TREE:
+                out.extend(s.parents)
+        return out
+
+    def q_offsets(self) -> List[int]:
+        off, acc = [], 0
+        for s in self.seqs:
+            off.append(acc)
+            acc += s.query_len
+        return off
+
+    def kv_offsets(self) -> List[int]:
+        off, acc = [], 0
+        for s in self.seqs:
+            off.append(acc)
+            acc += s.seq_len
+        return off
+
+    def seq_q(self, i: int) -> torch.Tensor:
+        o = self.q_offsets()[i]
+        return self.q[o:o + self.seqs[i].query_len]
+
+    def seq_kv(self, i: int):
+        if self.k is None:
+            raise ValueError("contiguous K/V were dropped for this batch")
+        o = self.kv_offsets()[i]
+        L = self.seqs[i].seq_len
+        return self.k[o:o + L], self.v[o:o + L]
+
+    @property
+    def total_q(self) -> int:
+        return sum(s.query_len for s in self.seqs)
+
+    @property
+    def total_kv(self) -> int:
+        return sum(s.seq_len for s in self.seqs)
+
+
+# ---------------------------------------------------------------------------------
+# Named configurations (sizes of the five benchmark batches)
+# ---------------------------------------------------------------------------------
+
+CONFIG_NAMES = [
+    "tiny_decode",          # 4 seqs, ctx {17,64,100,255}, 8q/2kv, d64
+    "llama3_8b_decode",     # 128 seqs, ctx U[512,8192], 32q/8kv, d128
+    "llama33_70b_prefill",  # 8 seqs x 2048-token chunk on ctx U[0,16384], 64q/8kv, d128
+    "qwen2_7b_unified",     # 4x512 prefill + 192 decode + 32 verify(5-node tree), 28q/4kv
+    "long_ctx_split",       # 16 seqs, ctx U[32768,131072], 128q/8kv, 1% outlier keys x8
+]
+
+
+def _randint(gen: torch.Generator, lo: int, hi: int, n: int) -> List[int]:
+    """n integers uniform on [lo, hi] inclusive."""
+    return torch.randint(lo, hi + 1, (n,), generator=gen).tolist()
+
+
+def random_tree(gen: torch.Generator, n: int) -> List[int]:
+    """Parent array of a random draft tree: parents[0] = -1, parents[i] ~ U{-1..i-1}."""
+    par = [-1]
+    for i in range(1, n):
+        par.append(int(torch.randint(-1, i, (1,), generator=gen).item()))
+    return par
+
+
+def config_seqs(name: str, gen: torch.Generator) -> tuple:
+    """(seqs, Hq, Hkv, d, outlier_frac) for a named configuration."""
+    if name == "tiny_decode":
+        seqs = [SeqSpec(L, 1, CAUSAL, []) for L in (17, 64, 100, 255)]
+        return seqs, 8, 2, 64, 0.0
+    if name == "llama3_8b_decode":
+        seqs = [SeqSpec(L, 1, CAUSAL, []) for L in _randint(gen, 512, 8192, 128)]
+        return seqs, 32, 8, 128, 0.0
+    if name == "llama33_70b_prefill":
+        seqs = [SeqSpec(c + 2048, 2048, CAUSAL, []) for c in _randint(gen, 0, 16384, 8)]
+        return seqs, 64, 8, 128, 0.0
+    if name == "qwen2_7b_unified":
+        seqs = [SeqSpec(512, 512, CAUSAL, []) for _ in range(4)]
+        seqs += [SeqSpec(L, 1, CAUSAL, []) for L in _randint(gen, 256, 4096, 192)]
+        for ctx in _randint(gen, 256, 4096, 32):
+            seqs.append(SeqSpec(ctx + 5, 5, TREE, random_tree(gen, 5)))
+        return seqs, 28, 4, 128, 0.0
+    if name == "long_ctx_split":
+        seqs = [SeqSpec(L, 1, CAUSAL, []) for L in _randint(gen, 32768, 131072, 16)]
+        return seqs, 128, 8, 128, 0.01
+    raise KeyError(name)
+
+
+def build_batch(name: str, seqs: Sequence[SeqSpec], num_q_heads: int, num_kv_heads: int,
+                head_dim: int, seed: int, device="cpu", page_size: int = 16,
+                outlier_frac: float = 0.0, outlier_scale: float = 8.0,
+                keep_contiguous: bool = True, bt_extra: int = 0,
+                perm_seed: Optional[int] = None) -> Batch:
+    """Draw Q/K/V for ``seqs`` and lay K/V out in a shuffled paged pool.
+
+    ``seed`` seeds the page permutation (CPU) and ``seed + 1`` the values (device);
+    ``perm_seed`` overrides the permutation seed alone, keeping the values.
+    ``bt_extra`` adds unused (-1) columns to the block table to exercise a stride
+    larger than the longest sequence needs.
+    """
+    device = torch.device(device)
+    sgen = torch.Generator().manual_seed(seed if perm_seed is None else perm_seed)
+    vgen = torch.Generator(device=device).manual_seed(seed + 1)     # bulk values
+    Hq, Hkv, d, P = num_q_heads, num_kv_heads, head_dim, page_size
+    B = len(seqs)
+    total_q = sum(s.query_len for s in seqs)
+    total_kv = sum(s.seq_len for s in seqs)
+
+    def randn_bf16(*shape):
+        return torch.randn(*shape, generator=vgen, device=device,
+                           dtype=torch.float32).to(torch.bfloat16)
+
+    q = randn_bf16(total_q, Hq, d)
+    k = randn_bf16(total_kv, Hkv, d)
+    v = randn_bf16(total_kv, Hkv, d)
+    if outlier_frac > 0:
+        flags = torch.rand(total_kv, Hkv, 1, generator=vgen, device=device) < outlier_frac
+        k = torch.where(flags, (k.float() * outlier_scale).to(torch.bfloat16), k)
+
+    pages_per_seq = [(s.seq_len + P - 1) // P for s in seqs]
+    num_pages = sum(pages_per_seq)
+    max_pages = max(pages_per_seq) + bt_extra
+    perm = torch.randperm(num_pages, generator=sgen)                # logical -> physical
+
+    block_table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    page_off = 0
+    tok_page = []      # per token: logical global page index
+    tok_slot = []
+    for i, s in enumerate(seqs):
+        n = pages_per_seq[i]
+        block_table[i, :n] = perm[page_off:page_off + n].to(torch.int32)
+        pos = torch.arange(s.seq_len)
+        tok_page.append(page_off + pos // P)
+        tok_slot.append(pos % P)
+        page_off += n
+    tok_phys = perm[torch.cat(tok_page)].to(device)
+    tok_slot = torch.cat(tok_slot).to(device)
+
+    # page-tail filler: finite, large, so an unmasked tail slot ruins parity
+    k_cache = (randn_bf16(num_pages, Hkv, P, d).float() * 50.0).to(torch.bfloat16)
+    v_cache = (randn_bf16(num_pages, Hkv, P, d).float() * 50.0).to(torch.bfloat16)
+    k_cache[tok_phys, :, tok_slot] = k
+    v_cache[tok_phys, :, tok_slot] = v
+    del tok_phys, tok_slot
+
+    return Batch(name=name, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=d, page_size=P,
+                 seqs=list(seqs), q=q, k=k if keep_contiguous else None,
+                 v=v if keep_contiguous else None, k_cache=k_cache, v_cache=v_cache,
+                 block_table=block_table.to(device), page_perm=perm,
+                 seed=seed, outlier_frac=outlier_frac)
+
+
+def make_config(name: str, device="cpu", seed: Optional[int] = None,
+                keep_contiguous: bool = True) -> Batch:
+    """One of the five named batches, seeded by its index unless ``seed`` is given."""
+    if seed is None:
+        seed = CONFIG_NAMES.index(name)
+    sgen = torch.Generator().manual_seed(seed)
+    seqs, Hq, Hkv, d, outl = config_seqs(name, sgen)
+    # structure draws above advance sgen; build_batch re-seeds its own structure stream
+    return build_batch(name, seqs, Hq, Hkv, d, seed=seed + 1000, device=device,
+                       outlier_frac=outl, keep_contiguous=keep_contiguous)
+
+
+def repage(batch: Batch, perm_seed: int) -> Batch:
+    """Same Q/K/V values, a different random page permutation (for invariance tests)."""
+    return build_batch(batch.name, batch.seqs, batch.num_q_heads, batch.num_kv_heads,
+                       batch.head_dim, seed=batch.seed, device=batch.q.device,
+                       page_size=batch.page_size, perm_seed=perm_seed,
+                       outlier_frac=batch.outlier_frac)
+
+
+def random_small(seed: int, num_seqs: int = 4, Hq: int = 8, Hkv: int = 2, d: int = 64,
+                 max_ctx: int = 80, max_q: int = 40, tree_frac: float = 0.3,
+                 max_draft: int = 8, device="cpu", bt_extra: int = 0) -> Batch:
+    """A small mixed batch: causal chunks of random length on random prefixes, decode
+    steps, and verify rows on random draft trees; sized for the CPU oracle."""
+    gen = torch.Generator().manual_seed(seed)
+    seqs = []
+    for _ in range(num_seqs):
+        r = torch.rand((), generator=gen).item()
+        prefix = int(torch.randint(0, max_ctx + 1, (1,), generator=gen).item())
+        if r < tree_frac:
+            T = int(torch.randint(1, max_draft + 1, (1,), generator=gen).item())
+            seqs.append(SeqSpec(prefix + T, T, TREE, random_tree(gen, T)))
+        else:
+            T = int(torch.randint(1, max_q + 1, (1,), generator=gen).item())
+            seqs.append(SeqSpec(prefix + T, T, CAUSAL, []))
+    return build_batch(f"random_small_{seed}", seqs, Hq, Hkv, d, seed=seed + 7,
+                       device=device, bt_extra=bt_extra)
