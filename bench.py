@@ -1,0 +1,315 @@
+"""Benchmark: mixed-batch paged attention on B200 through the library's C ABI.
+
+One step = one ``attn_run`` over the unified prefill / decode / verify batch shaped like
+Qwen2-7B (28 query / 4 KV heads, head_dim 128, page 16): 4 prefill chunks of 512 tokens,
+192 decode sequences (context U[256, 4096]) and 32 verify sequences with a random 5-node
+draft tree. Inputs are seeded synthetic bf16 N(0,1) values resident in HBM; the KV cache
+(about 1 GB) is larger than L2, so no flush is needed between steps.
+
+Prints ONE JSON line (rank 0). ``--impl reference`` times the float64 CPU oracle on the
+host cores on the same workload instead (the reference arm of this benchmark).
+Under torchrun each rank runs an independent replica on its own GPU (no data exchange);
+timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "mixed-batch paged attention: tokens/s; KV GB/s vs HBM peak; prefill TFLOP/s"
+DEFAULT_CONFIG = "qwen2_7b_unified"
+WORKLOADS = {
+    "tiny_decode": "4 decode seqs, ctx {17,64,100,255}, 8q/2kv heads, d64, page 16",
+    "llama3_8b_decode": "128 decode seqs, ctx U[512,8192], 32q/8kv heads, d128, page 16",
+    "llama33_70b_prefill": "8 x 2048-token causal chunks on ctx U[0,16384], 64q/8kv, d128, page 16",
+    "qwen2_7b_unified": "4 x 512 prefill + 192 decode (ctx U[256,4096]) + 32 verify (5-node tree), "
+                        "28q/4kv heads, d128, page 16",
+    "long_ctx_split": "16 decode seqs, ctx U[32768,131072], 128q/8kv, d128, page 16, 1% outlier keys x8",
+}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            pass
+        self.period = period_s
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._ok:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        s = sorted(self.samples)
+        return {"sm_mhz": s[len(s) // 2], "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(s)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class OracleRunner:
+    """The float64 oracle, as it stands, run over whole sequences of a batch in a cycle.
+
+    Host float64 copies are made up front (not timed); ``run(seconds)`` processes
+    sequences in order, wrapping around, until ``seconds`` have elapsed (at least one)."""
+
+    def __init__(self, batch):
+        import oracle
+        self._oracle = oracle
+        self.batch = batch
+        self.data = []
+        for i, sp in enumerate(batch.seqs):
+            k, v = batch.seq_kv(i)
+            self.data.append((batch.seq_q(i).double().cpu().numpy(), k.double().cpu().numpy(),
+                              v.double().cpu().numpy(), sp))
+        self.pos = 0
+        self.passes = 0.0
+        try:
+            import threadpoolctl
+            self.threads = max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()
+                               if i.get("user_api") == "blas")
+        except Exception:
+            self.threads = len(os.sched_getaffinity(0))
+
+    def run(self, seconds: float):
+        tokens, t0 = 0, time.perf_counter()
+        while True:
+            q, k, v, sp = self.data[self.pos]
+            self._oracle.attention([q], [k], [v], [sp.query_len], [sp.mask_kind], [sp.parents])
+            tokens += sp.query_len
+            self.pos = (self.pos + 1) % len(self.data)
+            self.passes += 1.0 / len(self.data)
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                return tokens, el
+
+    def sample_text(self):
+        return (f"whole sequences of the same batch taken in order, {self.passes:.2f} passes over "
+                f"all {len(self.data)} sequences")
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import workloads as W
+    batch = W.make_config(args.config, device="cpu")
+    runner = OracleRunner(batch)
+    step_s = args.ref_seconds / (args.warmup + args.steps)
+    for _ in range(args.warmup):
+        runner.run(step_s)
+    tok, sec = 0, 0.0
+    for _ in range(args.steps):
+        t, e = runner.run(step_s)
+        tok += t
+        sec += e
+    value = tok / sec
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": f"{args.config}: {WORKLOADS[args.config]}"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": runner.threads, "kind": "oracle",
+                             "sample": "each step: " + runner.sample_text()},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_attention_verify_b200 as pk
+    import workloads as W
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = load_peaks()
+
+    batch = W.make_config(args.config, device=dev)
+    plan = pk.plan_for_batch(batch)
+    info = plan.info()
+    stream = torch.cuda.current_stream()
+    out = torch.empty_like(batch.q)
+
+    def step():
+        plan.run(batch.q, batch.k_cache, batch.v_cache, out, stream)
+
+    for _ in range(args.warmup):
+        step()
+    if plan.check(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+    torch.cuda.synchronize()
+
+    n_ev = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev + 1)]
+    with ClockSampler(dev.index) as clk:
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(n_ev)]   # ms, one launch per step
+    elapsed_ms = ev[0].elapsed_time(ev[-1])
+    if ws > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    if plan.check(stream) != 0:
+        raise RuntimeError("device error during the timed region")
+
+    # end to end through the C ABI with host buffers (pinned), copies inside the region
+    q_host = batch.q.cpu().pin_memory()
+    o_host = torch.empty(q_host.shape, dtype=torch.bfloat16).pin_memory()
+    for _ in range(args.warmup):
+        plan.run_host(q_host, batch.k_cache, batch.v_cache, o_host, stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        plan.run_host(q_host, batch.k_cache, batch.v_cache, o_host, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if ws > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    tokens = batch.total_q
+    value = ws * tokens * args.steps / (elapsed_ms * 1e-3)
+    e2e_value = ws * tokens * args.steps / (e2e_ms * 1e-3)
+    avg_launch_s = (sum(per) / len(per)) * 1e-3
+    kv_gbs = info["kv_bytes"] / avg_launch_s / 1e9
+    tflops = info["attn_flops"] / avg_launch_s / 1e12
+    io_bytes = tokens * batch.num_q_heads * batch.head_dim * 2
+
+    result = None
+    if rank == 0:
+        cpu = None
+        if ws == 1 and not args.no_cpu_baseline:
+            runner = OracleRunner(batch)
+            tk, sec = runner.run(args.cpu_seconds)
+            cpu = {"value": tk / sec, "unit": "tokens/s", "cores": runner.threads, "kind": "oracle",
+                   "sample": runner.sample_text()}
+        result = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{args.config}: {WORKLOADS[args.config]}",
+                       "query_tokens_per_step": tokens, "kv_bytes_per_step": info["kv_bytes"],
+                       "l2": "inputs larger than L2 (KV cache read each step exceeds 126 MB)",
+                       "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+            "kv_gbs": kv_gbs, "kv_frac_of_hbm": kv_gbs / peaks["hbm_gbs"], "prefill_tflops": tflops,
+            "roofline": {"bound": "hbm", "achieved": kv_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": kv_gbs / peaks["hbm_gbs"], "traffic": None,
+                         "kernel": "decode_kernel", "peak_source": peaks["source"]},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
+                    "d2h_bytes_per_step": io_bytes},
+            "gpu_launches": args.steps * 1,
+            "clocks": clk.summary(),
+            "plan": {k: info[k] for k in ("num_decode_items", "num_split_units", "decode_rows")},
+        }
+        print(json.dumps(result))
+    plan.close()
+    if ws > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="host time for the oracle baseline line of our arm")
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="total host time the reference arm spreads over warm-up + steps")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,197 @@
+/*
+ * pkva.h — C ABI of a B200 (sm_100a) library for attention over a paged KV cache, serving
+ * one mixed batch of prefill chunks, decode steps and speculative-verify tokens under
+ * grouped-query attention.
+ *
+ * The operation (stated once; every entry point below refers to it):
+ *   For each sequence s with total KV length L_s (committed prefix plus new tokens) and
+ *   T_s new query tokens, query row i sits at absolute position L_s - T_s + i. Query head
+ *   h reads KV head h / (Hq / Hkv) (grouped-query attention). The output row is
+ *       out[i, h] = sum_j softmax_j(scale * <q[i, h], k[j, g]>) v[j, g]
+ *   over the allowed keys j:
+ *     PKVA_CAUSAL  j <= L_s - T_s + i   (a prefill chunk on a cached prefix; a decode step)
+ *     PKVA_TREE    j <  L_s - T_s, or j = L_s - T_s + a with a = i or an ancestor of i in
+ *                  the draft tree given as a parent array (speculative-decoding verify).
+ *   Sources: XY-Serve (arXiv 2412.18106), verdict page — core_discovery (prefill, decode
+ *   and verify tokens share one budgeted batch over a paged block cache, with chunked
+ *   prefill and prefix caching), forward_implications[2] (a single attention kernel that
+ *   picks the visible keys row by row covers all three kinds of row),
+ *   referee_report.significance (verify runs over a tree of draft tokens); Understanding
+ *   Inference Scaling for LLMs (arXiv 2605.19775), reference list (PagedAttention;
+ *   grouped-query attention).
+ *
+ * Memory layout (all device tensors are dense, row-major, bf16 unless noted):
+ *   q, out      [sum_s T_s, Hq, D]  — ragged: the new tokens of sequence 0, then of 1, ...
+ *   k_cache,
+ *   v_cache     [num_pages, Hkv, page_size, D] — one (page, kv head) block is contiguous
+ *   block_table int32 [num_seqs, bt_stride]; entry (s, p) is the physical page that holds
+ *               keys p*page_size .. p*page_size+page_size-1 of sequence s. Entries past
+ *               ceil(L_s / page_size) are never read.
+ *   The K/V of the new tokens must already be in the cache (at positions L_s-T_s .. L_s-1).
+ *   Cache slots past L_s in a sequence's last page are never attended to but are read by
+ *   the tensor-core path; they must hold finite values (any stale bf16 data is fine).
+ *
+ * Threading and errors: every call returns a pkva_status. On failure, attn_last_error()
+ * returns a message for the calling thread. A plan may be used from one stream at a time;
+ * distinct plans are independent. attn_run is asynchronous: it never synchronizes.
+ */
+#ifndef PKVA_H
+#define PKVA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PKVA_API __attribute__((visibility("default")))
+#else
+#define PKVA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct pkva_plan* pkva_plan_t;
+
+enum pkva_mask_kind {
+    PKVA_CAUSAL = 0,   /* prefill chunk or decode step: bottom-right causal mask        */
+    PKVA_TREE = 1      /* verify: committed prefix + ancestors-or-self in the draft tree */
+};
+
+enum pkva_status {
+    PKVA_OK = 0,
+    PKVA_EINVAL = -1,        /* bad argument (message says which)                        */
+    PKVA_EUNSUPPORTED = -2,  /* valid but not supported: head_dim, page_size, device     */
+    PKVA_ECUDA = -3,         /* a CUDA runtime call or a launch failed                   */
+    PKVA_ENOMEM = -4,        /* device or host allocation failed                         */
+    PKVA_EDEVICE = -5        /* the kernels flagged an error (see attn_check)            */
+};
+
+/* Device error bits reported by attn_check (PKVA_EDEVICE). */
+#define PKVA_DEVERR_BAD_PAGE   0x1  /* a block-table entry was outside [0, num_pages)      */
+#define PKVA_DEVERR_TIMEOUT    0x2  /* a bounded wait on an asynchronous copy gave up       */
+
+/*
+ * attn_plan — decompose one batch into tile tasks and upload them (host call, may block).
+ *
+ * Cites: XY-Serve verdict page, core_discovery (the mixed batch is broken into fixed-size
+ * tile tasks, kept in its Token-Table / Task-Table, which are then reordered so that the
+ * cores get balanced work) and key_machinery (attention tiles are ordered by how much work
+ * they hold and dealt out to the cores in a symmetric round-robin).
+ *
+ *   out_plan      receives the plan handle (set to NULL on failure).
+ *   num_seqs      number of sequences B (0 is allowed: attn_run then does nothing).
+ *   seq_lens      host int32[B]: L_s, total KV length including the new tokens (>= 1).
+ *   query_lens    host int32[B]: T_s, number of new query tokens, 1 <= T_s <= L_s.
+ *   block_table   device int32[B * bt_stride] (see layout above). Read at every attn_run,
+ *                 so its contents may change between runs without re-planning. Owned by
+ *                 the caller; must stay allocated while the plan is used.
+ *   bt_stride     row stride of block_table in entries; >= ceil(L_s / page_size) for all s.
+ *   num_pages     number of pages in k_cache / v_cache (bounds every block-table entry).
+ *   mask_kind     host int32[B]: PKVA_CAUSAL or PKVA_TREE per sequence.
+ *   parents       host int32[sum of T_s over TREE sequences]: the draft trees, concatenated
+ *                 in sequence order; parents[i] is -1 (hangs off the committed prefix) or
+ *                 an earlier node of the same tree. May be NULL if no sequence is TREE.
+ *                 TREE sequences need T_s <= 64.
+ *   num_q_heads   Hq; num_kv_heads Hkv; Hq must be a multiple of Hkv.
+ *   head_dim      D: 64 or 128.
+ *   page_size     16.
+ *   sm_scale      softmax scale; <= 0 selects 1/sqrt(D).
+ *
+ * Returns PKVA_OK, PKVA_EINVAL (inputs), PKVA_EUNSUPPORTED (head_dim, page_size, a device
+ * that is not sm_100), PKVA_ENOMEM or PKVA_ECUDA. The plan owns its device work lists and
+ * split-KV scratch; all are freed by attn_plan_destroy.
+ */
+PKVA_API int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq_lens,
+              const int32_t* query_lens, const int32_t* block_table, int bt_stride,
+              int num_pages, const int32_t* mask_kind, const int32_t* parents,
+              int num_q_heads, int num_kv_heads, int head_dim, int page_size, float sm_scale);
+
+/*
+ * attn_run — compute the batch's attention on `stream` (asynchronous).
+ *
+ *   q        device bf16 [sum T_s, Hq, D]
+ *   k_cache  device bf16 [num_pages, Hkv, page_size, D]; v_cache likewise.
+ *   out      device bf16 [sum T_s, Hq, D]; must not overlap q or the caches.
+ *   stream   a cudaStream_t (NULL = legacy default stream).
+ *
+ * All pointers must be 16-byte aligned. Results are bf16 (fp32 accumulation inside).
+ * Returns PKVA_OK, PKVA_EINVAL (NULL or misaligned pointer, NULL plan) or PKVA_ECUDA
+ * (launch failure). Device-side problems (a block-table entry out of range) do not fault:
+ * the page reads as zeros and attn_check reports PKVA_EDEVICE.
+ */
+PKVA_API int attn_run(pkva_plan_t plan, const void* q, const void* k_cache, const void* v_cache,
+             void* out, void* stream);
+
+/*
+ * attn_run_host — attn_run with q and out in HOST memory (the end-to-end call).
+ *
+ * Copies q (host, [sum T_s, Hq, D] bf16) to a plan-owned device buffer, runs, and copies
+ * the result back to out (host), all on `stream`; returns after enqueueing. The caller
+ * synchronizes the stream before reading `out`. Pinned host memory makes the copies
+ * asynchronous; pageable memory works but the copies then block. The caches stay in
+ * device memory (they are the resident KV state).
+ */
+PKVA_API int attn_run_host(pkva_plan_t plan, const void* q_host, const void* k_cache,
+                  const void* v_cache, void* out_host, void* stream);
+
+/*
+ * attn_check — synchronize `stream`, read and clear the plan's device error word.
+ * Returns PKVA_OK, PKVA_EDEVICE (bits in *device_error if not NULL) or PKVA_ECUDA.
+ */
+PKVA_API int attn_check(pkva_plan_t plan, void* stream, int32_t* device_error);
+
+/* attn_plan_destroy — free a plan (NULL is ignored). Synchronizes the plan's device. */
+PKVA_API void attn_plan_destroy(pkva_plan_t plan);
+
+/* attn_last_error — message for the last failing call on this thread ("" if none). */
+PKVA_API const char* attn_last_error(void);
+
+/* Summary of a plan's decomposition (for logging and tests). */
+typedef struct pkva_plan_info {
+    int32_t num_seqs;
+    int32_t num_decode_items;    /* CUDA-core decode/verify tile tasks (one CTA each)      */
+    int32_t num_prefill_items;   /* tensor-core prefill tile tasks                          */
+    int32_t num_split_units;     /* (seq, kv head, row chunk) units split over several CTAs */
+    int32_t num_partial_slots;   /* split-KV partial results held in plan scratch           */
+    int32_t decode_rows;         /* rows per decode task the launch is compiled for         */
+    int64_t kv_bytes;            /* algorithmic K+V bytes one run reads (each element once)  */
+    int64_t attn_flops;          /* algorithmic 4*D*Hq flops per allowed (query, key) pair  */
+    int64_t scratch_bytes;       /* device scratch the plan owns                            */
+} pkva_plan_info;
+
+PKVA_API int attn_plan_get_info(pkva_plan_t plan, pkva_plan_info* info);
+
+/* One tile task as the planner emitted it (host-side inspection only). */
+typedef struct pkva_work_desc {
+    int32_t kind;        /* 0 = decode/verify task, 1 = prefill task                      */
+    int32_t seq;         /* sequence index                                                 */
+    int32_t kv_head;     /* KV head; the task covers query heads of this head's group      */
+    int32_t row_begin;   /* first packed row (row = token * group + head-in-group)         */
+    int32_t row_count;   /* packed rows in the task                                        */
+    int32_t key_begin;   /* first key position covered                                     */
+    int32_t key_end;     /* one past the last key position covered                          */
+    int32_t split;       /* split index within its unit, -1 if the unit is not split       */
+    int32_t num_splits;  /* number of splits of its unit (1 if not split)                  */
+} pkva_work_desc;
+
+/*
+ * attn_plan_inspect — run the planner on the host only (no device, nothing allocated on
+ * it) and return its tile tasks in launch order. Arguments as attn_plan, plus:
+ *   num_sms, ctas_per_sm   the machine the plan should balance for;
+ *   items, max_items       output array (may be NULL to query the count);
+ *   num_items              receives the number of tasks.
+ * Returns PKVA_OK, PKVA_EINVAL / PKVA_EUNSUPPORTED (same checks as attn_plan), or
+ * PKVA_EINVAL if max_items is too small (num_items still set).
+ */
+PKVA_API int attn_plan_inspect(int num_seqs, const int32_t* seq_lens, const int32_t* query_lens,
+                      int bt_stride, int num_pages, const int32_t* mask_kind,
+                      const int32_t* parents, int num_q_heads, int num_kv_heads,
+                      int head_dim, int page_size, int num_sms, int ctas_per_sm,
+                      pkva_work_desc* items, int max_items, int* num_items);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKVA_H */

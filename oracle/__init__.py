@@ -26,11 +26,11 @@ What it computes (exact softmax attention, written out as its definition):
 
 Passages followed:
   * XY-Serve (arXiv 2412.18106), verdict page, ``pith_extraction.forward_implications[2]``:
-    one attention meta-kernel with row-wise mask control serves prefill, decode and
-    verify rows; ``core_discovery``: chunked prefill, prefix caching and a
-    PagedAttention-style block cache are all instances of one tiled attention;
-    ``referee_report.significance``: tree-based speculative decoding; supporting
-    citation [1]: FlashAttention's QK / softmax / SV pattern.
+    a single attention kernel, choosing the visible keys row by row, covers prefill,
+    decode and verify rows; ``core_discovery``: chunked prefill, prefix caching and a
+    paged block cache are all cases of one tiled attention; ``referee_report.significance``:
+    verify runs over a tree of draft tokens; supporting citation [1]: FlashAttention's
+    QK / softmax / SV pattern.
   * Understanding Inference Scaling for LLMs (arXiv 2605.19775), reference list:
     PagedAttention and grouped-query attention (the GQA head grouping).
 
@@ -59,8 +59,8 @@ TREE = 1
 def ancestors_or_self(parents: Sequence[int]) -> List[List[int]]:
     """For each draft node i, the sorted list {i} U ancestors(i) under the parent array.
 
-    Tree encoding (reading of 'tree-based speculative decoding', XY-Serve verdict page,
-    ``referee_report.significance``): parents[i] is -1 or an earlier node index.
+    Tree encoding (a reading of the draft tree of speculative decoding, XY-Serve verdict
+    page, ``referee_report.significance``): parents[i] is -1 or an earlier node index.
     """
     out = []
     for i in range(len(parents)):
@@ -77,10 +77,10 @@ def ancestors_or_self(parents: Sequence[int]) -> List[List[int]]:
 
 def allowed_mask(seq_len: int, query_len: int, mask_kind: int,
                  parents: Optional[Sequence[int]] = None) -> np.ndarray:
-    """Boolean [T, L]: which keys each new query row may attend to (row-wise mask).
+    """Boolean [T, L]: which keys each new query row may attend to.
 
-    XY-Serve verdict page, ``forward_implications[2]`` (row-wise mask control for
-    prefill, decode and verify rows).
+    XY-Serve verdict page, ``forward_implications[2]`` (the visible keys are chosen per
+    row, for prefill, decode and verify rows alike).
     """
     L, T = seq_len, query_len
     if not (1 <= T <= L):

@@ -1,0 +1,224 @@
+"""Paged-KV attention for unified prefill / decode / verify batches on B200 (sm_100a).
+
+Thin ctypes binding over the C ABI in ``include/pkva.h`` (library: ``lib/libpkva.so``,
+built in-tree by ``python -m paged_kv_attention_verify_b200.build``). This module only
+marshals arguments: host integer arrays go in as int32 buffers, device tensors as raw
+pointers, the stream as a ``cudaStream_t``. Every step of the computation runs in the
+library's kernels; there is no fallback of any kind, so a missing library is an error.
+
+    plan = Plan(seq_lens, query_lens, block_table, mask_kind, parents,
+                num_q_heads=32, num_kv_heads=8, head_dim=128, num_pages=P)
+    out = plan.run(q, k_cache, v_cache)        # q, caches, out: bf16 CUDA tensors
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libpkva.so")
+
+CAUSAL = 0
+TREE = 1
+
+PKVA_OK = 0
+STATUS_NAMES = {0: "PKVA_OK", -1: "PKVA_EINVAL", -2: "PKVA_EUNSUPPORTED", -3: "PKVA_ECUDA",
+                -4: "PKVA_ENOMEM", -5: "PKVA_EDEVICE"}
+DEVERR_BAD_PAGE = 0x1
+DEVERR_TIMEOUT = 0x2
+
+# every entry point that include/pkva.h declares
+EXPORTED = ["attn_plan", "attn_run", "attn_run_host", "attn_check", "attn_plan_destroy",
+            "attn_last_error", "attn_plan_get_info", "attn_plan_inspect"]
+
+
+class PkvaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("num_decode_items", ctypes.c_int32),
+                ("num_prefill_items", ctypes.c_int32), ("num_split_units", ctypes.c_int32),
+                ("num_partial_slots", ctypes.c_int32), ("decode_rows", ctypes.c_int32),
+                ("kv_bytes", ctypes.c_int64), ("attn_flops", ctypes.c_int64),
+                ("scratch_bytes", ctypes.c_int64)]
+
+
+class WorkDesc(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("seq", ctypes.c_int32), ("kv_head", ctypes.c_int32),
+                ("row_begin", ctypes.c_int32), ("row_count", ctypes.c_int32),
+                ("key_begin", ctypes.c_int32), ("key_end", ctypes.c_int32),
+                ("split", ctypes.c_int32), ("num_splits", ctypes.c_int32)]
+
+
+_lib = None
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_vp = ctypes.c_void_p
+
+
+def lib() -> ctypes.CDLL:
+    """Load the in-tree library (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m paged_kv_attention_verify_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    L.attn_plan.argtypes = [ctypes.POINTER(_vp), ctypes.c_int, _i32p, _i32p, _vp, ctypes.c_int,
+                            ctypes.c_int, _i32p, _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                            ctypes.c_int, ctypes.c_float]
+    L.attn_run.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp]
+    L.attn_run_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp]
+    L.attn_check.argtypes = [_vp, _vp, _i32p]
+    L.attn_plan_destroy.argtypes = [_vp]
+    L.attn_plan_destroy.restype = None
+    L.attn_last_error.restype = ctypes.c_char_p
+    L.attn_plan_get_info.argtypes = [_vp, ctypes.POINTER(PlanInfo)]
+    L.attn_plan_inspect.argtypes = [ctypes.c_int, _i32p, _i32p, ctypes.c_int, ctypes.c_int, _i32p,
+                                    _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_int, ctypes.c_int, ctypes.POINTER(WorkDesc),
+                                    ctypes.c_int, _i32p]
+    for name in ("attn_plan", "attn_run", "attn_run_host", "attn_check", "attn_plan_get_info",
+                 "attn_plan_inspect"):
+        getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _check(rc: int):
+    if rc != PKVA_OK:
+        raise PkvaError(rc, lib().attn_last_error().decode())
+
+
+def _i32(values) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(values, dtype=np.int32).reshape(-1))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(_i32p) if a.size else None
+
+
+def _stream_handle(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+class Plan:
+    """A planned batch (``attn_plan``); run it any number of times with ``run``."""
+
+    def __init__(self, seq_lens: Sequence[int], query_lens: Sequence[int], block_table,
+                 mask_kind: Sequence[int], parents: Optional[Sequence[int]] = None, *,
+                 num_q_heads: int, num_kv_heads: int, head_dim: int, num_pages: int,
+                 page_size: int = 16, sm_scale: Optional[float] = None):
+        import torch
+        self._handle = None
+        sl, ql, mk = _i32(seq_lens), _i32(query_lens), _i32(mask_kind)
+        par = _i32(parents if parents is not None else [])
+        if len(sl) != len(ql) or len(sl) != len(mk):
+            raise ValueError("seq_lens, query_lens and mask_kind must have one entry per sequence")
+        if len(sl):
+            if not (isinstance(block_table, torch.Tensor) and block_table.is_cuda
+                    and block_table.dtype == torch.int32 and block_table.dim() == 2
+                    and block_table.is_contiguous() and block_table.shape[0] == len(sl)):
+                raise ValueError("block_table must be a contiguous int32 CUDA tensor [num_seqs, bt_stride]")
+            bt_ptr, bt_stride = block_table.data_ptr(), block_table.shape[1]
+        else:
+            bt_ptr, bt_stride = None, 0
+        self.block_table = block_table          # keep the caller's table alive with the plan
+        self.num_q_heads, self.num_kv_heads, self.head_dim = num_q_heads, num_kv_heads, head_dim
+        self.num_pages, self.page_size = num_pages, page_size
+        self.total_q = int(ql.sum()) if len(ql) else 0
+        h = _vp()
+        _check(lib().attn_plan(ctypes.byref(h), len(sl), _ptr(sl), _ptr(ql), bt_ptr, bt_stride,
+                               num_pages, _ptr(mk), _ptr(par), num_q_heads, num_kv_heads, head_dim,
+                               page_size, float(sm_scale) if sm_scale else 0.0))
+        self._handle = h
+
+    # -- marshalling checks (shapes, dtypes, devices) ---------------------------------
+    def _check_tensors(self, q, k_cache, v_cache, out):
+        import torch
+        D, Hq, Hkv = self.head_dim, self.num_q_heads, self.num_kv_heads
+        for name, t, shape in (("q", q, (self.total_q, Hq, D)), ("out", out, (self.total_q, Hq, D)),
+                               ("k_cache", k_cache, (self.num_pages, Hkv, self.page_size, D)),
+                               ("v_cache", v_cache, (self.num_pages, Hkv, self.page_size, D))):
+            if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.bfloat16:
+                raise ValueError(f"{name} must be a bf16 CUDA tensor")
+            if tuple(t.shape) != shape or not t.is_contiguous():
+                raise ValueError(f"{name} must be contiguous with shape {shape}, got {tuple(t.shape)}")
+
+    def run(self, q, k_cache, v_cache, out=None, stream=None):
+        """out = attention(q, paged K/V); asynchronous on ``stream`` (default: current)."""
+        import torch
+        if out is None:
+            out = torch.empty_like(q)
+        self._check_tensors(q, k_cache, v_cache, out)
+        _check(lib().attn_run(self._handle, q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                              out.data_ptr(), _stream_handle(stream)))
+        return out
+
+    def run_host(self, q_host, k_cache, v_cache, out_host, stream=None):
+        """End-to-end call: q and out in (pinned) host memory; copies ride on ``stream``."""
+        import torch
+        for name, t in (("q_host", q_host), ("out_host", out_host)):
+            if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or \
+                    tuple(t.shape) != (self.total_q, self.num_q_heads, self.head_dim):
+                raise ValueError(f"{name} must be a contiguous bf16 host tensor "
+                                 f"[{self.total_q}, {self.num_q_heads}, {self.head_dim}]")
+        _check(lib().attn_run_host(self._handle, q_host.data_ptr(), k_cache.data_ptr(),
+                                   v_cache.data_ptr(), out_host.data_ptr(), _stream_handle(stream)))
+        return out_host
+
+    def check(self, stream=None) -> int:
+        """Synchronize and return the device error bits (0 if none); raises on CUDA errors."""
+        err = ctypes.c_int32(0)
+        rc = lib().attn_check(self._handle, _stream_handle(stream), ctypes.byref(err))
+        if rc not in (PKVA_OK, -5):
+            _check(rc)
+        return int(err.value)
+
+    def info(self) -> Dict[str, int]:
+        inf = PlanInfo()
+        _check(lib().attn_plan_get_info(self._handle, ctypes.byref(inf)))
+        return {f: getattr(inf, f) for f, _ in PlanInfo._fields_}
+
+    def close(self):
+        if self._handle:
+            lib().attn_plan_destroy(self._handle)
+            self._handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def inspect(seq_lens, query_lens, mask_kind, parents=None, *, num_q_heads: int,
+            num_kv_heads: int, head_dim: int, num_pages: int, bt_stride: int,
+            num_sms: int = 148, ctas_per_sm: int = 2, page_size: int = 16) -> List[Dict[str, int]]:
+    """Host-only planner run (``attn_plan_inspect``): the tile tasks in launch order."""
+    sl, ql, mk = _i32(seq_lens), _i32(query_lens), _i32(mask_kind)
+    par = _i32(parents if parents is not None else [])
+    n = ctypes.c_int32(0)
+    args = (len(sl), _ptr(sl), _ptr(ql), bt_stride, num_pages, _ptr(mk), _ptr(par), num_q_heads,
+            num_kv_heads, head_dim, page_size, num_sms, ctas_per_sm)
+    _check(lib().attn_plan_inspect(*args, None, 0, ctypes.byref(n)))
+    arr = (WorkDesc * max(1, n.value))()
+    _check(lib().attn_plan_inspect(*args, arr, n.value, ctypes.byref(n)))
+    return [{f: getattr(arr[i], f) for f, _ in WorkDesc._fields_} for i in range(n.value)]
+
+
+def plan_for_batch(batch, sm_scale: Optional[float] = None) -> Plan:
+    """Plan a ``workloads.Batch`` (a convenience for tests and the benchmark)."""
+    return Plan(batch.seq_lens, batch.query_lens, batch.block_table, batch.mask_kinds,
+                batch.parents_flat, num_q_heads=batch.num_q_heads, num_kv_heads=batch.num_kv_heads,
+                head_dim=batch.head_dim, num_pages=batch.k_cache.shape[0],
+                page_size=batch.page_size, sm_scale=sm_scale)

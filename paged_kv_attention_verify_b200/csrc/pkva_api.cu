@@ -1,0 +1,347 @@
+// The C ABI (include/pkva.h): plan objects, device buffers, tensor maps and launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <math.h>
+#include <stdio.h>
+
+#include <mutex>
+#include <new>
+#include <string>
+
+#include "pkva.h"
+#include "pkva_internal.h"
+#include "pkva_kernels.h"
+
+namespace pkva {
+
+static thread_local std::string g_last_error;
+
+void set_last_error(const std::string& msg) { g_last_error = msg; }
+
+static int cuda_fail(cudaError_t e, const char* what) {
+    std::string m = std::string(what) + ": " + cudaGetErrorString(e);
+    set_last_error(m);
+    return e == cudaErrorMemoryAllocation ? PKVA_ENOMEM : PKVA_ECUDA;
+}
+
+#define PKVA_CUDA(call, what)                          \
+    do {                                               \
+        cudaError_t e_ = (call);                       \
+        if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+    } while (0)
+
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// The cache viewed as a 2-D bf16 tensor [num_pages * Hkv * 16 rows, D columns]; one box
+// is 16 rows (one page of one KV head) x 64 columns, stored with the 128-byte swizzle.
+static bool encode_cache_map(CUtensorMap* map, const void* base, int num_pages, int Hkv, int D) {
+    auto fn = tensor_map_encoder();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)num_pages * Hkv * kPageSize};
+    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)kPageSize};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <class T>
+static int upload(T** dst, const std::vector<T>& src, int64_t* bytes) {
+    *dst = nullptr;
+    if (src.empty()) return PKVA_OK;
+    PKVA_CUDA(cudaMalloc(dst, src.size() * sizeof(T)), "cudaMalloc(plan tables)");
+    PKVA_CUDA(cudaMemcpy(*dst, src.data(), src.size() * sizeof(T), cudaMemcpyHostToDevice), "upload plan");
+    *bytes += (int64_t)(src.size() * sizeof(T));
+    return PKVA_OK;
+}
+
+}  // namespace pkva
+
+struct pkva_plan {
+    pkva::HostPlan hp;
+    int device = 0;
+    int num_sms = 0;
+    int decode_ctas = 0;
+    const int32_t* block_table = nullptr;
+    pkva::SeqInfo* d_seqs = nullptr;
+    pkva::DecodeWork* d_dwork = nullptr;
+    pkva::SplitUnit* d_units = nullptr;
+    uint64_t* d_anc = nullptr;
+    float* d_part_o = nullptr;
+    float* d_part_ml = nullptr;
+    int32_t* d_counters = nullptr;
+    int32_t* d_err = nullptr;
+    void* d_qstage = nullptr;
+    void* d_ostage = nullptr;
+    CUtensorMap tmK, tmV;
+    const void* tm_k = nullptr;
+    const void* tm_v = nullptr;
+    int64_t scratch_bytes = 0;
+};
+
+using namespace pkva;
+
+static void free_plan(pkva_plan* p) {
+    if (!p) return;
+    cudaFree(p->d_seqs);
+    cudaFree(p->d_dwork);
+    cudaFree(p->d_units);
+    cudaFree(p->d_anc);
+    cudaFree(p->d_part_o);
+    cudaFree(p->d_part_ml);
+    cudaFree(p->d_counters);
+    cudaFree(p->d_err);
+    cudaFree(p->d_qstage);
+    cudaFree(p->d_ostage);
+    delete p;
+}
+
+extern "C" const char* attn_last_error(void) { return g_last_error.c_str(); }
+
+extern "C" int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq_lens, const int32_t* query_lens,
+                         const int32_t* block_table, int bt_stride, int num_pages, const int32_t* mask_kind,
+                         const int32_t* parents, int num_q_heads, int num_kv_heads, int head_dim, int page_size,
+                         float sm_scale) {
+    if (!out_plan) {
+        set_last_error("attn_plan: out_plan is NULL");
+        return PKVA_EINVAL;
+    }
+    *out_plan = nullptr;
+    if (num_seqs > 0 && !block_table) {
+        set_last_error("attn_plan: block_table is NULL");
+        return PKVA_EINVAL;
+    }
+    // validate on the host first (a bad batch never touches the device)
+    PlanArgs a{num_seqs, seq_lens, query_lens, bt_stride, num_pages, mask_kind, parents, num_q_heads,
+               num_kv_heads, head_dim, page_size, sm_scale, 1, 1};
+    {
+        HostPlan probe;
+        std::string err;
+        const int rc = build_host_plan(a, &probe, &err);
+        if (rc != PKVA_OK) {
+            set_last_error("attn_plan: " + err);
+            return rc;
+        }
+    }
+
+    int dev = 0, major = 0, sms = 0;
+    PKVA_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    PKVA_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev), "device attribute");
+    PKVA_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "device attribute");
+    if (major != 10) {
+        set_last_error("attn_plan: this library is built for sm_100a (B200); the current device is not");
+        return PKVA_EUNSUPPORTED;
+    }
+
+    pkva_plan* p = new (std::nothrow) pkva_plan();
+    if (!p) {
+        set_last_error("attn_plan: out of host memory");
+        return PKVA_ENOMEM;
+    }
+    p->device = dev;
+    p->num_sms = sms;
+    p->block_table = block_table;
+
+    // the decode kernel's residency decides how many CTA slots the planner balances for
+    {
+        HostPlan probe;
+        std::string err;
+        build_host_plan(a, &probe, &err);
+        p->decode_ctas = decode_ctas_per_sm(head_dim, probe.decode_rows);
+        if (p->decode_ctas < 1) {
+            free_plan(p);
+            set_last_error("attn_plan: decode kernel cannot be resident (shared memory)");
+            return PKVA_ECUDA;
+        }
+    }
+    a.num_sms = sms;
+    a.ctas_per_sm = p->decode_ctas;
+    std::string err;
+    int rc = build_host_plan(a, &p->hp, &err);
+    if (rc != PKVA_OK) {
+        free_plan(p);
+        set_last_error("attn_plan: " + err);
+        return rc;
+    }
+    // the kernel set for the final row count may differ from the probe's; re-query
+    p->decode_ctas = decode_ctas_per_sm(head_dim, p->hp.decode_rows);
+
+    const HostPlan& hp = p->hp;
+#define PKVA_TRY(x)              \
+    do {                         \
+        int rc_ = (x);           \
+        if (rc_ != PKVA_OK) {    \
+            free_plan(p);        \
+            return rc_;          \
+        }                        \
+    } while (0)
+    PKVA_TRY(upload(&p->d_seqs, hp.seqs, &p->scratch_bytes));
+    PKVA_TRY(upload(&p->d_dwork, hp.dwork, &p->scratch_bytes));
+    PKVA_TRY(upload(&p->d_units, hp.units, &p->scratch_bytes));
+    PKVA_TRY(upload(&p->d_anc, hp.anc, &p->scratch_bytes));
+    auto alloc_zero = [&](void** ptr, size_t bytes, const char* what) -> int {
+        if (bytes == 0) return PKVA_OK;
+        cudaError_t e = cudaMalloc(ptr, bytes);
+        if (e != cudaSuccess) return cuda_fail(e, what);
+        e = cudaMemset(*ptr, 0, bytes);
+        if (e != cudaSuccess) return cuda_fail(e, what);
+        p->scratch_bytes += (int64_t)bytes;
+        return PKVA_OK;
+    };
+    PKVA_TRY(alloc_zero((void**)&p->d_part_o, (size_t)hp.num_slots * kDecodeRowsMax * hp.D * sizeof(float),
+                        "cudaMalloc(split partials)"));
+    PKVA_TRY(alloc_zero((void**)&p->d_part_ml, (size_t)hp.num_slots * kDecodeRowsMax * 2 * sizeof(float),
+                        "cudaMalloc(split partials)"));
+    PKVA_TRY(alloc_zero((void**)&p->d_counters, hp.units.size() * sizeof(int32_t), "cudaMalloc(split counters)"));
+    PKVA_TRY(alloc_zero((void**)&p->d_err, sizeof(int32_t), "cudaMalloc(error word)"));
+#undef PKVA_TRY
+    set_last_error("");
+    *out_plan = p;
+    return PKVA_OK;
+}
+
+extern "C" void attn_plan_destroy(pkva_plan_t plan) {
+    if (!plan) return;
+    const int dev = plan->device;
+    int cur = 0;
+    cudaGetDevice(&cur);
+    if (cur != dev) cudaSetDevice(dev);
+    cudaDeviceSynchronize();
+    free_plan(plan);
+    if (cur != dev) cudaSetDevice(cur);
+}
+
+extern "C" int attn_plan_get_info(pkva_plan_t plan, pkva_plan_info* info) {
+    if (!plan || !info) {
+        set_last_error("attn_plan_get_info: NULL argument");
+        return PKVA_EINVAL;
+    }
+    const HostPlan& hp = plan->hp;
+    info->num_seqs = hp.num_seqs;
+    info->num_decode_items = (int32_t)hp.dwork.size();
+    info->num_prefill_items = 0;
+    info->num_split_units = (int32_t)hp.units.size();
+    info->num_partial_slots = hp.num_slots;
+    info->decode_rows = hp.decode_rows;
+    info->kv_bytes = hp.kv_bytes;
+    info->attn_flops = hp.attn_flops;
+    info->scratch_bytes = plan->scratch_bytes;
+    return PKVA_OK;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+extern "C" int attn_run(pkva_plan_t plan, const void* q, const void* k_cache, const void* v_cache, void* out,
+                        void* stream) {
+    if (!plan) {
+        set_last_error("attn_run: plan is NULL");
+        return PKVA_EINVAL;
+    }
+    const HostPlan& hp = plan->hp;
+    if (hp.num_seqs == 0) return PKVA_OK;
+    if (!q || !k_cache || !v_cache || !out) {
+        set_last_error("attn_run: NULL tensor pointer");
+        return PKVA_EINVAL;
+    }
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) {
+        set_last_error("attn_run: tensor pointers must be 16-byte aligned");
+        return PKVA_EINVAL;
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (plan->tm_k != k_cache) {
+        if (!encode_cache_map(&plan->tmK, k_cache, hp.num_pages, hp.Hkv, hp.D)) {
+            set_last_error("attn_run: cuTensorMapEncodeTiled failed for k_cache");
+            return PKVA_ECUDA;
+        }
+        plan->tm_k = k_cache;
+    }
+    if (plan->tm_v != v_cache) {
+        if (!encode_cache_map(&plan->tmV, v_cache, hp.num_pages, hp.Hkv, hp.D)) {
+            set_last_error("attn_run: cuTensorMapEncodeTiled failed for v_cache");
+            return PKVA_ECUDA;
+        }
+        plan->tm_v = v_cache;
+    }
+    DecodeParams dp;
+    dp.q = static_cast<const __nv_bfloat16*>(q);
+    dp.out = static_cast<__nv_bfloat16*>(out);
+    dp.block_table = plan->block_table;
+    dp.seqs = plan->d_seqs;
+    dp.work = plan->d_dwork;
+    dp.units = plan->d_units;
+    dp.anc = plan->d_anc;
+    dp.part_o = plan->d_part_o;
+    dp.part_ml = plan->d_part_ml;
+    dp.counters = plan->d_counters;
+    dp.err = plan->d_err;
+    dp.bt_stride = hp.bt_stride;
+    dp.Hq = hp.Hq;
+    dp.Hkv = hp.Hkv;
+    dp.G = hp.G;
+    dp.num_pages = hp.num_pages;
+    dp.scale_log2 = hp.scale * 1.4426950408889634f;
+    cudaError_t e = launch_decode(dp, (int)hp.dwork.size(), hp.D, hp.decode_rows, plan->tmK, plan->tmV, st);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_run: decode launch");
+    return PKVA_OK;
+}
+
+extern "C" int attn_run_host(pkva_plan_t plan, const void* q_host, const void* k_cache, const void* v_cache,
+                             void* out_host, void* stream) {
+    if (!plan) {
+        set_last_error("attn_run_host: plan is NULL");
+        return PKVA_EINVAL;
+    }
+    const HostPlan& hp = plan->hp;
+    if (hp.num_seqs == 0) return PKVA_OK;
+    if (!q_host || !out_host) {
+        set_last_error("attn_run_host: NULL host pointer");
+        return PKVA_EINVAL;
+    }
+    const size_t bytes = (size_t)hp.total_q * hp.Hq * hp.D * 2;
+    if (!plan->d_qstage) {
+        PKVA_CUDA(cudaMalloc(&plan->d_qstage, bytes), "cudaMalloc(q staging)");
+        PKVA_CUDA(cudaMalloc(&plan->d_ostage, bytes), "cudaMalloc(out staging)");
+        plan->scratch_bytes += 2 * (int64_t)bytes;
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    PKVA_CUDA(cudaMemcpyAsync(plan->d_qstage, q_host, bytes, cudaMemcpyHostToDevice, st), "copy q to device");
+    const int rc = attn_run(plan, plan->d_qstage, k_cache, v_cache, plan->d_ostage, stream);
+    if (rc != PKVA_OK) return rc;
+    PKVA_CUDA(cudaMemcpyAsync(out_host, plan->d_ostage, bytes, cudaMemcpyDeviceToHost, st), "copy out to host");
+    return PKVA_OK;
+}
+
+extern "C" int attn_check(pkva_plan_t plan, void* stream, int32_t* device_error) {
+    if (!plan) {
+        set_last_error("attn_check: plan is NULL");
+        return PKVA_EINVAL;
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    PKVA_CUDA(cudaStreamSynchronize(st), "attn_check: stream synchronize");
+    int32_t e = 0;
+    PKVA_CUDA(cudaMemcpy(&e, plan->d_err, sizeof e, cudaMemcpyDeviceToHost), "attn_check: read error word");
+    if (device_error) *device_error = e;
+    if (e != 0) {
+        PKVA_CUDA(cudaMemset(plan->d_err, 0, sizeof(int32_t)), "attn_check: clear error word");
+        char buf[96];
+        snprintf(buf, sizeof buf, "attn_check: device error bits 0x%x", (unsigned)e);
+        set_last_error(buf);
+        return PKVA_EDEVICE;
+    }
+    return PKVA_OK;
+}

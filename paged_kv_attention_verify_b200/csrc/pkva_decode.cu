@@ -1,0 +1,472 @@
+// Decode / verify attention over the paged KV cache on CUDA cores (K-D).
+//
+// One CTA runs one tile task: up to 16 packed rows (token x query head of one GQA group)
+// of one sequence against a range of its KV pages for one KV head. Every K and V page
+// block is loaded once per task by TMA (128-byte swizzle, so the lane patterns below read
+// shared memory without bank conflicts) and reused by all rows of the group: the whole
+// query-head group shares one read of the page. Each of the four warps streams every
+// fourth page through its own ring of stages and keeps its own online-softmax state; the
+// warps merge their states at the end, and a task that is one split of a long context
+// writes a partial that the last split to finish merges (flash-decoding combine).
+//
+// Sources: XY-Serve (arXiv 2412.18106), verdict page — core_discovery (decode and verify
+// tokens read a paged block cache; FlashAttention-style tiling) and forward_implications[2]
+// (the visible keys are chosen per row: a causal limit for prefill/decode rows, ancestors
+// in the draft tree for verify rows); supporting citation [1] (FlashAttention's QK /
+// softmax / SV pattern, here with a running max and sum per row).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "pkva.h"
+#include "pkva_kernels.h"
+#include "pkva_ptx.cuh"
+
+namespace pkva {
+
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr int kBoxBytes = kPageSize * 128;     // one TMA box: 16 rows x 64 bf16
+constexpr int kBtSlice = kDecodeMaxPages;      // block-table entries staged per task
+
+constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
+
+template <int D, int NR>
+struct DecodeCfg {
+    static constexpr int NS = (D == 64) ? 4 : (NR <= 8 ? 3 : 2);    // stages per warp
+    static constexpr int PAGE_BYTES = kPageSize * D * 2;
+    static constexpr int STAGE_BYTES = 2 * PAGE_BYTES;              // K page + V page
+    static constexpr int HALF = D / 2;                              // columns per lane half
+    static constexpr int QROW = D + 8;                              // floats per staged Q row
+    static constexpr int OPL = D / 32;                              // output columns per lane
+    static constexpr int RING = kWarps * NS * STAGE_BYTES;
+    static constexpr int OFF_Q = RING;
+    static constexpr int OFF_P = OFF_Q + NR * QROW * 4;
+    static constexpr int OFF_BT = OFF_P + kWarps * kPageSize * NR * 4;
+    static constexpr int OFF_LIM = OFF_BT + kBtSlice * 4;
+    static constexpr int OFF_ANC = align_up(OFF_LIM + NR * 4, 8);
+    static constexpr int OFF_OUT = OFF_ANC + NR * 8;
+    static constexpr int OFF_BAR = align_up(OFF_OUT + NR * 4, 8);
+    static constexpr int OFF_FLAG = OFF_BAR + kWarps * NS * 8;
+    static constexpr int BYTES = OFF_FLAG + 16;
+    static constexpr int ALLOC = BYTES + 1008;                     // room to align to 1024
+    static_assert(kWarps * NR * (D + 2) * 4 <= RING, "combine buffers must fit in the ring");
+    static_assert(D == 64 || D == 128, "head_dim");
+};
+
+__device__ __forceinline__ int q_row_index(const DecodeParams& p, const SeqInfo& si, const DecodeWork& w,
+                                           int r) {
+    const int rr = w.row_begin + r;
+    const int t = rr / p.G;
+    const int g = rr - t * p.G;
+    return (si.q_start + t) * p.Hq + w.kv_head * p.G + g;
+}
+
+template <int D, int NR>
+__global__ void __launch_bounds__(kThreads)
+decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV) {
+    using C = DecodeCfg<D, NR>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const DecodeWork w = p.work[blockIdx.x];
+    const SeqInfo si = p.seqs[w.seq];
+
+    float* qs = reinterpret_cast<float*>(sm + C::OFF_Q);
+    float* ps = reinterpret_cast<float*>(sm + C::OFF_P);
+    int* bts = reinterpret_cast<int*>(sm + C::OFF_BT);
+    int* rlim = reinterpret_cast<int*>(sm + C::OFF_LIM);
+    uint64_t* ranc = reinterpret_cast<uint64_t*>(sm + C::OFF_ANC);
+    int* rout = reinterpret_cast<int*>(sm + C::OFF_OUT);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
+    int* flag = reinterpret_cast<int*>(sm + C::OFF_FLAG);
+
+    const int R = w.row_count;
+    const int npg = w.page_end - w.page_begin;
+    const int prefix = si.seq_len - si.query_len;
+
+    if (tid == 0) {
+        for (int i = 0; i < kWarps * C::NS; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+        flag[0] = 0;
+        flag[1] = 0;
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+    }
+    // block-table slice of this task; an entry out of range is flagged and its page is
+    // loaded from a fully out-of-bounds box, which TMA fills with zeros
+    const int32_t* btrow = p.block_table + (int64_t)w.seq * p.bt_stride + w.page_begin;
+    for (int i = tid; i < npg; i += kThreads) {
+        const int ph = btrow[i];
+        const bool bad = ph < 0 || ph >= p.num_pages;
+        if (bad) atomicOr(p.err, PKVA_DEVERR_BAD_PAGE);
+        bts[i] = bad ? -1 : ph;
+    }
+    // per-row records: output row, causal limit, tree ancestor mask
+    if (tid < NR) {
+        const int r = tid;
+        if (r < R) {
+            const int t = (w.row_begin + r) / p.G;
+            rout[r] = q_row_index(p, si, w, r);
+            if (si.mask_kind == PKVA_CAUSAL) {
+                rlim[r] = prefix + t;
+                ranc[r] = 0ull;
+            } else {
+                rlim[r] = prefix - 1;
+                ranc[r] = p.anc[si.anc_off + t];
+            }
+        } else {
+            rout[r] = -1;
+            rlim[r] = 0x7fffffff;
+            ranc[r] = 0ull;
+        }
+    }
+    // Q rows in fp32, pre-scaled by scale*log2(e); each row is stored as two halves with a
+    // 4-float pad so that the two lane halves read different banks
+    for (int idx = tid; idx < NR * (D / 8); idx += kThreads) {
+        const int r = idx / (D / 8);
+        const int c8 = (idx - r * (D / 8)) * 8;
+        float f[8];
+        if (r < R) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(p.q + (int64_t)q_row_index(p, si, w, r) * D + c8);
+            bf16x8_to_f32(raw, f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] *= p.scale_log2;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = 0.f;
+        }
+        const int hh = c8 / C::HALF;
+        float* dst = qs + r * C::QROW + hh * (C::HALF + 4) + (c8 - hh * C::HALF);
+        *reinterpret_cast<float4*>(dst) = make_float4(f[0], f[1], f[2], f[3]);
+        *reinterpret_cast<float4*>(dst + 4) = make_float4(f[4], f[5], f[6], f[7]);
+    }
+    __syncthreads();
+
+    int min_lim = 0x7fffffff;
+    for (int r = 0; r < R; ++r) min_lim = min(min_lim, rlim[r]);
+
+    // ---- page stream of this warp: pages warp, warp+4, ... of the task -----------------
+    const int n_my = npg > warp ? (npg - warp + kWarps - 1) / kWarps : 0;
+    uint8_t* ring = sm + warp * C::NS * C::STAGE_BYTES;
+    uint64_t* bar = bars + warp * C::NS;
+
+    auto issue = [&](int i) {     // lane 0 only: load page #i of this warp into its stage
+        const int stage = i % C::NS;
+        const int ph = bts[warp + kWarps * i];
+        const int row = ph >= 0 ? (ph * p.Hkv + w.kv_head) * kPageSize : -kPageSize;
+        uint8_t* dst = ring + stage * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(&bar[stage], C::STAGE_BYTES);
+#pragma unroll
+        for (int b = 0; b < D / 64; ++b) {
+            tma_load_2d(dst + b * kBoxBytes, &tmK, &bar[stage], b * 64, row);
+            tma_load_2d(dst + C::PAGE_BYTES + b * kBoxBytes, &tmV, &bar[stage], b * 64, row);
+        }
+    };
+
+    float o[NR][C::OPL];
+    float m_run[NR], l_run[NR];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+        m_run[r] = -INFINITY;
+        l_run[r] = 0.f;
+#pragma unroll
+        for (int c = 0; c < C::OPL; ++c) o[r][c] = 0.f;
+    }
+
+    if (lane == 0)
+        for (int i = 0; i < C::NS && i < n_my; ++i) issue(i);
+    __syncwarp();
+
+    const int j = lane & 15;       // key slot of this lane in the QK phase
+    const int hh = lane >> 4;      // which half of the head dimension it sums
+    float* pw = ps + warp * kPageSize * NR;
+    bool ok = true;
+    int waited = 0;
+
+    for (int i = 0; i < n_my; ++i) {
+        const int stage = i % C::NS;
+        const bool got = mbar_wait_bounded(&bar[stage], (i / C::NS) & 1, p.err, PKVA_DEVERR_TIMEOUT);
+        waited = i + 1;
+        if (__any_sync(0xffffffffu, !got)) {
+            ok = false;
+            break;
+        }
+        const uint8_t* Ks = ring + stage * C::STAGE_BYTES;
+        const uint8_t* Vs = Ks + C::PAGE_BYTES;
+        const int kbase = (w.page_begin + warp + kWarps * i) * kPageSize;
+
+        // -- scores: lane (j, hh) sums half hh of <q_r, k_j> for every row r ------------
+        float acc[NR];
+#pragma unroll
+        for (int r = 0; r < NR; ++r) acc[r] = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < C::HALF / 8; ++cc) {
+            const int col = hh * C::HALF + cc * 8;
+            const int box = col >> 6, ch = (col & 63) >> 3;
+            const uint4 kr = *reinterpret_cast<const uint4*>(Ks + box * kBoxBytes + j * 128 + ((ch ^ (j & 7)) << 4));
+            float kf[8];
+            bf16x8_to_f32(kr, kf);
+            const float* qp = qs + hh * (C::HALF + 4) + cc * 8;
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                if (r < R) {
+                    const float4 a = *reinterpret_cast<const float4*>(qp + r * C::QROW);
+                    const float4 b = *reinterpret_cast<const float4*>(qp + r * C::QROW + 4);
+                    float t = acc[r];
+                    t = fmaf(kf[0], a.x, t);
+                    t = fmaf(kf[1], a.y, t);
+                    t = fmaf(kf[2], a.z, t);
+                    t = fmaf(kf[3], a.w, t);
+                    t = fmaf(kf[4], b.x, t);
+                    t = fmaf(kf[5], b.y, t);
+                    t = fmaf(kf[6], b.z, t);
+                    t = fmaf(kf[7], b.w, t);
+                    acc[r] = t;
+                }
+            }
+        }
+        // -- mask, online softmax (warp-shuffle max over the page's 16 keys) --------------
+        const int kpos = kbase + j;
+        const bool page_all = (kbase + kPageSize - 1) <= min_lim;
+        float alpha[NR];
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+            alpha[r] = 1.f;
+            if (r < R) {
+                float s = acc[r] + __shfl_xor_sync(0xffffffffu, acc[r], 16);
+                bool allow = page_all || kpos <= rlim[r];
+                if (!allow && kpos >= prefix && kpos < si.seq_len)
+                    allow = (ranc[r] >> (kpos - prefix)) & 1ull;
+                s = allow ? s : -INFINITY;
+                float mx = s;
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                const float mnew = fmaxf(m_run[r], mx);
+                const float ref = (mnew == -INFINITY) ? 0.f : mnew;
+                const float pr = exp2f(s - ref);
+                alpha[r] = exp2f(m_run[r] - ref);
+                m_run[r] = mnew;
+                l_run[r] = fmaf(l_run[r], alpha[r], pr);
+                acc[r] = pr;
+            } else {
+                acc[r] = 0.f;
+            }
+        }
+        if (hh == 0) {
+#pragma unroll
+            for (int r4 = 0; r4 < NR / 4; ++r4)
+                *reinterpret_cast<float4*>(pw + j * NR + 4 * r4) =
+                    make_float4(acc[4 * r4], acc[4 * r4 + 1], acc[4 * r4 + 2], acc[4 * r4 + 3]);
+        }
+        __syncwarp();
+
+        // -- o_r = alpha_r * o_r + sum_j p_rj v_j; lane owns D/32 output columns ------------
+#pragma unroll
+        for (int r = 0; r < NR; ++r)
+            if (r < R)
+#pragma unroll
+                for (int c = 0; c < C::OPL; ++c) o[r][c] *= alpha[r];
+        const int nvalid = min(kPageSize, si.seq_len - kbase);   // slots past L are skipped
+#pragma unroll 4
+        for (int jj = 0; jj < nvalid; ++jj) {
+            float vf[C::OPL];
+            if constexpr (D == 128) {
+                const int box = lane >> 4, ch = (lane & 15) >> 1;
+                const uint2 vr = *reinterpret_cast<const uint2*>(Vs + box * kBoxBytes + jj * 128 +
+                                                                 ((ch ^ (jj & 7)) << 4) + (lane & 1) * 8);
+                bf16x2_to_f32(vr.x, vf[0], vf[1]);
+                bf16x2_to_f32(vr.y, vf[2], vf[3]);
+            } else {
+                const int ch = lane >> 2;
+                const uint32_t vr = *reinterpret_cast<const uint32_t*>(Vs + jj * 128 + ((ch ^ (jj & 7)) << 4) +
+                                                                       (lane & 3) * 4);
+                bf16x2_to_f32(vr, vf[0], vf[1]);
+            }
+#pragma unroll
+            for (int r4 = 0; r4 < NR / 4; ++r4) {
+                const float4 pp = *reinterpret_cast<const float4*>(pw + jj * NR + 4 * r4);
+                const float pv[4] = {pp.x, pp.y, pp.z, pp.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = 4 * r4 + e;
+                    if (r < R)
+#pragma unroll
+                        for (int c = 0; c < C::OPL; ++c) o[r][c] = fmaf(pv[e], vf[c], o[r][c]);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0 && i + C::NS < n_my) {
+            fence_proxy_async_smem();
+            issue(i + C::NS);
+        }
+    }
+    if (!ok) {
+        // drain this warp's copies still in flight (bounded) before the ring is reused
+        for (int i = waited; i < n_my && i < waited + C::NS; ++i)
+            mbar_wait_bounded(&bar[i % C::NS], (i / C::NS) & 1, p.err, PKVA_DEVERR_TIMEOUT);
+        if (lane == 0) atomicOr(&flag[1], 1);
+    }
+
+    // row sums: lanes j and j+16 hold the same keys, so reduce within each half
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+        float l = l_run[r];
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        l += __shfl_xor_sync(0xffffffffu, l, 4);
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l_run[r] = l;
+    }
+
+    // ---- merge the four warps' states (ring space is free now) --------------------------
+    __syncthreads();
+    float* cm = reinterpret_cast<float*>(sm);       // [kWarps][NR] running max (log2 units)
+    float* cl = cm + kWarps * NR;                   // [kWarps][NR] running sum
+    float* co = cl + kWarps * NR;                   // [kWarps][NR][D] unnormalised output
+    if (lane == 0) {
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+            cm[warp * NR + r] = m_run[r];
+            cl[warp * NR + r] = l_run[r];
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+        if (r < R) {
+            float* dst = co + (warp * NR + r) * D + lane * C::OPL;
+            if constexpr (C::OPL == 4)
+                *reinterpret_cast<float4*>(dst) = make_float4(o[r][0], o[r][1], o[r][2], o[r][3]);
+            else
+                *reinterpret_cast<float2*>(dst) = make_float2(o[r][0], o[r][1]);
+        }
+    }
+    __syncthreads();
+
+    const bool split = w.unit >= 0;
+    int slot = 0;
+    if (split) slot = p.units[w.unit].slot_base + w.split;
+    for (int idx = tid; idx < R * (D / 2); idx += kThreads) {
+        const int r = idx / (D / 2);
+        const int c = (idx - r * (D / 2)) * 2;
+        float M = -INFINITY;
+#pragma unroll
+        for (int ww = 0; ww < kWarps; ++ww) M = fmaxf(M, cm[ww * NR + r]);
+        float o0 = 0.f, o1 = 0.f, L = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int ww = 0; ww < kWarps; ++ww) {
+                const float f = exp2f(cm[ww * NR + r] - M);
+                const float2 v = *reinterpret_cast<const float2*>(co + (ww * NR + r) * D + c);
+                o0 = fmaf(f, v.x, o0);
+                o1 = fmaf(f, v.y, o1);
+                L = fmaf(f, cl[ww * NR + r], L);
+            }
+        }
+        if (!split) {
+            const float inv = L > 0.f ? 1.f / L : 0.f;
+            *reinterpret_cast<__nv_bfloat162*>(p.out + (int64_t)rout[r] * D + c) =
+                __floats2bfloat162_rn(o0 * inv, o1 * inv);
+        } else {
+            *reinterpret_cast<float2*>(p.part_o + ((int64_t)slot * kDecodeRowsMax + r) * D + c) =
+                make_float2(o0, o1);
+            if (c == 0)
+                *reinterpret_cast<float2*>(p.part_ml + ((int64_t)slot * kDecodeRowsMax + r) * 2) =
+                    make_float2(M, L);
+        }
+    }
+    if (!split) return;
+
+    // ---- split-KV combine: the last split of the unit to finish merges all partials -----
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const int prev = atomicAdd(&p.counters[w.unit], 1);
+        flag[0] = (prev == p.units[w.unit].num_splits - 1);
+    }
+    __syncthreads();
+    if (!flag[0]) return;
+    __threadfence();
+    const SplitUnit u = p.units[w.unit];
+    for (int idx = tid; idx < R * (D / 2); idx += kThreads) {
+        const int r = idx / (D / 2);
+        const int c = (idx - r * (D / 2)) * 2;
+        float M = -INFINITY;
+        for (int s = 0; s < u.num_splits; ++s)
+            M = fmaxf(M, __ldcg(p.part_ml + ((int64_t)(u.slot_base + s) * kDecodeRowsMax + r) * 2));
+        float o0 = 0.f, o1 = 0.f, L = 0.f;
+        if (M != -INFINITY) {
+            for (int s = 0; s < u.num_splits; ++s) {
+                const int64_t base = (int64_t)(u.slot_base + s) * kDecodeRowsMax + r;
+                const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + base * 2));
+                const float f = exp2f(ml.x - M);
+                const float2 v = __ldcg(reinterpret_cast<const float2*>(p.part_o + base * D + c));
+                o0 = fmaf(f, v.x, o0);
+                o1 = fmaf(f, v.y, o1);
+                L = fmaf(f, ml.y, L);
+            }
+        }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        *reinterpret_cast<__nv_bfloat162*>(p.out + (int64_t)rout[r] * D + c) =
+            __floats2bfloat162_rn(o0 * inv, o1 * inv);
+    }
+    if (tid == 0) p.counters[w.unit] = 0;     // ready for the next run of the plan
+}
+
+template <int D, int NR>
+cudaError_t launch_t(const DecodeParams& p, int num_work, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                     cudaStream_t stream) {
+    using C = DecodeCfg<D, NR>;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::ALLOC);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    decode_kernel<D, NR><<<num_work, kThreads, C::ALLOC, stream>>>(p, tmK, tmV);
+    return cudaGetLastError();
+}
+
+template <int D, int NR>
+int ctas_t() {
+    using C = DecodeCfg<D, NR>;
+    int n = 0;
+    if (cudaFuncSetAttribute(decode_kernel<D, NR>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::ALLOC) !=
+        cudaSuccess)
+        return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<D, NR>, kThreads, C::ALLOC) !=
+        cudaSuccess)
+        return 0;
+    return n;
+}
+
+}  // namespace
+
+int decode_ctas_per_sm(int D, int rows) {
+    if (D == 64) return rows <= 4 ? ctas_t<64, 4>() : rows <= 8 ? ctas_t<64, 8>() : ctas_t<64, 16>();
+    if (D == 128) return rows <= 4 ? ctas_t<128, 4>() : rows <= 8 ? ctas_t<128, 8>() : ctas_t<128, 16>();
+    return 0;
+}
+
+cudaError_t launch_decode(const DecodeParams& p, int num_work, int D, int rows, const CUtensorMap& tmK,
+                          const CUtensorMap& tmV, cudaStream_t stream) {
+    if (num_work == 0) return cudaSuccess;
+    if (D == 64) {
+        if (rows <= 4) return launch_t<64, 4>(p, num_work, tmK, tmV, stream);
+        if (rows <= 8) return launch_t<64, 8>(p, num_work, tmK, tmV, stream);
+        return launch_t<64, 16>(p, num_work, tmK, tmV, stream);
+    }
+    if (rows <= 4) return launch_t<128, 4>(p, num_work, tmK, tmV, stream);
+    if (rows <= 8) return launch_t<128, 8>(p, num_work, tmK, tmV, stream);
+    return launch_t<128, 16>(p, num_work, tmK, tmV, stream);
+}
+
+}  // namespace pkva

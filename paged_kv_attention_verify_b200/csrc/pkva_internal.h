@@ -1,0 +1,80 @@
+// Internal types shared by the host planner and the kernels (not part of the C ABI).
+#pragma once
+
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+namespace pkva {
+
+constexpr int kPageSize = 16;          // keys per page (the only page size supported)
+constexpr int kMaxTreeTokens = 64;     // draft tokens per TREE sequence (one 64-bit mask)
+constexpr int kDecodeRowsMax = 16;     // packed (token, head) rows per decode task
+constexpr int kDecodeMaxPages = 1024;  // pages per decode task (block-table slice in smem)
+
+// Per-sequence record (the "Token-Table" row of the batch).
+struct SeqInfo {
+    int32_t seq_len;     // L: total keys, new tokens included
+    int32_t query_len;   // T: new query tokens
+    int32_t q_start;     // first row of this sequence in q / out
+    int32_t mask_kind;   // 0 causal, 1 tree
+    int32_t anc_off;     // TREE: index of token 0's ancestor mask in the mask array
+    int32_t pad0, pad1, pad2;
+};
+static_assert(sizeof(SeqInfo) == 32, "SeqInfo layout");
+
+// One decode/verify tile task (the "Task-Table" row): packed rows [row_begin,
+// row_begin + row_count) of (seq, kv_head), keys of pages [page_begin, page_end).
+struct DecodeWork {
+    int32_t seq;
+    int32_t kv_head;
+    int32_t row_begin;   // packed row = token * group + head-in-group
+    int32_t row_count;   // <= kDecodeRowsMax
+    int32_t page_begin;  // logical pages of the sequence
+    int32_t page_end;
+    int32_t unit;        // split unit id, -1 when the task covers its whole unit
+    int32_t split;       // split index within the unit
+};
+static_assert(sizeof(DecodeWork) == 32, "DecodeWork layout");
+
+// A (seq, kv_head, row chunk) split over several tasks: where its partials live.
+struct SplitUnit {
+    int32_t slot_base;   // first partial slot
+    int32_t num_splits;
+};
+
+// Host-side result of planning, before anything is uploaded.
+struct HostPlan {
+    int num_seqs = 0, Hq = 0, Hkv = 0, G = 0, D = 0;
+    int bt_stride = 0, num_pages = 0;
+    int total_q = 0;
+    float scale = 0.f;
+    int decode_rows = 4;                  // rows per decode task the launch compiles for
+    std::vector<SeqInfo> seqs;
+    std::vector<uint64_t> anc;            // per TREE token: ancestor-or-self bit mask
+    std::vector<DecodeWork> dwork;        // launch order
+    std::vector<SplitUnit> units;
+    int num_slots = 0;
+    int64_t kv_bytes = 0;
+    int64_t attn_flops = 0;
+};
+
+struct PlanArgs {
+    int num_seqs;
+    const int32_t* seq_lens;
+    const int32_t* query_lens;
+    int bt_stride;
+    int num_pages;
+    const int32_t* mask_kind;
+    const int32_t* parents;
+    int Hq, Hkv, D, page_size;
+    float sm_scale;
+    int num_sms;
+    int ctas_per_sm;
+};
+
+// Validates and decomposes; returns a pkva_status and fills `err` on failure.
+int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err);
+
+}  // namespace pkva

@@ -1,0 +1,37 @@
+// Launch interface between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "pkva_internal.h"
+
+namespace pkva {
+
+struct DecodeParams {
+    const __nv_bfloat16* q;      // [sum T, Hq, D]
+    __nv_bfloat16* out;          // [sum T, Hq, D]
+    const int32_t* block_table;  // [B, bt_stride]
+    const SeqInfo* seqs;
+    const DecodeWork* work;
+    const SplitUnit* units;
+    const uint64_t* anc;         // TREE ancestor-or-self masks
+    float* part_o;               // [slots, kDecodeRowsMax, D]: unnormalised split outputs
+    float* part_ml;              // [slots, kDecodeRowsMax, 2]: (max, sum) in log2 units
+    int32_t* counters;           // [units]: split tasks finished (reset by the last one)
+    int32_t* err;                // device error word
+    int32_t bt_stride;
+    int32_t Hq, Hkv, G;
+    int32_t num_pages;
+    float scale_log2;            // softmax scale * log2(e)
+};
+
+// Resident CTAs per SM of the decode kernel compiled for (D, rows); 0 if unsupported.
+int decode_ctas_per_sm(int D, int rows);
+
+// Launch the decode/verify kernel over `num_work` tasks.
+cudaError_t launch_decode(const DecodeParams& p, int num_work, int D, int rows,
+                          const CUtensorMap& tmK, const CUtensorMap& tmV, cudaStream_t stream);
+
+}  // namespace pkva

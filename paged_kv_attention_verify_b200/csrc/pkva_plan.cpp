@@ -1,0 +1,223 @@
+// Host tile planner: validates one mixed prefill / decode / verify batch and decomposes it
+// into fixed-shape tile tasks, then orders them for the launch.
+//
+// XY-Serve (arXiv 2412.18106), verdict page, core_discovery: the batch is broken into
+// tile-level tasks (its Token-Table / Task-Table) that are then reordered to balance the
+// cores; key_machinery: attention tiles are ordered by how much work they carry and dealt
+// to the cores round-robin. Here the "cores" are the CTA slots of the B200 (SMs x resident
+// CTAs), the task list is uploaded once per plan, and the hardware block scheduler deals
+// the tasks out in list order, so heaviest-first order gives a longest-task-first schedule.
+#include <math.h>
+#include <stdio.h>
+
+#include <algorithm>
+#include <cstring>
+
+#include "pkva.h"
+#include "pkva_internal.h"
+
+namespace pkva {
+
+namespace {
+
+constexpr int kMinSplitPages = 8;      // never split a unit into tasks below 128 keys
+constexpr int kTasksPerSlot = 3;       // aim for ~3 tasks per CTA slot before splitting stops
+
+int fail(std::string* err, int code, const char* fmt, long a = 0, long b = 0, long c = 0) {
+    char buf[256];
+    snprintf(buf, sizeof buf, fmt, a, b, c);
+    if (err) *err = buf;
+    return code;
+}
+
+}  // namespace
+
+int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
+    HostPlan& p = *out;
+    p = HostPlan();
+    if (a.num_seqs < 0) return fail(err, PKVA_EINVAL, "num_seqs must be >= 0 (got %ld)", a.num_seqs);
+    if (a.num_seqs > 0 && (!a.seq_lens || !a.query_lens || !a.mask_kind))
+        return fail(err, PKVA_EINVAL, "seq_lens, query_lens and mask_kind must not be NULL");
+    if (a.Hkv < 1 || a.Hq < 1 || a.Hq % a.Hkv != 0)
+        return fail(err, PKVA_EINVAL, "num_q_heads (%ld) must be a positive multiple of num_kv_heads (%ld)",
+                    a.Hq, a.Hkv);
+    if (a.D != 64 && a.D != 128)
+        return fail(err, PKVA_EUNSUPPORTED, "head_dim %ld not supported (64 or 128)", a.D);
+    if (a.page_size != kPageSize)
+        return fail(err, PKVA_EUNSUPPORTED, "page_size %ld not supported (16)", a.page_size);
+    if (a.sm_scale != a.sm_scale) return fail(err, PKVA_EINVAL, "sm_scale is NaN");
+    if (a.num_sms < 1 || a.ctas_per_sm < 1)
+        return fail(err, PKVA_EINVAL, "num_sms and ctas_per_sm must be >= 1");
+
+    p.num_seqs = a.num_seqs;
+    p.Hq = a.Hq;
+    p.Hkv = a.Hkv;
+    p.G = a.Hq / a.Hkv;
+    p.D = a.D;
+    p.bt_stride = a.bt_stride;
+    p.num_pages = a.num_pages;
+    p.scale = a.sm_scale > 0.f ? a.sm_scale : 1.0f / sqrtf((float)a.D);
+
+    if (a.num_seqs > 0) {
+        if (a.num_pages < 1) return fail(err, PKVA_EINVAL, "num_pages must be >= 1");
+        if ((int64_t)a.num_pages * a.Hkv * kPageSize >= (int64_t(1) << 31))
+            return fail(err, PKVA_EUNSUPPORTED, "cache too large: num_pages*Hkv*16 must be < 2^31");
+    }
+
+    // -- per-sequence records and tree masks ------------------------------------------
+    int64_t q_acc = 0;
+    int par_off = 0;
+    for (int s = 0; s < a.num_seqs; ++s) {
+        const int L = a.seq_lens[s], T = a.query_lens[s], mk = a.mask_kind[s];
+        if (L < 1) return fail(err, PKVA_EINVAL, "seq_lens[%ld] = %ld must be >= 1", s, L);
+        if (T < 1 || T > L)
+            return fail(err, PKVA_EINVAL, "query_lens[%ld] = %ld must be in [1, seq_len = %ld]", s, T, L);
+        if (mk != PKVA_CAUSAL && mk != PKVA_TREE)
+            return fail(err, PKVA_EINVAL, "mask_kind[%ld] = %ld is not CAUSAL (0) or TREE (1)", s, mk);
+        const int pages = (L + kPageSize - 1) / kPageSize;
+        if (pages > a.bt_stride)
+            return fail(err, PKVA_EINVAL, "sequence %ld needs %ld block-table entries; bt_stride is %ld",
+                        s, pages, a.bt_stride);
+        SeqInfo si{};
+        si.seq_len = L;
+        si.query_len = T;
+        si.q_start = (int32_t)q_acc;
+        si.mask_kind = mk;
+        si.anc_off = -1;
+        if (mk == PKVA_TREE) {
+            if (T > kMaxTreeTokens)
+                return fail(err, PKVA_EINVAL, "TREE sequence %ld has %ld draft tokens (max 64)", s, T);
+            if (!a.parents) return fail(err, PKVA_EINVAL, "parents is NULL but sequence %ld is TREE", s);
+            si.anc_off = (int32_t)p.anc.size();
+            for (int i = 0; i < T; ++i) {
+                const int par = a.parents[par_off + i];
+                if (par < -1 || par >= i)
+                    return fail(err, PKVA_EINVAL,
+                                "parents of sequence %ld, node %ld = %ld: must be -1 or an earlier node",
+                                s, i, par);
+                uint64_t m = uint64_t(1) << i;
+                if (par >= 0) m |= p.anc[si.anc_off + par];
+                p.anc.push_back(m);
+            }
+            par_off += T;
+        }
+        p.seqs.push_back(si);
+        q_acc += T;
+        if (q_acc > (int64_t(1) << 31) / a.Hq)
+            return fail(err, PKVA_EUNSUPPORTED, "too many query rows");
+
+        // algorithmic work: every K and V element once; 4*D*Hq flops per allowed pair
+        p.kv_bytes += (int64_t)L * a.Hkv * a.D * 2 /*K,V*/ * 2 /*bf16*/;
+        int64_t pairs = (int64_t)T * (L - T);
+        if (mk == PKVA_CAUSAL) {
+            pairs += (int64_t)T * (T + 1) / 2;
+        } else {
+            for (int i = 0; i < T; ++i) pairs += __builtin_popcountll(p.anc[si.anc_off + i]);
+        }
+        p.attn_flops += pairs * a.Hq * 4 * a.D;
+    }
+    p.total_q = (int)q_acc;
+
+    // -- decode/verify units: (seq, kv head, chunk of packed rows) --------------------
+    struct Unit { int seq, kvh, rb, rc, pages; };
+    std::vector<Unit> units;
+    int64_t total_pages = 0;
+    int max_rc = 0;
+    for (int s = 0; s < a.num_seqs; ++s) {
+        const SeqInfo& si = p.seqs[s];
+        const int rows = si.query_len * p.G;
+        for (int h = 0; h < a.Hkv; ++h) {
+            for (int rb = 0; rb < rows; rb += kDecodeRowsMax) {
+                const int rc = std::min(kDecodeRowsMax, rows - rb);
+                const int t_last = (rb + rc - 1) / p.G;
+                // keys past the last row's own position are masked for every row of the
+                // chunk (causal and tree alike), so the task never loads them
+                const int kend = si.seq_len - si.query_len + t_last + 1;
+                const int pages = (kend + kPageSize - 1) / kPageSize;
+                units.push_back({s, h, rb, rc, pages});
+                total_pages += pages;
+                max_rc = std::max(max_rc, rc);
+            }
+        }
+    }
+    p.decode_rows = max_rc <= 4 ? 4 : (max_rc <= 8 ? 8 : 16);
+
+    // -- split long units so the grid has ~kTasksPerSlot tasks per CTA slot -------------
+    const int64_t slots = (int64_t)a.num_sms * a.ctas_per_sm;
+    int64_t target = (total_pages + slots * kTasksPerSlot - 1) / (slots * kTasksPerSlot);
+    target = std::max<int64_t>(target, kMinSplitPages);
+    target = std::min<int64_t>(target, kDecodeMaxPages);
+    for (const Unit& u : units) {
+        const int ns = (int)((u.pages + target - 1) / target);
+        int unit_id = -1;
+        if (ns > 1) {
+            unit_id = (int)p.units.size();
+            p.units.push_back({p.num_slots, ns});
+            p.num_slots += ns;
+        }
+        for (int k = 0; k < ns; ++k) {
+            DecodeWork w{};
+            w.seq = u.seq;
+            w.kv_head = u.kvh;
+            w.row_begin = u.rb;
+            w.row_count = u.rc;
+            w.page_begin = (int)((int64_t)u.pages * k / ns);
+            w.page_end = (int)((int64_t)u.pages * (k + 1) / ns);
+            w.unit = unit_id;
+            w.split = ns > 1 ? k : -1;
+            p.dwork.push_back(w);
+        }
+    }
+    // heaviest first; ties keep (seq, head, chunk) order so chunks of one head stay adjacent
+    std::stable_sort(p.dwork.begin(), p.dwork.end(), [](const DecodeWork& x, const DecodeWork& y) {
+        return (x.page_end - x.page_begin) > (y.page_end - y.page_begin);
+    });
+    return PKVA_OK;
+}
+
+}  // namespace pkva
+
+namespace pkva {
+void set_last_error(const std::string& msg);   // defined with the rest of the C ABI
+}
+
+extern "C" int attn_plan_inspect(int num_seqs, const int32_t* seq_lens, const int32_t* query_lens,
+                                 int bt_stride, int num_pages, const int32_t* mask_kind,
+                                 const int32_t* parents, int num_q_heads, int num_kv_heads,
+                                 int head_dim, int page_size, int num_sms, int ctas_per_sm,
+                                 pkva_work_desc* items, int max_items, int* num_items) {
+    using namespace pkva;
+    PlanArgs a{num_seqs, seq_lens, query_lens, bt_stride, num_pages, mask_kind, parents,
+               num_q_heads, num_kv_heads, head_dim, page_size, 0.f, num_sms, ctas_per_sm};
+    HostPlan hp;
+    std::string err;
+    int rc = build_host_plan(a, &hp, &err);
+    if (rc != PKVA_OK) {
+        set_last_error(err);
+        return rc;
+    }
+    const int n = (int)hp.dwork.size();
+    if (num_items) *num_items = n;
+    if (!items) return PKVA_OK;
+    if (max_items < n) {
+        set_last_error("attn_plan_inspect: max_items is smaller than the number of tasks");
+        return PKVA_EINVAL;
+    }
+    for (int i = 0; i < n; ++i) {
+        const DecodeWork& w = hp.dwork[i];
+        const SeqInfo& si = hp.seqs[w.seq];
+        pkva_work_desc d;
+        d.kind = 0;
+        d.seq = w.seq;
+        d.kv_head = w.kv_head;
+        d.row_begin = w.row_begin;
+        d.row_count = w.row_count;
+        d.key_begin = w.page_begin * kPageSize;
+        d.key_end = std::min(w.page_end * kPageSize, si.seq_len);
+        d.split = w.split;
+        d.num_splits = w.unit >= 0 ? hp.units[w.unit].num_splits : 1;
+        items[i] = d;
+    }
+    set_last_error("");
+    return PKVA_OK;
+}

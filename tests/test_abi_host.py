@@ -1,0 +1,151 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every entry point
+the header declares, validates its inputs, and the planner's tile tasks cover the batch
+exactly once."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import paged_kv_attention_verify_b200 as pk
+import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_symbols():
+    src = open(os.path.join(ROOT, "include", "pkva.h")).read()
+    return sorted(set(re.findall(r"PKVA_API\s+[\w\s\*]*?\b(attn_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = pk.lib()
+    syms = header_symbols()
+    assert len(syms) >= 8
+    assert set(syms) == set(pk.EXPORTED)
+    for s in syms:
+        assert hasattr(L, s), s
+
+
+def _plan_args(**over):
+    a = dict(seq_lens=[40, 17], query_lens=[8, 1], mask_kind=[W.CAUSAL, W.CAUSAL], parents=None,
+             num_q_heads=8, num_kv_heads=2, head_dim=64, num_pages=8, bt_stride=4)
+    a.update(over)
+    return a
+
+
+def _inspect(**over):
+    a = _plan_args(**over)
+    return pk.inspect(a.pop("seq_lens"), a.pop("query_lens"), a.pop("mask_kind"), a.pop("parents"), **a)
+
+
+@pytest.mark.parametrize("over, code", [
+    (dict(query_lens=[0, 1]), -1),                          # query_len = 0
+    (dict(query_lens=[41, 1]), -1),                         # query_len > seq_len
+    (dict(seq_lens=[0, 17], query_lens=[0, 1]), -1),        # empty sequence
+    (dict(num_q_heads=6, num_kv_heads=4), -1),              # Hq not a multiple of Hkv
+    (dict(head_dim=96), -2),                                # unsupported head_dim
+    (dict(bt_stride=2), -1),                                # block table too narrow
+    (dict(mask_kind=[2, 0]), -1),                           # unknown mask kind
+    (dict(mask_kind=[W.TREE, 0], parents=None), -1),        # tree without parents
+    (dict(mask_kind=[W.TREE, 0], parents=[-1, 0, 1, 3, 0, 0, 0, 0]), -1),  # parent not earlier
+    (dict(mask_kind=[W.TREE, 0], parents=[-1, 0, -2, 0, 0, 0, 0, 0]), -1), # parent < -1
+    (dict(seq_lens=[100, 17], query_lens=[65, 1], mask_kind=[W.TREE, 0],
+          parents=[-1] * 65, bt_stride=8), -1),             # tree too large
+])
+def test_planner_rejects_bad_batches(over, code):
+    with pytest.raises(pk.PkvaError) as ei:
+        _inspect(**over)
+    assert ei.value.code == code
+    assert pk.lib().attn_last_error().decode()
+
+
+def test_attn_plan_validates_before_touching_the_device():
+    # a non-NULL block-table pointer that is never dereferenced: validation fails first
+    L = pk.lib()
+    h = ctypes.c_void_p()
+    sl = (ctypes.c_int32 * 1)(5)
+    ql = (ctypes.c_int32 * 1)(6)
+    mk = (ctypes.c_int32 * 1)(0)
+    rc = L.attn_plan(ctypes.byref(h), 1, sl, ql, ctypes.c_void_p(0x1000), 1, 1, mk, None, 8, 2, 64, 16, 0.0)
+    assert rc == -1 and not h.value
+    assert b"query_lens" in L.attn_last_error()
+    rc = L.attn_plan(ctypes.byref(h), 1, sl, sl, None, 1, 1, mk, None, 8, 2, 64, 16, 0.0)
+    assert rc == -1 and b"block_table" in L.attn_last_error()
+    assert L.attn_run(None, None, None, None, None, None) == -1
+    assert L.attn_check(None, None, None) == -1
+    L.attn_plan_destroy(None)
+
+
+def _coverage(batch, items):
+    """Every (seq, kv head, packed row) must see exactly the keys it needs, once."""
+    G = batch.num_q_heads // batch.num_kv_heads
+    seen = {}
+    for it in items:
+        assert it["row_count"] >= 1 and it["row_count"] <= 16
+        assert it["key_begin"] % 16 == 0 and it["key_end"] > it["key_begin"]
+        for r in range(it["row_begin"], it["row_begin"] + it["row_count"]):
+            seen.setdefault((it["seq"], it["kv_head"], r), []).append((it["key_begin"], it["key_end"],
+                                                                      it["split"], it["num_splits"]))
+    for s, sp in enumerate(batch.seqs):
+        for h in range(batch.num_kv_heads):
+            for r in range(sp.query_len * G):
+                rngs = sorted(seen.pop((s, h, r)))
+                # contiguous, non-overlapping, starting at 0
+                assert rngs[0][0] == 0
+                for a, b in zip(rngs[:-1], rngs[1:]):
+                    assert a[1] == b[0]
+                # must reach this row's own position (the last key it may see)
+                t = r // G
+                assert rngs[-1][1] >= sp.seq_len - sp.query_len + t + 1
+                assert rngs[-1][1] <= sp.seq_len
+                n = rngs[0][3]
+                assert len(rngs) == n and sorted(x[2] for x in rngs) == (list(range(n)) if n > 1 else [-1])
+    assert not seen
+
+
+@pytest.mark.parametrize("name", W.CONFIG_NAMES)
+def test_planner_covers_configs(name):
+    gen = __import__("torch").Generator().manual_seed(W.CONFIG_NAMES.index(name))
+    seqs, Hq, Hkv, d, _ = W.config_seqs(name, gen)
+
+    class B:  # structure only: no tensors needed for the planner
+        pass
+    b = B()
+    b.seqs, b.num_q_heads, b.num_kv_heads = seqs, Hq, Hkv
+    if name == "llama33_70b_prefill":
+        b.seqs = seqs[:2]                       # keep the pure-Python coverage check fast
+    pages = sum((s.seq_len + 15) // 16 for s in b.seqs)
+    items = pk.inspect([s.seq_len for s in b.seqs], [s.query_len for s in b.seqs],
+                       [s.mask_kind for s in b.seqs], [p for s in b.seqs for p in s.parents],
+                       num_q_heads=Hq, num_kv_heads=Hkv, head_dim=d, num_pages=pages,
+                       bt_stride=max((s.seq_len + 15) // 16 for s in b.seqs))
+    _coverage(b, items)
+    sizes = [it["key_end"] - it["key_begin"] for it in items]
+    # heaviest first (page-granular: the last page of a task may be partial)
+    pg = [(it["key_end"] + 15) // 16 - it["key_begin"] // 16 for it in items]
+    assert pg == sorted(pg, reverse=True)
+    assert max(sizes) <= 1024 * 16
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_planner_covers_random_batches(seed):
+    b = W.random_small(seed, num_seqs=6, max_ctx=300, max_q=40, tree_frac=0.4)
+    items = pk.inspect(b.seq_lens, b.query_lens, b.mask_kinds, b.parents_flat,
+                       num_q_heads=b.num_q_heads, num_kv_heads=b.num_kv_heads, head_dim=b.head_dim,
+                       num_pages=b.k_cache.shape[0], bt_stride=b.block_table.shape[1],
+                       num_sms=4, ctas_per_sm=1)
+    _coverage(b, items)
+
+
+def test_empty_batch_plans_to_nothing():
+    assert pk.inspect([], [], [], num_q_heads=8, num_kv_heads=2, head_dim=64, num_pages=0,
+                      bt_stride=0) == []
+
+
+def test_long_context_is_split():
+    items = pk.inspect([100000] * 2, [1, 1], [0, 0], num_q_heads=128, num_kv_heads=8,
+                       head_dim=128, num_pages=12500, bt_stride=6250)
+    assert all(it["num_splits"] > 1 for it in items)
+    assert len(items) >= 148

@@ -1,0 +1,155 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Tolerance (bf16 inputs, fp32 accumulation, bf16 output): max abs <= 2e-2 and mean abs
+<= 2e-3 per compared set of rows. Small batches are compared on every row; the
+full-size batches on sampled sequences and tokens, in the launch configuration the
+benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_attention_verify_b200 as pk
+import workloads as W
+from _util import assert_close, oracle_rows
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def run_batch(b, plan=None):
+    plan = plan or pk.plan_for_batch(b)
+    out = plan.run(b.q, b.k_cache, b.v_cache)
+    assert plan.check() == 0
+    return out, plan
+
+
+def test_tiny_decode_config_all_rows():
+    b = W.make_config("tiny_decode", device=DEV)
+    out, plan = run_batch(b)
+    rows, exp = oracle_rows(b)
+    assert_close(out[rows], exp, "tiny_decode")
+    assert plan.info()["num_decode_items"] > 0
+
+
+SMALL = [
+    dict(seed=1, Hq=8, Hkv=2, d=64, max_ctx=80, max_q=40),
+    dict(seed=2, Hq=8, Hkv=2, d=128, max_ctx=300, max_q=20),
+    dict(seed=3, Hq=28, Hkv=4, d=128, max_ctx=500, max_q=12, tree_frac=0.6),
+    dict(seed=4, Hq=16, Hkv=16, d=128, max_ctx=200, max_q=33),
+    dict(seed=5, Hq=32, Hkv=2, d=64, max_ctx=700, max_q=5, tree_frac=0.5),
+    dict(seed=6, Hq=4, Hkv=1, d=128, max_ctx=40, max_q=64, tree_frac=0.5, max_draft=64),
+    dict(seed=7, Hq=64, Hkv=8, d=128, max_ctx=2000, max_q=9, num_seqs=5),
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: f"seed{c['seed']}_H{c['Hq']}x{c['Hkv']}_d{c['d']}")
+def test_small_mixed_batches_all_rows(cfg):
+    cfg = dict(cfg)
+    b = W.random_small(cfg.pop("seed"), device=DEV, bt_extra=3, **cfg)
+    out, _ = run_batch(b)
+    rows, exp = oracle_rows(b)
+    assert_close(out[rows], exp, "small batch")
+
+
+def test_edge_lengths():
+    """ctx 1, ctx at a page boundary, page + 1, a query longer than a page, a 64-node tree."""
+    seqs = [W.SeqSpec(1, 1, W.CAUSAL, []), W.SeqSpec(16, 1, W.CAUSAL, []),
+            W.SeqSpec(17, 1, W.CAUSAL, []), W.SeqSpec(32, 32, W.CAUSAL, []),
+            W.SeqSpec(48, 17, W.CAUSAL, []),
+            W.SeqSpec(64 + 3, 64, W.TREE, W.random_tree(torch.Generator().manual_seed(5), 64)),
+            W.SeqSpec(5, 5, W.TREE, [-1, 0, 0, 1, 3])]
+    for d in (64, 128):
+        b = W.build_batch("edges", seqs, 8, 2, d, seed=77, device=DEV)
+        out, _ = run_batch(b)
+        rows, exp = oracle_rows(b)
+        assert_close(out[rows], exp, f"edges d{d}")
+
+
+def test_page_permutation_gives_bitwise_identical_output():
+    b1 = W.random_small(21, num_seqs=5, Hq=16, Hkv=4, d=128, max_ctx=900, max_q=10, device=DEV)
+    b2 = W.repage(b1, perm_seed=4242)
+    assert not torch.equal(b1.block_table, b2.block_table)
+    o1, _ = run_batch(b1)
+    o2, _ = run_batch(b2)
+    assert torch.equal(o1, o2)
+
+
+def test_repeated_runs_are_identical_and_reset_split_state():
+    b = W.build_batch("long", [W.SeqSpec(20000, 1, W.CAUSAL, []), W.SeqSpec(9000, 3, W.TREE, [-1, 0, 0])],
+                      32, 2, 128, seed=3, device=DEV)
+    plan = pk.plan_for_batch(b)
+    assert plan.info()["num_split_units"] > 0
+    o1 = plan.run(b.q, b.k_cache, b.v_cache).clone()
+    o2 = plan.run(b.q, b.k_cache, b.v_cache)
+    assert torch.equal(o1, o2)
+    rows, exp = oracle_rows(b)
+    assert_close(o2[rows], exp, "split")
+
+
+def test_decode_steps_match_prefill_rows_on_gpu():
+    L, T = 300, 24
+    full = W.build_batch("pf", [W.SeqSpec(L, T, W.CAUSAL, [])], 8, 2, 128, seed=9, device=DEV)
+    o_full, _ = run_batch(full)
+    k, v = full.seq_kv(0)
+    for i in (0, 7, 23):
+        Li = L - T + i + 1
+        step = W.build_batch("st", [W.SeqSpec(Li, 1, W.CAUSAL, [])], 8, 2, 128, seed=9, device=DEV)
+        step.q = full.q[i:i + 1].clone()
+        # same keys/values, laid out in the step batch's own pool
+        step.k_cache.zero_()
+        step.v_cache.zero_()
+        P = 16
+        for pos in range(Li):
+            pg = step.block_table[0, pos // P].item()
+            step.k_cache[pg, :, pos % P] = k[pos]
+            step.v_cache[pg, :, pos % P] = v[pos]
+        o_step, _ = run_batch(step)
+        d = (o_step[0].float() - o_full[i].float()).abs().max().item()
+        assert d <= 2e-2, (i, d)
+
+
+def test_run_host_matches_run():
+    b = W.random_small(31, num_seqs=6, Hq=8, Hkv=2, d=128, max_ctx=400, max_q=8, device=DEV)
+    plan = pk.plan_for_batch(b)
+    o_dev = plan.run(b.q, b.k_cache, b.v_cache)
+    q_host = b.q.cpu().pin_memory()
+    o_host = torch.empty(q_host.shape, dtype=torch.bfloat16).pin_memory()
+    plan.run_host(q_host, b.k_cache, b.v_cache, o_host)
+    torch.cuda.current_stream().synchronize()
+    assert torch.equal(o_host, o_dev.cpu())
+
+
+def test_run_rejects_misaligned_pointer():
+    b = W.make_config("tiny_decode", device=DEV)
+    plan = pk.plan_for_batch(b)
+    L = pk.lib()
+    rc = L.attn_run(plan._handle, b.q.data_ptr() + 2, b.k_cache.data_ptr(), b.v_cache.data_ptr(),
+                    b.q.data_ptr(), None)
+    assert rc == -1
+
+
+FULL = ["llama3_8b_decode", "qwen2_7b_unified", "long_ctx_split", "llama33_70b_prefill"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_config_sampled(name):
+    b = W.make_config(name, device=DEV)
+    out, plan = run_batch(b)
+    n = len(b.seqs)
+    if name == "llama33_70b_prefill":
+        seq_ids = [0, 5]
+        picker = lambda sp: [0, 1, 127, 128, 1000, sp.query_len - 1]
+    elif name == "qwen2_7b_unified":
+        seq_ids = [0, 3, 4, 100, n - 32, n - 1]
+        picker = None
+    elif name == "long_ctx_split":
+        seq_ids = [0, 7, 15]
+        picker = None
+    else:
+        seq_ids = [0, 31, 64, 127]
+        picker = None
+    rows, exp = oracle_rows(b, seq_ids, picker)
+    assert_close(out[rows], exp, name)
+    # every output row is finite
+    assert torch.isfinite(out.float()).all()
