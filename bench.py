@@ -192,7 +192,7 @@ def run_ours(args):
     dev = torch.device("cuda", torch.cuda.current_device())
     peaks = load_peaks()
 
-    batch = W.make_config(args.config, device=dev)
+    batch = W.make_config(args.config, device=dev, max_seqs=args.seqs)
     plan = pk.plan_for_batch(batch)
     info = plan.info()
     stream = torch.cuda.current_stream()
@@ -230,28 +230,30 @@ def run_ours(args):
         raise RuntimeError("device error during the timed region")
 
     # end to end through the C ABI with host buffers (pinned), copies inside the region
-    q_host = batch.q.cpu().pin_memory()
-    o_host = torch.empty(q_host.shape, dtype=torch.bfloat16).pin_memory()
-    for _ in range(args.warmup):
-        plan.run_host(q_host, batch.k_cache, batch.v_cache, o_host, stream)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if ws > 1:
-        dist.barrier()
-    e0.record(stream)
-    for _ in range(args.steps):
-        plan.run_host(q_host, batch.k_cache, batch.v_cache, o_host, stream)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if ws > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = None
+    if not args.no_e2e:
+        q_host = batch.q.cpu().pin_memory()
+        o_host = torch.empty(q_host.shape, dtype=torch.bfloat16).pin_memory()
+        for _ in range(args.warmup):
+            plan.run_host(q_host, batch.k_cache, batch.v_cache, o_host, stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if ws > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            plan.run_host(q_host, batch.k_cache, batch.v_cache, o_host, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if ws > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
 
     tokens = batch.total_q
     value = ws * tokens * args.steps / (elapsed_ms * 1e-3)
-    e2e_value = ws * tokens * args.steps / (e2e_ms * 1e-3)
+    e2e_value = ws * tokens * args.steps / (e2e_ms * 1e-3) if e2e_ms else None
     avg_launch_s = (sum(per) / len(per)) * 1e-3
     kv_gbs = info["kv_bytes"] / avg_launch_s / 1e9
     tflops = info["attn_flops"] / avg_launch_s / 1e12
@@ -269,7 +271,8 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{args.config}: {WORKLOADS[args.config]}",
+            "config": {"workload": f"{args.config}: {WORKLOADS[args.config]}"
+                       + (f" (first {args.seqs} sequences)" if args.seqs else ""),
                        "query_tokens_per_step": tokens, "kv_bytes_per_step": info["kv_bytes"],
                        "l2": "inputs larger than L2 (KV cache read each step exceeds 126 MB)",
                        "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
@@ -299,6 +302,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
+    ap.add_argument("--seqs", type=int, default=None,
+                    help="keep only the first N sequences of the batch (smaller profiler captures)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="host time for the oracle baseline line of our arm")
     ap.add_argument("--ref-seconds", type=float, default=120.0,

@@ -232,12 +232,17 @@ def build_batch(name: str, seqs: Sequence[SeqSpec], num_q_heads: int, num_kv_hea
 
 
 def make_config(name: str, device="cpu", seed: Optional[int] = None,
-                keep_contiguous: bool = True) -> Batch:
-    """One of the five named batches, seeded by its index unless ``seed`` is given."""
+                keep_contiguous: bool = True, max_seqs: Optional[int] = None) -> Batch:
+    """One of the five named batches, seeded by its index unless ``seed`` is given.
+
+    ``max_seqs`` keeps only the first sequences (smaller cases of the same shape, e.g.
+    for profiler captures)."""
     if seed is None:
         seed = CONFIG_NAMES.index(name)
     sgen = torch.Generator().manual_seed(seed)
     seqs, Hq, Hkv, d, outl = config_seqs(name, sgen)
+    if max_seqs is not None:
+        seqs = seqs[:max_seqs]
     # structure draws above advance sgen; build_batch re-seeds its own structure stream
     return build_batch(name, seqs, Hq, Hkv, d, seed=seed + 1000, device=device,
                        outlier_frac=outl, keep_contiguous=keep_contiguous)
