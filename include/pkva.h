@@ -147,6 +147,38 @@ PKVA_API void attn_plan_destroy(pkva_plan_t plan);
 /* attn_last_error — message for the last failing call on this thread ("" if none). */
 PKVA_API const char* attn_last_error(void);
 
+/*
+ * attn_run_static — plan and run one batch in a single call that allocates no device memory.
+ *
+ * The paper has no counterpart to this call; it exists for callers that cannot call
+ * cudaMalloc where they need attention (an engine that owns all device memory through its
+ * own pool, or code running where allocation is not allowed). attn_plan allocates the
+ * plan's tables and split-KV scratch; this call instead keeps them in one fixed array
+ * that the library reserves on every GPU that loads it (about 9 MiB, held until the
+ * process exits), and plans on the host each time. It calls no cudaMalloc, cudaFree or
+ * other allocating routine; the caller still passes all inputs and outputs.
+ *
+ * Arguments are those of attn_plan followed by those of attn_run. Limits of the fixed
+ * scratch: at most 4096 sequences, 16384 tile tasks, 4096 split units, 16384 draft-tree
+ * tokens and 8 MiB of split partials (1024 split tasks at head_dim 128, 2048 at 64);
+ * a batch beyond any of them is rejected with PKVA_EUNSUPPORTED and a message naming
+ * the limit, before anything is launched.
+ *
+ * Set-up: the first call on a device (with that device current) looks up the array's
+ * device address; make that first call before any stream capture. Every call shares the
+ * one array, which keeps the last call's contents (the call clears the parts that must
+ * start at zero), so calls that overlap on the GPU (on different streams, or from
+ * different threads) race: serialize them. Device-side error bits (a block-table entry
+ * out of range) are not reported by this call. The task tables are copied from host
+ * memory with cudaMemcpyAsync, which may wait for `stream` before returning.
+ */
+PKVA_API int attn_run_static(int num_seqs, const int32_t* seq_lens, const int32_t* query_lens,
+                             const int32_t* block_table, int bt_stride, int num_pages,
+                             const int32_t* mask_kind, const int32_t* parents, int num_q_heads,
+                             int num_kv_heads, int head_dim, int page_size, float sm_scale,
+                             const void* q, const void* k_cache, const void* v_cache, void* out,
+                             void* stream);
+
 /* Summary of a plan's decomposition (for logging and tests). */
 typedef struct pkva_plan_info {
     int32_t num_seqs;

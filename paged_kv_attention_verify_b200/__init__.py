@@ -32,7 +32,7 @@ DEVERR_TIMEOUT = 0x2
 
 # every entry point that include/pkva.h declares
 EXPORTED = ["attn_plan", "attn_run", "attn_run_host", "attn_check", "attn_plan_destroy",
-            "attn_last_error", "attn_plan_get_info", "attn_plan_inspect"]
+            "attn_last_error", "attn_plan_get_info", "attn_plan_inspect", "attn_run_static"]
 
 
 class PkvaError(RuntimeError):
@@ -84,8 +84,11 @@ def lib() -> ctypes.CDLL:
                                     _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                     ctypes.c_int, ctypes.c_int, ctypes.POINTER(WorkDesc),
                                     ctypes.c_int, _i32p]
+    L.attn_run_static.argtypes = [ctypes.c_int, _i32p, _i32p, _vp, ctypes.c_int, ctypes.c_int, _i32p,
+                                  _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                  ctypes.c_float, _vp, _vp, _vp, _vp, _vp]
     for name in ("attn_plan", "attn_run", "attn_run_host", "attn_check", "attn_plan_get_info",
-                 "attn_plan_inspect"):
+                 "attn_plan_inspect", "attn_run_static"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -214,6 +217,26 @@ def inspect(seq_lens, query_lens, mask_kind, parents=None, *, num_q_heads: int,
     arr = (WorkDesc * max(1, n.value))()
     _check(lib().attn_plan_inspect(*args, arr, n.value, ctypes.byref(n)))
     return [{f: getattr(arr[i], f) for f, _ in WorkDesc._fields_} for i in range(n.value)]
+
+
+def run_static(seq_lens, query_lens, block_table, mask_kind, parents, q, k_cache, v_cache, out, *,
+               num_q_heads: int, num_kv_heads: int, head_dim: int, num_pages: int,
+               page_size: int = 16, sm_scale: Optional[float] = None, stream=None):
+    """``attn_run_static``: plan and run in one call without allocating device memory.
+
+    For callers that cannot allocate where they need attention; ``out`` must be
+    allocated by the caller beforehand. The library keeps the call's tables and split
+    scratch in a fixed array it reserves per GPU, so overlapping calls race (serialize
+    them), and batches beyond that array's limits raise PKVA_EUNSUPPORTED."""
+    sl, ql, mk = _i32(seq_lens), _i32(query_lens), _i32(mask_kind)
+    par = _i32(parents if parents is not None else [])
+    bt_stride = block_table.shape[1] if len(sl) else 0
+    _check(lib().attn_run_static(len(sl), _ptr(sl), _ptr(ql), block_table.data_ptr() if len(sl) else None,
+                                 bt_stride, num_pages, _ptr(mk), _ptr(par), num_q_heads, num_kv_heads,
+                                 head_dim, page_size, float(sm_scale) if sm_scale else 0.0,
+                                 q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), out.data_ptr(),
+                                 _stream_handle(stream)))
+    return out
 
 
 def plan_for_batch(batch, sm_scale: Optional[float] = None) -> Plan:
