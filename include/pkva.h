@@ -160,9 +160,10 @@ PKVA_API const char* attn_last_error(void);
  *
  * Arguments are those of attn_plan followed by those of attn_run. Limits of the fixed
  * scratch: at most 4096 sequences, 16384 tile tasks, 4096 split units, 16384 draft-tree
- * tokens and 8 MiB of split partials (1024 split tasks at head_dim 128, 2048 at 64);
- * a batch beyond any of them is rejected with PKVA_EUNSUPPORTED and a message naming
- * the limit, before anything is launched.
+ * tokens and 8 MiB of split partials (1024 split tasks at head_dim 128, 2048 at 64; long
+ * contexts are split more coarsely than attn_plan would split them until they fit). A
+ * batch beyond any limit is rejected with PKVA_EUNSUPPORTED and a message naming the
+ * limit, before anything is launched.
  *
  * Set-up: the first call on a device (with that device current) looks up the array's
  * device address; make that first call before any stream capture. Every call shares the

@@ -23,7 +23,8 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden",
           "-I", os.path.join(ROOT, "include"), "-I", CSRC]
-CU_FLAGS = ARCH + COMMON + ["--expt-relaxed-constexpr", "-use_fast_math", "-Xptxas", "-v"]
+CU_FLAGS = ARCH + COMMON + ["--expt-relaxed-constexpr", "-use_fast_math", "-diag-suppress=177",
+                            "-Xptxas", "-v"]
 
 
 def _sources():

@@ -5,6 +5,8 @@
 
 #include <math.h>
 #include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include <mutex>
 #include <new>
@@ -31,6 +33,11 @@ static int cuda_fail(cudaError_t e, const char* what) {
         cudaError_t e_ = (call);                       \
         if (e_ != cudaSuccess) return cuda_fail(e_, what); \
     } while (0)
+
+bool decode_body_is_mma() {
+    const char* v = getenv("PKVA_DECODE_BODY");
+    return !(v && strcmp(v, "fma") == 0);
+}
 
 static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -77,6 +84,7 @@ struct pkva_plan {
     int device = 0;
     int num_sms = 0;
     int decode_ctas = 0;
+    bool decode_mma = true;
     const int32_t* block_table = nullptr;
     pkva::SeqInfo* d_seqs = nullptr;
     pkva::DecodeWork* d_dwork = nullptr;
@@ -156,13 +164,14 @@ extern "C" int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq
     p->device = dev;
     p->num_sms = sms;
     p->block_table = block_table;
+    p->decode_mma = decode_body_is_mma();
 
     // the decode kernel's residency decides how many CTA slots the planner balances for
     {
         HostPlan probe;
         std::string err;
         build_host_plan(a, &probe, &err);
-        p->decode_ctas = decode_ctas_per_sm(head_dim, probe.decode_rows);
+        p->decode_ctas = decode_ctas_per_sm(head_dim, probe.decode_rows, p->decode_mma);
         if (p->decode_ctas < 1) {
             free_plan(p);
             set_last_error("attn_plan: decode kernel cannot be resident (shared memory)");
@@ -179,7 +188,7 @@ extern "C" int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq
         return rc;
     }
     // the kernel set for the final row count may differ from the probe's; re-query
-    p->decode_ctas = decode_ctas_per_sm(head_dim, p->hp.decode_rows);
+    p->decode_ctas = decode_ctas_per_sm(head_dim, p->hp.decode_rows, p->decode_mma);
 
     const HostPlan& hp = p->hp;
 #define PKVA_TRY(x)              \
@@ -295,7 +304,8 @@ extern "C" int attn_run(pkva_plan_t plan, const void* q, const void* k_cache, co
     dp.G = hp.G;
     dp.num_pages = hp.num_pages;
     dp.scale_log2 = hp.scale * 1.4426950408889634f;
-    cudaError_t e = launch_decode(dp, (int)hp.dwork.size(), hp.D, hp.decode_rows, plan->tmK, plan->tmV, st);
+    cudaError_t e = launch_decode(dp, (int)hp.dwork.size(), hp.D, hp.decode_rows, plan->decode_mma, plan->tmK,
+                                  plan->tmV, st);
     if (e != cudaSuccess) return cuda_fail(e, "attn_run: decode launch");
     return PKVA_OK;
 }

@@ -28,10 +28,15 @@ struct DecodeParams {
 };
 
 // Resident CTAs per SM of the decode kernel compiled for (D, rows); 0 if unsupported.
-int decode_ctas_per_sm(int D, int rows);
+// `mma` selects the tensor-core page body, otherwise the CUDA-core one.
+int decode_ctas_per_sm(int D, int rows, bool mma);
 
 // Launch the decode/verify kernel over `num_work` tasks.
-cudaError_t launch_decode(const DecodeParams& p, int num_work, int D, int rows,
+cudaError_t launch_decode(const DecodeParams& p, int num_work, int D, int rows, bool mma,
                           const CUtensorMap& tmK, const CUtensorMap& tmV, cudaStream_t stream);
+
+// Page body for decode/verify tasks: tensor cores unless PKVA_DECODE_BODY=fma is set in
+// the environment when the plan is made (the CUDA-core body, kept for comparison).
+bool decode_body_is_mma();
 
 }  // namespace pkva

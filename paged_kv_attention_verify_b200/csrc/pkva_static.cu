@@ -156,18 +156,25 @@ extern "C" int attn_run_static(int num_seqs, const int32_t* seq_lens, const int3
         return PKVA_EUNSUPPORTED;
     }
     a.num_sms = sms;
-    a.ctas_per_sm = decode_ctas_per_sm(head_dim, hp.decode_rows);
+    const bool mma = decode_body_is_mma();
+    a.ctas_per_sm = decode_ctas_per_sm(head_dim, hp.decode_rows, mma);
     if (a.ctas_per_sm < 1) {
         set_last_error("attn_run_static: decode kernel cannot be resident");
         return PKVA_ECUDA;
     }
-    rc = build_host_plan(a, &hp, &err);
-    if (rc != PKVA_OK) {
-        set_last_error("attn_run_static: " + err);
-        return rc;
+    // capacity checks: reject what the fixed scratch cannot hold. Splitting long contexts
+    // is the planner's choice, so first plan for fewer CTA slots (coarser splits) until
+    // the split partials fit.
+    const long max_slots = (long)(kStPartialBytes / ((size_t)kDecodeRowsMax * head_dim * sizeof(float)));
+    while (true) {
+        rc = build_host_plan(a, &hp, &err);
+        if (rc != PKVA_OK) {
+            set_last_error("attn_run_static: " + err);
+            return rc;
+        }
+        if ((long)hp.num_slots <= max_slots || a.num_sms == 1) break;
+        a.num_sms = (a.num_sms + 1) / 2;
     }
-    // capacity checks: reject what the fixed scratch cannot hold
-    const long max_slots = (long)(kStPartialBytes / ((size_t)kDecodeRowsMax * hp.D * sizeof(float)));
     if ((long)hp.seqs.size() > kStMaxSeqs) return too_big("sequences", (long)hp.seqs.size(), kStMaxSeqs);
     if ((long)hp.dwork.size() > kStMaxTasks) return too_big("tile tasks", (long)hp.dwork.size(), kStMaxTasks);
     if ((long)hp.units.size() > kStMaxUnits) return too_big("split units", (long)hp.units.size(), kStMaxUnits);
@@ -216,7 +223,7 @@ extern "C" int attn_run_static(int num_seqs, const int32_t* seq_lens, const int3
     dp.G = hp.G;
     dp.num_pages = hp.num_pages;
     dp.scale_log2 = hp.scale * 1.4426950408889634f;
-    e = launch_decode(dp, (int)hp.dwork.size(), hp.D, hp.decode_rows, tmK, tmV, st);
+    e = launch_decode(dp, (int)hp.dwork.size(), hp.D, hp.decode_rows, mma, tmK, tmV, st);
     if (e != cudaSuccess) {
         set_last_error(std::string("attn_run_static: launch: ") + cudaGetErrorString(e));
         return PKVA_ECUDA;

@@ -52,6 +52,17 @@ def test_small_mixed_batches_all_rows(cfg):
     assert_close(out[rows], exp, "small batch")
 
 
+@pytest.mark.parametrize("cfg", SMALL[:5], ids=lambda c: f"fma_seed{c['seed']}")
+def test_cuda_core_body_small_batches(cfg, monkeypatch):
+    """The CUDA-core page body (kept for comparison) against the oracle too."""
+    monkeypatch.setenv("PKVA_DECODE_BODY", "fma")
+    cfg = dict(cfg)
+    b = W.random_small(cfg.pop("seed"), device=DEV, bt_extra=3, **cfg)
+    out, _ = run_batch(b)
+    rows, exp = oracle_rows(b)
+    assert_close(out[rows], exp, "small batch, CUDA-core body")
+
+
 def test_edge_lengths():
     """ctx 1, ctx at a page boundary, page + 1, a query longer than a page, a 64-node tree."""
     seqs = [W.SeqSpec(1, 1, W.CAUSAL, []), W.SeqSpec(16, 1, W.CAUSAL, []),
