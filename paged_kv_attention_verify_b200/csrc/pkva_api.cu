@@ -67,6 +67,21 @@ static bool encode_cache_map(CUtensorMap* map, const void* base, int num_pages, 
     return r == CUDA_SUCCESS;
 }
 
+// q viewed as the 3-D bf16 tensor [sum T][Hq][D]; one box is 128 tokens x 64 columns of
+// one head, stored with the 128-byte swizzle (the prefill kernel's A operand layout).
+static bool encode_q_map(CUtensorMap* map, const void* base, int total_q, int Hq, int D) {
+    auto fn = tensor_map_encoder();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)total_q};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)kPrefillTileM};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <class T>
 static int upload(T** dst, const std::vector<T>& src, int64_t* bytes) {
     *dst = nullptr;
@@ -88,6 +103,11 @@ struct pkva_plan {
     const int32_t* block_table = nullptr;
     pkva::SeqInfo* d_seqs = nullptr;
     pkva::DecodeWork* d_dwork = nullptr;
+    pkva::PrefillWork* d_pwork = nullptr;
+    cudaStream_t side = nullptr;            // prefill tasks run here, overlapping decode tasks
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+    CUtensorMap tmQ;
+    const void* tm_q = nullptr;
     pkva::SplitUnit* d_units = nullptr;
     uint64_t* d_anc = nullptr;
     float* d_part_o = nullptr;
@@ -108,6 +128,10 @@ static void free_plan(pkva_plan* p) {
     if (!p) return;
     cudaFree(p->d_seqs);
     cudaFree(p->d_dwork);
+    cudaFree(p->d_pwork);
+    if (p->side) cudaStreamDestroy(p->side);
+    if (p->ev_fork) cudaEventDestroy(p->ev_fork);
+    if (p->ev_join) cudaEventDestroy(p->ev_join);
     cudaFree(p->d_units);
     cudaFree(p->d_anc);
     cudaFree(p->d_part_o);
@@ -201,6 +225,16 @@ extern "C" int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq
     } while (0)
     PKVA_TRY(upload(&p->d_seqs, hp.seqs, &p->scratch_bytes));
     PKVA_TRY(upload(&p->d_dwork, hp.dwork, &p->scratch_bytes));
+    PKVA_TRY(upload(&p->d_pwork, hp.pwork, &p->scratch_bytes));
+    if (!hp.pwork.empty() && !hp.dwork.empty()) {
+        cudaError_t e = cudaStreamCreateWithFlags(&p->side, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->ev_fork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->ev_join, cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            free_plan(p);
+            return cuda_fail(e, "attn_plan: side stream");
+        }
+    }
     PKVA_TRY(upload(&p->d_units, hp.units, &p->scratch_bytes));
     PKVA_TRY(upload(&p->d_anc, hp.anc, &p->scratch_bytes));
     auto alloc_zero = [&](void** ptr, size_t bytes, const char* what) -> int {
@@ -243,7 +277,7 @@ extern "C" int attn_plan_get_info(pkva_plan_t plan, pkva_plan_info* info) {
     const HostPlan& hp = plan->hp;
     info->num_seqs = hp.num_seqs;
     info->num_decode_items = (int32_t)hp.dwork.size();
-    info->num_prefill_items = 0;
+    info->num_prefill_items = (int32_t)hp.pwork.size();
     info->num_split_units = (int32_t)hp.units.size();
     info->num_partial_slots = hp.num_slots;
     info->decode_rows = hp.decode_rows;
@@ -286,6 +320,36 @@ extern "C" int attn_run(pkva_plan_t plan, const void* q, const void* k_cache, co
         }
         plan->tm_v = v_cache;
     }
+    if (!hp.pwork.empty() && plan->tm_q != q) {
+        if (!encode_q_map(&plan->tmQ, q, hp.total_q, hp.Hq, hp.D)) {
+            set_last_error("attn_run: cuTensorMapEncodeTiled failed for q");
+            return PKVA_ECUDA;
+        }
+        plan->tm_q = q;
+    }
+    // prefill tiles on a side stream that forks from and joins back into `stream`
+    cudaStream_t pst = st;
+    if (!hp.pwork.empty() && plan->side) {
+        PKVA_CUDA(cudaEventRecord(plan->ev_fork, st), "attn_run: fork");
+        PKVA_CUDA(cudaStreamWaitEvent(plan->side, plan->ev_fork, 0), "attn_run: fork");
+        pst = plan->side;
+    }
+    if (!hp.pwork.empty()) {
+        PrefillParams pp;
+        pp.out = static_cast<__nv_bfloat16*>(out);
+        pp.block_table = plan->block_table;
+        pp.seqs = plan->d_seqs;
+        pp.work = plan->d_pwork;
+        pp.err = plan->d_err;
+        pp.bt_stride = hp.bt_stride;
+        pp.Hq = hp.Hq;
+        pp.Hkv = hp.Hkv;
+        pp.G = hp.G;
+        pp.num_pages = hp.num_pages;
+        pp.scale_log2 = hp.scale * 1.4426950408889634f;
+        cudaError_t e = launch_prefill(pp, (int)hp.pwork.size(), plan->tmQ, plan->tmK, plan->tmV, pst);
+        if (e != cudaSuccess) return cuda_fail(e, "attn_run: prefill launch");
+    }
     DecodeParams dp;
     dp.q = static_cast<const __nv_bfloat16*>(q);
     dp.out = static_cast<__nv_bfloat16*>(out);
@@ -307,6 +371,10 @@ extern "C" int attn_run(pkva_plan_t plan, const void* q, const void* k_cache, co
     cudaError_t e = launch_decode(dp, (int)hp.dwork.size(), hp.D, hp.decode_rows, plan->decode_mma, plan->tmK,
                                   plan->tmV, st);
     if (e != cudaSuccess) return cuda_fail(e, "attn_run: decode launch");
+    if (pst != st) {
+        PKVA_CUDA(cudaEventRecord(plan->ev_join, pst), "attn_run: join");
+        PKVA_CUDA(cudaStreamWaitEvent(st, plan->ev_join, 0), "attn_run: join");
+    }
     return PKVA_OK;
 }
 

@@ -12,6 +12,10 @@ constexpr int kPageSize = 16;          // keys per page (the only page size supp
 constexpr int kMaxTreeTokens = 64;     // draft tokens per TREE sequence (one 64-bit mask)
 constexpr int kDecodeRowsMax = 16;     // packed (token, head) rows per decode task
 constexpr int kDecodeMaxPages = 1024;  // pages per decode task (block-table slice in smem)
+constexpr int kPrefillTileM = 128;     // query tokens per prefill tile (tcgen05 M)
+constexpr int kPrefillTileN = 128;     // keys per prefill KV tile (8 pages)
+constexpr int kPrefillMinTokens = 64;  // causal sequences with at least this many new tokens
+                                       // (and head_dim 128) run on the tensor-core prefill kernel
 
 // Per-sequence record (the "Token-Table" row of the batch).
 struct SeqInfo {
@@ -38,6 +42,18 @@ struct DecodeWork {
 };
 static_assert(sizeof(DecodeWork) == 32, "DecodeWork layout");
 
+// One prefill tile task: 128 query tokens [tok0, tok0 + ntok) of one query head against
+// KV tiles [0, num_kv_tiles) of 128 keys.
+struct PrefillWork {
+    int32_t seq;
+    int32_t q_head;
+    int32_t tok0;
+    int32_t ntok;
+    int32_t num_kv_tiles;
+    int32_t pad0, pad1, pad2;
+};
+static_assert(sizeof(PrefillWork) == 32, "PrefillWork layout");
+
 // A (seq, kv_head, row chunk) split over several tasks: where its partials live.
 struct SplitUnit {
     int32_t slot_base;   // first partial slot
@@ -54,6 +70,7 @@ struct HostPlan {
     std::vector<SeqInfo> seqs;
     std::vector<uint64_t> anc;            // per TREE token: ancestor-or-self bit mask
     std::vector<DecodeWork> dwork;        // launch order
+    std::vector<PrefillWork> pwork;       // launch order
     std::vector<SplitUnit> units;
     int num_slots = 0;
     int64_t kv_bytes = 0;
@@ -72,6 +89,7 @@ struct PlanArgs {
     float sm_scale;
     int num_sms;
     int ctas_per_sm;
+    bool use_prefill_kernel = true;       // false: every sequence goes to the decode kernel
 };
 
 // Validates and decomposes; returns a pkva_status and fills `err` on failure.

@@ -27,6 +27,25 @@ struct DecodeParams {
     float scale_log2;            // softmax scale * log2(e)
 };
 
+struct PrefillParams {
+    __nv_bfloat16* out;          // [sum T, Hq, 128]
+    const int32_t* block_table;  // [B, bt_stride]
+    const SeqInfo* seqs;
+    const PrefillWork* work;
+    int32_t* err;
+    int32_t bt_stride;
+    int32_t Hq, Hkv, G;
+    int32_t num_pages;
+    float scale_log2;
+};
+
+int prefill_ctas_per_sm();
+
+// Launch the tensor-core prefill kernel (head_dim 128). tmQ views q as the 3-D tensor
+// [sum T][Hq][128] with a {64, 1, 128} box; tmK/tmV as the decode kernel's cache maps.
+cudaError_t launch_prefill(const PrefillParams& p, int num_work, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                           const CUtensorMap& tmV, cudaStream_t stream);
+
 // Resident CTAs per SM of the decode kernel compiled for (D, rows); 0 if unsupported.
 // `mma` selects the tensor-core page body, otherwise the CUDA-core one.
 int decode_ctas_per_sm(int D, int rows, bool mma);

@@ -118,12 +118,44 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
     }
     p.total_q = (int)q_acc;
 
+    // -- prefill tiles: long causal chunks go to the tensor-core prefill kernel ---------
+    std::vector<char> on_prefill(a.num_seqs, 0);
+    if (a.use_prefill_kernel && a.D == 128) {
+        for (int s = 0; s < a.num_seqs; ++s) {
+            const SeqInfo& si = p.seqs[s];
+            if (si.mask_kind != PKVA_CAUSAL || si.query_len < kPrefillMinTokens) continue;
+            on_prefill[s] = 1;
+            const int prefix = si.seq_len - si.query_len;
+            for (int t0 = 0; t0 < si.query_len; t0 += kPrefillTileM) {
+                const int ntok = std::min(kPrefillTileM, si.query_len - t0);
+                // keys up to the last row's own position (causal tile skipping)
+                const int kend = prefix + t0 + ntok;
+                const int tiles = (kend + kPrefillTileN - 1) / kPrefillTileN;
+                for (int h = 0; h < a.Hq; ++h) {
+                    PrefillWork pw{};
+                    pw.seq = s;
+                    pw.q_head = h;
+                    pw.tok0 = t0;
+                    pw.ntok = ntok;
+                    pw.num_kv_tiles = tiles;
+                    p.pwork.push_back(pw);
+                }
+            }
+        }
+        // heaviest first; equal tiles keep (seq, tile, head) order so that the query heads
+        // of one GQA group run side by side and share their K/V tiles through L2
+        std::stable_sort(p.pwork.begin(), p.pwork.end(), [](const PrefillWork& x, const PrefillWork& y) {
+            return x.num_kv_tiles > y.num_kv_tiles;
+        });
+    }
+
     // -- decode/verify units: (seq, kv head, chunk of packed rows) --------------------
     struct Unit { int seq, kvh, rb, rc, pages; };
     std::vector<Unit> units;
     int64_t total_pages = 0;
     int max_rc = 0;
     for (int s = 0; s < a.num_seqs; ++s) {
+        if (on_prefill[s]) continue;
         const SeqInfo& si = p.seqs[s];
         const int rows = si.query_len * p.G;
         for (int h = 0; h < a.Hkv; ++h) {
@@ -141,6 +173,7 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
         }
     }
     p.decode_rows = max_rc <= 4 ? 4 : (max_rc <= 8 ? 8 : 16);
+    if (units.empty()) p.decode_rows = 4;
 
     // -- split long units so the grid has ~kTasksPerSlot tasks per CTA slot -------------
     const int64_t slots = (int64_t)a.num_sms * a.ctas_per_sm;
@@ -196,14 +229,30 @@ extern "C" int attn_plan_inspect(int num_seqs, const int32_t* seq_lens, const in
         set_last_error(err);
         return rc;
     }
-    const int n = (int)hp.dwork.size();
+    const int nd = (int)hp.dwork.size();
+    const int n = nd + (int)hp.pwork.size();
     if (num_items) *num_items = n;
     if (!items) return PKVA_OK;
     if (max_items < n) {
         set_last_error("attn_plan_inspect: max_items is smaller than the number of tasks");
         return PKVA_EINVAL;
     }
-    for (int i = 0; i < n; ++i) {
+    for (int i = nd; i < n; ++i) {
+        const PrefillWork& w = hp.pwork[i - nd];
+        const SeqInfo& si = hp.seqs[w.seq];
+        pkva_work_desc d;
+        d.kind = 1;
+        d.seq = w.seq;
+        d.kv_head = w.q_head / hp.G;
+        d.row_begin = w.tok0 * hp.G + w.q_head % hp.G;   // packed row of its first token
+        d.row_count = w.ntok;
+        d.key_begin = 0;
+        d.key_end = std::min(si.seq_len - si.query_len + w.tok0 + w.ntok, si.seq_len);
+        d.split = -1;
+        d.num_splits = 1;
+        items[i] = d;
+    }
+    for (int i = 0; i < nd; ++i) {
         const DecodeWork& w = hp.dwork[i];
         const SeqInfo& si = hp.seqs[w.seq];
         pkva_work_desc d;

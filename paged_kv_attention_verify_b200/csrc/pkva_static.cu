@@ -137,6 +137,7 @@ extern "C" int attn_run_static(int num_seqs, const int32_t* seq_lens, const int3
     // validate with the host planner before touching the device
     PlanArgs a{num_seqs, seq_lens, query_lens, bt_stride, num_pages, mask_kind, parents, num_q_heads,
                num_kv_heads, head_dim, page_size, sm_scale, 1, 1};
+    a.use_prefill_kernel = false;          // everything on the decode kernel (no TMEM, no extra tables)
     HostPlan hp;
     std::string err;
     int rc = build_host_plan(a, &hp, &err);

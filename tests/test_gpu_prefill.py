@@ -1,0 +1,78 @@
+"""GPU parity of the tensor-core prefill path (causal chunks of >= 64 new tokens, d = 128)
+against the float64 oracle, including chunk lengths that leave a ragged last tile, cached
+prefixes that do not align with the 128-key tiles, and GQA groups of several sizes."""
+import pytest
+import torch
+
+import paged_kv_attention_verify_b200 as pk
+import workloads as W
+from _util import assert_close, oracle_rows
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+CASES = [
+    # (prefix, T, Hq, Hkv)
+    (0, 128, 8, 2),
+    (0, 64, 8, 2),
+    (37, 200, 8, 2),
+    (500, 300, 28, 4),
+    (129, 129, 16, 16),
+    (1000, 513, 64, 8),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"p{c[0]}_T{c[1]}_H{c[2]}x{c[3]}")
+def test_prefill_chunk(case):
+    prefix, T, Hq, Hkv = case
+    b = W.build_batch("pf", [W.SeqSpec(prefix + T, T, W.CAUSAL, [])], Hq, Hkv, 128, seed=prefix + T,
+                      device=DEV)
+    plan = pk.plan_for_batch(b)
+    assert plan.info()["num_prefill_items"] > 0
+    out = plan.run(b.q, b.k_cache, b.v_cache)
+    assert plan.check() == 0
+    rows, exp = oracle_rows(b)
+    assert_close(out[rows], exp, f"prefill {case}")
+
+
+def test_prefill_mixed_with_decode_and_verify():
+    gen = torch.Generator().manual_seed(8)
+    seqs = [W.SeqSpec(300, 100, W.CAUSAL, []), W.SeqSpec(900, 1, W.CAUSAL, []),
+            W.SeqSpec(77, 77, W.CAUSAL, []), W.SeqSpec(1500 + 7, 7, W.TREE, W.random_tree(gen, 7)),
+            W.SeqSpec(2048, 256, W.CAUSAL, [])]
+    b = W.build_batch("mixed", seqs, 28, 4, 128, seed=5, device=DEV)
+    plan = pk.plan_for_batch(b)
+    info = plan.info()
+    assert info["num_prefill_items"] > 0 and info["num_decode_items"] > 0
+    for _ in range(2):
+        out = plan.run(b.q, b.k_cache, b.v_cache)
+        assert plan.check() == 0
+        rows, exp = oracle_rows(b)
+        assert_close(out[rows], exp, "mixed batch")
+
+
+def test_prefill_page_permutation_bitwise():
+    b1 = W.build_batch("pp", [W.SeqSpec(700, 256, W.CAUSAL, [])], 16, 4, 128, seed=3, device=DEV)
+    b2 = W.repage(b1, perm_seed=99)
+    o1 = pk.plan_for_batch(b1).run(b1.q, b1.k_cache, b1.v_cache)
+    o2 = pk.plan_for_batch(b2).run(b2.q, b2.k_cache, b2.v_cache)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+
+
+def test_prefill_matches_decode_body_on_same_rows(monkeypatch):
+    """The same causal chunk through the tensor-core prefill tiles and through the
+    decode/verify tasks (forced by planning with prefill off is not exposed, so compare
+    the chunk's last row against a one-token decode of that position)."""
+    L, T = 1000, 200
+    full = W.build_batch("pf", [W.SeqSpec(L, T, W.CAUSAL, [])], 8, 2, 128, seed=21, device=DEV)
+    o_full = pk.plan_for_batch(full).run(full.q, full.k_cache, full.v_cache)
+    step = W.build_batch("st", [W.SeqSpec(L, 1, W.CAUSAL, [])], 8, 2, 128, seed=21, device=DEV)
+    step.q = full.q[T - 1:T].clone()
+    step.k_cache.copy_(full.k_cache)
+    step.v_cache.copy_(full.v_cache)
+    step.block_table.copy_(full.block_table)
+    o_step = pk.plan_for_batch(step).run(step.q, step.k_cache, step.v_cache)
+    torch.cuda.synchronize()
+    d = (o_step[0].float() - o_full[T - 1].float()).abs().max().item()
+    assert d <= 2e-2
