@@ -7,11 +7,12 @@
 // mask leaves visible; tiles past the last row's own position are never loaded (causal
 // tile skipping), and only tiles that cross the diagonal are masked element by element.
 //
-// Warp roles (192 threads):
+// Warp roles (224 threads):
 //   warps 0-3  softmax: thread r owns row r = TMEM lane r. Reads S, keeps the running
 //              max / sum, writes P (bf16) back to TMEM, rescales O in TMEM only when a
 //              row max moved by more than 2^8 (rare after the first tiles), and writes O.
-//   warp 4     TMA producer: Q once, then K and V tiles into a 2-stage ring.
+//   warp 4     TMA producer of Q and of K tiles (3-stage ring, a stage is freed as soon as
+//              its QK^T is done); warp 6 produces V tiles (2-stage ring, freed after PV).
 //   warp 5     MMA issuer (one thread) and TMEM owner: QK^T of tile j+1 overlaps the
 //              softmax of tile j; PV of tile j reads P straight from TMEM.
 // TMEM (512 columns): S double buffer [0,256), O [256,384), P double buffer [384,512).
@@ -32,17 +33,19 @@ namespace pkva {
 
 namespace {
 
-constexpr int kPThreads = 192;
+constexpr int kPThreads = 224;
 constexpr int kD = 128;
-constexpr int kNS = 2;                                   // K/V stages
+constexpr int kNK = 3;                                   // K stages (freed when QK^T is done)
+constexpr int kNV = 2;                                   // V stages (freed when PV is done)
 constexpr int kHalfBytes = kPrefillTileM * 128;          // 128 rows x 64 bf16 (one swizzle column)
 constexpr int kTileBytes = 2 * kHalfBytes;               // 128 x 128 bf16
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kTileBytes;
-constexpr int kOffV = kOffK + kNS * kTileBytes;
-constexpr int kOffBar = kOffV + kNS * kTileBytes;
-// barriers: q_full, k_full[2], v_full[2], kv_empty[2], s_full[2], p_full[2], pv_done[2], mma_done
-constexpr int kNumBars = 1 + 3 * kNS + 2 + 2 + 2 + 1;
+constexpr int kOffV = kOffK + kNK * kTileBytes;
+constexpr int kOffBar = kOffV + kNV * kTileBytes;
+// barriers: q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2], p_full[2],
+// pv_done[2], mma_done
+constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 2 + 2 + 2 + 1;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kOffFlag = kOffTmemSlot + 16;
 constexpr int kSmemBytes = kOffFlag + 16;
@@ -57,8 +60,9 @@ constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);    // P fro
 struct Bars {
     uint64_t* q_full;
     uint64_t* k_full;
+    uint64_t* k_empty;
     uint64_t* v_full;
-    uint64_t* kv_empty;
+    uint64_t* v_empty;
     uint64_t* s_full;
     uint64_t* p_full;
     uint64_t* pv_done;
@@ -70,13 +74,41 @@ __device__ __forceinline__ Bars bars_at(uint8_t* sm) {
     Bars r;
     r.q_full = b;
     r.k_full = b + 1;
-    r.v_full = b + 1 + kNS;
-    r.kv_empty = b + 1 + 2 * kNS;
-    r.s_full = b + 1 + 3 * kNS;
+    r.k_empty = r.k_full + kNK;
+    r.v_full = r.k_empty + kNK;
+    r.v_empty = r.v_full + kNV;
+    r.s_full = r.v_empty + kNV;
     r.p_full = r.s_full + 2;
     r.pv_done = r.p_full + 2;
     r.mma_done = r.pv_done + 2;
     return r;
+}
+
+// Physical cache rows of the 8 pages of KV tile j (row -16 reads as zeros: past the end of
+// the sequence, or a block-table entry out of range, which is also flagged).
+__device__ __forceinline__ void tile_rows(const PrefillParams& p, const int32_t* btrow, int seq_pages, int kvh,
+                                          int j, int rows[8]) {
+#pragma unroll
+    for (int pg = 0; pg < 8; ++pg) {
+        const int lp = j * 8 + pg;
+        int ph = -1;
+        if (lp < seq_pages) {
+            ph = btrow[lp];
+            if (ph < 0 || ph >= p.num_pages) {
+                atomicOr(p.err, PKVA_DEVERR_BAD_PAGE);
+                ph = -1;
+            }
+        }
+        rows[pg] = ph >= 0 ? (ph * p.Hkv + kvh) * kPageSize : -kPageSize;
+    }
+}
+
+__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, const int rows[8]) {
+    mbar_arrive_expect_tx(bar, kTileBytes);
+#pragma unroll
+    for (int pg = 0; pg < 8; ++pg)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) tma_load_2d(dst + h * kHalfBytes + pg * (kPageSize * 128), map, bar, h * 64, rows[pg]);
 }
 
 // Bounded wait that also gives up at once when another role already gave up.
@@ -106,10 +138,13 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
 
     if (tid == 0) {
         mbar_init(B.q_full, 1);
-        for (int s = 0; s < kNS; ++s) {
+        for (int s = 0; s < kNK; ++s) {
             mbar_init(&B.k_full[s], 1);
+            mbar_init(&B.k_empty[s], 1);
+        }
+        for (int s = 0; s < kNV; ++s) {
             mbar_init(&B.v_full[s], 1);
-            mbar_init(&B.kv_empty[s], 1);
+            mbar_init(&B.v_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&B.s_full[b], 1);
@@ -129,51 +164,32 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
-        // ------------------------------ TMA producer ---------------------------------------
+    if (warp == 4 || warp == 6) {
+        // ------------------ TMA producers: warp 4 loads Q and K, warp 6 loads V -------------
         if (lane == 0) {
-            prefetch_tensormap(&tmQ);
-            prefetch_tensormap(&tmK);
-            prefetch_tensormap(&tmV);
-            const int qrow0 = si.q_start + w.tok0;
-            mbar_arrive_expect_tx(B.q_full, kTileBytes);
-            tma_load_3d(sm + kOffQ, &tmQ, B.q_full, 0, w.q_head, qrow0);
-            tma_load_3d(sm + kOffQ + kHalfBytes, &tmQ, B.q_full, 64, w.q_head, qrow0);
+            const bool is_k = warp == 4;
             const int seq_pages = (si.seq_len + kPageSize - 1) / kPageSize;
             const int32_t* btrow = p.block_table + (int64_t)w.seq * p.bt_stride;
+            if (is_k) {
+                prefetch_tensormap(&tmQ);
+                prefetch_tensormap(&tmK);
+                const int qrow0 = si.q_start + w.tok0;
+                mbar_arrive_expect_tx(B.q_full, kTileBytes);
+                tma_load_3d(sm + kOffQ, &tmQ, B.q_full, 0, w.q_head, qrow0);
+                tma_load_3d(sm + kOffQ + kHalfBytes, &tmQ, B.q_full, 64, w.q_head, qrow0);
+            } else {
+                prefetch_tensormap(&tmV);
+            }
+            const int NSt = is_k ? kNK : kNV;
+            uint64_t* full = is_k ? B.k_full : B.v_full;
+            uint64_t* empty = is_k ? B.k_empty : B.v_empty;
+            uint8_t* base = sm + (is_k ? kOffK : kOffV);
             for (int j = 0; j < n; ++j) {
-                const int st = j % kNS;
-                if (j >= kNS && !wait_or_abort(&B.kv_empty[st], ((j / kNS) - 1) & 1, p.err, abort_flag)) break;
+                const int st = j % NSt;
+                if (j >= NSt && !wait_or_abort(&empty[st], ((j / NSt) - 1) & 1, p.err, abort_flag)) break;
                 int rows[8];
-#pragma unroll
-                for (int pg = 0; pg < 8; ++pg) {
-                    const int lp = j * 8 + pg;
-                    int ph = -1;
-                    if (lp < seq_pages) {
-                        ph = btrow[lp];
-                        if (ph < 0 || ph >= p.num_pages) {
-                            atomicOr(p.err, PKVA_DEVERR_BAD_PAGE);
-                            ph = -1;
-                        }
-                    }
-                    rows[pg] = ph >= 0 ? (ph * p.Hkv + kvh) * kPageSize : -kPageSize;
-                }
-                uint8_t* kdst = sm + kOffK + st * kTileBytes;
-                uint8_t* vdst = sm + kOffV + st * kTileBytes;
-                mbar_arrive_expect_tx(&B.k_full[st], kTileBytes);
-#pragma unroll
-                for (int pg = 0; pg < 8; ++pg)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        tma_load_2d(kdst + h * kHalfBytes + pg * (kPageSize * 128), &tmK, &B.k_full[st], h * 64,
-                                    rows[pg]);
-                mbar_arrive_expect_tx(&B.v_full[st], kTileBytes);
-#pragma unroll
-                for (int pg = 0; pg < 8; ++pg)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        tma_load_2d(vdst + h * kHalfBytes + pg * (kPageSize * 128), &tmV, &B.v_full[st], h * 64,
-                                    rows[pg]);
+                tile_rows(p, btrow, seq_pages, kvh, j, rows);
+                load_tile(base + st * kTileBytes, is_k ? &tmK : &tmV, &full[st], rows);
             }
         }
     } else if (warp == 5) {
@@ -183,7 +199,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
             const uint32_t k_base = smem_addr(sm + kOffK);
             const uint32_t v_base = smem_addr(sm + kOffV);
             auto issue_qk = [&](int j) {
-                const int st = j % kNS;
+                const int st = j % kNK;
                 const uint32_t d = tmem + kColS + (j & 1) * 128;
 #pragma unroll
                 for (int ks = 0; ks < kD / 16; ++ks) {
@@ -193,6 +209,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
                     tc_mma_ss(d, ad, bd, kIdescQK, ks > 0);
                 }
                 tc_commit(&B.s_full[j & 1]);
+                tc_commit(&B.k_empty[st]);
             };
             bool ok = wait_or_abort(B.q_full, 0, p.err, abort_flag) &&
                       wait_or_abort(&B.k_full[0], 0, p.err, abort_flag);
@@ -202,14 +219,14 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
             }
             for (int j = 0; ok && j < n; ++j) {
                 if (j + 1 < n) {
-                    const int st = (j + 1) % kNS;
-                    if (!wait_or_abort(&B.k_full[st], ((j + 1) / kNS) & 1, p.err, abort_flag)) break;
+                    const int kst = (j + 1) % kNK;
+                    if (!wait_or_abort(&B.k_full[kst], ((j + 1) / kNK) & 1, p.err, abort_flag)) break;
                     tc_fence_after();
                     issue_qk(j + 1);
                 }
-                const int st = j % kNS;
+                const int st = j % kNV;
                 if (!wait_or_abort(&B.p_full[j & 1], (j >> 1) & 1, p.err, abort_flag)) break;
-                if (!wait_or_abort(&B.v_full[st], (j / kNS) & 1, p.err, abort_flag)) break;
+                if (!wait_or_abort(&B.v_full[st], (j / kNV) & 1, p.err, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t pcol = tmem + kColP + (j & 1) * 64;
 #pragma unroll
@@ -218,7 +235,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
                     tc_mma_ts(tmem + kColO, pcol + ks * 8, bd, kIdescPV, (j > 0 || ks > 0) ? 1u : 0u);
                 }
                 tc_commit(&B.pv_done[j & 1]);
-                tc_commit(&B.kv_empty[st]);
+                tc_commit(&B.v_empty[st]);
             }
             // every MMA this thread issued must finish before TMEM is released
             tc_commit(B.mma_done);
@@ -258,9 +275,15 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
                 for (int c = 0; c < 128; ++c)
                     if (c > vis) s[c] = -INFINITY;
             }
-            float mx = s[0];
+            // row max as eight independent chains (short dependency depth)
+            float mx8[8];
 #pragma unroll
-            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+            for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+#pragma unroll
+            for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) mx8[i] = fmaxf(mx8[i], mx8[i + 4]);
+            const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3]));
             const float m_tile = mx * p.scale_log2;
             bool need = false;
             float m_new = m_ref;
@@ -296,15 +319,15 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
             }
             const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
             uint32_t pk[64];
-            float lsum_t = 0.f;
+            float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
                 const float p0 = exp2f(fmaf(s[2 * c], p.scale_log2, -ref));
                 const float p1 = exp2f(fmaf(s[2 * c + 1], p.scale_log2, -ref));
-                lsum_t += p0 + p1;
+                ls4[c & 3] += p0 + p1;
                 pk[c] = pack_bf16x2(p0, p1);
             }
-            l_sum += lsum_t;
+            l_sum += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
             // P buffer (j & 1) was last read by PV of tile j-2
             if (j >= 2 &&
                 !__all_sync(0xffffffffu, wait_or_abort(&B.pv_done[j & 1], ((j - 2) >> 1) & 1, p.err, abort_flag))) {
