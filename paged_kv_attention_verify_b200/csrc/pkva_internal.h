@@ -13,6 +13,7 @@ constexpr int kMaxTreeTokens = 64;     // draft tokens per TREE sequence (one 64
 constexpr int kDecodeRowsMax = 16;     // packed (token, head) rows per decode task
 constexpr int kDecodeMaxPages = 1024;  // pages per decode task (block-table slice in smem)
 constexpr int kPrefillTileM = 128;     // query tokens per prefill tile (tcgen05 M)
+constexpr int kPrefillTaskTokens = 256; // query tokens per prefill task (two tiles, ping-pong)
 constexpr int kPrefillTileN = 128;     // keys per prefill KV tile (8 pages)
 constexpr int kPrefillMinTokens = 64;  // causal sequences with at least this many new tokens
                                        // (and head_dim 128) run on the tensor-core prefill kernel
@@ -42,15 +43,17 @@ struct DecodeWork {
 };
 static_assert(sizeof(DecodeWork) == 32, "DecodeWork layout");
 
-// One prefill tile task: 128 query tokens [tok0, tok0 + ntok) of one query head against
-// KV tiles [0, num_kv_tiles) of 128 keys.
+// One prefill task: up to 256 query tokens [tok0, tok0 + ntok) of one query head, as two
+// 128-token tiles; tile 0 needs KV tiles [0, kv_tiles0) of 128 keys, tile 1 [0, kv_tiles1)
+// (0 when the task has at most 128 tokens).
 struct PrefillWork {
     int32_t seq;
     int32_t q_head;
     int32_t tok0;
     int32_t ntok;
-    int32_t num_kv_tiles;
-    int32_t pad0, pad1, pad2;
+    int32_t kv_tiles0;
+    int32_t kv_tiles1;
+    int32_t pad0, pad1;
 };
 static_assert(sizeof(PrefillWork) == 32, "PrefillWork layout");
 

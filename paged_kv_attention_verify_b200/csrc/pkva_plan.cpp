@@ -126,26 +126,29 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
             if (si.mask_kind != PKVA_CAUSAL || si.query_len < kPrefillMinTokens) continue;
             on_prefill[s] = 1;
             const int prefix = si.seq_len - si.query_len;
-            for (int t0 = 0; t0 < si.query_len; t0 += kPrefillTileM) {
-                const int ntok = std::min(kPrefillTileM, si.query_len - t0);
-                // keys up to the last row's own position (causal tile skipping)
-                const int kend = prefix + t0 + ntok;
-                const int tiles = (kend + kPrefillTileN - 1) / kPrefillTileN;
+            for (int t0 = 0; t0 < si.query_len; t0 += kPrefillTaskTokens) {
+                const int ntok = std::min(kPrefillTaskTokens, si.query_len - t0);
+                // each tile needs keys up to its last row's own position (causal tile skipping)
+                const int n0tok = std::min(kPrefillTileM, ntok);
+                const int tiles0 = (prefix + t0 + n0tok + kPrefillTileN - 1) / kPrefillTileN;
+                const int tiles1 =
+                    ntok > kPrefillTileM ? (prefix + t0 + ntok + kPrefillTileN - 1) / kPrefillTileN : 0;
                 for (int h = 0; h < a.Hq; ++h) {
                     PrefillWork pw{};
                     pw.seq = s;
                     pw.q_head = h;
                     pw.tok0 = t0;
                     pw.ntok = ntok;
-                    pw.num_kv_tiles = tiles;
+                    pw.kv_tiles0 = tiles0;
+                    pw.kv_tiles1 = tiles1;
                     p.pwork.push_back(pw);
                 }
             }
         }
-        // heaviest first; equal tiles keep (seq, tile, head) order so that the query heads
+        // heaviest first; equal work keeps (seq, tile, head) order so that the query heads
         // of one GQA group run side by side and share their K/V tiles through L2
         std::stable_sort(p.pwork.begin(), p.pwork.end(), [](const PrefillWork& x, const PrefillWork& y) {
-            return x.num_kv_tiles > y.num_kv_tiles;
+            return x.kv_tiles0 + x.kv_tiles1 > y.kv_tiles0 + y.kv_tiles1;
         });
     }
 
@@ -248,6 +251,7 @@ extern "C" int attn_plan_inspect(int num_seqs, const int32_t* seq_lens, const in
         d.row_count = w.ntok;
         d.key_begin = 0;
         d.key_end = std::min(si.seq_len - si.query_len + w.tok0 + w.ntok, si.seq_len);
+        (void)w.kv_tiles0;
         d.split = -1;
         d.num_splits = 1;
         items[i] = d;

@@ -2,20 +2,24 @@
 // (K-P): S = Q K^T and O += P V are tcgen05.mma BF16 tiles with fp32 accumulators in
 // tensor memory (TMEM).
 //
-// One CTA runs one tile task: 128 query tokens of one query head (tcgen05 M = 128) against
-// the 128-key KV tiles (8 pages, gathered by TMA through the block table) that the causal
-// mask leaves visible; tiles past the last row's own position are never loaded (causal
-// tile skipping), and only tiles that cross the diagonal are masked element by element.
+// One CTA runs one task: up to 256 query tokens of one query head, as two 128-token tiles
+// (tcgen05 M = 128) that share every 128-key KV tile (8 pages, gathered by TMA through the
+// block table). KV tiles past a tile's last row are never loaded (causal tile skipping)
+// and only tiles that cross the diagonal are masked element by element.
 //
-// Warp roles (224 threads):
-//   warps 0-3  softmax: thread r owns row r = TMEM lane r. Reads S, keeps the running
-//              max / sum, writes P (bf16) back to TMEM, rescales O in TMEM only when a
-//              row max moved by more than 2^8 (rare after the first tiles), and writes O.
-//   warp 4     TMA producer of Q and of K tiles (3-stage ring, a stage is freed as soon as
-//              its QK^T is done); warp 6 produces V tiles (2-stage ring, freed after PV).
-//   warp 5     MMA issuer (one thread) and TMEM owner: QK^T of tile j+1 overlaps the
-//              softmax of tile j; PV of tile j reads P straight from TMEM.
-// TMEM (512 columns): S double buffer [0,256), O [256,384), P double buffer [384,512).
+// Warp roles (352 threads):
+//   warps 0-3, 4-7  two softmax warpgroups, one per query tile: thread r owns row r =
+//              TMEM lane r. Each reads S, keeps the running max / sum, writes P (bf16) over
+//              the first half of S in TMEM, rescales O in TMEM only when a row max moved by
+//              more than 2^8, and finally writes its O rows.
+//   warp 8     TMA producer of Q and of K tiles (2-stage ring, freed after both QK^T).
+//   warp 9     MMA issuer (one thread) and TMEM owner. The two tiles ping-pong: while one
+//              warpgroup runs its softmax, the tensor cores run the other tile's PV and
+//              next QK^T. PV takes P straight from TMEM as its A operand.
+//   warp 10    TMA producer of V tiles (2-stage ring, freed after both PV).
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512); P_b lives in
+// columns [0,64) of S_b (bf16 pairs). Tensor-core operations of one issuing thread run in
+// issue order, so the next QK^T into S_b is issued right after the PV that reads P_b.
 //
 // Sources: XY-Serve (arXiv 2412.18106), verdict page — key_machinery (the attention
 // primitive is a matmul-softmax-matmul tile whose QK and SV products overlap the softmax),
@@ -33,26 +37,26 @@ namespace pkva {
 
 namespace {
 
-constexpr int kPThreads = 224;
+constexpr int kPThreads = 352;
 constexpr int kD = 128;
-constexpr int kNK = 3;                                   // K stages (freed when QK^T is done)
-constexpr int kNV = 2;                                   // V stages (freed when PV is done)
+constexpr int kNK = 2;                                   // K stages
+constexpr int kNV = 2;                                   // V stages
 constexpr int kHalfBytes = kPrefillTileM * 128;          // 128 rows x 64 bf16 (one swizzle column)
 constexpr int kTileBytes = 2 * kHalfBytes;               // 128 x 128 bf16
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kTileBytes;
+constexpr int kOffQ = 0;                                 // Q0, Q1
+constexpr int kOffK = kOffQ + 2 * kTileBytes;
 constexpr int kOffV = kOffK + kNK * kTileBytes;
 constexpr int kOffBar = kOffV + kNV * kTileBytes;
-// barriers: q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2], p_full[2],
-// pv_done[2], mma_done
+// q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2], p_full[2], o_ready[2], mma_done
 constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 2 + 2 + 2 + 1;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kOffFlag = kOffTmemSlot + 16;
 constexpr int kSmemBytes = kOffFlag + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1008;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
+constexpr uint32_t kColS = 0, kColO = 256;
 constexpr float kRescaleSlack = 8.f;
+constexpr int kWarpKProd = 8, kWarpMma = 9, kWarpVProd = 10;
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);   // Q, K both K-major
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);    // P from TMEM, V MN-major
@@ -65,7 +69,7 @@ struct Bars {
     uint64_t* v_empty;
     uint64_t* s_full;
     uint64_t* p_full;
-    uint64_t* pv_done;
+    uint64_t* o_ready;
     uint64_t* mma_done;
 };
 
@@ -79,9 +83,19 @@ __device__ __forceinline__ Bars bars_at(uint8_t* sm) {
     r.v_empty = r.v_full + kNV;
     r.s_full = r.v_empty + kNV;
     r.p_full = r.s_full + 2;
-    r.pv_done = r.p_full + 2;
-    r.mma_done = r.pv_done + 2;
+    r.o_ready = r.p_full + 2;
+    r.mma_done = r.o_ready + 2;
     return r;
+}
+
+// Bounded wait that also gives up at once when another role already gave up.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* err, volatile int* abort_flag) {
+    if (*abort_flag) return false;
+    if (!mbar_wait_bounded(bar, parity, err, PKVA_DEVERR_TIMEOUT)) {
+        *abort_flag = 1;
+        return false;
+    }
+    return true;
 }
 
 // Physical cache rows of the 8 pages of KV tile j (row -16 reads as zeros: past the end of
@@ -111,16 +125,6 @@ __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, 
         for (int h = 0; h < 2; ++h) tma_load_2d(dst + h * kHalfBytes + pg * (kPageSize * 128), map, bar, h * 64, rows[pg]);
 }
 
-// Bounded wait that also gives up at once when another role already gave up.
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* err, volatile int* abort_flag) {
-    if (*abort_flag) return false;
-    if (!mbar_wait_bounded(bar, parity, err, PKVA_DEVERR_TIMEOUT)) {
-        *abort_flag = 1;
-        return false;
-    }
-    return true;
-}
-
 __global__ void __launch_bounds__(kPThreads, 1)
 prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
@@ -132,7 +136,8 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
     const Bars B = bars_at(sm);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffTmemSlot);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffFlag);
-    const int n = w.num_kv_tiles;
+    const int n0 = w.kv_tiles0, n1 = w.kv_tiles1;
+    const int nmax = n0 > n1 ? n0 : n1;
     const int kvh = w.q_head / p.G;
     const int prefix = si.seq_len - si.query_len;
 
@@ -149,13 +154,13 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
         for (int b = 0; b < 2; ++b) {
             mbar_init(&B.s_full[b], 1);
             mbar_init(&B.p_full[b], 128);
-            mbar_init(&B.pv_done[b], 1);
+            mbar_init(&B.o_ready[b], 1);
         }
         mbar_init(B.mma_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
@@ -164,19 +169,23 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4 || warp == 6) {
-        // ------------------ TMA producers: warp 4 loads Q and K, warp 6 loads V -------------
+    if (warp == kWarpKProd || warp == kWarpVProd) {
+        // ------------------ TMA producers: warp 8 loads Q and K, warp 10 loads V ------------
         if (lane == 0) {
-            const bool is_k = warp == 4;
+            const bool is_k = warp == kWarpKProd;
             const int seq_pages = (si.seq_len + kPageSize - 1) / kPageSize;
             const int32_t* btrow = p.block_table + (int64_t)w.seq * p.bt_stride;
             if (is_k) {
                 prefetch_tensormap(&tmQ);
                 prefetch_tensormap(&tmK);
                 const int qrow0 = si.q_start + w.tok0;
-                mbar_arrive_expect_tx(B.q_full, kTileBytes);
-                tma_load_3d(sm + kOffQ, &tmQ, B.q_full, 0, w.q_head, qrow0);
-                tma_load_3d(sm + kOffQ + kHalfBytes, &tmQ, B.q_full, 64, w.q_head, qrow0);
+                mbar_arrive_expect_tx(B.q_full, 2 * kTileBytes);
+#pragma unroll
+                for (int b = 0; b < 2; ++b)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_3d(sm + kOffQ + b * kTileBytes + h * kHalfBytes, &tmQ, B.q_full, h * 64,
+                                    w.q_head, qrow0 + b * kPrefillTileM);
             } else {
                 prefetch_tensormap(&tmV);
             }
@@ -184,7 +193,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
             uint64_t* full = is_k ? B.k_full : B.v_full;
             uint64_t* empty = is_k ? B.k_empty : B.v_empty;
             uint8_t* base = sm + (is_k ? kOffK : kOffV);
-            for (int j = 0; j < n; ++j) {
+            for (int j = 0; j < nmax; ++j) {
                 const int st = j % NSt;
                 if (j >= NSt && !wait_or_abort(&empty[st], ((j / NSt) - 1) & 1, p.err, abort_flag)) break;
                 int rows[8];
@@ -192,50 +201,77 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
                 load_tile(base + st * kTileBytes, is_k ? &tmK : &tmV, &full[st], rows);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == kWarpMma) {
         // ------------------------------ MMA issuer -------------------------------------------
         if (lane == 0) {
             const uint32_t q_base = smem_addr(sm + kOffQ);
             const uint32_t k_base = smem_addr(sm + kOffK);
             const uint32_t v_base = smem_addr(sm + kOffV);
-            auto issue_qk = [&](int j) {
+            auto issue_qk = [&](int b, int j) {           // S_b = Q_b K_j^T
                 const int st = j % kNK;
-                const uint32_t d = tmem + kColS + (j & 1) * 128;
+                const uint32_t d = tmem + kColS + b * 128;
 #pragma unroll
                 for (int ks = 0; ks < kD / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * kHalfBytes + (ks & 3) * 32;
-                    const uint64_t ad = smem_desc_sw128(q_base + off, 16, 1024);
+                    const uint64_t ad = smem_desc_sw128(q_base + b * kTileBytes + off, 16, 1024);
                     const uint64_t bd = smem_desc_sw128(k_base + st * kTileBytes + off, 16, 1024);
                     tc_mma_ss(d, ad, bd, kIdescQK, ks > 0);
                 }
-                tc_commit(&B.s_full[j & 1]);
-                tc_commit(&B.k_empty[st]);
+                tc_commit(&B.s_full[b]);
+            };
+            auto issue_pv = [&](int b, int j) {           // O_b += P_b V_j
+                const int st = j % kNV;
+                const uint32_t pcol = tmem + kColS + b * 128;
+#pragma unroll
+                for (int ks = 0; ks < kPrefillTileN / 16; ++ks) {
+                    const uint64_t bd = smem_desc_sw128(v_base + st * kTileBytes + ks * 2048, kHalfBytes, 1024);
+                    tc_mma_ts(tmem + kColO + b * 128, pcol + ks * 8, bd, kIdescPV, (j > 0 || ks > 0) ? 1u : 0u);
+                }
             };
             bool ok = wait_or_abort(B.q_full, 0, p.err, abort_flag) &&
                       wait_or_abort(&B.k_full[0], 0, p.err, abort_flag);
             if (ok) {
                 tc_fence_after();
-                issue_qk(0);
+                if (n0 > 0) issue_qk(0, 0);
+                if (n1 > 0) issue_qk(1, 0);
+                tc_commit(&B.k_empty[0]);
             }
-            for (int j = 0; ok && j < n; ++j) {
-                if (j + 1 < n) {
-                    const int kst = (j + 1) % kNK;
-                    if (!wait_or_abort(&B.k_full[kst], ((j + 1) / kNK) & 1, p.err, abort_flag)) break;
-                    tc_fence_after();
-                    issue_qk(j + 1);
-                }
-                const int st = j % kNV;
-                if (!wait_or_abort(&B.p_full[j & 1], (j >> 1) & 1, p.err, abort_flag)) break;
-                if (!wait_or_abort(&B.v_full[st], (j / kNV) & 1, p.err, abort_flag)) break;
-                tc_fence_after();
-                const uint32_t pcol = tmem + kColP + (j & 1) * 64;
+            for (int j = 0; ok && j < nmax; ++j) {
+                const int vst = j % kNV;
+                bool vwaited = false, kwaited = false;
 #pragma unroll
-                for (int ks = 0; ks < kPrefillTileN / 16; ++ks) {
-                    const uint64_t bd = smem_desc_sw128(v_base + st * kTileBytes + ks * 2048, kHalfBytes, 1024);
-                    tc_mma_ts(tmem + kColO, pcol + ks * 8, bd, kIdescPV, (j > 0 || ks > 0) ? 1u : 0u);
+                for (int b = 0; b < 2; ++b) {
+                    const int nb = b ? n1 : n0;
+                    if (j >= nb) continue;
+                    if (!wait_or_abort(&B.p_full[b], j & 1, p.err, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!vwaited) {
+                        if (!wait_or_abort(&B.v_full[vst], (j / kNV) & 1, p.err, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        vwaited = true;
+                    }
+                    tc_fence_after();
+                    issue_pv(b, j);
+                    if (j == nb - 1) tc_commit(&B.o_ready[b]);
+                    if (j + 1 < nb) {
+                        if (!kwaited) {
+                            if (!wait_or_abort(&B.k_full[(j + 1) % kNK], ((j + 1) / kNK) & 1, p.err, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            kwaited = true;
+                            tc_fence_after();
+                        }
+                        issue_qk(b, j + 1);
+                    }
                 }
-                tc_commit(&B.pv_done[j & 1]);
-                tc_commit(&B.v_empty[st]);
+                if (!ok) break;
+                tc_commit(&B.v_empty[vst]);
+                if (kwaited) tc_commit(&B.k_empty[(j + 1) % kNK]);
             }
             // every MMA this thread issued must finish before TMEM is released
             tc_commit(B.mma_done);
@@ -243,48 +279,46 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
         }
     } else {
         // ------------------------------ softmax (rows) ---------------------------------------
-        const int r = tid;                                   // row = TMEM lane
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const int tok = w.tok0 + r;
-        const bool real_row = r < w.ntok;
-        const int lim = real_row ? prefix + tok : 0x7fffffff;   // last visible key of this row
-        const int lim0 = prefix + w.tok0;                        // row 0's limit
+        const int b = warp >> 2;                             // query tile of this warpgroup
+        const int r = tid & 127;                             // row = TMEM lane
+        const int nb = b ? n1 : n0;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t s_addr = tmem + lane_off + kColS + b * 128;
+        const uint32_t o_addr = tmem + lane_off + kColO + b * 128;
+        const int row_in_task = b * kPrefillTileM + r;
+        const int tok = w.tok0 + row_in_task;
+        const bool real_row = row_in_task < w.ntok;
+        const int lim = real_row ? prefix + tok : 0x7fffffff;        // last visible key of this row
+        const int lim_first = prefix + w.tok0 + b * kPrefillTileM;    // the tile's first row
         float m_ref = -INFINITY, l_sum = 0.f;
         bool alive = true;
         // every break below is taken by the whole warp (tcgen05.ld/st are warp-collective)
-        for (int j = 0; j < n; ++j) {
-            if (!__all_sync(0xffffffffu, wait_or_abort(&B.s_full[j & 1], (j >> 1) & 1, p.err, abort_flag))) {
+        for (int j = 0; j < nb; ++j) {
+            if (!__all_sync(0xffffffffu, wait_or_abort(&B.s_full[b], j & 1, p.err, abort_flag))) {
                 alive = false;
                 break;
             }
             tc_fence_after();
             uint32_t sr[128];
-            {
-                const uint32_t sa = tmem + lane_off + kColS + (j & 1) * 128;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(sa + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-                tmem_wait_ld();
-            }
-            float s[128];
-#pragma unroll
-            for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
+            for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+            tmem_wait_ld();
             const int kb = j * kPrefillTileN;
-            if (kb + kPrefillTileN - 1 > lim0) {            // tile crosses the diagonal
-                const int vis = lim - kb;                      // columns <= vis are visible
+            if (kb + kPrefillTileN - 1 > lim_first) {          // tile crosses the diagonal
+                const int vis = lim - kb;                          // columns <= vis are visible
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
-                    if (c > vis) s[c] = -INFINITY;
+                    if (c > vis) sr[c] = __float_as_uint(-INFINITY);
             }
             // row max as eight independent chains (short dependency depth)
             float mx8[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+            for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(sr[i]);
 #pragma unroll
-            for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+            for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
 #pragma unroll
             for (int i = 0; i < 4; ++i) mx8[i] = fmaxf(mx8[i], mx8[i + 4]);
-            const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3]));
-            const float m_tile = mx * p.scale_log2;
+            const float m_tile = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])) * p.scale_log2;
             bool need = false;
             float m_new = m_ref;
             if (j == 0) {
@@ -293,65 +327,50 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
                 need = m_tile > m_ref + kRescaleSlack;
                 m_new = fmaxf(m_ref, m_tile);
             }
+            const float alpha = need ? exp2f(m_ref - m_new) : 1.f;
+            if (need) {
+                m_ref = m_new;
+                l_sum *= alpha;
+            }
+            const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
+            float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+            // P in place: pair c goes to word c (already consumed), then out to S_b[0, 64)
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                const float p0 = exp2f(fmaf(__uint_as_float(sr[2 * c]), p.scale_log2, -ref));
+                const float p1 = exp2f(fmaf(__uint_as_float(sr[2 * c + 1]), p.scale_log2, -ref));
+                ls4[c & 3] += p0 + p1;
+                sr[c] = pack_bf16x2(p0, p1);
+            }
+            l_sum += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+            tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
             if (__any_sync(0xffffffffu, need)) {
-                // rescale this warp's rows of O (needs PV of tile j-1 to have landed)
-                if (!__all_sync(0xffffffffu,
-                                wait_or_abort(&B.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p.err, abort_flag))) {
-                    alive = false;
-                    break;
-                }
-                tc_fence_after();
-                const float alpha = need ? exp2f(m_ref - m_new) : 1.f;
-                if (need) {
-                    m_ref = m_new;
-                    l_sum *= alpha;
-                }
-                const uint32_t oa = tmem + lane_off + kColO;
+                // rescale O_b (done with S, so its registers are free). O_b is complete for
+                // tile j-1: S_b of tile j was committed after that PV was issued.
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t ov[32];
-                    tmem_ld32(oa + c * 32, ov);
+                    tmem_ld32(o_addr + c * 32, ov);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-                    tmem_st32(oa + c * 32, ov);
+                    tmem_st32(o_addr + c * 32, ov);
                 }
             }
-            const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
-            uint32_t pk[64];
-            float ls4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                const float p0 = exp2f(fmaf(s[2 * c], p.scale_log2, -ref));
-                const float p1 = exp2f(fmaf(s[2 * c + 1], p.scale_log2, -ref));
-                ls4[c & 3] += p0 + p1;
-                pk[c] = pack_bf16x2(p0, p1);
-            }
-            l_sum += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
-            // P buffer (j & 1) was last read by PV of tile j-2
-            if (j >= 2 &&
-                !__all_sync(0xffffffffu, wait_or_abort(&B.pv_done[j & 1], ((j - 2) >> 1) & 1, p.err, abort_flag))) {
-                alive = false;
-                break;
-            }
-            const uint32_t pa = tmem + lane_off + kColP + (j & 1) * 64;
-            tmem_st32(pa, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-            tmem_st32(pa + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&B.p_full[j & 1]);
+            mbar_arrive(&B.p_full[b]);
         }
         // ---- epilogue: O / l -> bf16 rows --------------------------------------------------
-        if (alive && __all_sync(0xffffffffu, wait_or_abort(&B.pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, p.err,
-                                                          abort_flag))) {
+        if (nb > 0 && alive && __all_sync(0xffffffffu, wait_or_abort(&B.o_ready[b], 0, p.err, abort_flag))) {
             tc_fence_after();
             const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-            const uint32_t oa = tmem + lane_off + kColO;
             __nv_bfloat16* dst = p.out + ((int64_t)(si.q_start + tok) * p.Hq + w.q_head) * kD;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t ov[32];
-                tmem_ld32(oa + c * 32, ov);
+                tmem_ld32(o_addr + c * 32, ov);
                 tmem_wait_ld();
                 if (real_row) {
 #pragma unroll
@@ -371,7 +390,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 5) tmem_dealloc(tmem, kTmemCols);
+    if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace
