@@ -57,6 +57,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;
 constexpr float kRescaleSlack = 8.f;
 constexpr int kWarpKProd = 8, kWarpMma = 9, kWarpVProd = 10;
+constexpr bool kSpinOnS = true;    // softmax warps poll S without suspending
 
 // 2^x on the FMA pipe: 2^x = 2^n * p(f), n = round(x), f = x - n in [-1/2, 1/2], p the cubic
 // interpolating 2^f at the Chebyshev nodes of [-1/2, 1/2] (max relative error 1.0e-4, below
@@ -114,6 +115,16 @@ __device__ __forceinline__ Bars bars_at(uint8_t* sm) {
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* err, volatile int* abort_flag) {
     if (*abort_flag) return false;
     if (!mbar_wait_bounded(bar, parity, err, PKVA_DEVERR_TIMEOUT)) {
+        *abort_flag = 1;
+        return false;
+    }
+    return true;
+}
+
+// As wait_or_abort, polling without suspending (for waits on the critical path).
+__device__ __forceinline__ bool spin_or_abort(uint64_t* bar, uint32_t parity, int* err, volatile int* abort_flag) {
+    if (*abort_flag) return false;
+    if (!mbar_spin_bounded(bar, parity, err, PKVA_DEVERR_TIMEOUT)) {
         *abort_flag = 1;
         return false;
     }
@@ -265,16 +276,16 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
                 for (int b = 0; b < 2; ++b) {
                     const int nb = b ? n1 : n0;
                     if (j >= nb) continue;
-                    if (!wait_or_abort(&B.p_full[b], j & 1, p.err, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
                     if (!vwaited) {
                         if (!wait_or_abort(&B.v_full[vst], (j / kNV) & 1, p.err, abort_flag)) {
                             ok = false;
                             break;
                         }
                         vwaited = true;
+                    }
+                    if (!spin_or_abort(&B.p_full[b], j & 1, p.err, abort_flag)) {   // critical path
+                        ok = false;
+                        break;
                     }
                     tc_fence_after();
                     issue_pv(b, j);
@@ -316,7 +327,8 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
         bool alive = true;
         // every break below is taken by the whole warp (tcgen05.ld/st are warp-collective)
         for (int j = 0; j < nb; ++j) {
-            if (!__all_sync(0xffffffffu, wait_or_abort(&B.s_full[b], j & 1, p.err, abort_flag))) {
+            if (!__all_sync(0xffffffffu, kSpinOnS ? spin_or_abort(&B.s_full[b], j & 1, p.err, abort_flag)
+                                                  : wait_or_abort(&B.s_full[b], j & 1, p.err, abort_flag))) {
                 alive = false;
                 break;
             }
