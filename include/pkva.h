@@ -183,8 +183,8 @@ PKVA_API int attn_run_static(int num_seqs, const int32_t* seq_lens, const int32_
 /* Summary of a plan's decomposition (for logging and tests). */
 typedef struct pkva_plan_info {
     int32_t num_seqs;
-    int32_t num_decode_items;    /* CUDA-core decode/verify tile tasks (one CTA each)      */
-    int32_t num_prefill_items;   /* tensor-core prefill tile tasks                          */
+    int32_t num_decode_items;    /* decode/verify tile tasks (one block each)              */
+    int32_t num_prefill_items;   /* prefill tile tasks (one block each, 256 tokens, 1 head)  */
     int32_t num_split_units;     /* (seq, kv head, row chunk) units split over several CTAs */
     int32_t num_partial_slots;   /* split-KV partial results held in plan scratch           */
     int32_t decode_rows;         /* rows per decode task the launch is compiled for         */
@@ -199,9 +199,12 @@ PKVA_API int attn_plan_get_info(pkva_plan_t plan, pkva_plan_info* info);
 typedef struct pkva_work_desc {
     int32_t kind;        /* 0 = decode/verify task, 1 = prefill task                      */
     int32_t seq;         /* sequence index                                                 */
-    int32_t kv_head;     /* KV head; the task covers query heads of this head's group      */
-    int32_t row_begin;   /* first packed row (row = token * group + head-in-group)         */
-    int32_t row_count;   /* packed rows in the task                                        */
+    int32_t kv_head;     /* KV head whose keys and values the task reads                   */
+    int32_t q_head;      /* prefill: the one query head; decode/verify: -1 (all heads of   */
+                         /* the KV head's group, as packed rows)                           */
+    int32_t row_begin;   /* decode/verify: first packed row (token * group + head-in-group);*/
+                         /* prefill: first query token                                     */
+    int32_t row_count;   /* packed rows (decode/verify) or query tokens (prefill)          */
     int32_t key_begin;   /* first key position covered                                     */
     int32_t key_end;     /* one past the last key position covered                          */
     int32_t split;       /* split index within its unit, -1 if the unit is not split       */
@@ -210,7 +213,9 @@ typedef struct pkva_work_desc {
 
 /*
  * attn_plan_inspect — run the planner on the host only (no device, nothing allocated on
- * it) and return its tile tasks in launch order. Arguments as attn_plan, plus:
+ * it) and return its tile tasks grouped by kind: prefill tasks, then decode/verify tasks,
+ * each in its launch order (heaviest first; the single launch interleaves the two lists in
+ * proportion, three decode/verify tasks to a block). Arguments as attn_plan, plus:
  *   num_sms, ctas_per_sm   the machine the plan should balance for;
  *   items, max_items       output array (may be NULL to query the count);
  *   num_items              receives the number of tasks.

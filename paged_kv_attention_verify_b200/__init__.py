@@ -51,7 +51,7 @@ class PlanInfo(ctypes.Structure):
 
 class WorkDesc(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("seq", ctypes.c_int32), ("kv_head", ctypes.c_int32),
-                ("row_begin", ctypes.c_int32), ("row_count", ctypes.c_int32),
+                ("q_head", ctypes.c_int32), ("row_begin", ctypes.c_int32), ("row_count", ctypes.c_int32),
                 ("key_begin", ctypes.c_int32), ("key_end", ctypes.c_int32),
                 ("split", ctypes.c_int32), ("num_splits", ctypes.c_int32)]
 

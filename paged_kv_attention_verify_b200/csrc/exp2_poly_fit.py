@@ -5,7 +5,7 @@ Method: range reduction 2^x = 2^n * 2^f with n = round(x), f = x - n in [-1/2, 1
 degree-3 polynomial that interpolates 2^f at the four Chebyshev nodes of [-1/2, 1/2]
 (Chebyshev interpolation, which is within a small factor of the minimax polynomial). Run
 this file to print the coefficients and the worst relative error on a fine grid; the
-kernel's constants (kExp2C0..kExp2C3 in pkva_prefill.cu) are its output, and the CPU test
+kernel's constants (kExp2C0..kExp2C3 in pkva_prefill_body.cuh) are its output, and the CPU test
 tests/test_exp2_poly.py re-derives them and checks the error bound.
 """
 import numpy as np

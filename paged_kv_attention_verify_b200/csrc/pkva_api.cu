@@ -104,8 +104,8 @@ struct pkva_plan {
     pkva::SeqInfo* d_seqs = nullptr;
     pkva::DecodeWork* d_dwork = nullptr;
     pkva::PrefillWork* d_pwork = nullptr;
-    cudaStream_t side = nullptr;            // prefill tasks run here, overlapping decode tasks
-    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+    int32_t* d_order = nullptr;             // unified launch order
+    int32_t* d_order_prefill = nullptr;     // prefill tasks only (comparison mode)
     CUtensorMap tmQ;
     const void* tm_q = nullptr;
     pkva::SplitUnit* d_units = nullptr;
@@ -129,9 +129,8 @@ static void free_plan(pkva_plan* p) {
     cudaFree(p->d_seqs);
     cudaFree(p->d_dwork);
     cudaFree(p->d_pwork);
-    if (p->side) cudaStreamDestroy(p->side);
-    if (p->ev_fork) cudaEventDestroy(p->ev_fork);
-    if (p->ev_join) cudaEventDestroy(p->ev_join);
+    cudaFree(p->d_order);
+    cudaFree(p->d_order_prefill);
     cudaFree(p->d_units);
     cudaFree(p->d_anc);
     cudaFree(p->d_part_o);
@@ -190,17 +189,21 @@ extern "C" int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq
     p->block_table = block_table;
     p->decode_mma = decode_body_is_mma();
 
-    // the decode kernel's residency decides how many CTA slots the planner balances for
+    // Decode tasks are balanced over slots of four page-streaming warps: the unified kernel
+    // runs one block per SM holding three decode tasks, the stand-alone CUDA-core kernel its
+    // own residency.
     {
         HostPlan probe;
         std::string err;
         build_host_plan(a, &probe, &err);
-        p->decode_ctas = decode_ctas_per_sm(head_dim, probe.decode_rows, p->decode_mma);
-        if (p->decode_ctas < 1) {
+        const int blocks = p->decode_mma ? attn_ctas_per_sm(head_dim, probe.decode_rows)
+                                         : decode_ctas_per_sm(head_dim, probe.decode_rows, false);
+        if (blocks < 1) {
             free_plan(p);
-            set_last_error("attn_plan: decode kernel cannot be resident (shared memory)");
+            set_last_error("attn_plan: attention kernel cannot be resident (shared memory)");
             return PKVA_ECUDA;
         }
+        p->decode_ctas = p->decode_mma ? kDecTasksPerBlock * blocks : blocks;
     }
     a.num_sms = sms;
     a.ctas_per_sm = p->decode_ctas;
@@ -211,8 +214,6 @@ extern "C" int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq
         set_last_error("attn_plan: " + err);
         return rc;
     }
-    // the kernel set for the final row count may differ from the probe's; re-query
-    p->decode_ctas = decode_ctas_per_sm(head_dim, p->hp.decode_rows, p->decode_mma);
 
     const HostPlan& hp = p->hp;
 #define PKVA_TRY(x)              \
@@ -226,14 +227,11 @@ extern "C" int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq
     PKVA_TRY(upload(&p->d_seqs, hp.seqs, &p->scratch_bytes));
     PKVA_TRY(upload(&p->d_dwork, hp.dwork, &p->scratch_bytes));
     PKVA_TRY(upload(&p->d_pwork, hp.pwork, &p->scratch_bytes));
-    if (!hp.pwork.empty() && !hp.dwork.empty()) {
-        cudaError_t e = cudaStreamCreateWithFlags(&p->side, cudaStreamNonBlocking);
-        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->ev_fork, cudaEventDisableTiming);
-        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->ev_join, cudaEventDisableTiming);
-        if (e != cudaSuccess) {
-            free_plan(p);
-            return cuda_fail(e, "attn_plan: side stream");
-        }
+    PKVA_TRY(upload(&p->d_order, hp.order, &p->scratch_bytes));
+    {
+        std::vector<int32_t> po(hp.pwork.size());
+        for (size_t i = 0; i < po.size(); ++i) po[i] = (int32_t)i;
+        PKVA_TRY(upload(&p->d_order_prefill, po, &p->scratch_bytes));
     }
     PKVA_TRY(upload(&p->d_units, hp.units, &p->scratch_bytes));
     PKVA_TRY(upload(&p->d_anc, hp.anc, &p->scratch_bytes));
@@ -327,29 +325,18 @@ extern "C" int attn_run(pkva_plan_t plan, const void* q, const void* k_cache, co
         }
         plan->tm_q = q;
     }
-    // prefill tiles on a side stream that forks from and joins back into `stream`
-    cudaStream_t pst = st;
-    if (!hp.pwork.empty() && plan->side) {
-        PKVA_CUDA(cudaEventRecord(plan->ev_fork, st), "attn_run: fork");
-        PKVA_CUDA(cudaStreamWaitEvent(plan->side, plan->ev_fork, 0), "attn_run: fork");
-        pst = plan->side;
-    }
-    if (!hp.pwork.empty()) {
-        PrefillParams pp;
-        pp.out = static_cast<__nv_bfloat16*>(out);
-        pp.block_table = plan->block_table;
-        pp.seqs = plan->d_seqs;
-        pp.work = plan->d_pwork;
-        pp.err = plan->d_err;
-        pp.bt_stride = hp.bt_stride;
-        pp.Hq = hp.Hq;
-        pp.Hkv = hp.Hkv;
-        pp.G = hp.G;
-        pp.num_pages = hp.num_pages;
-        pp.scale_log2 = hp.scale * 1.4426950408889634f;
-        cudaError_t e = launch_prefill(pp, (int)hp.pwork.size(), plan->tmQ, plan->tmK, plan->tmV, pst);
-        if (e != cudaSuccess) return cuda_fail(e, "attn_run: prefill launch");
-    }
+    PrefillParams pp;
+    pp.out = static_cast<__nv_bfloat16*>(out);
+    pp.block_table = plan->block_table;
+    pp.seqs = plan->d_seqs;
+    pp.work = plan->d_pwork;
+    pp.err = plan->d_err;
+    pp.bt_stride = hp.bt_stride;
+    pp.Hq = hp.Hq;
+    pp.Hkv = hp.Hkv;
+    pp.G = hp.G;
+    pp.num_pages = hp.num_pages;
+    pp.scale_log2 = hp.scale * 1.4426950408889634f;
     DecodeParams dp;
     dp.q = static_cast<const __nv_bfloat16*>(q);
     dp.out = static_cast<__nv_bfloat16*>(out);
@@ -367,14 +354,29 @@ extern "C" int attn_run(pkva_plan_t plan, const void* q, const void* k_cache, co
     dp.Hkv = hp.Hkv;
     dp.G = hp.G;
     dp.num_pages = hp.num_pages;
-    dp.scale_log2 = hp.scale * 1.4426950408889634f;
-    cudaError_t e = launch_decode(dp, (int)hp.dwork.size(), hp.D, hp.decode_rows, plan->decode_mma, plan->tmK,
-                                  plan->tmV, st);
-    if (e != cudaSuccess) return cuda_fail(e, "attn_run: decode launch");
-    if (pst != st) {
-        PKVA_CUDA(cudaEventRecord(plan->ev_join, pst), "attn_run: join");
-        PKVA_CUDA(cudaStreamWaitEvent(st, plan->ev_join, 0), "attn_run: join");
+    dp.scale_log2 = pp.scale_log2;
+    AttnParams ap;
+    ap.pre = pp;
+    ap.dec = dp;
+    const bool has_prefill = !hp.pwork.empty();
+    cudaError_t e;
+    if (plan->decode_mma) {
+        // the whole batch in one launch
+        ap.order = plan->d_order;
+        ap.num_blocks = (int32_t)hp.order.size();
+        ap.num_decode = (int32_t)hp.dwork.size();
+        e = launch_attn(ap, hp.D, hp.decode_rows, has_prefill, plan->tmQ, plan->tmK, plan->tmV, st);
+    } else {
+        // comparison mode: decode tasks on the CUDA-core kernel, prefill tasks after them
+        e = launch_decode(dp, (int)hp.dwork.size(), hp.D, hp.decode_rows, false, plan->tmK, plan->tmV, st);
+        if (e == cudaSuccess && has_prefill) {
+            ap.order = plan->d_order_prefill;
+            ap.num_blocks = (int32_t)hp.pwork.size();
+            ap.num_decode = 0;
+            e = launch_attn(ap, hp.D, hp.decode_rows, has_prefill, plan->tmQ, plan->tmK, plan->tmV, st);
+        }
     }
+    if (e != cudaSuccess) return cuda_fail(e, "attn_run: launch");
     return PKVA_OK;
 }
 

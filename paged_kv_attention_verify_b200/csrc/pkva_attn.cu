@@ -1,0 +1,111 @@
+// One launch for a whole mixed prefill / decode / verify batch.
+//
+// The planner's task list is one grid: prefill tasks first (heaviest first), then the
+// decode/verify tasks (heaviest first). A block whose index falls in the prefill range
+// runs the tensor-core prefill task (TMEM, tcgen05.mma, four warp roles); any other block
+// runs three decode/verify tasks side by side, each on four page-streaming warps with its own
+// third of shared memory and its own named barrier (warp-level tensor-core page body).
+// Both kinds use the same 352-thread block and the same dynamic shared memory (one block
+// per SM), so the hardware block scheduler deals the mixed work out as one
+// longest-task-first schedule and decode blocks fill the SMs as prefill blocks finish.
+//
+// XY-Serve (arXiv 2412.18106), verdict page — forward_implications[2] (one attention kernel
+// for prefill, decode and verify rows, the visible keys chosen row by row) and
+// core_discovery (a budgeted mixed batch decomposed into tile tasks, reordered for balance).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "pkva_decode_body.cuh"
+#include "pkva_prefill_body.cuh"
+
+namespace pkva {
+
+namespace {
+
+constexpr int kAttnThreads = 384;                 // prefill uses 352; decode 3 x 128
+constexpr int kDecWarps = 4;                      // page-streaming warps per decode task
+static_assert(kAttnThreads >= pre::kPThreads, "block too small for a prefill task");
+static_assert(kAttnThreads == kDecTasksPerBlock * 128, "one 128-thread group per decode task");
+
+template <int D>
+struct AttnNS {
+    static constexpr int value = D == 64 ? 4 : 2;  // decode stages per warp
+};
+
+template <int D, int NT>
+struct AttnSmem {
+    using DC = dec::DecodeCfg<D, NT * 8, false, kDecWarps, AttnNS<D>::value>;
+    static constexpr int GROUP_BYTES = (DC::BYTES + 1023) / 1024 * 1024;    // one decode task
+    static constexpr int DEC_BYTES = kDecTasksPerBlock * GROUP_BYTES;
+    static constexpr int BYTES = (D == 128 && pre::kSmemBytes > DEC_BYTES) ? pre::kSmemBytes : DEC_BYTES;
+    static constexpr int ALLOC = BYTES + 1008;    // room to align to 1024
+    static_assert(ALLOC <= 227 * 1024, "shared memory");
+};
+
+template <int D, int NT>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+            const __grid_constant__ CUtensorMap tmV) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int e = p.order[blockIdx.x];
+    if constexpr (D == 128) {
+        if (e >= 0) {
+            pre::prefill_task(p.pre, e, tmQ, tmK, tmV, sm);
+            return;
+        }
+    }
+    if (e >= 0) return;                          // (never planned: prefill needs head_dim 128)
+    // decode block: warps 4g .. 4g+3 run task g of the block's three
+    const int g = threadIdx.x >> 7;
+    const int task = (-1 - e) * kDecTasksPerBlock + g;
+    if (task >= p.num_decode) return;
+    const dec::Group grp{(int)threadIdx.x & 127, 128, 1 + g};
+    dec::decode_mma_task<D, NT, kDecWarps, AttnNS<D>::value>(grp, p.dec, task, tmK, tmV,
+                                                             sm + g * AttnSmem<D, NT>::GROUP_BYTES);
+}
+
+template <int D, int NT>
+cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                     const CUtensorMap& tmV, cudaStream_t stream) {
+    using S = AttnSmem<D, NT>;
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::ALLOC);
+    if (e != cudaSuccess) return e;
+    const int grid = p.num_blocks;
+    if (grid == 0) return cudaSuccess;
+    attn_kernel<D, NT><<<grid, kAttnThreads, S::ALLOC, stream>>>(p, tmQ, tmK, tmV);
+    return cudaGetLastError();
+}
+
+template <int D, int NT>
+int ctas_t() {
+    using S = AttnSmem<D, NT>;
+    int n = 0;
+    if (cudaFuncSetAttribute(attn_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::ALLOC) !=
+        cudaSuccess)
+        return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_kernel<D, NT>, kAttnThreads, S::ALLOC) !=
+        cudaSuccess)
+        return 0;
+    return n;
+}
+
+}  // namespace
+
+int attn_ctas_per_sm(int D, int rows) {
+    if (D == 64) return rows <= 8 ? ctas_t<64, 1>() : ctas_t<64, 2>();
+    if (D == 128) return rows <= 8 ? ctas_t<128, 1>() : ctas_t<128, 2>();
+    return 0;
+}
+
+cudaError_t launch_attn(const AttnParams& p, int D, int rows, bool has_prefill, const CUtensorMap& tmQ,
+                        const CUtensorMap& tmK, const CUtensorMap& tmV, cudaStream_t stream) {
+    if (D == 64) {
+        if (has_prefill) return cudaErrorInvalidValue;   // prefill tasks need head_dim 128
+        return rows <= 8 ? launch_t<64, 1>(p, tmQ, tmK, tmV, stream) : launch_t<64, 2>(p, tmQ, tmK, tmV, stream);
+    }
+    return rows <= 8 ? launch_t<128, 1>(p, tmQ, tmK, tmV, stream) : launch_t<128, 2>(p, tmQ, tmK, tmV, stream);
+}
+
+}  // namespace pkva

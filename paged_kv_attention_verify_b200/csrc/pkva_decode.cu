@@ -29,698 +29,38 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
-#include "pkva.h"
-#include "pkva_kernels.h"
-#include "pkva_ptx.cuh"
+
+#include "pkva_decode_body.cuh"
 
 namespace pkva {
 
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kThreads = kWarps * 32;
-constexpr int kBoxBytes = kPageSize * 128;     // one TMA box: 16 rows x 64 bf16
-constexpr int kBtSlice = kDecodeMaxPages;      // block-table entries staged per task
-constexpr float kRescaleSlack = 8.f;           // log2 units a stale row max may lag (mma body)
-
-constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
-
-// Shared-memory map of one task. NR = rows the launch is compiled for; QF = whether the
-// CUDA-core body's staged Q and P buffers are present.
-template <int D, int NR, bool QF>
-struct DecodeCfg {
-    static constexpr int NS = (D == 64) ? 4 : (NR <= 8 ? 3 : 2);    // stages per warp
-    static constexpr int PAGE_BYTES = kPageSize * D * 2;
-    static constexpr int STAGE_BYTES = 2 * PAGE_BYTES;              // K page + V page
-    static constexpr int HALF = D / 2;                              // columns per lane half
-    static constexpr int QROW = D + 8;                              // floats per staged Q row
-    static constexpr int OPL = D / 32;                              // output columns per lane
-    static constexpr int RING = kWarps * NS * STAGE_BYTES;
-    static constexpr int OFF_Q = RING;
-    static constexpr int OFF_P = OFF_Q + (QF ? NR * QROW * 4 : 0);
-    static constexpr int OFF_BT = OFF_P + (QF ? kWarps * kPageSize * NR * 4 : 0);
-    static constexpr int OFF_LIM = OFF_BT + kBtSlice * 4;
-    static constexpr int OFF_ANC = align_up(OFF_LIM + NR * 4, 8);
-    static constexpr int OFF_OUT = OFF_ANC + NR * 8;
-    static constexpr int OFF_BAR = align_up(OFF_OUT + NR * 4, 8);
-    static constexpr int OFF_FLAG = OFF_BAR + kWarps * NS * 8;
-    static constexpr int BYTES = OFF_FLAG + 16;
-    static constexpr int ALLOC = BYTES + 1008;                     // room to align to 1024
-    static_assert(kWarps * NR * (D + 2) * 4 <= RING, "combine buffers must fit in the ring");
-    static_assert(D == 64 || D == 128, "head_dim");
+// Stand-alone decode kernels: four page-streaming warps per CTA (128 threads).
+constexpr int kDecThreads = 128;
+template <int D, int NR>
+struct StandaloneNS {
+    static constexpr int value = (D == 64) ? 4 : (NR <= 8 ? 3 : 2);
 };
 
-__device__ __forceinline__ int q_row_index(const DecodeParams& p, const SeqInfo& si, const DecodeWork& w,
-                                           int r) {
-    const int rr = w.row_begin + r;
-    const int t = rr / p.G;
-    const int g = rr - t * p.G;
-    return (si.q_start + t) * p.Hq + w.kv_head * p.G + g;
-}
-
-// Per-task set-up shared by both bodies: barriers, block-table slice, row records.
-template <int NR, int NS>
-__device__ __forceinline__ void task_setup(const DecodeParams& p, const DecodeWork& w, const SeqInfo& si,
-                                           int* bts, int* rlim, uint64_t* ranc, int* rout, uint64_t* bars,
-                                           int* flag, const CUtensorMap* tmK, const CUtensorMap* tmV) {
-    const int tid = threadIdx.x;
-    const int R = w.row_count;
-    const int npg = w.page_end - w.page_begin;
-    const int prefix = si.seq_len - si.query_len;
-    if (tid == 0) {
-        for (int i = 0; i < kWarps * NS; ++i) mbar_init(&bars[i], 1);
-        fence_mbar_init();
-        flag[0] = 0;
-        flag[1] = 0;
-        prefetch_tensormap(tmK);
-        prefetch_tensormap(tmV);
-    }
-    // block-table slice of this task; an entry out of range is flagged and its page is
-    // loaded from a fully out-of-bounds box, which TMA fills with zeros
-    const int32_t* btrow = p.block_table + (int64_t)w.seq * p.bt_stride + w.page_begin;
-    for (int i = tid; i < npg; i += kThreads) {
-        const int ph = btrow[i];
-        const bool bad = ph < 0 || ph >= p.num_pages;
-        if (bad) atomicOr(p.err, PKVA_DEVERR_BAD_PAGE);
-        bts[i] = bad ? -1 : ph;
-    }
-    // per-row records: output row, causal limit, tree ancestor mask
-    if (tid < NR) {
-        const int r = tid;
-        if (r < R) {
-            const int t = (w.row_begin + r) / p.G;
-            rout[r] = q_row_index(p, si, w, r);
-            if (si.mask_kind == PKVA_CAUSAL) {
-                rlim[r] = prefix + t;
-                ranc[r] = 0ull;
-            } else {
-                rlim[r] = prefix - 1;
-                ranc[r] = p.anc[si.anc_off + t];
-            }
-        } else {
-            rout[r] = -1;
-            rlim[r] = 0x7fffffff;
-            ranc[r] = 0ull;
-        }
-    }
-}
-
-// Load page #i of this warp's stream (lane 0 only).
-template <int D, int NS, int STAGE_BYTES, int PAGE_BYTES>
-__device__ __forceinline__ void issue_page(const DecodeParams& p, const DecodeWork& w, const int* bts,
-                                           uint8_t* ring, uint64_t* bar, int warp, int i,
-                                           const CUtensorMap* tmK, const CUtensorMap* tmV) {
-    const int stage = i % NS;
-    const int ph = bts[warp + kWarps * i];
-    const int row = ph >= 0 ? (ph * p.Hkv + w.kv_head) * kPageSize : -kPageSize;
-    uint8_t* dst = ring + stage * STAGE_BYTES;
-    mbar_arrive_expect_tx(&bar[stage], STAGE_BYTES);
-#pragma unroll
-    for (int b = 0; b < D / 64; ++b) {
-        tma_load_2d(dst + b * kBoxBytes, tmK, &bar[stage], b * 64, row);
-        tma_load_2d(dst + PAGE_BYTES + b * kBoxBytes, tmV, &bar[stage], b * 64, row);
-    }
-}
-
-// Merge the four warps' (max, sum, unnormalised output) held in cm/cl/co, then either
-// write the rows (whole unit) or a split partial; the last split of a unit merges all
-// partials. Every thread of the CTA calls this.
-template <int D, int NR>
-__device__ __forceinline__ void merge_and_store(const DecodeParams& p, const DecodeWork& w, const float* cm,
-                                                const float* cl, const float* co, const int* rout, int* flag) {
-    const int tid = threadIdx.x;
-    const int R = w.row_count;
-    const bool split = w.unit >= 0;
-    int slot = 0;
-    if (split) slot = p.units[w.unit].slot_base + w.split;
-    for (int idx = tid; idx < R * (D / 2); idx += kThreads) {
-        const int r = idx / (D / 2);
-        const int c = (idx - r * (D / 2)) * 2;
-        float M = -INFINITY;
-#pragma unroll
-        for (int ww = 0; ww < kWarps; ++ww) M = fmaxf(M, cm[ww * NR + r]);
-        float o0 = 0.f, o1 = 0.f, L = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int ww = 0; ww < kWarps; ++ww) {
-                const float f = exp2f(cm[ww * NR + r] - M);
-                const float2 v = *reinterpret_cast<const float2*>(co + (ww * NR + r) * D + c);
-                o0 = fmaf(f, v.x, o0);
-                o1 = fmaf(f, v.y, o1);
-                L = fmaf(f, cl[ww * NR + r], L);
-            }
-        }
-        if (!split) {
-            const float inv = L > 0.f ? 1.f / L : 0.f;
-            *reinterpret_cast<__nv_bfloat162*>(p.out + (int64_t)rout[r] * D + c) =
-                __floats2bfloat162_rn(o0 * inv, o1 * inv);
-        } else {
-            *reinterpret_cast<float2*>(p.part_o + ((int64_t)slot * kDecodeRowsMax + r) * D + c) =
-                make_float2(o0, o1);
-            if (c == 0)
-                *reinterpret_cast<float2*>(p.part_ml + ((int64_t)slot * kDecodeRowsMax + r) * 2) =
-                    make_float2(M, L);
-        }
-    }
-    if (!split) return;
-
-    // ---- split-KV combine: the last split of the unit to finish merges all partials -----
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        const int prev = atomicAdd(&p.counters[w.unit], 1);
-        flag[0] = (prev == p.units[w.unit].num_splits - 1);
-    }
-    __syncthreads();
-    if (!flag[0]) return;
-    __threadfence();
-    const SplitUnit u = p.units[w.unit];
-    for (int idx = tid; idx < R * (D / 2); idx += kThreads) {
-        const int r = idx / (D / 2);
-        const int c = (idx - r * (D / 2)) * 2;
-        float M = -INFINITY;
-        for (int s = 0; s < u.num_splits; ++s)
-            M = fmaxf(M, __ldcg(p.part_ml + ((int64_t)(u.slot_base + s) * kDecodeRowsMax + r) * 2));
-        float o0 = 0.f, o1 = 0.f, L = 0.f;
-        if (M != -INFINITY) {
-            for (int s = 0; s < u.num_splits; ++s) {
-                const int64_t base = (int64_t)(u.slot_base + s) * kDecodeRowsMax + r;
-                const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + base * 2));
-                const float f = exp2f(ml.x - M);
-                const float2 v = __ldcg(reinterpret_cast<const float2*>(p.part_o + base * D + c));
-                o0 = fmaf(f, v.x, o0);
-                o1 = fmaf(f, v.y, o1);
-                L = fmaf(f, ml.y, L);
-            }
-        }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        *reinterpret_cast<__nv_bfloat162*>(p.out + (int64_t)rout[r] * D + c) =
-            __floats2bfloat162_rn(o0 * inv, o1 * inv);
-    }
-    if (tid == 0) p.counters[w.unit] = 0;     // ready for the next run of the plan
-}
-
-// =====================================================================================
-// Tensor-core page body (mma.sync): keys on M, the group's rows on N.
-// =====================================================================================
 template <int D, int NT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kDecThreads)
 decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV) {
-    constexpr int NR = NT * 8;
-    using C = DecodeCfg<D, NR, false>;
-    constexpr int KS = D / 16;                    // k-steps of QK^T; d-tiles of PV
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, t4 = lane & 3;       // fragment row group / thread-in-group
-    const DecodeWork w = p.work[blockIdx.x];
-    const SeqInfo si = p.seqs[w.seq];
-
-    int* bts = reinterpret_cast<int*>(sm + C::OFF_BT);
-    int* rlim = reinterpret_cast<int*>(sm + C::OFF_LIM);
-    uint64_t* ranc = reinterpret_cast<uint64_t*>(sm + C::OFF_ANC);
-    int* rout = reinterpret_cast<int*>(sm + C::OFF_OUT);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
-    int* flag = reinterpret_cast<int*>(sm + C::OFF_FLAG);
-
-    const int R = w.row_count;
-    const int npg = w.page_end - w.page_begin;
-    const int prefix = si.seq_len - si.query_len;
-
-    task_setup<NR, C::NS>(p, w, si, bts, rlim, ranc, rout, bars, flag, &tmK, &tmV);
-
-    // Q^T as the B operand: row (column of S^T) nt*8+g, k = d; pairs straight from global
-    uint32_t qf[NT][KS][2];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        const int r = nt * 8 + g;
-        if (r < R) {
-            const __nv_bfloat16* qp = p.q + (int64_t)q_row_index(p, si, w, r) * D + 2 * t4;
-#pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
-                qf[nt][ks][0] = *reinterpret_cast<const uint32_t*>(qp + ks * 16);
-                qf[nt][ks][1] = *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8);
-            }
-        } else {
-#pragma unroll
-            for (int ks = 0; ks < KS; ++ks) qf[nt][ks][0] = qf[nt][ks][1] = 0u;
-        }
-    }
-    __syncthreads();
-
-    // this thread's columns: c = nt*8 + 2*t4 + e
-    int lim[NT][2];
-    uint64_t anc[NT][2];
-    int min_lim = 0x7fffffff;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int c = nt * 8 + 2 * t4 + e;
-            lim[nt][e] = rlim[c];
-            anc[nt][e] = ranc[c];
-        }
-    for (int r = 0; r < R; ++r) min_lim = min(min_lim, rlim[r]);
-
-    const int n_my = npg > warp ? (npg - warp + kWarps - 1) / kWarps : 0;
-    uint8_t* ring = sm + warp * C::NS * C::STAGE_BYTES;
-    uint64_t* bar = bars + warp * C::NS;
-
-    float o[KS][NT][4];           // O^T tiles: [d-tile][n-tile]{(d g, c), (d g, c+1), (d g+8, c), (d g+8, c+1)}
-    float mref[NT][2], lsum[NT][2];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            mref[nt][e] = -INFINITY;
-            lsum[nt][e] = 0.f;
-        }
-#pragma unroll
-        for (int dt = 0; dt < KS; ++dt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) o[dt][nt][i] = 0.f;
-    }
-
-    if (lane == 0)
-        for (int i = 0; i < C::NS && i < n_my; ++i)
-            issue_page<D, C::NS, C::STAGE_BYTES, C::PAGE_BYTES>(p, w, bts, ring, bar, warp, i, &tmK, &tmV);
-    __syncwarp();
-
-    // ldmatrix row addresses: matrix mi = lane >> 3 supplies its rows from lanes 8mi..8mi+7
-    const int mi = lane >> 3, mr = lane & 7;
-    const int k_key = mr + (mi & 1) * 8, k_chunk = mi >> 1;          // K: A operand, keys on M
-    const int v_key = mr + (mi >> 1) * 8, v_chunk = mi & 1;          // V: A operand of V^T (trans)
-    bool ok = true;
-    int waited = 0;
-
-    for (int i = 0; i < n_my; ++i) {
-        const int stage = i % C::NS;
-        const bool got = mbar_wait_bounded(&bar[stage], (i / C::NS) & 1, p.err, PKVA_DEVERR_TIMEOUT);
-        waited = i + 1;
-        if (__any_sync(0xffffffffu, !got)) {
-            ok = false;
-            break;
-        }
-        uint8_t* Ks = ring + stage * C::STAGE_BYTES;
-        uint8_t* Vs = Ks + C::PAGE_BYTES;
-        const int kbase = (w.page_begin + warp + kWarps * i) * kPageSize;
-
-        // -- S^T = K Q^T (16 keys x 8 rows per n-tile) ------------------------------------
-        float s[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            const int cg = ks * 2 + k_chunk;
-            uint32_t a[4];
-            ldmatrix_x4(a, Ks + (cg >> 3) * kBoxBytes + k_key * 128 + (((cg & 7) ^ (k_key & 7)) << 4));
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a, qf[nt][ks]);
-        }
-
-        // -- mask and per-row (column) max over the page's 16 keys ------------------------
-        const bool page_all = (kbase + kPageSize - 1) <= min_lim;
-        float cmax[NT][2];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int kpos = kbase + g + 8 * h;
-                    float v = s[nt][2 * h + e] * p.scale_log2;
-                    if (!page_all) {
-                        bool allow = kpos <= lim[nt][e];
-                        if (!allow && kpos >= prefix && kpos < si.seq_len)
-                            allow = (anc[nt][e] >> (kpos - prefix)) & 1ull;
-                        v = allow ? v : -INFINITY;
-                    }
-                    s[nt][2 * h + e] = v;
-                }
-                float mx = fmaxf(s[nt][e], s[nt][2 + e]);
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                cmax[nt][e] = mx;
-            }
-        // -- lazy rescale: only when some row's max passed its reference by the slack ------
-        bool need = false;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e)
-                need |= cmax[nt][e] > mref[nt][e] + kRescaleSlack ||
-                        (mref[nt][e] == -INFINITY && cmax[nt][e] != -INFINITY);
-        if (__any_sync(0xffffffffu, need)) {
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const float mnew = fmaxf(mref[nt][e], cmax[nt][e]);
-                    if (mnew != mref[nt][e]) {
-                        const float alpha = mref[nt][e] == -INFINITY ? 0.f : exp2f(mref[nt][e] - mnew);
-                        mref[nt][e] = mnew;
-                        lsum[nt][e] *= alpha;
-#pragma unroll
-                        for (int dt = 0; dt < KS; ++dt) {
-                            o[dt][nt][e] *= alpha;
-                            o[dt][nt][2 + e] *= alpha;
-                        }
-                    }
-                }
-        }
-        // -- P = exp2(S - ref), row sums, P^T as the B operand (transpose in registers) -----
-        uint32_t pb[NT][2];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            float pv[4];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const float ref = mref[nt][e] == -INFINITY ? 0.f : mref[nt][e];
-                pv[e] = exp2f(s[nt][e] - ref);
-                pv[2 + e] = exp2f(s[nt][2 + e] - ref);
-                lsum[nt][e] += pv[e] + pv[2 + e];
-            }
-            pb[nt][0] = movmatrix_trans(pack_bf16x2(pv[0], pv[1]));   // keys 0..7
-            pb[nt][1] = movmatrix_trans(pack_bf16x2(pv[2], pv[3]));   // keys 8..15
-        }
-        // slots past the sequence's end hold stale cache data: zero those V rows so that
-        // P = 0 times a non-finite value cannot reach the accumulators
-        const int nvalid = si.seq_len - kbase;
-        if (nvalid < kPageSize) {
-            for (int idx = lane; idx < (kPageSize - nvalid) * (D / 8); idx += 32) {
-                const int row = nvalid + idx / (D / 8);
-                const int cg = idx % (D / 8);
-                *reinterpret_cast<uint4*>(Vs + (cg >> 3) * kBoxBytes + row * 128 + (cg & 7) * 16) =
-                    make_uint4(0u, 0u, 0u, 0u);
-            }
-            __syncwarp();
-        }
-        // -- O^T += V^T P^T -----------------------------------------------------------------
-#pragma unroll
-        for (int dt = 0; dt < KS; ++dt) {
-            const int cg = dt * 2 + v_chunk;
-            uint32_t a[4];
-            ldmatrix_x4_trans(a, Vs + (cg >> 3) * kBoxBytes + v_key * 128 + (((cg & 7) ^ (v_key & 7)) << 4));
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[dt][nt], a, pb[nt]);
-        }
-        __syncwarp();
-        if (lane == 0 && i + C::NS < n_my) {
-            fence_proxy_async_smem();
-            issue_page<D, C::NS, C::STAGE_BYTES, C::PAGE_BYTES>(p, w, bts, ring, bar, warp, i + C::NS, &tmK,
-                                                                 &tmV);
-        }
-    }
-    if (!ok) {
-        for (int i = waited; i < n_my && i < waited + C::NS; ++i)
-            mbar_wait_bounded(&bar[i % C::NS], (i / C::NS) & 1, p.err, PKVA_DEVERR_TIMEOUT);
-        if (lane == 0) atomicOr(&flag[1], 1);
-    }
-    // row sums over the 16 keys: lanes with the same t4 hold the column
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            float l = lsum[nt][e];
-            l += __shfl_xor_sync(0xffffffffu, l, 4);
-            l += __shfl_xor_sync(0xffffffffu, l, 8);
-            l += __shfl_xor_sync(0xffffffffu, l, 16);
-            lsum[nt][e] = l;
-        }
-
-    __syncthreads();
-    float* cm = reinterpret_cast<float*>(sm);       // [kWarps][NR]
-    float* cl = cm + kWarps * NR;                   // [kWarps][NR]
-    float* co = cl + kWarps * NR;                   // [kWarps][NR][D]
-    if (g == 0) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int c = nt * 8 + 2 * t4 + e;
-                cm[warp * NR + c] = mref[nt][e];
-                cl[warp * NR + c] = lsum[nt][e];
-            }
-    }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int dt = 0; dt < KS; ++dt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int c = nt * 8 + 2 * t4 + (i & 1);
-                const int d = dt * 16 + g + 8 * (i >> 1);
-                co[(warp * NR + c) * D + d] = o[dt][nt][i];
-            }
-    __syncthreads();
-    merge_and_store<D, NR>(p, w, cm, cl, co, rout, flag);
+    const dec::Group grp{(int)threadIdx.x, kDecThreads, 0};
+    dec::decode_mma_task<D, NT, 4, StandaloneNS<D, NT * 8>::value>(grp, p, blockIdx.x, tmK, tmV, sm);
 }
 
-// =====================================================================================
-// CUDA-core page body (fp32 FMA).
-// =====================================================================================
 template <int D, int NR>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kDecThreads)
 decode_fma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV) {
-    using C = DecodeCfg<D, NR, true>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const DecodeWork w = p.work[blockIdx.x];
-    const SeqInfo si = p.seqs[w.seq];
-
-    float* qs = reinterpret_cast<float*>(sm + C::OFF_Q);
-    float* ps = reinterpret_cast<float*>(sm + C::OFF_P);
-    int* bts = reinterpret_cast<int*>(sm + C::OFF_BT);
-    int* rlim = reinterpret_cast<int*>(sm + C::OFF_LIM);
-    uint64_t* ranc = reinterpret_cast<uint64_t*>(sm + C::OFF_ANC);
-    int* rout = reinterpret_cast<int*>(sm + C::OFF_OUT);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
-    int* flag = reinterpret_cast<int*>(sm + C::OFF_FLAG);
-
-    const int R = w.row_count;
-    const int npg = w.page_end - w.page_begin;
-    const int prefix = si.seq_len - si.query_len;
-
-    task_setup<NR, C::NS>(p, w, si, bts, rlim, ranc, rout, bars, flag, &tmK, &tmV);
-    // Q rows in fp32, pre-scaled by scale*log2(e); each row is stored as two halves with a
-    // 4-float pad so that the two lane halves read different banks
-    for (int idx = tid; idx < NR * (D / 8); idx += kThreads) {
-        const int r = idx / (D / 8);
-        const int c8 = (idx - r * (D / 8)) * 8;
-        float f[8];
-        if (r < R) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(p.q + (int64_t)q_row_index(p, si, w, r) * D + c8);
-            bf16x8_to_f32(raw, f);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] *= p.scale_log2;
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = 0.f;
-        }
-        const int hh = c8 / C::HALF;
-        float* dst = qs + r * C::QROW + hh * (C::HALF + 4) + (c8 - hh * C::HALF);
-        *reinterpret_cast<float4*>(dst) = make_float4(f[0], f[1], f[2], f[3]);
-        *reinterpret_cast<float4*>(dst + 4) = make_float4(f[4], f[5], f[6], f[7]);
-    }
-    __syncthreads();
-
-    int min_lim = 0x7fffffff;
-    for (int r = 0; r < R; ++r) min_lim = min(min_lim, rlim[r]);
-
-    const int n_my = npg > warp ? (npg - warp + kWarps - 1) / kWarps : 0;
-    uint8_t* ring = sm + warp * C::NS * C::STAGE_BYTES;
-    uint64_t* bar = bars + warp * C::NS;
-
-    float o[NR][C::OPL];
-    float m_run[NR], l_run[NR];
-#pragma unroll
-    for (int r = 0; r < NR; ++r) {
-        m_run[r] = -INFINITY;
-        l_run[r] = 0.f;
-#pragma unroll
-        for (int c = 0; c < C::OPL; ++c) o[r][c] = 0.f;
-    }
-
-    if (lane == 0)
-        for (int i = 0; i < C::NS && i < n_my; ++i)
-            issue_page<D, C::NS, C::STAGE_BYTES, C::PAGE_BYTES>(p, w, bts, ring, bar, warp, i, &tmK, &tmV);
-    __syncwarp();
-
-    const int j = lane & 15;       // key slot of this lane in the QK phase
-    const int hh = lane >> 4;      // which half of the head dimension it sums
-    float* pw = ps + warp * kPageSize * NR;
-    bool ok = true;
-    int waited = 0;
-
-    for (int i = 0; i < n_my; ++i) {
-        const int stage = i % C::NS;
-        const bool got = mbar_wait_bounded(&bar[stage], (i / C::NS) & 1, p.err, PKVA_DEVERR_TIMEOUT);
-        waited = i + 1;
-        if (__any_sync(0xffffffffu, !got)) {
-            ok = false;
-            break;
-        }
-        const uint8_t* Ks = ring + stage * C::STAGE_BYTES;
-        const uint8_t* Vs = Ks + C::PAGE_BYTES;
-        const int kbase = (w.page_begin + warp + kWarps * i) * kPageSize;
-
-        // -- scores: lane (j, hh) sums half hh of <q_r, k_j> for every row r ------------
-        float acc[NR];
-#pragma unroll
-        for (int r = 0; r < NR; ++r) acc[r] = 0.f;
-#pragma unroll
-        for (int cc = 0; cc < C::HALF / 8; ++cc) {
-            const int col = hh * C::HALF + cc * 8;
-            const int box = col >> 6, ch = (col & 63) >> 3;
-            const uint4 kr = *reinterpret_cast<const uint4*>(Ks + box * kBoxBytes + j * 128 + ((ch ^ (j & 7)) << 4));
-            float kf[8];
-            bf16x8_to_f32(kr, kf);
-            const float* qp = qs + hh * (C::HALF + 4) + cc * 8;
-#pragma unroll
-            for (int r = 0; r < NR; ++r) {
-                if (r < R) {
-                    const float4 a = *reinterpret_cast<const float4*>(qp + r * C::QROW);
-                    const float4 b = *reinterpret_cast<const float4*>(qp + r * C::QROW + 4);
-                    float t = acc[r];
-                    t = fmaf(kf[0], a.x, t);
-                    t = fmaf(kf[1], a.y, t);
-                    t = fmaf(kf[2], a.z, t);
-                    t = fmaf(kf[3], a.w, t);
-                    t = fmaf(kf[4], b.x, t);
-                    t = fmaf(kf[5], b.y, t);
-                    t = fmaf(kf[6], b.z, t);
-                    t = fmaf(kf[7], b.w, t);
-                    acc[r] = t;
-                }
-            }
-        }
-        // -- mask, online softmax (warp-shuffle max over the page's 16 keys) --------------
-        const int kpos = kbase + j;
-        const bool page_all = (kbase + kPageSize - 1) <= min_lim;
-        float alpha[NR];
-#pragma unroll
-        for (int r = 0; r < NR; ++r) {
-            alpha[r] = 1.f;
-            if (r < R) {
-                float s = acc[r] + __shfl_xor_sync(0xffffffffu, acc[r], 16);
-                bool allow = page_all || kpos <= rlim[r];
-                if (!allow && kpos >= prefix && kpos < si.seq_len)
-                    allow = (ranc[r] >> (kpos - prefix)) & 1ull;
-                s = allow ? s : -INFINITY;
-                float mx = s;
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                const float mnew = fmaxf(m_run[r], mx);
-                const float ref = (mnew == -INFINITY) ? 0.f : mnew;
-                const float pr = exp2f(s - ref);
-                alpha[r] = exp2f(m_run[r] - ref);
-                m_run[r] = mnew;
-                l_run[r] = fmaf(l_run[r], alpha[r], pr);
-                acc[r] = pr;
-            } else {
-                acc[r] = 0.f;
-            }
-        }
-        if (hh == 0) {
-#pragma unroll
-            for (int r4 = 0; r4 < NR / 4; ++r4)
-                *reinterpret_cast<float4*>(pw + j * NR + 4 * r4) =
-                    make_float4(acc[4 * r4], acc[4 * r4 + 1], acc[4 * r4 + 2], acc[4 * r4 + 3]);
-        }
-        __syncwarp();
-
-        // -- o_r = alpha_r * o_r + sum_j p_rj v_j; lane owns D/32 output columns ------------
-#pragma unroll
-        for (int r = 0; r < NR; ++r)
-            if (r < R)
-#pragma unroll
-                for (int c = 0; c < C::OPL; ++c) o[r][c] *= alpha[r];
-        const int nvalid = min(kPageSize, si.seq_len - kbase);   // slots past L are skipped
-#pragma unroll 4
-        for (int jj = 0; jj < nvalid; ++jj) {
-            float vf[C::OPL];
-            if constexpr (D == 128) {
-                const int box = lane >> 4, ch = (lane & 15) >> 1;
-                const uint2 vr = *reinterpret_cast<const uint2*>(Vs + box * kBoxBytes + jj * 128 +
-                                                                 ((ch ^ (jj & 7)) << 4) + (lane & 1) * 8);
-                bf16x2_to_f32(vr.x, vf[0], vf[1]);
-                bf16x2_to_f32(vr.y, vf[2], vf[3]);
-            } else {
-                const int ch = lane >> 2;
-                const uint32_t vr = *reinterpret_cast<const uint32_t*>(Vs + jj * 128 + ((ch ^ (jj & 7)) << 4) +
-                                                                       (lane & 3) * 4);
-                bf16x2_to_f32(vr, vf[0], vf[1]);
-            }
-#pragma unroll
-            for (int r4 = 0; r4 < NR / 4; ++r4) {
-                const float4 pp = *reinterpret_cast<const float4*>(pw + jj * NR + 4 * r4);
-                const float pv[4] = {pp.x, pp.y, pp.z, pp.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = 4 * r4 + e;
-                    if (r < R)
-#pragma unroll
-                        for (int c = 0; c < C::OPL; ++c) o[r][c] = fmaf(pv[e], vf[c], o[r][c]);
-                }
-            }
-        }
-        __syncwarp();
-        if (lane == 0 && i + C::NS < n_my) {
-            fence_proxy_async_smem();
-            issue_page<D, C::NS, C::STAGE_BYTES, C::PAGE_BYTES>(p, w, bts, ring, bar, warp, i + C::NS, &tmK,
-                                                                 &tmV);
-        }
-    }
-    if (!ok) {
-        for (int i = waited; i < n_my && i < waited + C::NS; ++i)
-            mbar_wait_bounded(&bar[i % C::NS], (i / C::NS) & 1, p.err, PKVA_DEVERR_TIMEOUT);
-        if (lane == 0) atomicOr(&flag[1], 1);
-    }
-
-    // row sums: lanes j and j+16 hold the same keys, so reduce within each half
-#pragma unroll
-    for (int r = 0; r < NR; ++r) {
-        float l = l_run[r];
-        l += __shfl_xor_sync(0xffffffffu, l, 1);
-        l += __shfl_xor_sync(0xffffffffu, l, 2);
-        l += __shfl_xor_sync(0xffffffffu, l, 4);
-        l += __shfl_xor_sync(0xffffffffu, l, 8);
-        l_run[r] = l;
-    }
-
-    __syncthreads();
-    float* cm = reinterpret_cast<float*>(sm);       // [kWarps][NR] running max (log2 units)
-    float* cl = cm + kWarps * NR;                   // [kWarps][NR] running sum
-    float* co = cl + kWarps * NR;                   // [kWarps][NR][D] unnormalised output
-    if (lane == 0) {
-#pragma unroll
-        for (int r = 0; r < NR; ++r) {
-            cm[warp * NR + r] = m_run[r];
-            cl[warp * NR + r] = l_run[r];
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < NR; ++r) {
-        if (r < R) {
-            float* dst = co + (warp * NR + r) * D + lane * C::OPL;
-            if constexpr (C::OPL == 4)
-                *reinterpret_cast<float4*>(dst) = make_float4(o[r][0], o[r][1], o[r][2], o[r][3]);
-            else
-                *reinterpret_cast<float2*>(dst) = make_float2(o[r][0], o[r][1]);
-        }
-    }
-    __syncthreads();
-    merge_and_store<D, NR>(p, w, cm, cl, co, rout, flag);
+    const dec::Group grp{(int)threadIdx.x, kDecThreads, 0};
+    dec::decode_fma_task<D, NR, 4, StandaloneNS<D, NR>::value>(grp, p, blockIdx.x, tmK, tmV, sm);
 }
 
 // ---- launch plumbing ---------------------------------------------------------------------
@@ -734,7 +74,7 @@ template <class K>
 int resident(K kernel, int bytes) {
     int n = 0;
     if (set_smem(kernel, bytes) != cudaSuccess) return 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads, bytes) != cudaSuccess) return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kDecThreads, bytes) != cudaSuccess) return 0;
     return n;
 }
 
@@ -743,15 +83,15 @@ cudaError_t launch_t(const DecodeParams& p, int num_work, bool mma, const CUtens
                      const CUtensorMap& tmV, cudaStream_t stream) {
     if (mma) {
         constexpr int NT = NR <= 8 ? 1 : 2;
-        using C = DecodeCfg<D, NT * 8, false>;
+        using C = dec::DecodeCfg<D, NT * 8, false, 4, StandaloneNS<D, NT * 8>::value>;
         cudaError_t e = set_smem(decode_mma_kernel<D, NT>, C::ALLOC);
         if (e != cudaSuccess) return e;
-        decode_mma_kernel<D, NT><<<num_work, kThreads, C::ALLOC, stream>>>(p, tmK, tmV);
+        decode_mma_kernel<D, NT><<<num_work, kDecThreads, C::ALLOC, stream>>>(p, tmK, tmV);
     } else {
-        using C = DecodeCfg<D, NR, true>;
+        using C = dec::DecodeCfg<D, NR, true, 4, StandaloneNS<D, NR>::value>;
         cudaError_t e = set_smem(decode_fma_kernel<D, NR>, C::ALLOC);
         if (e != cudaSuccess) return e;
-        decode_fma_kernel<D, NR><<<num_work, kThreads, C::ALLOC, stream>>>(p, tmK, tmV);
+        decode_fma_kernel<D, NR><<<num_work, kDecThreads, C::ALLOC, stream>>>(p, tmK, tmV);
     }
     return cudaGetLastError();
 }
@@ -760,9 +100,9 @@ template <int D, int NR>
 int ctas_t(bool mma) {
     if (mma) {
         constexpr int NT = NR <= 8 ? 1 : 2;
-        return resident(decode_mma_kernel<D, NT>, DecodeCfg<D, NT * 8, false>::ALLOC);
+        return resident(decode_mma_kernel<D, NT>, dec::DecodeCfg<D, NT * 8, false, 4, StandaloneNS<D, NT * 8>::value>::ALLOC);
     }
-    return resident(decode_fma_kernel<D, NR>, DecodeCfg<D, NR, true>::ALLOC);
+    return resident(decode_fma_kernel<D, NR>, dec::DecodeCfg<D, NR, true, 4, StandaloneNS<D, NR>::value>::ALLOC);
 }
 
 }  // namespace

@@ -15,6 +15,7 @@ constexpr int kDecodeMaxPages = 1024;  // pages per decode task (block-table sli
 constexpr int kPrefillTileM = 128;     // query tokens per prefill tile (tcgen05 M)
 constexpr int kPrefillTaskTokens = 256; // query tokens per prefill task (two tiles, ping-pong)
 constexpr int kPrefillTileN = 128;     // keys per prefill KV tile (8 pages)
+constexpr int kDecTasksPerBlock = 3;   // decode tasks side by side in one block of the unified kernel
 constexpr int kPrefillMinTokens = 64;  // causal sequences with at least this many new tokens
                                        // (and head_dim 128) run on the tensor-core prefill kernel
 
@@ -73,7 +74,11 @@ struct HostPlan {
     std::vector<SeqInfo> seqs;
     std::vector<uint64_t> anc;            // per TREE token: ancestor-or-self bit mask
     std::vector<DecodeWork> dwork;        // launch order
-    std::vector<PrefillWork> pwork;       // launch order
+    std::vector<PrefillWork> pwork;       // heaviest first
+    // Unified launch order, one entry per block: e >= 0 runs prefill task e; e < 0 runs
+    // decode tasks 3*(-1-e) .. 3*(-1-e)+2 side by side. Both kinds heaviest first, merged
+    // in proportion.
+    std::vector<int32_t> order;
     std::vector<SplitUnit> units;
     int num_slots = 0;
     int64_t kv_bytes = 0;

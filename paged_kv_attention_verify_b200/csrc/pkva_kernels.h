@@ -39,12 +39,23 @@ struct PrefillParams {
     float scale_log2;
 };
 
-int prefill_ctas_per_sm();
+// Everything one launch of the unified attention kernel needs.
+struct AttnParams {
+    PrefillParams pre;
+    DecodeParams dec;
+    const int32_t* order;         // per block: >= 0 prefill task, < 0 decode pair -1-e
+    int32_t num_blocks;
+    int32_t num_decode;           // decode/verify tasks (two per block)
+};
 
-// Launch the tensor-core prefill kernel (head_dim 128). tmQ views q as the 3-D tensor
-// [sum T][Hq][128] with a {64, 1, 128} box; tmK/tmV as the decode kernel's cache maps.
-cudaError_t launch_prefill(const PrefillParams& p, int num_work, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                           const CUtensorMap& tmV, cudaStream_t stream);
+// Resident blocks per SM of the unified kernel (one: each block takes most of an SM).
+int attn_ctas_per_sm(int D, int rows);
+
+// Launch the unified kernel over p.num_blocks blocks in the order p.order (prefill tasks
+// need head_dim 128). tmQ views q as the 3-D tensor [sum T][Hq][128] with a
+// {64, 1, 128} box; tmK/tmV are the cache maps (16 x 64 boxes).
+cudaError_t launch_attn(const AttnParams& p, int D, int rows, bool has_prefill, const CUtensorMap& tmQ,
+                        const CUtensorMap& tmK, const CUtensorMap& tmV, cudaStream_t stream);
 
 // Resident CTAs per SM of the decode kernel compiled for (D, rows); 0 if unsupported.
 // `mma` selects the tensor-core page body, otherwise the CUDA-core one.

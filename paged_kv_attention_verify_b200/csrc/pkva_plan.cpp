@@ -208,6 +208,22 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
     std::stable_sort(p.dwork.begin(), p.dwork.end(), [](const DecodeWork& x, const DecodeWork& y) {
         return (x.page_end - x.page_begin) > (y.page_end - y.page_begin);
     });
+
+    // -- one launch order for both kinds. Each kind keeps its heaviest-first order; the two
+    //    lists are merged in proportion, so prefill blocks (tensor cores, latency) run beside
+    //    decode blocks (HBM) from start to end instead of one kind forming the tail. Decode
+    //    tasks go three to a block, neighbours in the sorted list.
+    const int np = (int)p.pwork.size();
+    const int nd = (int)((p.dwork.size() + kDecTasksPerBlock - 1) / kDecTasksPerBlock);
+    int ip = 0, id = 0;
+    while (ip < np || id < nd) {
+        // take from the list that is further behind in its share of the launch
+        const bool take_p = id >= nd || (ip < np && (int64_t)ip * nd <= (int64_t)id * np);
+        if (take_p)
+            p.order.push_back(ip++);
+        else
+            p.order.push_back(-1 - id++);
+    }
     return PKVA_OK;
 }
 
@@ -232,37 +248,38 @@ extern "C" int attn_plan_inspect(int num_seqs, const int32_t* seq_lens, const in
         set_last_error(err);
         return rc;
     }
-    const int nd = (int)hp.dwork.size();
-    const int n = nd + (int)hp.pwork.size();
+    const int np = (int)hp.pwork.size();
+    const int n = np + (int)hp.dwork.size();
     if (num_items) *num_items = n;
     if (!items) return PKVA_OK;
     if (max_items < n) {
         set_last_error("attn_plan_inspect: max_items is smaller than the number of tasks");
         return PKVA_EINVAL;
     }
-    for (int i = nd; i < n; ++i) {
-        const PrefillWork& w = hp.pwork[i - nd];
+    for (int i = 0; i < np; ++i) {      // launch order: prefill tasks first
+        const PrefillWork& w = hp.pwork[i];
         const SeqInfo& si = hp.seqs[w.seq];
         pkva_work_desc d;
         d.kind = 1;
         d.seq = w.seq;
         d.kv_head = w.q_head / hp.G;
-        d.row_begin = w.tok0 * hp.G + w.q_head % hp.G;   // packed row of its first token
+        d.q_head = w.q_head;
+        d.row_begin = w.tok0;
         d.row_count = w.ntok;
         d.key_begin = 0;
         d.key_end = std::min(si.seq_len - si.query_len + w.tok0 + w.ntok, si.seq_len);
-        (void)w.kv_tiles0;
         d.split = -1;
         d.num_splits = 1;
         items[i] = d;
     }
-    for (int i = 0; i < nd; ++i) {
-        const DecodeWork& w = hp.dwork[i];
+    for (int i = np; i < n; ++i) {
+        const DecodeWork& w = hp.dwork[i - np];
         const SeqInfo& si = hp.seqs[w.seq];
         pkva_work_desc d;
         d.kind = 0;
         d.seq = w.seq;
         d.kv_head = w.kv_head;
+        d.q_head = -1;
         d.row_begin = w.row_begin;
         d.row_count = w.row_count;
         d.key_begin = w.page_begin * kPageSize;

@@ -1,4 +1,4 @@
-// Causal chunked-prefill attention over the paged KV cache on 5th-generation tensor cores
+// Prefill task body: causal chunked-prefill attention over the paged KV cache on 5th-generation tensor cores
 // (K-P): S = Q K^T and O += P V are tcgen05.mma BF16 tiles with fp32 accumulators in
 // tensor memory (TMEM).
 //
@@ -25,6 +25,8 @@
 // primitive is a matmul-softmax-matmul tile whose QK and SV products overlap the softmax),
 // core_discovery (chunked prefill on cached prefixes; fully masked tiles are skipped);
 // supporting citation [1] (FlashAttention's tiled online softmax).
+#pragma once
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -34,8 +36,8 @@
 #include "pkva_ptx.cuh"
 
 namespace pkva {
+namespace pre {
 
-namespace {
 
 constexpr int kPThreads = 352;
 constexpr int kD = 128;
@@ -158,13 +160,13 @@ __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, 
         for (int h = 0; h < 2; ++h) tma_load_2d(dst + h * kHalfBytes + pg * (kPageSize * 128), map, bar, h * 64, rows[pg]);
 }
 
-__global__ void __launch_bounds__(kPThreads, 1)
-prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
-               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+// One prefill task; every thread of the block (at least kPThreads) calls it; warps past
+// the V producer only take part in the block barriers. `sm` is the block's 1024-aligned
+// dynamic shared memory (kSmemBytes).
+__device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, const CUtensorMap& tmQ,
+                                             const CUtensorMap& tmK, const CUtensorMap& tmV, uint8_t* sm) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const PrefillWork w = p.work[blockIdx.x];
+    const PrefillWork w = p.work[task];
     const SeqInfo si = p.seqs[w.seq];
     const Bars B = bars_at(sm);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffTmemSlot);
@@ -310,7 +312,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
             tc_commit(B.mma_done);
             mbar_wait_bounded(B.mma_done, 0, p.err, PKVA_DEVERR_TIMEOUT);
         }
-    } else {
+    } else if (warp < 8) {
         // ------------------------------ softmax (rows) ---------------------------------------
         const int b = warp >> 2;                             // query tile of this warpgroup
         const int r = tid & 127;                             // row = TMEM lane
@@ -436,24 +438,6 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
     if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
 }
 
-}  // namespace
 
-int prefill_ctas_per_sm() {
-    int n = 0;
-    if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc) != cudaSuccess)
-        return 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, prefill_kernel, kPThreads, kSmemAlloc) != cudaSuccess)
-        return 0;
-    return n;
-}
-
-cudaError_t launch_prefill(const PrefillParams& p, int num_work, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                           const CUtensorMap& tmV, cudaStream_t stream) {
-    if (num_work == 0) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
-    if (e != cudaSuccess) return e;
-    prefill_kernel<<<num_work, kPThreads, kSmemAlloc, stream>>>(p, tmQ, tmK, tmV);
-    return cudaGetLastError();
-}
-
+}  // namespace pre
 }  // namespace pkva

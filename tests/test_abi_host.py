@@ -83,9 +83,14 @@ def _coverage(batch, items):
     G = batch.num_q_heads // batch.num_kv_heads
     seen = {}
     for it in items:
-        assert it["row_count"] >= 1 and it["row_count"] <= 16
         assert it["key_begin"] % 16 == 0 and it["key_end"] > it["key_begin"]
-        for r in range(it["row_begin"], it["row_begin"] + it["row_count"]):
+        if it["kind"] == 1:            # prefill: tokens [row_begin, +row_count) of one query head
+            assert 1 <= it["row_count"] <= 256 and it["q_head"] // G == it["kv_head"]
+            rows = [t * G + it["q_head"] % G for t in range(it["row_begin"], it["row_begin"] + it["row_count"])]
+        else:
+            assert 1 <= it["row_count"] <= 16 and it["q_head"] == -1
+            rows = range(it["row_begin"], it["row_begin"] + it["row_count"])
+        for r in rows:
             seen.setdefault((it["seq"], it["kv_head"], r), []).append((it["key_begin"], it["key_end"],
                                                                       it["split"], it["num_splits"]))
     for s, sp in enumerate(batch.seqs):
@@ -122,16 +127,18 @@ def test_planner_covers_configs(name):
                        num_q_heads=Hq, num_kv_heads=Hkv, head_dim=d, num_pages=pages,
                        bt_stride=max((s.seq_len + 15) // 16 for s in b.seqs))
     _coverage(b, items)
-    sizes = [it["key_end"] - it["key_begin"] for it in items]
-    # heaviest first (page-granular: the last page of a task may be partial)
-    pg = [(it["key_end"] + 15) // 16 - it["key_begin"] // 16 for it in items]
+    # launch order: prefill tasks, then decode/verify tasks, each heaviest first
+    kinds = [it["kind"] for it in items]
+    assert kinds == sorted(kinds, reverse=True)
+    dec = [it for it in items if it["kind"] == 0]
+    pg = [(it["key_end"] + 15) // 16 - it["key_begin"] // 16 for it in dec]
     assert pg == sorted(pg, reverse=True)
-    assert max(sizes) <= 1024 * 16
+    assert all(it["key_end"] - it["key_begin"] <= 1024 * 16 for it in dec)
 
 
-@pytest.mark.parametrize("seed", range(6))
-def test_planner_covers_random_batches(seed):
-    b = W.random_small(seed, num_seqs=6, max_ctx=300, max_q=40, tree_frac=0.4)
+@pytest.mark.parametrize("seed, d, max_q", [(s, 64, 40) for s in range(4)] + [(s, 128, 300) for s in range(4, 8)])
+def test_planner_covers_random_batches(seed, d, max_q):
+    b = W.random_small(seed, num_seqs=6, d=d, max_ctx=300, max_q=max_q, tree_frac=0.4)
     items = pk.inspect(b.seq_lens, b.query_lens, b.mask_kinds, b.parents_flat,
                        num_q_heads=b.num_q_heads, num_kv_heads=b.num_kv_heads, head_dim=b.head_dim,
                        num_pages=b.k_cache.shape[0], bt_stride=b.block_table.shape[1],

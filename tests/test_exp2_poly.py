@@ -20,7 +20,7 @@ def _fit():
 
 
 def kernel_coefficients():
-    src = open(os.path.join(CSRC, "pkva_prefill.cu")).read()
+    src = open(os.path.join(CSRC, "pkva_prefill_body.cuh")).read()
     vals = dict(re.findall(r"kExp2C(\d) = ([0-9.e+-]+)f", src))
     return [np.float32(vals[str(i)]) for i in range(4)]
 
