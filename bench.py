@@ -178,6 +178,76 @@ def run_reference(args):
     return 0
 
 
+def time_steps(plan, batch, out, steps, warmup, stream, ws=1, clk=None):
+    """Device time of `steps` consecutive attn_run calls (one kernel launch each), bracketed
+    by a barrier and a synchronize on both sides. Returns (per-step ms list, total ms)."""
+    import torch
+    import torch.distributed as dist
+    for _ in range(warmup):
+        plan.run(batch.q, batch.k_cache, batch.v_cache, out, stream)
+    if plan.check(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    if clk is not None:
+        clk.__enter__()
+    try:
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for i in range(steps):
+            plan.run(batch.q, batch.k_cache, batch.v_cache, out, stream)
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
+    finally:
+        if clk is not None:
+            clk.__exit__()
+    if plan.check(stream) != 0:
+        raise RuntimeError("device error during the timed region")
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    return per, ev[0].elapsed_time(ev[-1])
+
+
+def roofline(info, seconds, peaks, sustained=False):
+    """The binding resource of one launch and how close the launch comes to it.
+
+    HBM: algorithmic K+V bytes (each element once) per launch / launch time.
+    Tensor: algorithmic attention flops (4 * D * Hq per allowed query-key pair) / time.
+    The bound is whichever takes longer at its measured peak."""
+    tf_peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    t_hbm = info["kv_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_tc = info["attn_flops"] / (tf_peak * 1e12)
+    if t_hbm >= t_tc:
+        ach = info["kv_bytes"] / seconds / 1e9
+        return {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "frac_of_spec_8000": ach / 8000.0}
+    ach = info["attn_flops"] / seconds / 1e12
+    return {"bound": "tensor", "achieved": ach, "peak": tf_peak, "unit": "TFLOP/s",
+            "frac": ach / tf_peak, "frac_of_spec_2250": ach / 2250.0}
+
+
+def kernel_traffic(workload):
+    """DRAM bytes per launch of the attention kernel from the committed ncu summary, if it
+    was taken on this workload and on the current kernel sources (else None)."""
+    import glob
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "attn_kernel_traffic.json")))
+    except Exception:
+        return None
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "paged_kv_attention_verify_b200", "csrc", "*"))):
+        if f.endswith((".cu", ".cuh", ".h", ".cpp")):
+            h.update(open(f, "rb").read())
+    for e in rec.get("captures", []):
+        if e.get("workload") == workload and e.get("source_sha256") == h.hexdigest():
+            return e.get("dram_bytes_per_launch")
+    return None
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -191,43 +261,19 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     dev = torch.device("cuda", torch.cuda.current_device())
     peaks = load_peaks()
+    stream = torch.cuda.current_stream()
 
     batch = W.make_config(args.config, device=dev, max_seqs=args.seqs)
     plan = pk.plan_for_batch(batch)
     info = plan.info()
-    stream = torch.cuda.current_stream()
     out = torch.empty_like(batch.q)
 
-    def step():
-        plan.run(batch.q, batch.k_cache, batch.v_cache, out, stream)
-
-    for _ in range(args.warmup):
-        step()
-    if plan.check(stream) != 0:
-        raise RuntimeError("device error during warm-up")
-    torch.cuda.synchronize()
-
-    n_ev = args.steps
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev + 1)]
-    with ClockSampler(dev.index) as clk:
-        if ws > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        ev[0].record(stream)
-        for i in range(args.steps):
-            step()
-            ev[i + 1].record(stream)
-        torch.cuda.synchronize()
-        if ws > 1:
-            dist.barrier()
-    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(n_ev)]   # ms, one launch per step
-    elapsed_ms = ev[0].elapsed_time(ev[-1])
+    clk = ClockSampler(dev.index)
+    per, elapsed_ms = time_steps(plan, batch, out, args.steps, args.warmup, stream, ws, clk)
     if ws > 1:
         t = torch.tensor([elapsed_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         elapsed_ms = float(t.item())
-    if plan.check(stream) != 0:
-        raise RuntimeError("device error during the timed region")
 
     # end to end through the C ABI with host buffers (pinned), copies inside the region
     e2e_ms = None
@@ -258,37 +304,64 @@ def run_ours(args):
     kv_gbs = info["kv_bytes"] / avg_launch_s / 1e9
     tflops = info["attn_flops"] / avg_launch_s / 1e12
     io_bytes = tokens * batch.num_q_heads * batch.head_dim * 2
+    workload = f"{args.config}" + (f" (first {args.seqs} sequences)" if args.seqs else "")
+    rl = roofline(info, avg_launch_s, peaks)
+    rl.update({"traffic": kernel_traffic(workload), "kernel": "attn_kernel",
+               "peak_source": peaks["source"],
+               "per_launch": "algorithmic work of one attn_run (one kernel launch) / its mean CUDA-event time"})
+    plan.close()
+    del batch, out
 
-    result = None
+    # the other benchmark batches, same measurement (one launch per step)
+    per_config = {}
+    if ws == 1 and not args.seqs and not args.no_other_configs:
+        for name in ("llama3_8b_decode", "llama33_70b_prefill", "long_ctx_split"):
+            if name == args.config:
+                continue
+            b = W.make_config(name, device=dev, keep_contiguous=False)
+            pl = pk.plan_for_batch(b)
+            inf = pl.info()
+            o = torch.empty_like(b.q)
+            ps, _ = time_steps(pl, b, o, args.other_steps, args.warmup, stream)
+            sec = sum(ps) / len(ps) * 1e-3
+            per_config[name] = {"ms_per_launch": sec * 1e3, "tokens_per_s": b.total_q / sec,
+                                "kv_gbs": inf["kv_bytes"] / sec / 1e9,
+                                "attn_tflops": inf["attn_flops"] / sec / 1e12,
+                                "roofline": roofline(inf, sec, peaks)}
+            pl.close()
+            del b, o
+            torch.cuda.empty_cache()
+
     if rank == 0:
         cpu = None
         if ws == 1 and not args.no_cpu_baseline:
-            runner = OracleRunner(batch)
+            b = W.make_config(args.config, device=dev, max_seqs=args.seqs)
+            runner = OracleRunner(b)
             tk, sec = runner.run(args.cpu_seconds)
             cpu = {"value": tk / sec, "unit": "tokens/s", "cores": runner.threads, "kind": "oracle",
                    "sample": runner.sample_text()}
+            del b
         result = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{args.config}: {WORKLOADS[args.config]}"
-                       + (f" (first {args.seqs} sequences)" if args.seqs else ""),
+            "config": {"workload": f"{workload}: {WORKLOADS[args.config]}",
                        "query_tokens_per_step": tokens, "kv_bytes_per_step": info["kv_bytes"],
+                       "attn_flops_per_step": info["attn_flops"],
                        "l2": "inputs larger than L2 (KV cache read each step exceeds 126 MB)",
                        "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
             "kv_gbs": kv_gbs, "kv_frac_of_hbm": kv_gbs / peaks["hbm_gbs"], "prefill_tflops": tflops,
-            "roofline": {"bound": "hbm", "achieved": kv_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": kv_gbs / peaks["hbm_gbs"], "traffic": None,
-                         "kernel": "decode_kernel", "peak_source": peaks["source"]},
+            "roofline": rl,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
                     "d2h_bytes_per_step": io_bytes},
-            "gpu_launches": args.steps * 1,
+            "gpu_launches": args.steps,
             "clocks": clk.summary(),
-            "plan": {k: info[k] for k in ("num_decode_items", "num_split_units", "decode_rows")},
+            "plan": {k: info[k] for k in ("num_decode_items", "num_prefill_items", "num_split_units",
+                                          "decode_rows")},
+            "per_config": per_config,
         }
         print(json.dumps(result))
-    plan.close()
     if ws > 1:
         dist.destroy_process_group()
     return 0
@@ -297,12 +370,15 @@ def run_ours(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the per-config table of the other benchmark batches")
+    ap.add_argument("--other-steps", type=int, default=50)
     ap.add_argument("--seqs", type=int, default=None,
                     help="keep only the first N sequences of the batch (smaller profiler captures)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
