@@ -110,6 +110,22 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest `value` over all ranks (the job's time is its slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, steps: int, max_ms: float, world: int) -> float:
+    """Whole-job rate: the units every rank processed, over the slowest rank's time."""
+    return world * units_per_rank * steps / (max_ms * 1e-3)
+
+
 class OracleRunner:
     """The float64 oracle, as it stands, run over whole sequences of a batch in a cycle.
 
@@ -270,10 +286,7 @@ def run_ours(args):
 
     clk = ClockSampler(dev.index)
     per, elapsed_ms = time_steps(plan, batch, out, args.steps, args.warmup, stream, ws, clk)
-    if ws > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dev)
 
     # end to end through the C ABI with host buffers (pinned), copies inside the region
     e2e_ms = None
@@ -291,15 +304,11 @@ def run_ours(args):
             plan.run_host(q_host, batch.k_cache, batch.v_cache, o_host, stream)
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-        if ws > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
 
     tokens = batch.total_q
-    value = ws * tokens * args.steps / (elapsed_ms * 1e-3)
-    e2e_value = ws * tokens * args.steps / (e2e_ms * 1e-3) if e2e_ms else None
+    value = job_throughput(tokens, args.steps, elapsed_ms, ws)
+    e2e_value = job_throughput(tokens, args.steps, e2e_ms, ws) if e2e_ms else None
     avg_launch_s = (sum(per) / len(per)) * 1e-3
     kv_gbs = info["kv_bytes"] / avg_launch_s / 1e9
     tflops = info["attn_flops"] / avg_launch_s / 1e12

@@ -1,0 +1,66 @@
+"""The multi-rank plumbing of bench.py on CPU with gloo (world size 2): the job's time is
+the slowest rank's, throughput counts every rank's units, and the reference arm runs on
+rank 0 only (the other ranks exit 0 without work or output). Each rank of the GPU
+benchmark is an independent replica, so no data crosses ranks."""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    import bench
+    ws, r, local = bench.dist_env()
+    slow = bench.max_over_ranks(10.0 + 5.0 * rank)          # rank 1 is the slow one
+    q.put((r, ws, local, slow, bench.job_throughput(100, 4, slow, ws)))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_job_throughput_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, (r, ws, local, slow, thr) in enumerate(res):
+        assert (r, ws, local) == (rank, 2, rank)
+        assert slow == 15.0                                  # the slowest rank's time
+        assert thr == pytest.approx(2 * 100 * 4 / 15e-3)     # all ranks' units / that time
+
+
+def test_single_process_defaults():
+    import bench
+    assert bench.max_over_ranks(3.5) == 3.5
+    assert bench.job_throughput(10, 2, 4.0, 1) == pytest.approx(5000.0)
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "3", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == ""
