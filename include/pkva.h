@@ -180,6 +180,17 @@ PKVA_API int attn_run_static(int num_seqs, const int32_t* seq_lens, const int32_
                              const void* q, const void* k_cache, const void* v_cache, void* out,
                              void* stream);
 
+/*
+ * pkva_selftest_wait_timeout — exercise the bounded device wait (diagnostic).
+ *
+ * Launches one block that waits, with the kernels' polling loop, on an mbarrier nothing
+ * completes, giving up after `limit_ns` (0 < limit_ns <= 1 s). Synchronizes the device.
+ * On return *device_error holds PKVA_DEVERR_TIMEOUT if the wait gave up as it must (and
+ * 0 otherwise). Returns PKVA_OK, PKVA_EINVAL or PKVA_ECUDA. Not part of the attention
+ * path; it shows that a stuck asynchronous copy ends in an error word, not a hang.
+ */
+PKVA_API int pkva_selftest_wait_timeout(long long limit_ns, int32_t* device_error);
+
 /* Summary of a plan's decomposition (for logging and tests). */
 typedef struct pkva_plan_info {
     int32_t num_seqs;

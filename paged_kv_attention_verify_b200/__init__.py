@@ -32,7 +32,8 @@ DEVERR_TIMEOUT = 0x2
 
 # every entry point that include/pkva.h declares
 EXPORTED = ["attn_plan", "attn_run", "attn_run_host", "attn_check", "attn_plan_destroy",
-            "attn_last_error", "attn_plan_get_info", "attn_plan_inspect", "attn_run_static"]
+            "attn_last_error", "attn_plan_get_info", "attn_plan_inspect", "attn_run_static",
+            "pkva_selftest_wait_timeout"]
 
 
 class PkvaError(RuntimeError):
@@ -87,8 +88,9 @@ def lib() -> ctypes.CDLL:
     L.attn_run_static.argtypes = [ctypes.c_int, _i32p, _i32p, _vp, ctypes.c_int, ctypes.c_int, _i32p,
                                   _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                   ctypes.c_float, _vp, _vp, _vp, _vp, _vp]
+    L.pkva_selftest_wait_timeout.argtypes = [ctypes.c_longlong, _i32p]
     for name in ("attn_plan", "attn_run", "attn_run_host", "attn_check", "attn_plan_get_info",
-                 "attn_plan_inspect", "attn_run_static"):
+                 "attn_plan_inspect", "attn_run_static", "pkva_selftest_wait_timeout"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -237,6 +239,13 @@ def run_static(seq_lens, query_lens, block_table, mask_kind, parents, q, k_cache
                                  q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), out.data_ptr(),
                                  _stream_handle(stream)))
     return out
+
+
+def selftest_wait_timeout(limit_ns: int = 20_000_000) -> int:
+    """Run the bounded-wait self-test; returns the device error bits it reported."""
+    err = ctypes.c_int32(0)
+    _check(lib().pkva_selftest_wait_timeout(int(limit_ns), ctypes.byref(err)))
+    return int(err.value)
 
 
 def plan_for_batch(batch, sm_scale: Optional[float] = None) -> Plan:

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def header_symbols():
     src = open(os.path.join(ROOT, "include", "pkva.h")).read()
-    return sorted(set(re.findall(r"PKVA_API\s+[\w\s\*]*?\b(attn_\w+)\s*\(", src)))
+    return sorted(set(re.findall(r"PKVA_API\s+[\w\s\*]*?\b((?:attn|pkva)_\w+)\s*\(", src)))
 
 
 def test_library_exports_every_declared_symbol():
