@@ -27,9 +27,10 @@
  *   block_table int32 [num_seqs, bt_stride]; entry (s, p) is the physical page that holds
  *               keys p*page_size .. p*page_size+page_size-1 of sequence s. Entries past
  *               ceil(L_s / page_size) are never read.
- *   The K/V of the new tokens must already be in the cache (at positions L_s-T_s .. L_s-1).
- *   Cache slots past L_s in a sequence's last page are never attended to but are read by
- *   the tensor-core path; they must hold finite values (any stale bf16 data is fine).
+ *   For attn_run the K/V of the new tokens must already be in the cache (at positions
+ *   L_s-T_s .. L_s-1); attn_run_append writes them there itself. Cache slots past L_s in a
+ *   sequence's last page are loaded but never attended to and never reach the result, so
+ *   they may hold any bytes (stale data, NaN).
  *
  * Threading and errors: every call returns a pkva_status. On failure, attn_last_error()
  * returns a message for the calling thread. A plan may be used from one stream at a time;
@@ -134,6 +135,36 @@ PKVA_API int attn_run(pkva_plan_t plan, const void* q, const void* k_cache, cons
  */
 PKVA_API int attn_run_host(pkva_plan_t plan, const void* q_host, const void* k_cache,
                   const void* v_cache, void* out_host, void* stream);
+
+/*
+ * attn_run_append — write the new tokens' K/V into the paged cache and compute the batch's
+ * attention, in one launch on `stream` (asynchronous).
+ *
+ * Cites: XY-Serve verdict page, core_discovery (every step appends the new tokens' keys
+ * and values to the paged block cache that later steps read; chunked prefill extends a
+ * cached prefix) and forward_implications[2] (one attention kernel for all row kinds).
+ *
+ *   q          device bf16 [sum T_s, Hq, D], as for attn_run.
+ *   k_new,
+ *   v_new      device bf16 [sum T_s, Hkv, D]: the new tokens' keys and values, in q's token
+ *              order (the K/V of query row i of sequence s belong at position L_s - T_s + i).
+ *   k_cache,
+ *   v_cache    device bf16 [num_pages, Hkv, page_size, D]. Slots of the new tokens
+ *              (positions L_s - T_s .. L_s - 1, through the block table) are WRITTEN with
+ *              k_new / v_new; every other slot is only read. Their previous contents are
+ *              never used, so they may hold anything.
+ *   out        device bf16 [sum T_s, Hq, D].
+ *
+ * The result equals writing k_new / v_new into the cache and then calling attn_run: the
+ * attention reads the new tokens' K/V from k_new / v_new, so no task depends on another's
+ * cache writes. The pages holding the new tokens must be distinct for distinct sequences
+ * (a page shared by two sequences would be written twice). All pointers 16-byte aligned;
+ * k_new / v_new must not overlap the caches or out. Errors as attn_run; an out-of-range
+ * block-table entry skips that slot's write and sets PKVA_DEVERR_BAD_PAGE. Needs the
+ * tensor-core decode body (PKVA_EUNSUPPORTED when PKVA_DECODE_BODY=fma).
+ */
+PKVA_API int attn_run_append(pkva_plan_t plan, const void* q, const void* k_new, const void* v_new,
+                    void* k_cache, void* v_cache, void* out, void* stream);
 
 /*
  * attn_check — synchronize `stream`, read and clear the plan's device error word.

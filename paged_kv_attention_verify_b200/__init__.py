@@ -31,7 +31,7 @@ DEVERR_BAD_PAGE = 0x1
 DEVERR_TIMEOUT = 0x2
 
 # every entry point that include/pkva.h declares
-EXPORTED = ["attn_plan", "attn_run", "attn_run_host", "attn_check", "attn_plan_destroy",
+EXPORTED = ["attn_plan", "attn_run", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_destroy",
             "attn_last_error", "attn_plan_get_info", "attn_plan_inspect", "attn_run_static",
             "pkva_selftest_wait_timeout"]
 
@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
                             ctypes.c_int, _i32p, _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                             ctypes.c_int, ctypes.c_float]
     L.attn_run.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp]
+    L.attn_run_append.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
     L.attn_run_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp]
     L.attn_check.argtypes = [_vp, _vp, _i32p]
     L.attn_plan_destroy.argtypes = [_vp]
@@ -89,7 +90,7 @@ def lib() -> ctypes.CDLL:
                                   _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                   ctypes.c_float, _vp, _vp, _vp, _vp, _vp]
     L.pkva_selftest_wait_timeout.argtypes = [ctypes.c_longlong, _i32p]
-    for name in ("attn_plan", "attn_run", "attn_run_host", "attn_check", "attn_plan_get_info",
+    for name in ("attn_plan", "attn_run", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_get_info",
                  "attn_plan_inspect", "attn_run_static", "pkva_selftest_wait_timeout"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -167,6 +168,23 @@ class Plan:
         self._check_tensors(q, k_cache, v_cache, out)
         _check(lib().attn_run(self._handle, q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
                               out.data_ptr(), _stream_handle(stream)))
+        return out
+
+    def run_append(self, q, k_new, v_new, k_cache, v_cache, out=None, stream=None):
+        """Write the new tokens' K/V (``k_new``/``v_new`` [sum T, Hkv, D]) into the cache and
+        compute the attention, in one launch (``attn_run_append``)."""
+        import torch
+        if out is None:
+            out = torch.empty_like(q)
+        self._check_tensors(q, k_cache, v_cache, out)
+        shape = (self.total_q, self.num_kv_heads, self.head_dim)
+        for name, t in (("k_new", k_new), ("v_new", v_new)):
+            if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.bfloat16 \
+                    or tuple(t.shape) != shape or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor {shape}")
+        _check(lib().attn_run_append(self._handle, q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(),
+                                     k_cache.data_ptr(), v_cache.data_ptr(), out.data_ptr(),
+                                     _stream_handle(stream)))
         return out
 
     def run_host(self, q_host, k_cache, v_cache, out_host, stream=None):

@@ -68,7 +68,8 @@ static bool encode_cache_map(CUtensorMap* map, const void* base, int num_pages, 
 }
 
 // q viewed as the 3-D bf16 tensor [sum T][Hq][D]; one box is 128 tokens x 64 columns of
-// one head, stored with the 128-byte swizzle (the prefill kernel's A operand layout).
+// one head, stored with the 128-byte swizzle (the prefill kernel's A operand layout). The
+// new tokens' K and V ([sum T][Hkv][D]) use the same view with Hkv heads.
 static bool encode_q_map(CUtensorMap* map, const void* base, int total_q, int Hq, int D) {
     auto fn = tensor_map_encoder();
     if (!fn) return false;
@@ -119,6 +120,9 @@ struct pkva_plan {
     CUtensorMap tmK, tmV;
     const void* tm_k = nullptr;
     const void* tm_v = nullptr;
+    CUtensorMap tmKn, tmVn;                 // the new tokens' K / V (fused append)
+    const void* tm_kn = nullptr;
+    const void* tm_vn = nullptr;
     int64_t scratch_bytes = 0;
 };
 
@@ -287,43 +291,65 @@ extern "C" int attn_plan_get_info(pkva_plan_t plan, pkva_plan_info* info) {
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-extern "C" int attn_run(pkva_plan_t plan, const void* q, const void* k_cache, const void* v_cache, void* out,
-                        void* stream) {
+static int run_impl(pkva_plan_t plan, const void* q, const void* k_new, const void* v_new, const void* k_cache,
+                    const void* v_cache, void* out, void* stream, const char* who) {
+    const std::string name(who);
     if (!plan) {
-        set_last_error("attn_run: plan is NULL");
+        set_last_error(name + ": plan is NULL");
         return PKVA_EINVAL;
     }
     const HostPlan& hp = plan->hp;
+    const bool append = k_new != nullptr || v_new != nullptr;
     if (hp.num_seqs == 0) return PKVA_OK;
-    if (!q || !k_cache || !v_cache || !out) {
-        set_last_error("attn_run: NULL tensor pointer");
+    if (!q || !k_cache || !v_cache || !out || (append && (!k_new || !v_new))) {
+        set_last_error(name + ": NULL tensor pointer");
         return PKVA_EINVAL;
     }
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) {
-        set_last_error("attn_run: tensor pointers must be 16-byte aligned");
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        (append && (!aligned16(k_new) || !aligned16(v_new)))) {
+        set_last_error(name + ": tensor pointers must be 16-byte aligned");
         return PKVA_EINVAL;
+    }
+    if (append && !plan->decode_mma) {
+        set_last_error(name + ": the fused append runs on the tensor-core decode body only (PKVA_DECODE_BODY=fma)");
+        return PKVA_EUNSUPPORTED;
     }
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (plan->tm_k != k_cache) {
         if (!encode_cache_map(&plan->tmK, k_cache, hp.num_pages, hp.Hkv, hp.D)) {
-            set_last_error("attn_run: cuTensorMapEncodeTiled failed for k_cache");
+            set_last_error(name + ": cuTensorMapEncodeTiled failed for k_cache");
             return PKVA_ECUDA;
         }
         plan->tm_k = k_cache;
     }
     if (plan->tm_v != v_cache) {
         if (!encode_cache_map(&plan->tmV, v_cache, hp.num_pages, hp.Hkv, hp.D)) {
-            set_last_error("attn_run: cuTensorMapEncodeTiled failed for v_cache");
+            set_last_error(name + ": cuTensorMapEncodeTiled failed for v_cache");
             return PKVA_ECUDA;
         }
         plan->tm_v = v_cache;
     }
-    if (!hp.pwork.empty() && plan->tm_q != q) {
+    const bool has_prefill = !hp.pwork.empty();
+    if (has_prefill && plan->tm_q != q) {
         if (!encode_q_map(&plan->tmQ, q, hp.total_q, hp.Hq, hp.D)) {
-            set_last_error("attn_run: cuTensorMapEncodeTiled failed for q");
+            set_last_error(name + ": cuTensorMapEncodeTiled failed for q");
             return PKVA_ECUDA;
         }
         plan->tm_q = q;
+    }
+    if (has_prefill && append && plan->tm_kn != k_new) {
+        if (!encode_q_map(&plan->tmKn, k_new, hp.total_q, hp.Hkv, hp.D)) {
+            set_last_error(name + ": cuTensorMapEncodeTiled failed for k_new");
+            return PKVA_ECUDA;
+        }
+        plan->tm_kn = k_new;
+    }
+    if (has_prefill && append && plan->tm_vn != v_new) {
+        if (!encode_q_map(&plan->tmVn, v_new, hp.total_q, hp.Hkv, hp.D)) {
+            set_last_error(name + ": cuTensorMapEncodeTiled failed for v_new");
+            return PKVA_ECUDA;
+        }
+        plan->tm_vn = v_new;
     }
     PrefillParams pp;
     pp.out = static_cast<__nv_bfloat16*>(out);
@@ -355,17 +381,26 @@ extern "C" int attn_run(pkva_plan_t plan, const void* q, const void* k_cache, co
     dp.G = hp.G;
     dp.num_pages = hp.num_pages;
     dp.scale_log2 = pp.scale_log2;
+    if (append) {
+        pp.append = dp.append = 1;
+        pp.k_new = dp.k_new = static_cast<const __nv_bfloat16*>(k_new);
+        pp.v_new = dp.v_new = static_cast<const __nv_bfloat16*>(v_new);
+        // the cache is written only at the new tokens' slots, which no task reads
+        pp.k_cache = dp.k_cache = static_cast<__nv_bfloat16*>(const_cast<void*>(k_cache));
+        pp.v_cache = dp.v_cache = static_cast<__nv_bfloat16*>(const_cast<void*>(v_cache));
+    }
     AttnParams ap;
     ap.pre = pp;
     ap.dec = dp;
-    const bool has_prefill = !hp.pwork.empty();
+    const CUtensorMap& tmKn = append ? plan->tmKn : plan->tmQ;
+    const CUtensorMap& tmVn = append ? plan->tmVn : plan->tmQ;
     cudaError_t e;
     if (plan->decode_mma) {
         // the whole batch in one launch
         ap.order = plan->d_order;
         ap.num_blocks = (int32_t)hp.order.size();
         ap.num_decode = (int32_t)hp.dwork.size();
-        e = launch_attn(ap, hp.D, hp.decode_rows, has_prefill, plan->tmQ, plan->tmK, plan->tmV, st);
+        e = launch_attn(ap, hp.D, hp.decode_rows, has_prefill, plan->tmQ, plan->tmK, plan->tmV, tmKn, tmVn, st);
     } else {
         // comparison mode: decode tasks on the CUDA-core kernel, prefill tasks after them
         e = launch_decode(dp, (int)hp.dwork.size(), hp.D, hp.decode_rows, false, plan->tmK, plan->tmV, st);
@@ -373,11 +408,25 @@ extern "C" int attn_run(pkva_plan_t plan, const void* q, const void* k_cache, co
             ap.order = plan->d_order_prefill;
             ap.num_blocks = (int32_t)hp.pwork.size();
             ap.num_decode = 0;
-            e = launch_attn(ap, hp.D, hp.decode_rows, has_prefill, plan->tmQ, plan->tmK, plan->tmV, st);
+            e = launch_attn(ap, hp.D, hp.decode_rows, has_prefill, plan->tmQ, plan->tmK, plan->tmV, tmKn, tmVn, st);
         }
     }
-    if (e != cudaSuccess) return cuda_fail(e, "attn_run: launch");
+    if (e != cudaSuccess) return cuda_fail(e, (name + ": launch").c_str());
     return PKVA_OK;
+}
+
+extern "C" int attn_run(pkva_plan_t plan, const void* q, const void* k_cache, const void* v_cache, void* out,
+                        void* stream) {
+    return run_impl(plan, q, nullptr, nullptr, k_cache, v_cache, out, stream, "attn_run");
+}
+
+extern "C" int attn_run_append(pkva_plan_t plan, const void* q, const void* k_new, const void* v_new, void* k_cache,
+                               void* v_cache, void* out, void* stream) {
+    if (plan && plan->hp.num_seqs > 0 && (!k_new || !v_new)) {
+        set_last_error("attn_run_append: k_new / v_new is NULL");
+        return PKVA_EINVAL;
+    }
+    return run_impl(plan, q, k_new, v_new, k_cache, v_cache, out, stream, "attn_run_append");
 }
 
 extern "C" int attn_run_host(pkva_plan_t plan, const void* q_host, const void* k_cache, const void* v_cache,

@@ -25,7 +25,7 @@ namespace {
 
 constexpr int kAttnThreads = 384;                 // prefill uses 352; decode 3 x 128
 constexpr int kDecWarps = 4;                      // page-streaming warps per decode task
-static_assert(kAttnThreads >= pre::kPThreads, "block too small for a prefill task");
+static_assert(kAttnThreads >= pre::kPThreadsAppend, "block too small for a prefill task");
 static_assert(kAttnThreads == kDecTasksPerBlock * 128, "one 128-thread group per decode task");
 
 template <int D>
@@ -46,13 +46,14 @@ struct AttnSmem {
 template <int D, int NT>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-            const __grid_constant__ CUtensorMap tmV) {
+            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKn,
+            const __grid_constant__ CUtensorMap tmVn) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int e = p.order[blockIdx.x];
     if constexpr (D == 128) {
         if (e >= 0) {
-            pre::prefill_task(p.pre, e, tmQ, tmK, tmV, sm);
+            pre::prefill_task(p.pre, e, tmQ, tmK, tmV, tmKn, tmVn, sm);
             return;
         }
     }
@@ -67,14 +68,14 @@ attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const _
 }
 
 template <int D, int NT>
-cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                     const CUtensorMap& tmV, cudaStream_t stream) {
+cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                     const CUtensorMap& tmKn, const CUtensorMap& tmVn, cudaStream_t stream) {
     using S = AttnSmem<D, NT>;
     cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::ALLOC);
     if (e != cudaSuccess) return e;
     const int grid = p.num_blocks;
     if (grid == 0) return cudaSuccess;
-    attn_kernel<D, NT><<<grid, kAttnThreads, S::ALLOC, stream>>>(p, tmQ, tmK, tmV);
+    attn_kernel<D, NT><<<grid, kAttnThreads, S::ALLOC, stream>>>(p, tmQ, tmK, tmV, tmKn, tmVn);
     return cudaGetLastError();
 }
 
@@ -100,12 +101,15 @@ int attn_ctas_per_sm(int D, int rows) {
 }
 
 cudaError_t launch_attn(const AttnParams& p, int D, int rows, bool has_prefill, const CUtensorMap& tmQ,
-                        const CUtensorMap& tmK, const CUtensorMap& tmV, cudaStream_t stream) {
+                        const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKn,
+                        const CUtensorMap& tmVn, cudaStream_t stream) {
     if (D == 64) {
         if (has_prefill) return cudaErrorInvalidValue;   // prefill tasks need head_dim 128
-        return rows <= 8 ? launch_t<64, 1>(p, tmQ, tmK, tmV, stream) : launch_t<64, 2>(p, tmQ, tmK, tmV, stream);
+        return rows <= 8 ? launch_t<64, 1>(p, tmQ, tmK, tmV, tmKn, tmVn, stream)
+                         : launch_t<64, 2>(p, tmQ, tmK, tmV, tmKn, tmVn, stream);
     }
-    return rows <= 8 ? launch_t<128, 1>(p, tmQ, tmK, tmV, stream) : launch_t<128, 2>(p, tmQ, tmK, tmV, stream);
+    return rows <= 8 ? launch_t<128, 1>(p, tmQ, tmK, tmV, tmKn, tmVn, stream)
+                     : launch_t<128, 2>(p, tmQ, tmK, tmV, tmKn, tmVn, stream);
 }
 
 }  // namespace pkva

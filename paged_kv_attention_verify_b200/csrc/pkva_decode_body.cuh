@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include "pkva.h"
+#include "pkva_append.cuh"
 #include "pkva_kernels.h"
 #include "pkva_ptx.cuh"
 
@@ -314,6 +315,12 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
         uint8_t* Ks = ring + stage * C::STAGE_BYTES;
         uint8_t* Vs = Ks + C::PAGE_BYTES;
         const int kbase = (w.page_begin + warp + NW * i) * kPageSize;
+        if (p.append && kbase + kPageSize > prefix && kbase < si.seq_len) {
+            // fused append: the new tokens' rows come from the dense input, not the cache
+            const int r0 = max(prefix - kbase, 0), r1 = min(si.seq_len - kbase, kPageSize);
+            patch_page_rows<D>(Ks, Vs, p.k_new, p.v_new, si, p.Hkv, w.kv_head, r0, r1, kbase + r0 - prefix, lane);
+            __syncwarp();
+        }
 
         // -- S^T = K Q^T (16 keys x 8 rows per n-tile) ------------------------------------
         float s[NT][4];
@@ -469,6 +476,9 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
     }
     grp.sync();
     merge_and_store<D, NR, NW>(grp, p, w, cm, cl, co, rout, flag);
+    if (p.append && w.row_begin == 0 && w.split <= 0)   // one task per (sequence, KV head)
+        append_rows<D>(p.k_new, p.v_new, p.k_cache, p.v_cache, p.block_table, p.bt_stride, p.num_pages, p.Hkv,
+                       p.err, si, w.seq, w.kv_head, 0, si.query_len, tid, grp.n);
 }
 
 // =====================================================================================
@@ -556,9 +566,14 @@ __device__ __forceinline__ void decode_fma_task(const Group& grp, const DecodePa
             ok = false;
             break;
         }
-        const uint8_t* Ks = ring + stage * C::STAGE_BYTES;
-        const uint8_t* Vs = Ks + C::PAGE_BYTES;
+        uint8_t* Ks = ring + stage * C::STAGE_BYTES;
+        uint8_t* Vs = Ks + C::PAGE_BYTES;
         const int kbase = (w.page_begin + warp + NW * i) * kPageSize;
+        if (p.append && kbase + kPageSize > prefix && kbase < si.seq_len) {
+            const int r0 = max(prefix - kbase, 0), r1 = min(si.seq_len - kbase, kPageSize);
+            patch_page_rows<D>(Ks, Vs, p.k_new, p.v_new, si, p.Hkv, w.kv_head, r0, r1, kbase + r0 - prefix, lane);
+            __syncwarp();
+        }
 
         // -- scores: lane (j, hh) sums half hh of <q_r, k_j> for every row r ------------
         float acc[NR];
@@ -709,6 +724,9 @@ __device__ __forceinline__ void decode_fma_task(const Group& grp, const DecodePa
     }
     grp.sync();
     merge_and_store<D, NR, NW>(grp, p, w, cm, cl, co, rout, flag);
+    if (p.append && w.row_begin == 0 && w.split <= 0)   // one task per (sequence, KV head)
+        append_rows<D>(p.k_new, p.v_new, p.k_cache, p.v_cache, p.block_table, p.bt_stride, p.num_pages, p.Hkv,
+                       p.err, si, w.seq, w.kv_head, 0, si.query_len, tid, grp.n);
 }
 
 

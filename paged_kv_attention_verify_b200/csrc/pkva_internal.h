@@ -54,7 +54,11 @@ struct PrefillWork {
     int32_t ntok;
     int32_t kv_tiles0;
     int32_t kv_tiles1;
-    int32_t pad0, pad1;
+    // with a fused KV append, keys come from the cache for the committed prefix (tiles
+    // aligned at key 0) and from the new tokens' input for the chunk (tiles aligned at the
+    // chunk start): the tile counts of the two query tiles in that mode
+    int32_t kv_tiles0_append;
+    int32_t kv_tiles1_append;
 };
 static_assert(sizeof(PrefillWork) == 32, "PrefillWork layout");
 

@@ -25,6 +25,12 @@ struct DecodeParams {
     int32_t Hq, Hkv, G;
     int32_t num_pages;
     float scale_log2;            // softmax scale * log2(e)
+    // fused KV append (attn_run_append): the new tokens' K/V, in q's token order
+    int32_t append = 0;
+    const __nv_bfloat16* k_new = nullptr;  // [sum T, Hkv, D]
+    const __nv_bfloat16* v_new = nullptr;
+    __nv_bfloat16* k_cache = nullptr;      // written at the new tokens' slots
+    __nv_bfloat16* v_cache = nullptr;
 };
 
 struct PrefillParams {
@@ -37,6 +43,11 @@ struct PrefillParams {
     int32_t Hq, Hkv, G;
     int32_t num_pages;
     float scale_log2;
+    int32_t append = 0;          // fused KV append: see DecodeParams
+    const __nv_bfloat16* k_new = nullptr;
+    const __nv_bfloat16* v_new = nullptr;
+    __nv_bfloat16* k_cache = nullptr;
+    __nv_bfloat16* v_cache = nullptr;
 };
 
 // Everything one launch of the unified attention kernel needs.
@@ -54,8 +65,10 @@ int attn_ctas_per_sm(int D, int rows);
 // Launch the unified kernel over p.num_blocks blocks in the order p.order (prefill tasks
 // need head_dim 128). tmQ views q as the 3-D tensor [sum T][Hq][128] with a
 // {64, 1, 128} box; tmK/tmV are the cache maps (16 x 64 boxes).
+// tmKn/tmVn view k_new/v_new like tmQ ({64, 1, 128} boxes); read only when p.pre.append.
 cudaError_t launch_attn(const AttnParams& p, int D, int rows, bool has_prefill, const CUtensorMap& tmQ,
-                        const CUtensorMap& tmK, const CUtensorMap& tmV, cudaStream_t stream);
+                        const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKn,
+                        const CUtensorMap& tmVn, cudaStream_t stream);
 
 // Resident CTAs per SM of the decode kernel compiled for (D, rows); 0 if unsupported.
 // `mma` selects the tensor-core page body, otherwise the CUDA-core one.

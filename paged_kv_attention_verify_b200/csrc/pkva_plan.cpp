@@ -133,6 +133,10 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
                 const int tiles0 = (prefix + t0 + n0tok + kPrefillTileN - 1) / kPrefillTileN;
                 const int tiles1 =
                     ntok > kPrefillTileM ? (prefix + t0 + ntok + kPrefillTileN - 1) / kPrefillTileN : 0;
+                const int cache_tiles = (prefix + kPrefillTileN - 1) / kPrefillTileN;
+                const int tiles0_app = cache_tiles + (t0 + n0tok - 1) / kPrefillTileN + 1;
+                const int tiles1_app =
+                    ntok > kPrefillTileM ? cache_tiles + (t0 + ntok - 1) / kPrefillTileN + 1 : 0;
                 for (int h = 0; h < a.Hq; ++h) {
                     PrefillWork pw{};
                     pw.seq = s;
@@ -141,6 +145,8 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
                     pw.ntok = ntok;
                     pw.kv_tiles0 = tiles0;
                     pw.kv_tiles1 = tiles1;
+                    pw.kv_tiles0_append = tiles0_app;
+                    pw.kv_tiles1_append = tiles1_app;
                     p.pwork.push_back(pw);
                 }
             }

@@ -17,6 +17,7 @@
 //              warpgroup runs its softmax, the tensor cores run the other tile's PV and
 //              next QK^T. PV takes P straight from TMEM as its A operand.
 //   warp 10    TMA producer of V tiles (2-stage ring, freed after both PV).
+//   warp 11    (fused KV append only) copies a share of the new rows into the cache.
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512); P_b lives in
 // columns [0,64) of S_b (bf16 pairs). Tensor-core operations of one issuing thread run in
 // issue order, so the next QK^T into S_b is issued right after the PV that reads P_b.
@@ -32,6 +33,7 @@
 #include <cuda_runtime.h>
 
 #include "pkva.h"
+#include "pkva_append.cuh"
 #include "pkva_kernels.h"
 #include "pkva_ptx.cuh"
 
@@ -40,6 +42,7 @@ namespace pre {
 
 
 constexpr int kPThreads = 352;
+constexpr int kPThreadsAppend = 384;                     // with the cache-writing warp
 constexpr int kD = 128;
 constexpr int kNK = 2;                                   // K stages
 constexpr int kNV = 2;                                   // V stages
@@ -49,8 +52,9 @@ constexpr int kOffQ = 0;                                 // Q0, Q1
 constexpr int kOffK = kOffQ + 2 * kTileBytes;
 constexpr int kOffV = kOffK + kNK * kTileBytes;
 constexpr int kOffBar = kOffV + kNV * kTileBytes;
-// q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2], p_full[2], o_ready[2], mma_done
-constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 2 + 2 + 2 + 1;
+// q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2], p_full[2], o_ready[2], mma_done,
+// v_fix
+constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 2 + 2 + 2 + 1 + 1;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kOffFlag = kOffTmemSlot + 16;
 constexpr int kSmemBytes = kOffFlag + 16;
@@ -96,6 +100,7 @@ struct Bars {
     uint64_t* p_full;
     uint64_t* o_ready;
     uint64_t* mma_done;
+    uint64_t* v_fix;         // the V tile whose stale rows the producer zeroes first
 };
 
 __device__ __forceinline__ Bars bars_at(uint8_t* sm) {
@@ -110,6 +115,7 @@ __device__ __forceinline__ Bars bars_at(uint8_t* sm) {
     r.p_full = r.s_full + 2;
     r.o_ready = r.p_full + 2;
     r.mma_done = r.o_ready + 2;
+    r.v_fix = r.mma_done + 1;
     return r;
 }
 
@@ -133,15 +139,15 @@ __device__ __forceinline__ bool spin_or_abort(uint64_t* bar, uint32_t parity, in
     return true;
 }
 
-// Physical cache rows of the 8 pages of KV tile j (row -16 reads as zeros: past the end of
-// the sequence, or a block-table entry out of range, which is also flagged).
-__device__ __forceinline__ void tile_rows(const PrefillParams& p, const int32_t* btrow, int seq_pages, int kvh,
+// Physical cache rows of the 8 pages of KV tile j (row -16 reads as zeros: a page with no
+// key below key_limit, or a block-table entry out of range, which is also flagged).
+__device__ __forceinline__ void tile_rows(const PrefillParams& p, const int32_t* btrow, int key_limit, int kvh,
                                           int j, int rows[8]) {
 #pragma unroll
     for (int pg = 0; pg < 8; ++pg) {
         const int lp = j * 8 + pg;
         int ph = -1;
-        if (lp < seq_pages) {
+        if (lp * kPageSize < key_limit) {
             ph = btrow[lp];
             if (ph < 0 || ph >= p.num_pages) {
                 atomicOr(p.err, PKVA_DEVERR_BAD_PAGE);
@@ -163,18 +169,26 @@ __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, 
 // One prefill task; every thread of the block (at least kPThreads) calls it; warps past
 // the V producer only take part in the block barriers. `sm` is the block's 1024-aligned
 // dynamic shared memory (kSmemBytes).
+// With p.append, KV tiles [0, nc) come from the cache (the committed prefix, keys at and past
+// it masked) and tiles [nc, n) from the new tokens' K/V through tmKn / tmVn (tiles aligned
+// at the chunk start), and warp 11 writes a share of the task's new rows into the cache.
 __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, const CUtensorMap& tmQ,
-                                             const CUtensorMap& tmK, const CUtensorMap& tmV, uint8_t* sm) {
+                                             const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                             const CUtensorMap& tmKn, const CUtensorMap& tmVn, uint8_t* sm) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const PrefillWork w = p.work[task];
     const SeqInfo si = p.seqs[w.seq];
     const Bars B = bars_at(sm);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffTmemSlot);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffFlag);
-    const int n0 = w.kv_tiles0, n1 = w.kv_tiles1;
+    const bool append = p.append != 0;
+    const int n0 = append ? w.kv_tiles0_append : w.kv_tiles0;
+    const int n1 = append ? w.kv_tiles1_append : w.kv_tiles1;
     const int nmax = n0 > n1 ? n0 : n1;
     const int kvh = w.q_head / p.G;
     const int prefix = si.seq_len - si.query_len;
+    const int nc = append ? (prefix + kPrefillTileN - 1) / kPrefillTileN : nmax;   // tiles read from the cache
+    const int key_limit = append ? prefix : si.seq_len;                            // cache keys that hold data
 
     if (tid == 0) {
         mbar_init(B.q_full, 1);
@@ -192,6 +206,7 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
             mbar_init(&B.o_ready[b], 1);
         }
         mbar_init(B.mma_done, 1);
+        mbar_init(B.v_fix, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -208,11 +223,14 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         // ------------------ TMA producers: warp 8 loads Q and K, warp 10 loads V ------------
         if (lane == 0) {
             const bool is_k = warp == kWarpKProd;
-            const int seq_pages = (si.seq_len + kPageSize - 1) / kPageSize;
             const int32_t* btrow = p.block_table + (int64_t)w.seq * p.bt_stride;
+            // the cache page holding key_limit has stale rows from key_limit on (when it is
+            // not page-aligned): the V tile with that page is zeroed there before its PV
+            const int fix_tile = (key_limit % kPageSize) ? key_limit / kPageSize / 8 : -1;
             if (is_k) {
                 prefetch_tensormap(&tmQ);
                 prefetch_tensormap(&tmK);
+                if (append) prefetch_tensormap(&tmKn);
                 const int qrow0 = si.q_start + w.tok0;
                 mbar_arrive_expect_tx(B.q_full, 2 * kTileBytes);
 #pragma unroll
@@ -223,6 +241,7 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
                                     w.q_head, qrow0 + b * kPrefillTileM);
             } else {
                 prefetch_tensormap(&tmV);
+                if (append) prefetch_tensormap(&tmVn);
             }
             const int NSt = is_k ? kNK : kNV;
             uint64_t* full = is_k ? B.k_full : B.v_full;
@@ -231,9 +250,34 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
             for (int j = 0; j < nmax; ++j) {
                 const int st = j % NSt;
                 if (j >= NSt && !wait_or_abort(&empty[st], ((j / NSt) - 1) & 1, p.err, abort_flag)) break;
+                uint8_t* dst = base + st * kTileBytes;
+                if (j >= nc) {
+                    // new tokens [128 (j - nc), +128) of the chunk, straight from the input
+                    const int row0 = si.q_start + (j - nc) * kPrefillTileN;
+                    mbar_arrive_expect_tx(&full[st], kTileBytes);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_3d(dst + h * kHalfBytes, is_k ? &tmKn : &tmVn, &full[st], h * 64, kvh, row0);
+                    continue;
+                }
                 int rows[8];
-                tile_rows(p, btrow, seq_pages, kvh, j, rows);
-                load_tile(base + st * kTileBytes, is_k ? &tmK : &tmV, &full[st], rows);
+                tile_rows(p, btrow, key_limit, kvh, j, rows);
+                if (is_k || j != fix_tile) {
+                    load_tile(dst, is_k ? &tmK : &tmV, &full[st], rows);
+                    continue;
+                }
+                load_tile(dst, &tmV, B.v_fix, rows);
+                if (!wait_or_abort(B.v_fix, 0, p.err, abort_flag)) break;
+                const int pg = (key_limit / kPageSize) % 8;
+                for (int r = key_limit % kPageSize; r < kPageSize; ++r)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            *reinterpret_cast<uint4*>(dst + h * kHalfBytes + (pg * kPageSize + r) * 128 + c * 16) =
+                                make_uint4(0u, 0u, 0u, 0u);
+                fence_proxy_async_smem();
+                mbar_arrive(&full[st]);
             }
         }
     } else if (warp == kWarpMma) {
@@ -325,6 +369,9 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         const bool real_row = row_in_task < w.ntok;
         const int lim = real_row ? prefix + tok : 0x7fffffff;        // last visible key of this row
         const int lim_first = prefix + w.tok0 + b * kPrefillTileM;    // the tile's first row
+        // append mode: the cache tiles show keys [0, prefix) to every row; the new tiles are
+        // indexed from the chunk start, so a row sees new keys up to its own token index
+        const int lim_new = tok, lim_first_new = w.tok0 + b * kPrefillTileM;
         float m_ref = -INFINITY, l_sum = 0.f;
         bool alive = true;
         // every break below is taken by the whole warp (tcgen05.ld/st are warp-collective)
@@ -339,9 +386,18 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
 #pragma unroll
             for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
             tmem_wait_ld();
-            const int kb = j * kPrefillTileN;
-            if (kb + kPrefillTileN - 1 > lim_first) {          // tile crosses the diagonal
-                const int vis = lim - kb;                          // columns <= vis are visible
+            int kb = j * kPrefillTileN, lim_j = lim, lim_first_j = lim_first;
+            if (append) {
+                if (j < nc) {
+                    lim_j = lim_first_j = prefix - 1;
+                } else {
+                    kb = (j - nc) * kPrefillTileN;
+                    lim_j = lim_new;
+                    lim_first_j = lim_first_new;
+                }
+            }
+            if (kb + kPrefillTileN - 1 > lim_first_j) {        // tile crosses the diagonal
+                const int vis = lim_j - kb;                        // columns <= vis are visible
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
                     if (c > vis) sr[c] = __float_as_uint(-INFINITY);
@@ -430,6 +486,14 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
                 }
             }
         }
+    } else if (append) {
+        // ------------------- warp 11: this task's share of the cache writes -------------------
+        // the G query-head tasks of one KV head and token range each write 1/G of its rows
+        const int gi = w.q_head % p.G;
+        const int t_begin = w.tok0 + (int)((int64_t)w.ntok * gi / p.G);
+        const int t_end = w.tok0 + (int)((int64_t)w.ntok * (gi + 1) / p.G);
+        append_rows<kD>(p.k_new, p.v_new, p.k_cache, p.v_cache, p.block_table, p.bt_stride, p.num_pages, p.Hkv,
+                        p.err, si, w.seq, kvh, t_begin, t_end, lane, 32);
     }
     // all roles done (the MMA thread waited for its last MMA); release TMEM
     tc_fence_before();

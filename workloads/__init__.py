@@ -231,6 +231,42 @@ def build_batch(name: str, seqs: Sequence[SeqSpec], num_q_heads: int, num_kv_hea
                  seed=seed, outlier_frac=outlier_frac)
 
 
+def new_token_slots(batch: Batch):
+    """Physical (page, slot) of every new token, in q's token order (positions
+    L - T .. L - 1 of each sequence through its block table)."""
+    bt = batch.block_table.cpu()
+    pages, slots = [], []
+    for i, s in enumerate(batch.seqs):
+        pos = torch.arange(s.seq_len - s.query_len, s.seq_len)
+        pages.append(bt[i, pos // batch.page_size].long())
+        slots.append(pos % batch.page_size)
+    dev = batch.k_cache.device
+    return torch.cat(pages).to(dev), torch.cat(slots).to(dev)
+
+
+def tail_slots(batch: Batch):
+    """Physical (page, slot) of the unused slots past L in each sequence's last page."""
+    bt = batch.block_table.cpu()
+    pages, slots = [], []
+    for i, s in enumerate(batch.seqs):
+        n = (-s.seq_len) % batch.page_size
+        if n:
+            pos = torch.arange(s.seq_len, s.seq_len + n)
+            pages.append(bt[i, pos // batch.page_size].long())
+            slots.append(pos % batch.page_size)
+    dev = batch.k_cache.device
+    if not pages:
+        return torch.zeros(0, dtype=torch.long, device=dev), torch.zeros(0, dtype=torch.long, device=dev)
+    return torch.cat(pages).to(dev), torch.cat(slots).to(dev)
+
+
+def new_token_kv(batch: Batch):
+    """The new tokens' K and V as dense [sum T, Hkv, d] tensors in q's token order (the
+    inputs of a fused cache append), read from the cache where the batch placed them."""
+    pg, sl = new_token_slots(batch)
+    return batch.k_cache[pg, :, sl].contiguous(), batch.v_cache[pg, :, sl].contiguous()
+
+
 def make_config(name: str, device="cpu", seed: Optional[int] = None,
                 keep_contiguous: bool = True, max_seqs: Optional[int] = None) -> Batch:
     """One of the five named batches, seeded by its index unless ``seed`` is given.
