@@ -227,6 +227,21 @@ def time_steps(plan, batch, out, steps, warmup, stream, ws=1, clk=None):
     return per, ev[0].elapsed_time(ev[-1])
 
 
+def time_fn(fn, steps, warmup, stream):
+    """Per-step device times (ms) of `steps` calls of fn on `stream` (CUDA events)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record(stream)
+    for i in range(steps):
+        fn()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    return [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+
+
 def roofline(info, seconds, peaks, sustained=False):
     """The binding resource of one launch and how close the launch comes to it.
 
@@ -318,6 +333,36 @@ def run_ours(args):
     rl.update({"traffic": kernel_traffic(workload), "kernel": "attn_kernel",
                "peak_source": peaks["source"],
                "per_launch": "algorithmic work of one attn_run (one kernel launch) / its mean CUDA-event time"})
+    # fused KV append on the same batch: attn_run_append (one launch that also writes the
+    # new tokens' K/V into the cache) against attn_run alone and against a separate scatter
+    # (torch index_put) followed by attn_run
+    append = None
+    if ws == 1 and not args.no_append:
+        k_new, v_new = W.new_token_kv(batch)
+        pg, sl = W.new_token_slots(batch)
+        kc, vc = batch.k_cache, batch.v_cache
+
+        def fused():
+            plan.run_append(batch.q, k_new, v_new, kc, vc, out, stream)
+
+        def unfused():
+            kc[pg, :, sl] = k_new
+            vc[pg, :, sl] = v_new
+            plan.run(batch.q, kc, vc, out, stream)
+
+        n = 4 * args.other_steps
+        pf = time_fn(fused, n, args.warmup, stream)
+        pu = time_fn(unfused, n, args.warmup, stream)
+        if plan.check(stream) != 0:
+            raise RuntimeError("device error in the append measurement")
+        new_bytes = 2 * k_new.numel() * 2                      # K and V of the new tokens
+        sf, su = sum(pf) / len(pf) * 1e-3, sum(pu) / len(pu) * 1e-3
+        append = {"ms_per_launch": sf * 1e3, "tokens_per_s": tokens / sf,
+                  "attn_run_ms": avg_launch_s * 1e3, "scatter_then_attn_run_ms": su * 1e3,
+                  "new_kv_bytes": new_bytes,
+                  "gbs": (info["kv_bytes"] + 2 * new_bytes) / sf / 1e9,
+                  "what": "algorithmic bytes: cache K/V read once + new K/V read and written"}
+        del k_new, v_new, pg, sl
     plan.close()
     del batch, out
 
@@ -369,6 +414,7 @@ def run_ours(args):
             "plan": {k: info[k] for k in ("num_decode_items", "num_prefill_items", "num_split_units",
                                           "decode_rows")},
             "per_config": per_config,
+            "append": append,
         }
         print(json.dumps(result))
     if ws > 1:
@@ -385,6 +431,7 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
+    ap.add_argument("--no-append", action="store_true", help="skip the fused KV-append measurement")
     ap.add_argument("--no-other-configs", action="store_true",
                     help="skip the per-config table of the other benchmark batches")
     ap.add_argument("--other-steps", type=int, default=50)
