@@ -385,6 +385,29 @@ def run_ours(args):
             pl.close()
             del b, o
             torch.cuda.empty_cache()
+        # shared-prefix batch: cascade plan (attn_plan_shared) against the same batch planned
+        # without groups; algorithmic bytes count the shared keys once in both
+        for name in W.SHARED_CONFIG_NAMES:
+            b = W.make_shared_config(name, device=dev, keep_contiguous=False)
+            o = torch.empty_like(b.q)
+            res = {}
+            for tag, shared in (("cascade", True), ("no_cascade", False)):
+                pl = pk.plan_for_batch(b, shared=shared)
+                inf = pl.info()
+                ps, _ = time_steps(pl, b, o, args.other_steps, args.warmup, stream)
+                sec = sum(ps) / len(ps) * 1e-3
+                res[tag] = {"ms_per_launch": sec * 1e3, "tokens_per_s": b.total_q / sec,
+                            "kv_bytes_read_by_plan": inf["kv_bytes"],
+                            "cascade_tasks": inf["num_cascade_items"]}
+                if shared:
+                    kv_unique = inf["kv_bytes"]
+                    res[tag]["roofline"] = roofline(inf, sec, peaks)
+                pl.close()
+            res["kv_bytes_unique"] = kv_unique
+            res["speedup"] = res["no_cascade"]["ms_per_launch"] / res["cascade"]["ms_per_launch"]
+            per_config[name] = res
+            del b, o
+            torch.cuda.empty_cache()
 
     if rank == 0:
         cpu = None

@@ -109,6 +109,40 @@ PKVA_API int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq_l
               int num_q_heads, int num_kv_heads, int head_dim, int page_size, float sm_scale);
 
 /*
+ * attn_plan_shared — attn_plan for a batch in which groups of sequences share their first
+ * keys (a common prompt / system prefix held once in the cache), so that the shared keys
+ * are read once per group instead of once per sequence (cascade attention).
+ *
+ * Cites: XY-Serve verdict page, pith_inferences[0] and load_bearing_attack (automatic
+ * prefix caching and attention that reuses a cached prefix across requests); the split
+ * results are merged with the log-sum-exp rule of FlashAttention-style tiling
+ * (supporting_citations[1]).
+ *
+ *   (first fourteen arguments as attn_plan)
+ *   prefix_group  host int32[B]: -1, or the group of sequence s in [0, num_groups). The
+ *                 sequences of one group must be consecutive in the batch.
+ *   prefix_len    host int32[num_groups]: keys the group's sequences share, a multiple of
+ *                 page_size, at most L_s - T_s (the committed prefix) of every member.
+ *   num_groups    number of groups (0: same as attn_plan).
+ * The caller guarantees that the block-table entries 0 .. prefix_len/page_size - 1 are
+ * equal across a group's sequences (the pages are shared); the kernels read the group's
+ * first sequence's entries for those keys.
+ *
+ * The output is the same as attn_plan's on the same batch (up to rounding). Members that
+ * run as decode/verify tasks get their shared keys from cascade tasks: the stacked (token,
+ * head) rows of a run of members, floor(128 / (Hq/Hkv)) tokens x all heads of one KV head
+ * per tensor-core tile, against the shared keys in chunks of 1024; each member then merges
+ * those partial results with its own keys' (split-KV combine). Members that run as prefill
+ * tasks (causal chunks of >= 64 tokens) read their whole prefix as before. Needs head_dim
+ * 128 when any prefix_len > 0 (else PKVA_EUNSUPPORTED). Errors as attn_plan.
+ */
+PKVA_API int attn_plan_shared(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq_lens,
+              const int32_t* query_lens, const int32_t* block_table, int bt_stride,
+              int num_pages, const int32_t* mask_kind, const int32_t* parents,
+              int num_q_heads, int num_kv_heads, int head_dim, int page_size, float sm_scale,
+              const int32_t* prefix_group, const int32_t* prefix_len, int num_groups);
+
+/*
  * attn_run — compute the batch's attention on `stream` (asynchronous).
  *
  *   q        device bf16 [sum T_s, Hq, D]
@@ -233,14 +267,20 @@ typedef struct pkva_plan_info {
     int64_t kv_bytes;            /* algorithmic K+V bytes one run reads (each element once)  */
     int64_t attn_flops;          /* algorithmic 4*D*Hq flops per allowed (query, key) pair  */
     int64_t scratch_bytes;       /* device scratch the plan owns                            */
+    int32_t num_cascade_items;   /* shared-prefix tasks (attn_plan_shared)                  */
+    int32_t reserved;
 } pkva_plan_info;
 
 PKVA_API int attn_plan_get_info(pkva_plan_t plan, pkva_plan_info* info);
 
 /* One tile task as the planner emitted it (host-side inspection only). */
 typedef struct pkva_work_desc {
-    int32_t kind;        /* 0 = decode/verify task, 1 = prefill task                      */
-    int32_t seq;         /* sequence index                                                 */
+    int32_t kind;        /* 0 = decode/verify task, 1 = prefill task, 2 = shared-prefix     */
+                         /* (cascade) task: all heads of kv_head for q rows [row_begin,    */
+                         /* row_begin + row_count) of consecutive group members, keys      */
+                         /* [key_begin, key_end) of the shared prefix; split / num_splits  */
+                         /* count the cascade chunks of the prefix only                    */
+    int32_t seq;         /* sequence index (cascade: the group's first member in the run)  */
     int32_t kv_head;     /* KV head whose keys and values the task reads                   */
     int32_t q_head;      /* prefill: the one query head; decode/verify: -1 (all heads of   */
                          /* the KV head's group, as packed rows)                           */
@@ -255,9 +295,11 @@ typedef struct pkva_work_desc {
 
 /*
  * attn_plan_inspect — run the planner on the host only (no device, nothing allocated on
- * it) and return its tile tasks grouped by kind: prefill tasks, then decode/verify tasks,
- * each in its launch order (heaviest first; the single launch interleaves the two lists in
- * proportion, three decode/verify tasks to a block). Arguments as attn_plan, plus:
+ * it) and return its tile tasks grouped by kind: prefill tasks, then shared-prefix tasks,
+ * then decode/verify tasks, each in the planner's order (heaviest first; the single launch
+ * interleaves the tensor-core and decode/verify lists in proportion, three decode/verify
+ * tasks to a block). Arguments as attn_plan_shared (prefix_group / prefix_len may be NULL
+ * with num_groups 0), plus:
  *   num_sms, ctas_per_sm   the machine the plan should balance for;
  *   items, max_items       output array (may be NULL to query the count);
  *   num_items              receives the number of tasks.
@@ -267,7 +309,8 @@ typedef struct pkva_work_desc {
 PKVA_API int attn_plan_inspect(int num_seqs, const int32_t* seq_lens, const int32_t* query_lens,
                       int bt_stride, int num_pages, const int32_t* mask_kind,
                       const int32_t* parents, int num_q_heads, int num_kv_heads,
-                      int head_dim, int page_size, int num_sms, int ctas_per_sm,
+                      int head_dim, int page_size, const int32_t* prefix_group,
+                      const int32_t* prefix_len, int num_groups, int num_sms, int ctas_per_sm,
                       pkva_work_desc* items, int max_items, int* num_items);
 
 #ifdef __cplusplus

@@ -31,7 +31,7 @@ DEVERR_BAD_PAGE = 0x1
 DEVERR_TIMEOUT = 0x2
 
 # every entry point that include/pkva.h declares
-EXPORTED = ["attn_plan", "attn_run", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_destroy",
+EXPORTED = ["attn_plan", "attn_plan_shared", "attn_run", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_destroy",
             "attn_last_error", "attn_plan_get_info", "attn_plan_inspect", "attn_run_static",
             "pkva_selftest_wait_timeout"]
 
@@ -47,7 +47,8 @@ class PlanInfo(ctypes.Structure):
                 ("num_prefill_items", ctypes.c_int32), ("num_split_units", ctypes.c_int32),
                 ("num_partial_slots", ctypes.c_int32), ("decode_rows", ctypes.c_int32),
                 ("kv_bytes", ctypes.c_int64), ("attn_flops", ctypes.c_int64),
-                ("scratch_bytes", ctypes.c_int64)]
+                ("scratch_bytes", ctypes.c_int64), ("num_cascade_items", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 class WorkDesc(ctypes.Structure):
@@ -74,6 +75,7 @@ def lib() -> ctypes.CDLL:
     L.attn_plan.argtypes = [ctypes.POINTER(_vp), ctypes.c_int, _i32p, _i32p, _vp, ctypes.c_int,
                             ctypes.c_int, _i32p, _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                             ctypes.c_int, ctypes.c_float]
+    L.attn_plan_shared.argtypes = L.attn_plan.argtypes + [_i32p, _i32p, ctypes.c_int]
     L.attn_run.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp]
     L.attn_run_append.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
     L.attn_run_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp]
@@ -84,13 +86,14 @@ def lib() -> ctypes.CDLL:
     L.attn_plan_get_info.argtypes = [_vp, ctypes.POINTER(PlanInfo)]
     L.attn_plan_inspect.argtypes = [ctypes.c_int, _i32p, _i32p, ctypes.c_int, ctypes.c_int, _i32p,
                                     _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    _i32p, _i32p, ctypes.c_int,
                                     ctypes.c_int, ctypes.c_int, ctypes.POINTER(WorkDesc),
                                     ctypes.c_int, _i32p]
     L.attn_run_static.argtypes = [ctypes.c_int, _i32p, _i32p, _vp, ctypes.c_int, ctypes.c_int, _i32p,
                                   _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                   ctypes.c_float, _vp, _vp, _vp, _vp, _vp]
     L.pkva_selftest_wait_timeout.argtypes = [ctypes.c_longlong, _i32p]
-    for name in ("attn_plan", "attn_run", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_get_info",
+    for name in ("attn_plan", "attn_plan_shared", "attn_run", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_get_info",
                  "attn_plan_inspect", "attn_run_static", "pkva_selftest_wait_timeout"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -123,7 +126,11 @@ class Plan:
     def __init__(self, seq_lens: Sequence[int], query_lens: Sequence[int], block_table,
                  mask_kind: Sequence[int], parents: Optional[Sequence[int]] = None, *,
                  num_q_heads: int, num_kv_heads: int, head_dim: int, num_pages: int,
-                 page_size: int = 16, sm_scale: Optional[float] = None):
+                 page_size: int = 16, sm_scale: Optional[float] = None,
+                 prefix_group: Optional[Sequence[int]] = None,
+                 prefix_len: Optional[Sequence[int]] = None):
+        """``attn_plan``; with ``prefix_group`` / ``prefix_len`` (shared-prefix groups),
+        ``attn_plan_shared``."""
         import torch
         self._handle = None
         sl, ql, mk = _i32(seq_lens), _i32(query_lens), _i32(mask_kind)
@@ -143,9 +150,14 @@ class Plan:
         self.num_pages, self.page_size = num_pages, page_size
         self.total_q = int(ql.sum()) if len(ql) else 0
         h = _vp()
-        _check(lib().attn_plan(ctypes.byref(h), len(sl), _ptr(sl), _ptr(ql), bt_ptr, bt_stride,
-                               num_pages, _ptr(mk), _ptr(par), num_q_heads, num_kv_heads, head_dim,
-                               page_size, float(sm_scale) if sm_scale else 0.0))
+        args = (ctypes.byref(h), len(sl), _ptr(sl), _ptr(ql), bt_ptr, bt_stride, num_pages, _ptr(mk),
+                _ptr(par), num_q_heads, num_kv_heads, head_dim, page_size,
+                float(sm_scale) if sm_scale else 0.0)
+        if prefix_group is None:
+            _check(lib().attn_plan(*args))
+        else:
+            pg, pl = _i32(prefix_group), _i32(prefix_len if prefix_len is not None else [])
+            _check(lib().attn_plan_shared(*args, _ptr(pg), _ptr(pl), len(pl)))
         self._handle = h
 
     # -- marshalling checks (shapes, dtypes, devices) ---------------------------------
@@ -226,13 +238,17 @@ class Plan:
 
 def inspect(seq_lens, query_lens, mask_kind, parents=None, *, num_q_heads: int,
             num_kv_heads: int, head_dim: int, num_pages: int, bt_stride: int,
-            num_sms: int = 148, ctas_per_sm: int = 2, page_size: int = 16) -> List[Dict[str, int]]:
+            num_sms: int = 148, ctas_per_sm: int = 2, page_size: int = 16,
+            prefix_group=None, prefix_len=None) -> List[Dict[str, int]]:
     """Host-only planner run (``attn_plan_inspect``): the tile tasks in launch order."""
     sl, ql, mk = _i32(seq_lens), _i32(query_lens), _i32(mask_kind)
     par = _i32(parents if parents is not None else [])
+    pg = _i32(prefix_group if prefix_group is not None else [])
+    pl = _i32(prefix_len if prefix_len is not None else [])
     n = ctypes.c_int32(0)
     args = (len(sl), _ptr(sl), _ptr(ql), bt_stride, num_pages, _ptr(mk), _ptr(par), num_q_heads,
-            num_kv_heads, head_dim, page_size, num_sms, ctas_per_sm)
+            num_kv_heads, head_dim, page_size, _ptr(pg), _ptr(pl), len(pl) if prefix_group is not None else 0,
+            num_sms, ctas_per_sm)
     _check(lib().attn_plan_inspect(*args, None, 0, ctypes.byref(n)))
     arr = (WorkDesc * max(1, n.value))()
     _check(lib().attn_plan_inspect(*args, arr, n.value, ctypes.byref(n)))
@@ -266,9 +282,12 @@ def selftest_wait_timeout(limit_ns: int = 20_000_000) -> int:
     return int(err.value)
 
 
-def plan_for_batch(batch, sm_scale: Optional[float] = None) -> Plan:
-    """Plan a ``workloads.Batch`` (a convenience for tests and the benchmark)."""
+def plan_for_batch(batch, sm_scale: Optional[float] = None, shared: bool = True) -> Plan:
+    """Plan a ``workloads.Batch`` (a convenience for tests and the benchmark); a batch with
+    shared-prefix groups is planned with them unless ``shared`` is False."""
+    groups = getattr(batch, "prefix_group", None) if shared else None
     return Plan(batch.seq_lens, batch.query_lens, batch.block_table, batch.mask_kinds,
                 batch.parents_flat, num_q_heads=batch.num_q_heads, num_kv_heads=batch.num_kv_heads,
                 head_dim=batch.head_dim, num_pages=batch.k_cache.shape[0],
-                page_size=batch.page_size, sm_scale=sm_scale)
+                page_size=batch.page_size, sm_scale=sm_scale,
+                prefix_group=groups, prefix_len=batch.prefix_len if groups is not None else None)

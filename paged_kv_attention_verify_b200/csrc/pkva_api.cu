@@ -8,6 +8,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 #include <new>
 #include <string>
@@ -69,13 +70,16 @@ static bool encode_cache_map(CUtensorMap* map, const void* base, int num_pages, 
 
 // q viewed as the 3-D bf16 tensor [sum T][Hq][D]; one box is 128 tokens x 64 columns of
 // one head, stored with the 128-byte swizzle (the prefill kernel's A operand layout). The
-// new tokens' K and V ([sum T][Hkv][D]) use the same view with Hkv heads.
-static bool encode_q_map(CUtensorMap* map, const void* base, int total_q, int Hq, int D) {
+// new tokens' K and V ([sum T][Hkv][D]) use the same view with Hkv heads. Cascade tasks
+// read q in boxes of box_heads heads x box_tokens tokens (the (token, head) rows of one KV
+// head's group, still 128-byte rows in the same swizzle).
+static bool encode_q_map(CUtensorMap* map, const void* base, int total_q, int Hq, int D, int box_heads = 1,
+                         int box_tokens = kPrefillTileM) {
     auto fn = tensor_map_encoder();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)total_q};
     cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
-    cuuint32_t box[3] = {64, 1, (cuuint32_t)kPrefillTileM};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_tokens};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -106,7 +110,7 @@ struct pkva_plan {
     pkva::DecodeWork* d_dwork = nullptr;
     pkva::PrefillWork* d_pwork = nullptr;
     int32_t* d_order = nullptr;             // unified launch order
-    int32_t* d_order_prefill = nullptr;     // prefill tasks only (comparison mode)
+    int32_t* d_order_tensor = nullptr;      // tensor-core tasks only (comparison mode)
     CUtensorMap tmQ;
     const void* tm_q = nullptr;
     pkva::SplitUnit* d_units = nullptr;
@@ -123,6 +127,11 @@ struct pkva_plan {
     CUtensorMap tmKn, tmVn;                 // the new tokens' K / V (fused append)
     const void* tm_kn = nullptr;
     const void* tm_vn = nullptr;
+    CUtensorMap tmQc;                       // q in (token, head) tiles of one KV head (cascade)
+    const void* tm_qc = nullptr;
+    pkva::CascadeWork* d_cwork = nullptr;
+    int32_t* d_crowmap = nullptr;
+    int32_t* d_cunits = nullptr;
     int64_t scratch_bytes = 0;
 };
 
@@ -134,8 +143,11 @@ static void free_plan(pkva_plan* p) {
     cudaFree(p->d_dwork);
     cudaFree(p->d_pwork);
     cudaFree(p->d_order);
-    cudaFree(p->d_order_prefill);
+    cudaFree(p->d_order_tensor);
     cudaFree(p->d_units);
+    cudaFree(p->d_cwork);
+    cudaFree(p->d_crowmap);
+    cudaFree(p->d_cunits);
     cudaFree(p->d_anc);
     cudaFree(p->d_part_o);
     cudaFree(p->d_part_ml);
@@ -148,28 +160,25 @@ static void free_plan(pkva_plan* p) {
 
 extern "C" const char* attn_last_error(void) { return g_last_error.c_str(); }
 
-extern "C" int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq_lens, const int32_t* query_lens,
-                         const int32_t* block_table, int bt_stride, int num_pages, const int32_t* mask_kind,
-                         const int32_t* parents, int num_q_heads, int num_kv_heads, int head_dim, int page_size,
-                         float sm_scale) {
+static int plan_create(pkva_plan_t* out_plan, PlanArgs a, const int32_t* block_table, const char* who) {
+    const std::string name(who);
     if (!out_plan) {
-        set_last_error("attn_plan: out_plan is NULL");
+        set_last_error(name + ": out_plan is NULL");
         return PKVA_EINVAL;
     }
     *out_plan = nullptr;
+    const int num_seqs = a.num_seqs, head_dim = a.D;
     if (num_seqs > 0 && !block_table) {
-        set_last_error("attn_plan: block_table is NULL");
+        set_last_error(name + ": block_table is NULL");
         return PKVA_EINVAL;
     }
     // validate on the host first (a bad batch never touches the device)
-    PlanArgs a{num_seqs, seq_lens, query_lens, bt_stride, num_pages, mask_kind, parents, num_q_heads,
-               num_kv_heads, head_dim, page_size, sm_scale, 1, 1};
     {
         HostPlan probe;
         std::string err;
         const int rc = build_host_plan(a, &probe, &err);
         if (rc != PKVA_OK) {
-            set_last_error("attn_plan: " + err);
+            set_last_error(name + ": " + err);
             return rc;
         }
     }
@@ -179,13 +188,13 @@ extern "C" int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq
     PKVA_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev), "device attribute");
     PKVA_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "device attribute");
     if (major != 10) {
-        set_last_error("attn_plan: this library is built for sm_100a (B200); the current device is not");
+        set_last_error(name + ": this library is built for sm_100a (B200); the current device is not");
         return PKVA_EUNSUPPORTED;
     }
 
     pkva_plan* p = new (std::nothrow) pkva_plan();
     if (!p) {
-        set_last_error("attn_plan: out of host memory");
+        set_last_error(name + ": out of host memory");
         return PKVA_ENOMEM;
     }
     p->device = dev;
@@ -204,7 +213,7 @@ extern "C" int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq
                                          : decode_ctas_per_sm(head_dim, probe.decode_rows, false);
         if (blocks < 1) {
             free_plan(p);
-            set_last_error("attn_plan: attention kernel cannot be resident (shared memory)");
+            set_last_error(name + ": attention kernel cannot be resident (shared memory)");
             return PKVA_ECUDA;
         }
         p->decode_ctas = p->decode_mma ? kDecTasksPerBlock * blocks : blocks;
@@ -215,8 +224,13 @@ extern "C" int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq
     int rc = build_host_plan(a, &p->hp, &err);
     if (rc != PKVA_OK) {
         free_plan(p);
-        set_last_error("attn_plan: " + err);
+        set_last_error(name + ": " + err);
         return rc;
+    }
+    if (!p->decode_mma && !p->hp.cwork.empty()) {
+        free_plan(p);
+        set_last_error(name + ": shared-prefix groups need the tensor-core decode body (PKVA_DECODE_BODY=fma)");
+        return PKVA_EUNSUPPORTED;
     }
 
     const HostPlan& hp = p->hp;
@@ -233,12 +247,16 @@ extern "C" int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq
     PKVA_TRY(upload(&p->d_pwork, hp.pwork, &p->scratch_bytes));
     PKVA_TRY(upload(&p->d_order, hp.order, &p->scratch_bytes));
     {
-        std::vector<int32_t> po(hp.pwork.size());
-        for (size_t i = 0; i < po.size(); ++i) po[i] = (int32_t)i;
-        PKVA_TRY(upload(&p->d_order_prefill, po, &p->scratch_bytes));
+        std::vector<int32_t> po;
+        for (int32_t e : hp.order)
+            if (e >= 0) po.push_back(e);
+        PKVA_TRY(upload(&p->d_order_tensor, po, &p->scratch_bytes));
     }
     PKVA_TRY(upload(&p->d_units, hp.units, &p->scratch_bytes));
     PKVA_TRY(upload(&p->d_anc, hp.anc, &p->scratch_bytes));
+    PKVA_TRY(upload(&p->d_cwork, hp.cwork, &p->scratch_bytes));
+    PKVA_TRY(upload(&p->d_crowmap, hp.crowmap, &p->scratch_bytes));
+    PKVA_TRY(upload(&p->d_cunits, hp.cunits, &p->scratch_bytes));
     auto alloc_zero = [&](void** ptr, size_t bytes, const char* what) -> int {
         if (bytes == 0) return PKVA_OK;
         cudaError_t e = cudaMalloc(ptr, bytes);
@@ -258,6 +276,28 @@ extern "C" int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq
     set_last_error("");
     *out_plan = p;
     return PKVA_OK;
+}
+
+extern "C" int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq_lens, const int32_t* query_lens,
+                         const int32_t* block_table, int bt_stride, int num_pages, const int32_t* mask_kind,
+                         const int32_t* parents, int num_q_heads, int num_kv_heads, int head_dim, int page_size,
+                         float sm_scale) {
+    PlanArgs a{num_seqs, seq_lens, query_lens, bt_stride, num_pages, mask_kind, parents, num_q_heads,
+               num_kv_heads, head_dim, page_size, sm_scale, 1, 1};
+    return plan_create(out_plan, a, block_table, "attn_plan");
+}
+
+extern "C" int attn_plan_shared(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq_lens,
+                                const int32_t* query_lens, const int32_t* block_table, int bt_stride, int num_pages,
+                                const int32_t* mask_kind, const int32_t* parents, int num_q_heads, int num_kv_heads,
+                                int head_dim, int page_size, float sm_scale, const int32_t* prefix_group,
+                                const int32_t* prefix_len, int num_groups) {
+    PlanArgs a{num_seqs, seq_lens, query_lens, bt_stride, num_pages, mask_kind, parents, num_q_heads,
+               num_kv_heads, head_dim, page_size, sm_scale, 1, 1};
+    a.prefix_group = prefix_group;
+    a.prefix_len = prefix_len;
+    a.num_groups = num_groups;
+    return plan_create(out_plan, a, block_table, "attn_plan_shared");
 }
 
 extern "C" void attn_plan_destroy(pkva_plan_t plan) {
@@ -286,6 +326,8 @@ extern "C" int attn_plan_get_info(pkva_plan_t plan, pkva_plan_info* info) {
     info->kv_bytes = hp.kv_bytes;
     info->attn_flops = hp.attn_flops;
     info->scratch_bytes = plan->scratch_bytes;
+    info->num_cascade_items = (int32_t)hp.cwork.size();
+    info->reserved = 0;
     return PKVA_OK;
 }
 
@@ -329,7 +371,14 @@ static int run_impl(pkva_plan_t plan, const void* q, const void* k_new, const vo
         }
         plan->tm_v = v_cache;
     }
-    const bool has_prefill = !hp.pwork.empty();
+    const bool has_prefill = !hp.pwork.empty() || !hp.cwork.empty();
+    if (!hp.cwork.empty() && plan->tm_qc != q) {
+        if (!encode_q_map(&plan->tmQc, q, hp.total_q, hp.Hq, hp.D, hp.G, hp.cascade_tok)) {
+            set_last_error(name + ": cuTensorMapEncodeTiled failed for q (shared-prefix tiles)");
+            return PKVA_ECUDA;
+        }
+        plan->tm_qc = q;
+    }
     if (has_prefill && plan->tm_q != q) {
         if (!encode_q_map(&plan->tmQ, q, hp.total_q, hp.Hq, hp.D)) {
             set_last_error(name + ": cuTensorMapEncodeTiled failed for q");
@@ -363,6 +412,15 @@ static int run_impl(pkva_plan_t plan, const void* q, const void* k_new, const vo
     pp.G = hp.G;
     pp.num_pages = hp.num_pages;
     pp.scale_log2 = hp.scale * 1.4426950408889634f;
+    pp.num_prefill = (int32_t)hp.pwork.size();
+    pp.cascade_tok = hp.cascade_tok;
+    pp.cwork = plan->d_cwork;
+    pp.crowmap = plan->d_crowmap;
+    pp.cunits = plan->d_cunits;
+    pp.units = plan->d_units;
+    pp.part_o = plan->d_part_o;
+    pp.part_ml = plan->d_part_ml;
+    pp.counters = plan->d_counters;
     DecodeParams dp;
     dp.q = static_cast<const __nv_bfloat16*>(q);
     dp.out = static_cast<__nv_bfloat16*>(out);
@@ -400,15 +458,17 @@ static int run_impl(pkva_plan_t plan, const void* q, const void* k_new, const vo
         ap.order = plan->d_order;
         ap.num_blocks = (int32_t)hp.order.size();
         ap.num_decode = (int32_t)hp.dwork.size();
-        e = launch_attn(ap, hp.D, hp.decode_rows, has_prefill, plan->tmQ, plan->tmK, plan->tmV, tmKn, tmVn, st);
+        e = launch_attn(ap, hp.D, hp.decode_rows, has_prefill, plan->tmQ, plan->tmK, plan->tmV, tmKn, tmVn,
+                        plan->tmQc, st);
     } else {
         // comparison mode: decode tasks on the CUDA-core kernel, prefill tasks after them
         e = launch_decode(dp, (int)hp.dwork.size(), hp.D, hp.decode_rows, false, plan->tmK, plan->tmV, st);
         if (e == cudaSuccess && has_prefill) {
-            ap.order = plan->d_order_prefill;
-            ap.num_blocks = (int32_t)hp.pwork.size();
+            ap.order = plan->d_order_tensor;
+            ap.num_blocks = (int32_t)(hp.pwork.size() + hp.cwork.size());
             ap.num_decode = 0;
-            e = launch_attn(ap, hp.D, hp.decode_rows, has_prefill, plan->tmQ, plan->tmK, plan->tmV, tmKn, tmVn, st);
+            e = launch_attn(ap, hp.D, hp.decode_rows, has_prefill, plan->tmQ, plan->tmK, plan->tmV, tmKn, tmVn,
+                            plan->tmQc, st);
         }
     }
     if (e != cudaSuccess) return cuda_fail(e, (name + ": launch").c_str());

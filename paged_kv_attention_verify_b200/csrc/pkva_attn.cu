@@ -1,13 +1,18 @@
 // One launch for a whole mixed prefill / decode / verify batch.
 //
-// The planner's task list is one grid: prefill tasks first (heaviest first), then the
-// decode/verify tasks (heaviest first). A block whose index falls in the prefill range
-// runs the tensor-core prefill task (TMEM, tcgen05.mma, four warp roles); any other block
-// runs three decode/verify tasks side by side, each on four page-streaming warps with its own
-// third of shared memory and its own named barrier (warp-level tensor-core page body).
-// Both kinds use the same 352-thread block and the same dynamic shared memory (one block
-// per SM), so the hardware block scheduler deals the mixed work out as one
-// longest-task-first schedule and decode blocks fill the SMs as prefill blocks finish.
+// The planner's task list is one grid: shared-prefix (cascade) tasks first, then prefill
+// tasks and decode/verify tasks, each heaviest first, merged in proportion. A block whose
+// entry is a tensor-core task runs it with all its warps (TMEM, tcgen05.mma, four warp
+// roles); any other block runs three decode/verify tasks side by side, each on four
+// page-streaming warps with its own third of shared memory and its own named barrier
+// (warp-level tensor-core page body). Both kinds use the same 384-thread block and the
+// same dynamic shared memory (one block per SM), so the hardware block scheduler deals the
+// mixed work out as one longest-task-first schedule and decode blocks fill the SMs as
+// prefill blocks finish.
+//
+// (A persistent variant, blocks pulling tasks from two global queues with each decode
+// group taking its next task on its own, measured 3-13 % slower on B200 and was dropped:
+// the extra per-task fetch and the register pressure of the loop outweighed the gain.)
 //
 // XY-Serve (arXiv 2412.18106), verdict page — forward_implications[2] (one attention kernel
 // for prefill, decode and verify rows, the visible keys chosen row by row) and
@@ -38,7 +43,9 @@ struct AttnSmem {
     using DC = dec::DecodeCfg<D, NT * 8, false, kDecWarps, AttnNS<D>::value>;
     static constexpr int GROUP_BYTES = (DC::BYTES + 1023) / 1024 * 1024;    // one decode task
     static constexpr int DEC_BYTES = kDecTasksPerBlock * GROUP_BYTES;
-    static constexpr int BYTES = (D == 128 && pre::kSmemBytes > DEC_BYTES) ? pre::kSmemBytes : DEC_BYTES;
+    static constexpr int TASK_BYTES = (D == 128 && pre::kSmemBytes > DEC_BYTES) ? pre::kSmemBytes : DEC_BYTES;
+    static constexpr int OFF_SCHED = TASK_BYTES;  // the TMEM address of a tensor-core block
+    static constexpr int BYTES = TASK_BYTES + 64;
     static constexpr int ALLOC = BYTES + 1008;    // room to align to 1024
     static_assert(ALLOC <= 227 * 1024, "shared memory");
 };
@@ -47,35 +54,51 @@ template <int D, int NT>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKn,
-            const __grid_constant__ CUtensorMap tmVn) {
+            const __grid_constant__ CUtensorMap tmVn, const __grid_constant__ CUtensorMap tmQc) {
+    using S = AttnSmem<D, NT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int e = p.order[blockIdx.x];
     if constexpr (D == 128) {
         if (e >= 0) {
-            pre::prefill_task(p.pre, e, tmQ, tmK, tmV, tmKn, tmVn, sm);
+            // tensor-core task: 512 TMEM columns for the block (one block per SM)
+            uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + S::OFF_SCHED);
+            const int warp = threadIdx.x >> 5;
+            if (warp == pre::kWarpMma) {
+                tmem_alloc(tmem_slot, pre::kTmemCols);
+                tmem_relinquish();
+            }
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            const uint32_t tmem = *tmem_slot;
+            pre::prefill_task(p.pre, e, tmQ, tmK, tmV, tmKn, tmVn, tmQc, tmem, sm);
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            if (warp == pre::kWarpMma) tmem_dealloc(tmem, pre::kTmemCols);
             return;
         }
     }
-    if (e >= 0) return;                          // (never planned: prefill needs head_dim 128)
+    if (e >= 0) return;                          // (never planned: tensor-core tasks need head_dim 128)
     // decode block: warps 4g .. 4g+3 run task g of the block's three
     const int g = threadIdx.x >> 7;
     const int task = (-1 - e) * kDecTasksPerBlock + g;
     if (task >= p.num_decode) return;
     const dec::Group grp{(int)threadIdx.x & 127, 128, 1 + g};
-    dec::decode_mma_task<D, NT, kDecWarps, AttnNS<D>::value>(grp, p.dec, task, tmK, tmV,
-                                                             sm + g * AttnSmem<D, NT>::GROUP_BYTES);
+    dec::decode_mma_task<D, NT, kDecWarps, AttnNS<D>::value>(grp, p.dec, task, tmK, tmV, sm + g * S::GROUP_BYTES);
 }
 
 template <int D, int NT>
 cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                     const CUtensorMap& tmKn, const CUtensorMap& tmVn, cudaStream_t stream) {
+                     const CUtensorMap& tmKn, const CUtensorMap& tmVn, const CUtensorMap& tmQc,
+                     cudaStream_t stream) {
     using S = AttnSmem<D, NT>;
     cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::ALLOC);
     if (e != cudaSuccess) return e;
     const int grid = p.num_blocks;
     if (grid == 0) return cudaSuccess;
-    attn_kernel<D, NT><<<grid, kAttnThreads, S::ALLOC, stream>>>(p, tmQ, tmK, tmV, tmKn, tmVn);
+    attn_kernel<D, NT><<<grid, kAttnThreads, S::ALLOC, stream>>>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc);
     return cudaGetLastError();
 }
 
@@ -102,14 +125,14 @@ int attn_ctas_per_sm(int D, int rows) {
 
 cudaError_t launch_attn(const AttnParams& p, int D, int rows, bool has_prefill, const CUtensorMap& tmQ,
                         const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKn,
-                        const CUtensorMap& tmVn, cudaStream_t stream) {
+                        const CUtensorMap& tmVn, const CUtensorMap& tmQc, cudaStream_t stream) {
     if (D == 64) {
-        if (has_prefill) return cudaErrorInvalidValue;   // prefill tasks need head_dim 128
-        return rows <= 8 ? launch_t<64, 1>(p, tmQ, tmK, tmV, tmKn, tmVn, stream)
-                         : launch_t<64, 2>(p, tmQ, tmK, tmV, tmKn, tmVn, stream);
+        if (has_prefill) return cudaErrorInvalidValue;   // prefill and cascade tasks need head_dim 128
+        return rows <= 8 ? launch_t<64, 1>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
+                         : launch_t<64, 2>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
     }
-    return rows <= 8 ? launch_t<128, 1>(p, tmQ, tmK, tmV, tmKn, tmVn, stream)
-                     : launch_t<128, 2>(p, tmQ, tmK, tmV, tmKn, tmVn, stream);
+    return rows <= 8 ? launch_t<128, 1>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
+                     : launch_t<128, 2>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
 }
 
 }  // namespace pkva

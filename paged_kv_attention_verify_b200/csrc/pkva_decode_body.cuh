@@ -9,6 +9,7 @@
 #include "pkva.h"
 #include "pkva_append.cuh"
 #include "pkva_kernels.h"
+#include "pkva_merge.cuh"
 #include "pkva_ptx.cuh"
 
 namespace pkva {
@@ -52,7 +53,11 @@ struct DecodeCfg {
     static constexpr int OFF_OUT = OFF_ANC + NR * 8;
     static constexpr int OFF_BAR = align_up(OFF_OUT + NR * 4, 8);
     static constexpr int OFF_FLAG = OFF_BAR + NW * NS * 8;
-    static constexpr int BYTES = OFF_FLAG + 16;
+    // tensor-core body with two n-tiles: Q rows staged in shared memory (swizzled 16-byte
+    // chunks) and read per page with ldmatrix, instead of 32 registers held through the loop
+    static constexpr bool QB = !QF && NR > 8;
+    static constexpr int OFF_QB = align_up(OFF_FLAG + 16, 128);
+    static constexpr int BYTES = QB ? OFF_QB + NR * D * 2 : OFF_FLAG + 16;
     static constexpr int ALLOC = BYTES + 1008;                     // room to align to 1024
     static_assert(NW * NR * (D + 2) * 4 <= RING, "combine buffers must fit in the ring");
     static_assert(D == 64 || D == 128, "head_dim");
@@ -66,23 +71,27 @@ __device__ __forceinline__ int q_row_index(const DecodeParams& p, const SeqInfo&
     return (si.q_start + t) * p.Hq + w.kv_head * p.G + g;
 }
 
-// Per-task set-up shared by both bodies: barriers, block-table slice, row records.
+// Per-task set-up shared by both bodies: barriers (unless the warps set up their own),
+// block-table slice, row records.
 template <int NR, int NS, int NW>
 __device__ __forceinline__ void task_setup(const Group& grp, const DecodeParams& p, const DecodeWork& w,
                                            const SeqInfo& si,
                                            int* bts, int* rlim, uint64_t* ranc, int* rout, uint64_t* bars,
-                                           int* flag, const CUtensorMap* tmK, const CUtensorMap* tmV) {
+                                           int* flag, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                           bool init_bars = true) {
     const int tid = grp.tid;
     const int R = w.row_count;
     const int npg = w.page_end - w.page_begin;
     const int prefix = si.seq_len - si.query_len;
     if (tid == 0) {
-        for (int i = 0; i < NW * NS; ++i) mbar_init(&bars[i], 1);
-        fence_mbar_init();
+        if (init_bars) {
+            for (int i = 0; i < NW * NS; ++i) mbar_init(&bars[i], 1);
+            fence_mbar_init();
+            prefetch_tensormap(tmK);
+            prefetch_tensormap(tmV);
+        }
         flag[0] = 0;
         flag[1] = 0;
-        prefetch_tensormap(tmK);
-        prefetch_tensormap(tmV);
     }
     // block-table slice of this task; an entry out of range is flagged and its page is
     // loaded from a fully out-of-bounds box, which TMA fills with zeros
@@ -114,13 +123,11 @@ __device__ __forceinline__ void task_setup(const Group& grp, const DecodeParams&
     }
 }
 
-// Load page #i of this warp's stream (lane 0 only).
-template <int D, int NS, int STAGE_BYTES, int PAGE_BYTES, int NW>
-__device__ __forceinline__ void issue_page(const DecodeParams& p, const DecodeWork& w, const int* bts,
-                                           uint8_t* ring, uint64_t* bar, int warp, int i,
-                                           const CUtensorMap* tmK, const CUtensorMap* tmV) {
+// Load page #i of this warp's stream (lane 0 only); ph is its physical page, -1 for none.
+template <int D, int NS, int STAGE_BYTES, int PAGE_BYTES>
+__device__ __forceinline__ void issue_page_at(const DecodeParams& p, const DecodeWork& w, int ph, uint8_t* ring,
+                                              uint64_t* bar, int i, const CUtensorMap* tmK, const CUtensorMap* tmV) {
     const int stage = i % NS;
-    const int ph = bts[warp + NW * i];
     const int row = ph >= 0 ? (ph * p.Hkv + w.kv_head) * kPageSize : -kPageSize;
     uint8_t* dst = ring + stage * STAGE_BYTES;
     mbar_arrive_expect_tx(&bar[stage], STAGE_BYTES);
@@ -129,6 +136,14 @@ __device__ __forceinline__ void issue_page(const DecodeParams& p, const DecodeWo
         tma_load_2d(dst + b * kBoxBytes, tmK, &bar[stage], b * 64, row);
         tma_load_2d(dst + PAGE_BYTES + b * kBoxBytes, tmV, &bar[stage], b * 64, row);
     }
+}
+
+// Load page #i of this warp's stream from the staged block-table slice (lane 0 only).
+template <int D, int NS, int STAGE_BYTES, int PAGE_BYTES, int NW>
+__device__ __forceinline__ void issue_page(const DecodeParams& p, const DecodeWork& w, const int* bts,
+                                           uint8_t* ring, uint64_t* bar, int warp, int i,
+                                           const CUtensorMap* tmK, const CUtensorMap* tmV) {
+    issue_page_at<D, NS, STAGE_BYTES, PAGE_BYTES>(p, w, bts[warp + NW * i], ring, bar, i, tmK, tmV);
 }
 
 // Merge the four warps' (max, sum, unnormalised output) held in cm/cl/co, then either
@@ -174,40 +189,21 @@ __device__ __forceinline__ void merge_and_store(const Group& grp, const DecodePa
     }
     if (!split) return;
 
-    // ---- split-KV combine: the last split of the unit to finish merges all partials -----
+    // ---- split-KV combine: the last task of the unit to finish merges all partials -------
     __threadfence();
     grp.sync();
     if (tid == 0) {
         const int prev = atomicAdd(&p.counters[w.unit], 1);
-        flag[0] = (prev == p.units[w.unit].num_splits - 1);
+        flag[0] = (prev == p.units[w.unit].arrivals - 1);
+        if (flag[0]) p.counters[w.unit] = 0;        // every arrival is in: ready for the next run
     }
     grp.sync();
     if (!flag[0]) return;
     __threadfence();
-    const SplitUnit u = p.units[w.unit];
-    for (int idx = tid; idx < R * (D / 2); idx += grp.n) {
-        const int r = idx / (D / 2);
-        const int c = (idx - r * (D / 2)) * 2;
-        float M = -INFINITY;
-        for (int s = 0; s < u.num_splits; ++s)
-            M = fmaxf(M, __ldcg(p.part_ml + ((int64_t)(u.slot_base + s) * kDecodeRowsMax + r) * 2));
-        float o0 = 0.f, o1 = 0.f, L = 0.f;
-        if (M != -INFINITY) {
-            for (int s = 0; s < u.num_splits; ++s) {
-                const int64_t base = (int64_t)(u.slot_base + s) * kDecodeRowsMax + r;
-                const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + base * 2));
-                const float f = exp2f(ml.x - M);
-                const float2 v = __ldcg(reinterpret_cast<const float2*>(p.part_o + base * D + c));
-                o0 = fmaf(f, v.x, o0);
-                o1 = fmaf(f, v.y, o1);
-                L = fmaf(f, ml.y, L);
-            }
-        }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        *reinterpret_cast<__nv_bfloat162*>(p.out + (int64_t)rout[r] * D + c) =
-            __floats2bfloat162_rn(o0 * inv, o1 * inv);
-    }
-    if (tid == 0) p.counters[w.unit] = 0;     // ready for the next run of the plan
+    const int32_t uid = w.unit;
+    const int pref0 = 0;
+    merge_units<D>(tid >> 5, grp.n >> 5, tid & 31, &uid, &pref0, 1, w.row_count, p.units, p.part_o, p.part_ml,
+                   p.seqs, p.out, p.Hq, p.G);
 }
 
 // =====================================================================================
@@ -237,24 +233,55 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
     const int R = w.row_count;
     const int npg = w.page_end - w.page_begin;
     const int prefix = si.seq_len - si.query_len;
+    const int n_my = (warp < NW && npg > warp) ? (npg - warp + NW - 1) / NW : 0;
+    uint8_t* ring = sm + warp * C::NS * C::STAGE_BYTES;    // used only by warps < NW
+    uint64_t* bar = bars + warp * C::NS;
 
-    task_setup<NR, C::NS, NW>(grp, p, w, si, bts, rlim, ranc, rout, bars, flag, &tmK, &tmV);
+    // each streaming warp sets up its own stages and starts its first pages at once,
+    // reading their block-table entries directly; the rest of the set-up overlaps them
+    if (warp < NW && lane == 0) {
+        for (int i = 0; i < C::NS; ++i) mbar_init(&bar[i], 1);
+        fence_mbar_init();
+        fence_proxy_async_smem();                  // the previous task's generic accesses come first
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+        const int32_t* btrow = p.block_table + (int64_t)w.seq * p.bt_stride + w.page_begin;
+        for (int i = 0; i < C::NS && i < n_my; ++i) {
+            int ph = btrow[warp + NW * i];
+            if (ph < 0 || ph >= p.num_pages) ph = -1;     // flagged by the slice staging below
+            issue_page_at<D, C::NS, C::STAGE_BYTES, C::PAGE_BYTES>(p, w, ph, ring, bar, i, &tmK, &tmV);
+        }
+    }
+    task_setup<NR, C::NS, NW>(grp, p, w, si, bts, rlim, ranc, rout, bars, flag, &tmK, &tmV, false);
 
-    // Q^T as the B operand: row (column of S^T) nt*8+g, k = d; pairs straight from global
-    uint32_t qf[NT][KS][2];
+    // Q^T as the B operand: row (column of S^T) nt*8+g, k = d. One n-tile: pairs straight
+    // from global into registers. Two: rows staged in shared memory, chunk c of row r at
+    // chunk c ^ (r & 7), read per page with ldmatrix (keeps the page loop out of spilling).
+    constexpr int QREG = C::QB ? 1 : KS;
+    uint32_t qf[NT][QREG][2];
+    uint8_t* qs = sm + C::OFF_QB;
+    if constexpr (C::QB) {
+        for (int idx = tid; idx < NR * (D / 8); idx += grp.n) {
+            const int r = idx / (D / 8), c = idx - r * (D / 8);
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (r < R) v = *reinterpret_cast<const uint4*>(p.q + (int64_t)q_row_index(p, si, w, r) * D + c * 8);
+            *reinterpret_cast<uint4*>(qs + r * (D * 2) + ((c ^ (r & 7)) << 4)) = v;
+        }
+    } else {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        const int r = nt * 8 + g;
-        if (r < R) {
-            const __nv_bfloat16* qp = p.q + (int64_t)q_row_index(p, si, w, r) * D + 2 * t4;
+        for (int nt = 0; nt < NT; ++nt) {
+            const int r = nt * 8 + g;
+            if (r < R) {
+                const __nv_bfloat16* qp = p.q + (int64_t)q_row_index(p, si, w, r) * D + 2 * t4;
 #pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
-                qf[nt][ks][0] = *reinterpret_cast<const uint32_t*>(qp + ks * 16);
-                qf[nt][ks][1] = *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8);
+                for (int ks = 0; ks < QREG; ++ks) {
+                    qf[nt][ks][0] = *reinterpret_cast<const uint32_t*>(qp + ks * 16);
+                    qf[nt][ks][1] = *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8);
+                }
+            } else {
+#pragma unroll
+                for (int ks = 0; ks < QREG; ++ks) qf[nt][ks][0] = qf[nt][ks][1] = 0u;
             }
-        } else {
-#pragma unroll
-            for (int ks = 0; ks < KS; ++ks) qf[nt][ks][0] = qf[nt][ks][1] = 0u;
         }
     }
     grp.sync();
@@ -273,10 +300,6 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
         }
     for (int r = 0; r < R; ++r) min_lim = min(min_lim, rlim[r]);
 
-    const int n_my = (warp < NW && npg > warp) ? (npg - warp + NW - 1) / NW : 0;
-    uint8_t* ring = sm + warp * C::NS * C::STAGE_BYTES;    // used only by warps < NW
-    uint64_t* bar = bars + warp * C::NS;
-
     float o[KS][NT][4];           // O^T tiles: [d-tile][n-tile]{(d g, c), (d g, c+1), (d g+8, c), (d g+8, c+1)}
     float mref[NT][2], lsum[NT][2];
 #pragma unroll
@@ -291,11 +314,6 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
 #pragma unroll
             for (int i = 0; i < 4; ++i) o[dt][nt][i] = 0.f;
     }
-
-    if (lane == 0)
-        for (int i = 0; i < C::NS && i < n_my; ++i)
-            issue_page<D, C::NS, C::STAGE_BYTES, C::PAGE_BYTES, NW>(p, w, bts, ring, bar, warp, i, &tmK, &tmV);
-    __syncwarp();
 
     // ldmatrix row addresses: matrix mi = lane >> 3 supplies its rows from lanes 8mi..8mi+7
     const int mi = lane >> 3, mr = lane & 7;
@@ -328,13 +346,33 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
+        if constexpr (C::QB) {
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            const int cg = ks * 2 + k_chunk;
-            uint32_t a[4];
-            ldmatrix_x4(a, Ks + (cg >> 3) * kBoxBytes + k_key * 128 + (((cg & 7) ^ (k_key & 7)) << 4));
+            for (int k2 = 0; k2 < KS; k2 += 2) {
+                uint32_t qb[NT][4];              // b fragments of k-steps k2 and k2 + 1
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a, qf[nt][ks]);
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int qr = nt * 8 + (lane & 7), qc = 2 * k2 + (lane >> 3);
+                    ldmatrix_x4(qb[nt], qs + qr * (D * 2) + ((qc ^ (qr & 7)) << 4));
+                }
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk) {
+                    const int cg = (k2 + kk) * 2 + k_chunk;
+                    uint32_t a[4];
+                    ldmatrix_x4(a, Ks + (cg >> 3) * kBoxBytes + k_key * 128 + (((cg & 7) ^ (k_key & 7)) << 4));
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a, &qb[nt][2 * kk]);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                const int cg = ks * 2 + k_chunk;
+                uint32_t a[4];
+                ldmatrix_x4(a, Ks + (cg >> 3) * kBoxBytes + k_key * 128 + (((cg & 7) ^ (k_key & 7)) << 4));
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a, qf[nt][ks]);
+            }
         }
 
         // -- mask and per-row (column) max over the page's 16 keys ------------------------
@@ -436,6 +474,9 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
             mbar_wait_bounded(&bar[i % C::NS], (i / C::NS) & 1, p.err, PKVA_DEVERR_TIMEOUT);
         if (lane == 0) atomicOr(&flag[1], 1);
     }
+    __syncwarp();
+    if (warp < NW && lane == 0)                    // every phase of this warp's stages is complete
+        for (int i = 0; i < C::NS; ++i) mbar_inval(&bar[i]);
     // row sums over the 16 keys: lanes with the same t4 hold the column
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)

@@ -18,6 +18,7 @@ constexpr int kPrefillTileN = 128;     // keys per prefill KV tile (8 pages)
 constexpr int kDecTasksPerBlock = 3;   // decode tasks side by side in one block of the unified kernel
 constexpr int kPrefillMinTokens = 64;  // causal sequences with at least this many new tokens
                                        // (and head_dim 128) run on the tensor-core prefill kernel
+constexpr int kCascadeTilesPerTask = 8; // shared-prefix KV tiles (128 keys) per cascade task
 
 // Per-sequence record (the "Token-Table" row of the batch).
 struct SeqInfo {
@@ -26,7 +27,8 @@ struct SeqInfo {
     int32_t q_start;     // first row of this sequence in q / out
     int32_t mask_kind;   // 0 causal, 1 tree
     int32_t anc_off;     // TREE: index of token 0's ancestor mask in the mask array
-    int32_t pad0, pad1, pad2;
+    int32_t shared_len;  // keys shared with its prefix group and read by cascade tasks (else 0)
+    int32_t pad1, pad2;
 };
 static_assert(sizeof(SeqInfo) == 32, "SeqInfo layout");
 
@@ -62,11 +64,36 @@ struct PrefillWork {
 };
 static_assert(sizeof(PrefillWork) == 32, "PrefillWork layout");
 
-// A (seq, kv_head, row chunk) split over several tasks: where its partials live.
+// A (seq, kv_head, row chunk) whose keys are split over several tasks: where its partials
+// live, how many task arrivals complete it, and which output rows it owns (so that any
+// contributing task, decode or cascade, can merge it when it arrives last).
 struct SplitUnit {
     int32_t slot_base;   // first partial slot
-    int32_t num_splits;
+    int32_t num_splits;  // partial slots: decode splits, then cascade splits
+    int32_t arrivals;    // tasks that must finish before the merge
+    int32_t seq;
+    int32_t kv_head;
+    int32_t row_begin;   // packed rows [row_begin, row_begin + row_count)
+    int32_t row_count;
+    int32_t pad;
 };
+static_assert(sizeof(SplitUnit) == 32, "SplitUnit layout");
+
+// One shared-prefix (cascade) task: the stacked query rows of a run of sequences that share
+// their first prefix_len keys, against KV tiles [tile_begin, tile_end) of that prefix, as
+// two tcgen05 M = 128 tiles of (token, head) rows of one KV head. Each row's partial goes to
+// the split slot the row map gives; the units it touches are listed for the arrival count.
+struct CascadeWork {
+    int32_t lead_seq;    // the sequence whose block table supplies the shared pages
+    int32_t kv_head;
+    int32_t tok0;        // first q row (global token index) of the task
+    int32_t ntok;        // tokens in the task (<= 2 * tokens per tile)
+    int32_t tile_begin;  // KV tiles of 128 keys
+    int32_t tile_end;
+    int32_t unit_off;    // into the cascade unit list
+    int32_t unit_cnt;
+};
+static_assert(sizeof(CascadeWork) == 32, "CascadeWork layout");
 
 // Host-side result of planning, before anything is uploaded.
 struct HostPlan {
@@ -79,12 +106,19 @@ struct HostPlan {
     std::vector<uint64_t> anc;            // per TREE token: ancestor-or-self bit mask
     std::vector<DecodeWork> dwork;        // launch order
     std::vector<PrefillWork> pwork;       // heaviest first
-    // Unified launch order, one entry per block: e >= 0 runs prefill task e; e < 0 runs
-    // decode tasks 3*(-1-e) .. 3*(-1-e)+2 side by side. Both kinds heaviest first, merged
-    // in proportion.
+    // Unified launch order, one entry per block: e >= 0 runs tensor-core task e (prefill task
+    // e, or cascade task e - pwork.size()); e < 0 runs decode tasks 3*(-1-e) .. 3*(-1-e)+2
+    // side by side. Cascade tasks first, then prefill and decode tasks, each heaviest
+    // first, merged in proportion.
     std::vector<int32_t> order;
     std::vector<SplitUnit> units;
     int num_slots = 0;
+    // shared-prefix (cascade) tasks: launch-order entries e >= pwork.size() run cascade task
+    // e - pwork.size(); 2 * 128 row-map entries per task (partial index slot*16 + row, or -1)
+    std::vector<CascadeWork> cwork;
+    std::vector<int32_t> crowmap;
+    std::vector<int32_t> cunits;
+    int cascade_tok = 0;                  // tokens per cascade tile: floor(128 / G)
     int64_t kv_bytes = 0;
     int64_t attn_flops = 0;
 };
@@ -102,6 +136,11 @@ struct PlanArgs {
     int num_sms;
     int ctas_per_sm;
     bool use_prefill_kernel = true;       // false: every sequence goes to the decode kernel
+    // shared-prefix groups (may be NULL / 0): prefix_group[s] in {-1} U [0, num_groups),
+    // members of a group consecutive in the batch, prefix_len[g] keys shared (page multiple)
+    const int32_t* prefix_group = nullptr;
+    const int32_t* prefix_len = nullptr;
+    int num_groups = 0;
 };
 
 // Validates and decomposes; returns a pkva_status and fills `err` on failure.

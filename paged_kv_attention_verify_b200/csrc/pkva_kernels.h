@@ -48,15 +48,27 @@ struct PrefillParams {
     const __nv_bfloat16* v_new = nullptr;
     __nv_bfloat16* k_cache = nullptr;
     __nv_bfloat16* v_cache = nullptr;
+    // shared-prefix (cascade) tasks: task indices >= num_prefill
+    int32_t num_prefill = 0;
+    int32_t cascade_tok = 0;     // tokens per 128-row tile: floor(128 / G)
+    const CascadeWork* cwork = nullptr;
+    const int32_t* crowmap = nullptr;    // [tasks][256]: partial index slot*16 + row, or -1
+    const int32_t* cunits = nullptr;
+    const SplitUnit* units = nullptr;
+    float* part_o = nullptr;
+    float* part_ml = nullptr;
+    int32_t* counters = nullptr;
 };
 
 // Everything one launch of the unified attention kernel needs.
+// One entry of `order` per block: e >= 0 runs tensor-core task e (a prefill task, or
+// cascade task e - num_prefill); e < 0 runs decode tasks 3(-1-e) .. 3(-1-e)+2 side by side.
 struct AttnParams {
     PrefillParams pre;
     DecodeParams dec;
-    const int32_t* order;         // per block: >= 0 prefill task, < 0 decode pair -1-e
+    const int32_t* order;
     int32_t num_blocks;
-    int32_t num_decode;           // decode/verify tasks (two per block)
+    int32_t num_decode;           // decode/verify tasks
 };
 
 // Resident blocks per SM of the unified kernel (one: each block takes most of an SM).
@@ -66,9 +78,11 @@ int attn_ctas_per_sm(int D, int rows);
 // need head_dim 128). tmQ views q as the 3-D tensor [sum T][Hq][128] with a
 // {64, 1, 128} box; tmK/tmV are the cache maps (16 x 64 boxes).
 // tmKn/tmVn view k_new/v_new like tmQ ({64, 1, 128} boxes); read only when p.pre.append.
+// tmQc views q in boxes of {64 columns, G heads, floor(128 / G) tokens}; read only by
+// cascade tasks.
 cudaError_t launch_attn(const AttnParams& p, int D, int rows, bool has_prefill, const CUtensorMap& tmQ,
                         const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKn,
-                        const CUtensorMap& tmVn, cudaStream_t stream);
+                        const CUtensorMap& tmVn, const CUtensorMap& tmQc, cudaStream_t stream);
 
 // Resident CTAs per SM of the decode kernel compiled for (D, rows); 0 if unsupported.
 // `mma` selects the tensor-core page body, otherwise the CUDA-core one.

@@ -118,6 +118,44 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
     }
     p.total_q = (int)q_acc;
 
+    // -- shared-prefix groups ------------------------------------------------------------
+    std::vector<int> grp_of(a.num_seqs, -1);     // group of a sequence whose prefix is shared
+    if (a.num_groups < 0) return fail(err, PKVA_EINVAL, "num_groups must be >= 0 (got %ld)", a.num_groups);
+    if (a.num_groups > 0 && a.num_seqs > 0) {
+        if (!a.prefix_group || !a.prefix_len)
+            return fail(err, PKVA_EINVAL, "prefix_group and prefix_len must not be NULL when num_groups > 0");
+        std::vector<int> first(a.num_groups, -1), last(a.num_groups, -1), count(a.num_groups, 0);
+        for (int s = 0; s < a.num_seqs; ++s) {
+            const int g = a.prefix_group[s];
+            if (g < -1 || g >= a.num_groups)
+                return fail(err, PKVA_EINVAL, "prefix_group[%ld] = %ld must be -1 or in [0, num_groups)", s, g);
+            if (g < 0) continue;
+            if (first[g] < 0) first[g] = s;
+            last[g] = s;
+            ++count[g];
+        }
+        for (int g = 0; g < a.num_groups; ++g) {
+            const int P = a.prefix_len[g];
+            if (P < 0 || P % kPageSize)
+                return fail(err, PKVA_EINVAL, "prefix_len[%ld] = %ld must be a non-negative multiple of 16", g, P);
+            if (first[g] < 0) continue;
+            if (last[g] - first[g] + 1 != count[g])
+                return fail(err, PKVA_EINVAL, "the sequences of prefix group %ld are not consecutive in the batch", g);
+            for (int s = first[g]; s <= last[g]; ++s) {
+                const SeqInfo& si = p.seqs[s];
+                if (P > si.seq_len - si.query_len)
+                    return fail(err, PKVA_EINVAL,
+                                "prefix_len of group %ld (%ld) exceeds the committed prefix of sequence %ld", g, P, s);
+            }
+            if (P == 0) continue;
+            if (a.D != 128)
+                return fail(err, PKVA_EUNSUPPORTED, "shared-prefix groups need head_dim 128 (got %ld)", a.D);
+            if (p.G > kPrefillTileM)
+                return fail(err, PKVA_EUNSUPPORTED, "shared-prefix groups need at most 128 query heads per KV head");
+            for (int s = first[g]; s <= last[g]; ++s) grp_of[s] = g;
+        }
+    }
+
     // -- prefill tiles: long causal chunks go to the tensor-core prefill kernel ---------
     std::vector<char> on_prefill(a.num_seqs, 0);
     if (a.use_prefill_kernel && a.D == 128) {
@@ -159,14 +197,26 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
     }
 
     // -- decode/verify units: (seq, kv head, chunk of packed rows) --------------------
-    struct Unit { int seq, kvh, rb, rc, pages; };
+    // A sequence of a shared-prefix group leaves its first prefix_len keys to the cascade
+    // tasks: its units start at that page, and always merge partials.
+    struct Unit { int seq, kvh, rb, rc, pstart, pages, cs; };   // cs: cascade splits (0: none)
     std::vector<Unit> units;
+    std::vector<int> unit_base(a.num_seqs, -1);     // index of (s, head 0, chunk 0) in units
+    std::vector<char> on_cascade(a.num_seqs, 0);
     int64_t total_pages = 0;
     int max_rc = 0;
     for (int s = 0; s < a.num_seqs; ++s) {
         if (on_prefill[s]) continue;
         const SeqInfo& si = p.seqs[s];
         const int rows = si.query_len * p.G;
+        const int g = grp_of[s];
+        const int pstart = g >= 0 ? a.prefix_len[g] / kPageSize : 0;
+        const int cs = g >= 0 ? (a.prefix_len[g] + kPrefillTileN * kCascadeTilesPerTask - 1) /
+                                    (kPrefillTileN * kCascadeTilesPerTask)
+                              : 0;
+        on_cascade[s] = g >= 0;
+        p.seqs[s].shared_len = g >= 0 ? a.prefix_len[g] : 0;
+        unit_base[s] = (int)units.size();
         for (int h = 0; h < a.Hkv; ++h) {
             for (int rb = 0; rb < rows; rb += kDecodeRowsMax) {
                 const int rc = std::min(kDecodeRowsMax, rows - rb);
@@ -175,10 +225,22 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
                 // chunk (causal and tree alike), so the task never loads them
                 const int kend = si.seq_len - si.query_len + t_last + 1;
                 const int pages = (kend + kPageSize - 1) / kPageSize;
-                units.push_back({s, h, rb, rc, pages});
-                total_pages += pages;
+                units.push_back({s, h, rb, rc, pstart, pages, cs});
+                total_pages += pages - pstart;
                 max_rc = std::max(max_rc, rc);
             }
+        }
+    }
+    // algorithmic bytes: a shared prefix is one set of keys, counted once per group
+    if (a.num_groups > 0) {
+        std::vector<char> counted(a.num_groups, 0);
+        for (int s = 0; s < a.num_seqs; ++s) {
+            if (!on_cascade[s]) continue;
+            const int g = grp_of[s];
+            const int64_t per_key = (int64_t)a.Hkv * a.D * 2 * 2;
+            p.kv_bytes -= (int64_t)a.prefix_len[g] * per_key;
+            if (!counted[g]) p.kv_bytes += (int64_t)a.prefix_len[g] * per_key;
+            counted[g] = 1;
         }
     }
     p.decode_rows = max_rc <= 4 ? 4 : (max_rc <= 8 ? 8 : 16);
@@ -189,25 +251,108 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
     int64_t target = (total_pages + slots * kTasksPerSlot - 1) / (slots * kTasksPerSlot);
     target = std::max<int64_t>(target, kMinSplitPages);
     target = std::min<int64_t>(target, kDecodeMaxPages);
-    for (const Unit& u : units) {
-        const int ns = (int)((u.pages + target - 1) / target);
+    std::vector<int> unit_id_of(units.size(), -1);
+    std::vector<int> unit_ns(units.size(), 0);
+    for (size_t ui = 0; ui < units.size(); ++ui) {
+        const Unit& u = units[ui];
+        const int own = u.pages - u.pstart;
+        const int ns = (int)((own + target - 1) / target);
+        unit_ns[ui] = ns;
         int unit_id = -1;
-        if (ns > 1) {
+        if (ns > 1 || u.cs > 0) {
             unit_id = (int)p.units.size();
-            p.units.push_back({p.num_slots, ns});
-            p.num_slots += ns;
+            SplitUnit su{};
+            su.slot_base = p.num_slots;
+            su.num_splits = ns + u.cs;
+            su.arrivals = ns;                 // cascade tasks add theirs below
+            su.seq = u.seq;
+            su.kv_head = u.kvh;
+            su.row_begin = u.rb;
+            su.row_count = u.rc;
+            p.units.push_back(su);
+            p.num_slots += ns + u.cs;
         }
+        unit_id_of[ui] = unit_id;
         for (int k = 0; k < ns; ++k) {
             DecodeWork w{};
             w.seq = u.seq;
             w.kv_head = u.kvh;
             w.row_begin = u.rb;
             w.row_count = u.rc;
-            w.page_begin = (int)((int64_t)u.pages * k / ns);
-            w.page_end = (int)((int64_t)u.pages * (k + 1) / ns);
+            w.page_begin = u.pstart + (int)((int64_t)own * k / ns);
+            w.page_end = u.pstart + (int)((int64_t)own * (k + 1) / ns);
             w.unit = unit_id;
-            w.split = ns > 1 ? k : -1;
+            w.split = unit_id >= 0 ? k : -1;
             p.dwork.push_back(w);
+        }
+    }
+
+    // -- shared-prefix (cascade) tasks: per group, per run of consecutive decode-path
+    //    members (their q rows are contiguous), per KV head: tiles of floor(128 / G) tokens
+    //    x G heads, two tiles per task, the prefix split into chunks of tiles ---------------
+    p.cascade_tok = kPrefillTileM / p.G;
+    if (a.num_groups > 0) {
+        const int TOK = p.cascade_tok;
+        auto seq_of_token = [&](int tok) {
+            int lo = 0, hi = a.num_seqs - 1;       // last s with q_start <= tok
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) / 2;
+                if (p.seqs[mid].q_start <= tok) lo = mid; else hi = mid - 1;
+            }
+            return lo;
+        };
+        int s = 0;
+        while (s < a.num_seqs) {
+            if (!on_cascade[s]) { ++s; continue; }
+            const int g = grp_of[s];
+            int e = s;
+            while (e + 1 < a.num_seqs && on_cascade[e + 1] && grp_of[e + 1] == g) ++e;
+            const int run_t0 = p.seqs[s].q_start;
+            const int run_t1 = p.seqs[e].q_start + p.seqs[e].query_len;
+            const int tiles = (a.prefix_len[g] + kPrefillTileN - 1) / kPrefillTileN;
+            const int cs = units[unit_base[s]].cs;
+            for (int h = 0; h < a.Hkv; ++h) {
+                for (int t0 = run_t0; t0 < run_t1; t0 += 2 * TOK) {
+                    const int ntok = std::min(2 * TOK, run_t1 - t0);
+                    for (int k = 0; k < cs; ++k) {
+                        CascadeWork cw{};
+                        cw.lead_seq = s;
+                        cw.kv_head = h;
+                        cw.tok0 = t0;
+                        cw.ntok = ntok;
+                        cw.tile_begin = (int)((int64_t)tiles * k / cs);
+                        cw.tile_end = (int)((int64_t)tiles * (k + 1) / cs);
+                        cw.unit_off = (int)p.cunits.size();
+                        int last_unit = -1;
+                        for (int b = 0; b < 2; ++b) {
+                            for (int r = 0; r < kPrefillTileM; ++r) {
+                                const int tl = b * TOK + r / p.G;
+                                int entry = -1;
+                                if (r < TOK * p.G && tl < ntok) {
+                                    const int tok = t0 + tl;
+                                    const int sq = seq_of_token(tok);
+                                    const int pr = (tok - p.seqs[sq].q_start) * p.G + r % p.G;
+                                    const int chunks = (p.seqs[sq].query_len * p.G + kDecodeRowsMax - 1) /
+                                                       kDecodeRowsMax;
+                                    const int ui = unit_base[sq] + h * chunks + pr / kDecodeRowsMax;
+                                    const int uid = unit_id_of[ui];
+                                    entry = (p.units[uid].slot_base + unit_ns[ui] + k) * kDecodeRowsMax +
+                                            pr % kDecodeRowsMax;
+                                    if (uid != last_unit) {      // rows of one unit are adjacent
+                                        p.cunits.push_back(uid);
+                                        p.units[uid].arrivals += 1;
+                                        last_unit = uid;
+                                    }
+                                }
+                                p.crowmap.push_back(entry);
+                            }
+                        }
+                        cw.unit_cnt = (int)p.cunits.size() - cw.unit_off;
+                        p.cwork.push_back(cw);
+                    }
+                }
+            }
+            s = e + 1;
         }
     }
     // heaviest first; ties keep (seq, head, chunk) order so chunks of one head stay adjacent
@@ -215,10 +360,14 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
         return (x.page_end - x.page_begin) > (y.page_end - y.page_begin);
     });
 
-    // -- one launch order for both kinds. Each kind keeps its heaviest-first order; the two
-    //    lists are merged in proportion, so prefill blocks (tensor cores, latency) run beside
-    //    decode blocks (HBM) from start to end instead of one kind forming the tail. Decode
-    //    tasks go three to a block, neighbours in the sorted list.
+    // -- one launch order. Cascade tasks go first: few, long, and every unit of their rows
+    //    waits for them, so the units' own decode tasks tend to arrive last and do the
+    //    merges, spread over many blocks. Prefill and decode tasks each keep their
+    //    heaviest-first order; the two lists are merged in proportion, so prefill blocks
+    //    (tensor cores, latency) run beside decode blocks (HBM) from start to end instead of
+    //    one kind forming the tail. Decode tasks go three to a block, neighbours in the
+    //    sorted list.
+    for (size_t i = 0; i < p.cwork.size(); ++i) p.order.push_back((int32_t)(p.pwork.size() + i));
     const int np = (int)p.pwork.size();
     const int nd = (int)((p.dwork.size() + kDecTasksPerBlock - 1) / kDecTasksPerBlock);
     int ip = 0, id = 0;
@@ -242,11 +391,15 @@ void set_last_error(const std::string& msg);   // defined with the rest of the C
 extern "C" int attn_plan_inspect(int num_seqs, const int32_t* seq_lens, const int32_t* query_lens,
                                  int bt_stride, int num_pages, const int32_t* mask_kind,
                                  const int32_t* parents, int num_q_heads, int num_kv_heads,
-                                 int head_dim, int page_size, int num_sms, int ctas_per_sm,
+                                 int head_dim, int page_size, const int32_t* prefix_group,
+                                 const int32_t* prefix_len, int num_groups, int num_sms, int ctas_per_sm,
                                  pkva_work_desc* items, int max_items, int* num_items) {
     using namespace pkva;
     PlanArgs a{num_seqs, seq_lens, query_lens, bt_stride, num_pages, mask_kind, parents,
                num_q_heads, num_kv_heads, head_dim, page_size, 0.f, num_sms, ctas_per_sm};
+    a.prefix_group = prefix_group;
+    a.prefix_len = prefix_len;
+    a.num_groups = num_groups;
     HostPlan hp;
     std::string err;
     int rc = build_host_plan(a, &hp, &err);
@@ -255,14 +408,15 @@ extern "C" int attn_plan_inspect(int num_seqs, const int32_t* seq_lens, const in
         return rc;
     }
     const int np = (int)hp.pwork.size();
-    const int n = np + (int)hp.dwork.size();
+    const int nc = (int)hp.cwork.size();
+    const int n = np + nc + (int)hp.dwork.size();
     if (num_items) *num_items = n;
     if (!items) return PKVA_OK;
     if (max_items < n) {
         set_last_error("attn_plan_inspect: max_items is smaller than the number of tasks");
         return PKVA_EINVAL;
     }
-    for (int i = 0; i < np; ++i) {      // launch order: prefill tasks first
+    for (int i = 0; i < np; ++i) {      // prefill tasks first
         const PrefillWork& w = hp.pwork[i];
         const SeqInfo& si = hp.seqs[w.seq];
         pkva_work_desc d;
@@ -278,8 +432,28 @@ extern "C" int attn_plan_inspect(int num_seqs, const int32_t* seq_lens, const in
         d.num_splits = 1;
         items[i] = d;
     }
-    for (int i = np; i < n; ++i) {
-        const DecodeWork& w = hp.dwork[i - np];
+    for (int i = 0; i < nc; ++i) {      // then shared-prefix tasks
+        const CascadeWork& w = hp.cwork[i];
+        const int P = a.prefix_len[a.prefix_group[w.lead_seq]];
+        const int tiles = (P + kPrefillTileN - 1) / kPrefillTileN;
+        const int cs = (P + kPrefillTileN * kCascadeTilesPerTask - 1) / (kPrefillTileN * kCascadeTilesPerTask);
+        int k = 0;
+        while (k < cs && (int)((int64_t)tiles * k / cs) != w.tile_begin) ++k;
+        pkva_work_desc d;
+        d.kind = 2;
+        d.seq = w.lead_seq;
+        d.kv_head = w.kv_head;
+        d.q_head = -1;
+        d.row_begin = w.tok0;
+        d.row_count = w.ntok;
+        d.key_begin = w.tile_begin * kPrefillTileN;
+        d.key_end = std::min(w.tile_end * kPrefillTileN, P);
+        d.split = k;
+        d.num_splits = cs;
+        items[np + i] = d;
+    }
+    for (int i = np + nc; i < n; ++i) {
+        const DecodeWork& w = hp.dwork[i - np - nc];
         const SeqInfo& si = hp.seqs[w.seq];
         pkva_work_desc d;
         d.kind = 0;

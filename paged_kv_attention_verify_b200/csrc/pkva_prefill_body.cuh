@@ -35,6 +35,7 @@
 #include "pkva.h"
 #include "pkva_append.cuh"
 #include "pkva_kernels.h"
+#include "pkva_merge.cuh"
 #include "pkva_ptx.cuh"
 
 namespace pkva {
@@ -168,27 +169,50 @@ __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, 
 
 // One prefill task; every thread of the block (at least kPThreads) calls it; warps past
 // the V producer only take part in the block barriers. `sm` is the block's 1024-aligned
-// dynamic shared memory (kSmemBytes).
+// dynamic shared memory (kSmemBytes); `tmem` the block's 512 TMEM columns, allocated by
+// the caller for the block's lifetime (a persistent block runs many tasks). The task's
+// barriers are invalidated at its end, so the next task may reuse the memory.
 // With p.append, KV tiles [0, nc) come from the cache (the committed prefix, keys at and past
 // it masked) and tiles [nc, n) from the new tokens' K/V through tmKn / tmVn (tiles aligned
 // at the chunk start), and warp 11 writes a share of the task's new rows into the cache.
+//
+// Task indices >= p.num_prefill are shared-prefix (cascade) tasks: the two query tiles hold
+// (token, head) rows of one KV head for consecutive tokens of a group's members (tmQc), the
+// KV tiles are a chunk of the shared prefix (all keys visible to every row), and each row's
+// unnormalised output, max and sum go to the split slot its row-map entry names; the task
+// then counts one arrival on every unit it touched and merges those it completed.
 __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, const CUtensorMap& tmQ,
                                              const CUtensorMap& tmK, const CUtensorMap& tmV,
-                                             const CUtensorMap& tmKn, const CUtensorMap& tmVn, uint8_t* sm) {
+                                             const CUtensorMap& tmKn, const CUtensorMap& tmVn,
+                                             const CUtensorMap& tmQc, uint32_t tmem, uint8_t* sm) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const PrefillWork w = p.work[task];
+    const bool cascade = task >= p.num_prefill;
+    const int ci = task - p.num_prefill;
+    PrefillWork w{};
+    CascadeWork cw{};
+    if (cascade) {
+        cw = p.cwork[ci];
+        w.seq = cw.lead_seq;
+        w.tok0 = cw.tok0;
+        w.ntok = cw.ntok;
+    } else {
+        w = p.work[task];
+    }
     const SeqInfo si = p.seqs[w.seq];
     const Bars B = bars_at(sm);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffTmemSlot);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffFlag);
-    const bool append = p.append != 0;
-    const int n0 = append ? w.kv_tiles0_append : w.kv_tiles0;
-    const int n1 = append ? w.kv_tiles1_append : w.kv_tiles1;
+    const bool append = p.append != 0 && !cascade;
+    const int TOK = p.cascade_tok;                      // cascade: tokens per query tile
+    const int n0 = cascade ? cw.tile_end - cw.tile_begin : append ? w.kv_tiles0_append : w.kv_tiles0;
+    const int n1 = cascade ? (cw.ntok > TOK ? n0 : 0) : append ? w.kv_tiles1_append : w.kv_tiles1;
     const int nmax = n0 > n1 ? n0 : n1;
-    const int kvh = w.q_head / p.G;
+    const int jbase = cascade ? cw.tile_begin : 0;     // first KV tile (of 128 keys) of the task
+    const int kvh = cascade ? cw.kv_head : w.q_head / p.G;
     const int prefix = si.seq_len - si.query_len;
     const int nc = append ? (prefix + kPrefillTileN - 1) / kPrefillTileN : nmax;   // tiles read from the cache
-    const int key_limit = append ? prefix : si.seq_len;                            // cache keys that hold data
+    // cache keys that hold data: the shared prefix (cascade), the committed prefix
+    // (append), the whole sequence (otherwise)
+    const int key_limit = cascade ? si.shared_len : append ? prefix : si.seq_len;
 
     if (tid == 0) {
         mbar_init(B.q_full, 1);
@@ -210,24 +234,32 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == kWarpMma) {
-        tmem_alloc(tmem_slot, kTmemCols);
-        tmem_relinquish();
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
 
     if (warp == kWarpKProd || warp == kWarpVProd) {
         // ------------------ TMA producers: warp 8 loads Q and K, warp 10 loads V ------------
         if (lane == 0) {
+            fence_proxy_async_smem();              // the previous task's generic accesses come first
             const bool is_k = warp == kWarpKProd;
             const int32_t* btrow = p.block_table + (int64_t)w.seq * p.bt_stride;
             // the cache page holding key_limit has stale rows from key_limit on (when it is
             // not page-aligned): the V tile with that page is zeroed there before its PV
-            const int fix_tile = (key_limit % kPageSize) ? key_limit / kPageSize / 8 : -1;
-            if (is_k) {
+            const int fix_tile = (key_limit % kPageSize) ? key_limit / kPageSize / 8 - jbase : -1;
+            if (is_k && cascade) {
+                // G heads x TOK tokens per tile: rows (token, head) in the tile's first
+                // G * TOK rows, the same 128-byte rows as a one-head box
+                prefetch_tensormap(&tmQc);
+                prefetch_tensormap(&tmK);
+                mbar_arrive_expect_tx(B.q_full, 4u * (uint32_t)(p.G * TOK) * 128u);
+#pragma unroll
+                for (int b = 0; b < 2; ++b)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_3d(sm + kOffQ + b * kTileBytes + h * kHalfBytes, &tmQc, B.q_full, h * 64,
+                                    kvh * p.G, cw.tok0 + b * TOK);
+            } else if (is_k) {
                 prefetch_tensormap(&tmQ);
                 prefetch_tensormap(&tmK);
                 if (append) prefetch_tensormap(&tmKn);
@@ -261,7 +293,7 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
                     continue;
                 }
                 int rows[8];
-                tile_rows(p, btrow, key_limit, kvh, j, rows);
+                tile_rows(p, btrow, key_limit, kvh, jbase + j, rows);
                 if (is_k || j != fix_tile) {
                     load_tile(dst, is_k ? &tmK : &tmV, &full[st], rows);
                     continue;
@@ -279,6 +311,10 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
                 fence_proxy_async_smem();
                 mbar_arrive(&full[st]);
             }
+            // drain: the last stages' release arrives (from tcgen05.commit) must have landed
+            // before the task ends and its barriers are invalidated and reused
+            for (int j = nmax > NSt ? nmax - NSt : 0; j < nmax; ++j)
+                if (!wait_or_abort(&empty[j % NSt], (j / NSt) & 1, p.err, abort_flag)) break;
         }
     } else if (warp == kWarpMma) {
         // ------------------------------ MMA issuer -------------------------------------------
@@ -366,12 +402,18 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         const uint32_t o_addr = tmem + lane_off + kColO + b * 128;
         const int row_in_task = b * kPrefillTileM + r;
         const int tok = w.tok0 + row_in_task;
-        const bool real_row = row_in_task < w.ntok;
-        const int lim = real_row ? prefix + tok : 0x7fffffff;        // last visible key of this row
-        const int lim_first = prefix + w.tok0 + b * kPrefillTileM;    // the tile's first row
-        // append mode: the cache tiles show keys [0, prefix) to every row; the new tiles are
-        // indexed from the chunk start, so a row sees new keys up to its own token index
-        const int lim_new = tok, lim_first_new = w.tok0 + b * kPrefillTileM;
+        // Per KV tile j: its first key kb and the last key this row (lim) and the tile's
+        // first row (lim_first) may see. Tiles [0, na) are cache tiles j + jbase with limits
+        // (lim_a, lim_first_a); append mode's new tiles j >= na are indexed from the chunk
+        // start with limits (lim_b, lim_first_b).
+        //   plain: lim_a = prefix + tok (the causal diagonal), all tiles cache tiles;
+        //   append: cache tiles show keys [0, prefix) to every row, a new tile's row sees new
+        //           keys up to its own token index;
+        //   cascade: every shared key (below key_limit) is visible.
+        const int na = append ? nc : nmax;
+        const int lim_first_b = w.tok0 + b * kPrefillTileM, lim_b = tok;
+        const int lim_first_a = cascade || append ? key_limit - 1 : prefix + lim_first_b;
+        const int lim_a = cascade || append ? key_limit - 1 : (row_in_task < w.ntok ? prefix + tok : 0x7fffffff);
         float m_ref = -INFINITY, l_sum = 0.f;
         bool alive = true;
         // every break below is taken by the whole warp (tcgen05.ld/st are warp-collective)
@@ -386,16 +428,10 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
 #pragma unroll
             for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
             tmem_wait_ld();
-            int kb = j * kPrefillTileN, lim_j = lim, lim_first_j = lim_first;
-            if (append) {
-                if (j < nc) {
-                    lim_j = lim_first_j = prefix - 1;
-                } else {
-                    kb = (j - nc) * kPrefillTileN;
-                    lim_j = lim_new;
-                    lim_first_j = lim_first_new;
-                }
-            }
+            const bool tile_a = j < na;
+            const int kb = tile_a ? (jbase + j) * kPrefillTileN : (j - na) * kPrefillTileN;
+            const int lim_j = tile_a ? lim_a : lim_b;
+            const int lim_first_j = tile_a ? lim_first_a : lim_first_b;
             if (kb + kPrefillTileN - 1 > lim_first_j) {        // tile crosses the diagonal
                 const int vis = lim_j - kb;                        // columns <= vis are visible
 #pragma unroll
@@ -463,9 +499,71 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
             tc_fence_before();
             mbar_arrive(&B.p_full[b]);
         }
+        // ---- epilogue (cascade): unnormalised O, max and sum -> the row's split slot --------
+        if (cascade) {
+            // where this row's partial goes (slot * 16 + row in unit), or -1
+            const int part_idx = p.crowmap[(int64_t)ci * 2 * kPrefillTileM + row_in_task];
+            const bool real_row = part_idx >= 0;
+            if (nb > 0 && alive && __all_sync(0xffffffffu, wait_or_abort(&B.o_ready[b], 0, p.err, abort_flag))) {
+                tc_fence_after();
+                float* dst = p.part_o + (int64_t)(part_idx < 0 ? 0 : part_idx) * kD;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t ov[32];
+                    tmem_ld32(o_addr + c * 32, ov);
+                    tmem_wait_ld();
+                    if (real_row) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4)
+                            *reinterpret_cast<float4*>(dst + c * 32 + e) =
+                                make_float4(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1]),
+                                            __uint_as_float(ov[e + 2]), __uint_as_float(ov[e + 3]));
+                    }
+                }
+                if (real_row)
+                    *reinterpret_cast<float2*>(p.part_ml + (int64_t)part_idx * 2) = make_float2(m_ref, l_sum);
+            }
+            // all 256 softmax threads: count one arrival per unit touched, then merge the
+            // units this task completed. Every MMA has finished here (both warpgroups waited
+            // for their tiles' last PV), so the Q tiles' shared memory is free for the flags.
+            __threadfence();
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            int* cnt = reinterpret_cast<int*>(sm + kOffQ);      // [256] rows of each completed unit, else 0
+            int* uid = cnt + 256;                                // [256]
+            int* pref = uid + 256;                               // [256] compacted prefix sums
+            int* cuid = pref + 256;                              // [256] compacted unit ids
+            const bool aborted = *abort_flag != 0;
+            for (int i = tid; i < cw.unit_cnt; i += 256) {
+                const int u = p.cunits[cw.unit_off + i];
+                const bool done = !aborted && atomicAdd(&p.counters[u], 1) == p.units[u].arrivals - 1;
+                if (done) p.counters[u] = 0;        // every arrival is in: ready for the next run
+                cnt[i] = done ? p.units[u].row_count : 0;
+                uid[i] = u;
+            }
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            int* totals = cuid + 256;                            // [2]: rows, units
+            if (tid == 0) {                          // compact the completed units (a few hundred at most)
+                int n = 0, rows = 0;
+                for (int i = 0; i < cw.unit_cnt; ++i)
+                    if (cnt[i]) {
+                        pref[n] = rows;
+                        cuid[n++] = uid[i];
+                        rows += cnt[i];
+                    }
+                totals[0] = rows;
+                totals[1] = n;
+            }
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            __threadfence();
+            const int total = totals[0], n_done = totals[1];
+            if (n_done > 0)
+                merge_units<kD>(warp, 8, lane, cuid, pref, n_done, total, p.units, p.part_o, p.part_ml, p.seqs,
+                                p.out, p.Hq, p.G);
+        }
         // ---- epilogue: O / l -> bf16 rows --------------------------------------------------
-        if (nb > 0 && alive && __all_sync(0xffffffffu, wait_or_abort(&B.o_ready[b], 0, p.err, abort_flag))) {
+        else if (nb > 0 && alive && __all_sync(0xffffffffu, wait_or_abort(&B.o_ready[b], 0, p.err, abort_flag))) {
             tc_fence_after();
+            const bool real_row = row_in_task < w.ntok;
             const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
             __nv_bfloat16* dst = p.out + ((int64_t)(si.q_start + tok) * p.Hq + w.q_head) * kD;
 #pragma unroll
@@ -495,11 +593,15 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         append_rows<kD>(p.k_new, p.v_new, p.k_cache, p.v_cache, p.block_table, p.bt_stride, p.num_pages, p.Hkv,
                         p.err, si, w.seq, kvh, t_begin, t_end, lane, 32);
     }
-    // all roles done (the MMA thread waited for its last MMA); release TMEM
+    // all roles done (the MMA thread waited for its last MMA): TMEM and shared memory are
+    // free for the block's next task
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
+    if (tid == 0) {
+        uint64_t* b = reinterpret_cast<uint64_t*>(sm + kOffBar);
+        for (int i = 0; i < kNumBars; ++i) mbar_inval(&b[i]);
+    }
 }
 
 

@@ -78,21 +78,31 @@ def test_attn_plan_validates_before_touching_the_device():
     L.attn_plan_destroy(None)
 
 
-def _coverage(batch, items):
+def _coverage(batch, items, prefix_group=None, prefix_len=None):
     """Every (seq, kv head, packed row) must see exactly the keys it needs, once."""
     G = batch.num_q_heads // batch.num_kv_heads
+    q_start = np.cumsum([0] + [sp.query_len for sp in batch.seqs])
     seen = {}
     for it in items:
         assert it["key_begin"] % 16 == 0 and it["key_end"] > it["key_begin"]
         if it["kind"] == 1:            # prefill: tokens [row_begin, +row_count) of one query head
             assert 1 <= it["row_count"] <= 256 and it["q_head"] // G == it["kv_head"]
-            rows = [t * G + it["q_head"] % G for t in range(it["row_begin"], it["row_begin"] + it["row_count"])]
+            rows = [(it["seq"], t * G + it["q_head"] % G)
+                    for t in range(it["row_begin"], it["row_begin"] + it["row_count"])]
+        elif it["kind"] == 2:          # cascade: all heads of q rows [row_begin, +row_count)
+            assert it["q_head"] == -1 and 1 <= it["row_count"] <= 2 * (128 // G)
+            rows = []
+            for tok in range(it["row_begin"], it["row_begin"] + it["row_count"]):
+                s = int(np.searchsorted(q_start, tok, side="right") - 1)
+                assert prefix_group[s] == prefix_group[it["seq"]] >= 0
+                assert it["key_end"] <= prefix_len[prefix_group[s]]
+                rows += [(s, (tok - q_start[s]) * G + g) for g in range(G)]
         else:
             assert 1 <= it["row_count"] <= 16 and it["q_head"] == -1
-            rows = range(it["row_begin"], it["row_begin"] + it["row_count"])
-        for r in rows:
-            seen.setdefault((it["seq"], it["kv_head"], r), []).append((it["key_begin"], it["key_end"],
-                                                                      it["split"], it["num_splits"]))
+            rows = [(it["seq"], r) for r in range(it["row_begin"], it["row_begin"] + it["row_count"])]
+        for s, r in rows:
+            seen.setdefault((s, it["kv_head"], r), []).append((it["key_begin"], it["key_end"], it["kind"],
+                                                               it["split"], it["num_splits"]))
     for s, sp in enumerate(batch.seqs):
         for h in range(batch.num_kv_heads):
             for r in range(sp.query_len * G):
@@ -105,8 +115,17 @@ def _coverage(batch, items):
                 t = r // G
                 assert rngs[-1][1] >= sp.seq_len - sp.query_len + t + 1
                 assert rngs[-1][1] <= sp.seq_len
-                n = rngs[0][3]
-                assert len(rngs) == n and sorted(x[2] for x in rngs) == (list(range(n)) if n > 1 else [-1])
+                casc = [x for x in rngs if x[2] == 2]
+                own = [x for x in rngs if x[2] != 2]
+                if casc:               # cascade chunks then the sequence's own splits
+                    assert all(x[4] == len(casc) for x in casc)
+                    assert sorted(x[3] for x in casc) == list(range(len(casc)))
+                    assert all(x[2] == 0 and x[4] == len(own) + len(casc) for x in own)
+                    assert sorted(x[3] for x in own) == list(range(len(own)))
+                    assert casc[-1][1] == own[0][0] == prefix_len[prefix_group[s]]
+                else:
+                    n = rngs[0][4]
+                    assert len(rngs) == n and sorted(x[3] for x in rngs) == (list(range(n)) if n > 1 else [-1])
     assert not seen
 
 
@@ -156,3 +175,47 @@ def test_long_context_is_split():
                        head_dim=128, num_pages=12500, bt_stride=6250)
     assert all(it["num_splits"] > 1 for it in items)
     assert len(items) >= 148
+
+
+def _shared_inspect(b, **kw):
+    return pk.inspect(b.seq_lens, b.query_lens, b.mask_kinds, b.parents_flat, num_q_heads=b.num_q_heads,
+                      num_kv_heads=b.num_kv_heads, head_dim=b.head_dim, num_pages=b.k_cache.shape[0],
+                      bt_stride=b.block_table.shape[1], prefix_group=b.prefix_group,
+                      prefix_len=b.prefix_len, **kw)
+
+
+@pytest.mark.parametrize("seed, heads", [(0, (16, 4)), (1, (28, 4)), (2, (8, 8)), (3, (64, 2))])
+def test_planner_covers_shared_prefix_batches(seed, heads):
+    b = W.random_shared_small(seed, *heads)
+    items = _shared_inspect(b, num_sms=4, ctas_per_sm=1)
+    assert any(it["kind"] == 2 for it in items)
+    _coverage(b, items, b.prefix_group, b.prefix_len)
+
+
+def test_planner_covers_shared_prefix_config():
+    b = W.make_shared_config("llama3_8b_shared_prefix")
+    items = _shared_inspect(b)
+    _coverage(b, items, b.prefix_group, b.prefix_len)
+    casc = [it for it in items if it["kind"] == 2]
+    # 4 groups x 8 KV heads x (32 members' 48 query tokens / 64 tokens per task) x 4 chunks
+    assert len(casc) == 4 * 8 * 1 * 4
+
+
+@pytest.mark.parametrize("groups, lens, code", [
+    ([0, -1, 0], [16], -1),          # members not consecutive
+    ([0, 0, -1], [24], -1),          # not a page multiple
+    ([0, 0, -1], [48], -1),          # beyond the committed prefix of a member
+    ([0, 2, -1], [16], -1),          # group id out of range
+])
+def test_planner_rejects_bad_groups(groups, lens, code):
+    with pytest.raises(pk.PkvaError) as ei:
+        pk.inspect([40, 60, 30], [1, 1, 1], [0, 0, 0], num_q_heads=8, num_kv_heads=2, head_dim=128,
+                   num_pages=12, bt_stride=4, prefix_group=groups, prefix_len=lens)
+    assert ei.value.code == code
+
+
+def test_shared_prefix_needs_head_dim_128():
+    with pytest.raises(pk.PkvaError) as ei:
+        pk.inspect([40, 60], [1, 1], [0, 0], num_q_heads=8, num_kv_heads=2, head_dim=64,
+                   num_pages=12, bt_stride=4, prefix_group=[0, 0], prefix_len=[32])
+    assert ei.value.code == -2

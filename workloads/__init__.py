@@ -62,6 +62,10 @@ class Batch:
     page_perm: torch.Tensor          # [num_pages] int64 (CPU): logical page -> physical page
     seed: int = 0
     outlier_frac: float = 0.0
+    # shared-prefix groups: prefix_group[s] in {-1} U [0, G); the first prefix_len[g] keys of
+    # every member of group g are the same values on the same physical pages
+    prefix_group: Optional[List[int]] = None
+    prefix_len: Optional[List[int]] = None
 
     # -- convenience views (layout only) ---------------------------------------------
     @property
@@ -165,6 +169,132 @@ def config_seqs(name: str, gen: torch.Generator) -> tuple:
         seqs = [SeqSpec(L, 1, CAUSAL, []) for L in _randint(gen, 32768, 131072, 16)]
         return seqs, 128, 8, 128, 0.01
     raise KeyError(name)
+
+
+SHARED_CONFIG_NAMES = [
+    "llama3_8b_shared_prefix",   # 4 groups x 32 seqs on a shared 4096-key prefix, 32q/8kv, d128
+]
+
+
+def shared_config(name: str, gen: torch.Generator) -> tuple:
+    """(seqs, prefix_group, prefix_len, Hq, Hkv, d) for a named shared-prefix batch."""
+    if name == "llama3_8b_shared_prefix":
+        seqs, group = [], []
+        for g in range(4):
+            for i in range(32):
+                own = int(torch.randint(0, 1025, (1,), generator=gen).item())
+                if i % 4 == 3:          # every fourth member verifies a 5-node draft tree
+                    seqs.append(SeqSpec(4096 + own + 5, 5, TREE, random_tree(gen, 5)))
+                else:
+                    seqs.append(SeqSpec(4096 + own + 1, 1, CAUSAL, []))
+                group.append(g)
+        return seqs, group, [4096] * 4, 32, 8, 128
+    raise KeyError(name)
+
+
+def build_shared_batch(name: str, seqs: Sequence[SeqSpec], prefix_group: Sequence[int],
+                       prefix_len: Sequence[int], num_q_heads: int, num_kv_heads: int,
+                       head_dim: int, seed: int, device="cpu", page_size: int = 16,
+                       keep_contiguous: bool = True, bt_extra: int = 0) -> Batch:
+    """Like ``build_batch``, but the members of each group share the values and the physical
+    pages of their first ``prefix_len[g]`` keys (a common prompt held once in the cache).
+
+    Seeding as in ``build_batch``; the shared keys of group g are drawn once, after the
+    per-sequence values."""
+    device = torch.device(device)
+    sgen = torch.Generator().manual_seed(seed)
+    vgen = torch.Generator(device=device).manual_seed(seed + 1)
+    Hq, Hkv, d, P = num_q_heads, num_kv_heads, head_dim, page_size
+    B = len(seqs)
+    for s, g in zip(seqs, prefix_group):
+        if g >= 0 and (prefix_len[g] % P or prefix_len[g] > s.seq_len - s.query_len):
+            raise ValueError("a shared prefix must be page-aligned and within the committed prefix")
+
+    def randn_bf16(*shape):
+        return torch.randn(*shape, generator=vgen, device=device,
+                           dtype=torch.float32).to(torch.bfloat16)
+
+    total_q = sum(s.query_len for s in seqs)
+    total_kv = sum(s.seq_len for s in seqs)
+    q = randn_bf16(total_q, Hq, d)
+    k = randn_bf16(total_kv, Hkv, d)
+    v = randn_bf16(total_kv, Hkv, d)
+    shared_k = [randn_bf16(n, Hkv, d) for n in prefix_len]
+    shared_v = [randn_bf16(n, Hkv, d) for n in prefix_len]
+
+    # logical pages: each group's shared pages once, then every sequence's own pages
+    shared_pages = [n // P for n in prefix_len]
+    own_pages = [(s.seq_len + P - 1) // P - (shared_pages[g] if g >= 0 else 0)
+                 for s, g in zip(seqs, prefix_group)]
+    num_pages = sum(shared_pages) + sum(own_pages)
+    perm = torch.randperm(num_pages, generator=sgen)
+    group_first = []
+    acc = 0
+    for n in shared_pages:
+        group_first.append(acc)
+        acc += n
+    max_pages = max((s.seq_len + P - 1) // P for s in seqs) + bt_extra
+    block_table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    tok_page, tok_slot = [], []
+    kv_off = 0
+    for i, (s, g) in enumerate(zip(seqs, prefix_group)):
+        ns = shared_pages[g] if g >= 0 else 0
+        logical = list(range(group_first[g], group_first[g] + ns)) if g >= 0 else []
+        logical += list(range(acc, acc + own_pages[i]))
+        acc += own_pages[i]
+        block_table[i, :len(logical)] = perm[logical].to(torch.int32)
+        pos = torch.arange(s.seq_len)
+        tok_page.append(torch.tensor(logical, dtype=torch.long)[pos // P])
+        tok_slot.append(pos % P)
+        if g >= 0:
+            n = prefix_len[g]
+            k[kv_off:kv_off + n] = shared_k[g]
+            v[kv_off:kv_off + n] = shared_v[g]
+        kv_off += s.seq_len
+    tok_phys = perm[torch.cat(tok_page)].to(device)
+    tok_slot = torch.cat(tok_slot).to(device)
+    k_cache = (randn_bf16(num_pages, Hkv, P, d).float() * 50.0).to(torch.bfloat16)
+    v_cache = (randn_bf16(num_pages, Hkv, P, d).float() * 50.0).to(torch.bfloat16)
+    k_cache[tok_phys, :, tok_slot] = k
+    v_cache[tok_phys, :, tok_slot] = v
+    del tok_phys, tok_slot
+    return Batch(name=name, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=d, page_size=P,
+                 seqs=list(seqs), q=q, k=k if keep_contiguous else None,
+                 v=v if keep_contiguous else None, k_cache=k_cache, v_cache=v_cache,
+                 block_table=block_table.to(device), page_perm=perm, seed=seed,
+                 prefix_group=list(prefix_group), prefix_len=list(prefix_len))
+
+
+def random_shared_small(seed: int, Hq: int = 16, Hkv: int = 4, device="cpu") -> Batch:
+    """A small shared-prefix batch (head_dim 128): group 0 has six decode / verify members on
+    48 shared keys; one sequence belongs to no group; group 1 has three members on 160
+    shared keys, one of them a 100-token causal chunk (which runs as a prefill task)."""
+    gen = torch.Generator().manual_seed(seed)
+    seqs, group = [], []
+    for i in range(6):
+        own = int(torch.randint(0, 40, (1,), generator=gen).item())
+        T = 1 if i % 3 else 4
+        seqs.append(SeqSpec(48 + own + T, T, TREE if T == 4 else CAUSAL,
+                            random_tree(gen, 4) if T == 4 else []))
+        group.append(0)
+    seqs.append(SeqSpec(70, 2, CAUSAL, []))
+    group.append(-1)
+    for T in (3, 100, 1):
+        seqs.append(SeqSpec(160 + 20 + T, T, CAUSAL, []))
+        group.append(1)
+    return build_shared_batch(f"shared_small_{seed}", seqs, group, [48, 160], Hq, Hkv, 128, seed=seed,
+                              device=device)
+
+
+def make_shared_config(name: str, device="cpu", seed: Optional[int] = None,
+                       keep_contiguous: bool = True) -> Batch:
+    """A named shared-prefix batch (seeded by 100 + its index unless ``seed`` is given)."""
+    if seed is None:
+        seed = 100 + SHARED_CONFIG_NAMES.index(name)
+    sgen = torch.Generator().manual_seed(seed)
+    seqs, group, plen, Hq, Hkv, d = shared_config(name, sgen)
+    return build_shared_batch(name, seqs, group, plen, Hq, Hkv, d, seed=seed + 1000, device=device,
+                              keep_contiguous=keep_contiguous)
 
 
 def build_batch(name: str, seqs: Sequence[SeqSpec], num_q_heads: int, num_kv_heads: int,
