@@ -236,3 +236,37 @@ def gather_paged(cache: np.ndarray, block_table_row: Sequence[int], seq_len: int
         page = block_table_row[pos // P]
         rows.append(cache[page, :, pos % P, :])
     return np.stack(rows)
+
+
+# -------------------------------------------------------------------------------------
+# FP8 (E4M3) KV cache: decoding of the stored codes. The attention itself is unchanged:
+# the oracle decodes every code exactly (float64) and multiplies by the per-KV-head scale,
+# then runs the definition above on those values.
+# -------------------------------------------------------------------------------------
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """float64 value of each FP8 E4M3 code (one byte each).
+
+    The format, written out: bit 7 is the sign; bits 6..3 are a biased exponent e (bias 7);
+    bits 2..0 a mantissa m. e = 0 encodes subnormals m/8 * 2^-6; e in 1..15 encodes
+    (1 + m/8) * 2^(e-7), except e = 15 with m = 7, which is NaN. There are no infinities,
+    so the largest finite magnitude is (1 + 6/8) * 2^8 = 448.
+
+    Reading: the pages name FP8 and quantised KV-cache formats without fixing one (Arctic
+    Inference review page, section 3 comments); E4M3 of this form is taken as the FP8 KV
+    format, the plainest common choice.
+    """
+    c = np.asarray(codes).astype(np.int64) & 0xFF
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
+def dequantize_kv(codes: np.ndarray, scale_per_head: np.ndarray) -> np.ndarray:
+    """Values [L, Hkv, d] of an FP8 K or V tensor [L, Hkv, d] with one scale per KV head:
+    value = e4m3_decode(code) * scale[head]."""
+    s = np.asarray(scale_per_head, dtype=np.float64)
+    return e4m3_decode(codes) * s[None, :, None]

@@ -231,9 +231,34 @@ def pin9_split_merge():
             assert np.allclose(oracle.lse_merge(parts), full, atol=1e-12, rtol=0)
 
 
+def pin10_e4m3_codes():
+    """FP8 E4M3 decoding against values the format's definition fixes in closed form."""
+    d = oracle.e4m3_decode
+    fixed = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 / 8 * 2.0 ** -6, 0x08: 2.0 ** -6, 0x30: 0.5,
+             0x38: 1.0, 0x39: 1.125, 0x3F: 1.875, 0x40: 2.0, 0x44: 3.0, 0x70: 128.0, 0x78: 256.0,
+             0x7E: 448.0, 0xB8: -1.0, 0xC0: -2.0, 0xFE: -448.0, 0x81: -(2.0 ** -9)}
+    for c, val in fixed.items():
+        assert d(np.array([c]))[0] == val, hex(c)
+    assert np.signbit(d(np.array([0x80]))[0]) and d(np.array([0x80]))[0] == 0.0
+    assert np.isnan(d(np.array([0x7F, 0xFF]))).all()
+    pos = d(np.arange(0x00, 0x7F))
+    assert np.all(np.diff(pos) > 0)                        # codes 0..126 strictly increase
+    assert np.array_equal(d(np.arange(0x80, 0xFF)), -pos)  # the sign bit only negates
+    # consecutive normal codes in one binade are 1/8 of the binade apart
+    for e in range(1, 16):
+        base = 2.0 ** (e - 7)
+        vals = d(np.arange(e * 8, e * 8 + (7 if e == 15 else 8)))
+        assert np.allclose(np.diff(vals), base / 8, rtol=0, atol=0)
+    # dequantisation multiplies by the KV head's own scale
+    codes = np.array([[[0x38, 0x40]], [[0xC0, 0x08]]], dtype=np.uint8).repeat(2, axis=1)
+    deq = oracle.dequantize_kv(codes, np.array([0.5, 3.0]))
+    assert deq[0, 0, 0] == 0.5 and deq[0, 1, 0] == 3.0 and deq[1, 1, 0] == -6.0
+
+
 PINS = [pin1_rows_sum_to_one, pin2_single_key, pin3_identical_keys_give_mean,
         pin4_chain_tree_is_causal, pin5_decode_steps_match_prefill,
-        pin6_page_permutation_invariance, pin7_brute_force, pin8_sdpa, pin9_split_merge]
+        pin6_page_permutation_invariance, pin7_brute_force, pin8_sdpa, pin9_split_merge,
+        pin10_e4m3_codes]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -354,9 +379,39 @@ def _mut_merge_unweighted(orig):
     return {"lse_merge": lse_merge}
 
 
+def _mut_e4m3_bias_8(orig):
+    def e4m3_decode(codes):
+        return orig.e4m3_decode(codes) / 2.0                  # exponent bias 8 instead of 7
+    return {"e4m3_decode": e4m3_decode}
+
+
+def _mut_e4m3_no_subnormals(orig):
+    def e4m3_decode(codes):
+        c = np.asarray(codes).astype(np.int64) & 0xFF
+        v = orig.e4m3_decode(codes)
+        return np.where(((c >> 3) & 0xF) == 0, np.where(c & 0x80, -0.0, 0.0), v)   # flushed to zero
+    return {"e4m3_decode": e4m3_decode}
+
+
+def _mut_e4m3_ieee_style_inf(orig):
+    def e4m3_decode(codes):
+        c = np.asarray(codes).astype(np.int64) & 0xFF
+        v = orig.e4m3_decode(codes)
+        return np.where(((c >> 3) & 0xF) == 15, np.where(c & 7, np.nan, np.inf), v)   # top binade reserved
+    return {"e4m3_decode": e4m3_decode}
+
+
+def _mut_dequant_wrong_head(orig):
+    def dequantize_kv(codes, scale):
+        return orig.e4m3_decode(codes) * np.asarray(scale, np.float64)[::-1][None, :, None]
+    return {"dequantize_kv": dequantize_kv}
+
+
 MUTANTS = [_mut_gqa_modulo, _mut_causal_excludes_diagonal, _mut_tree_self_only,
            _mut_tree_parent_not_ancestors, _mut_no_max_subtraction_scale,
-           _mut_top_left_causal, _mut_transposed_value, _mut_merge_unweighted]
+           _mut_top_left_causal, _mut_transposed_value, _mut_merge_unweighted,
+           _mut_e4m3_bias_8, _mut_e4m3_no_subnormals, _mut_e4m3_ieee_style_inf,
+           _mut_dequant_wrong_head]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS, ids=lambda f: f.__name__)
