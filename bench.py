@@ -385,6 +385,33 @@ def run_ours(args):
             pl.close()
             del b, o
             torch.cuda.empty_cache()
+        # FP8 (E4M3) caches: the same batches through attn_plan_kv / attn_run_fp8 (every
+        # sequence as decode/verify tasks; algorithmic bytes are the FP8 bytes)
+        fp8 = {}
+        for name in ("llama3_8b_decode", "long_ctx_split", "qwen2_7b_unified"):
+            b = W.make_config(name, device=dev)
+            f = W.fp8_kv(b)
+            b.k = b.v = None
+            torch.cuda.empty_cache()
+            pl = pk.plan_for_batch(b, kv_fp8=True)
+            inf = pl.info()
+            o = torch.empty_like(b.q)
+
+            def step(pl=pl, b=b, f=f, o=o):
+                pl.run_fp8(b.q, f.k_cache, f.v_cache_t, f.k_scale, f.v_scale, o, stream)
+
+            ps = time_fn(step, args.other_steps, args.warmup, stream)
+            if pl.check(stream) != 0:
+                raise RuntimeError("device error in the FP8 measurement")
+            sec = sum(ps) / len(ps) * 1e-3
+            fp8[name] = {"ms_per_launch": sec * 1e3, "tokens_per_s": b.total_q / sec,
+                         "kv_bytes_fp8": inf["kv_bytes"], "roofline": roofline(inf, sec, peaks)}
+            if name in per_config:
+                fp8[name]["speedup_vs_bf16"] = per_config[name]["ms_per_launch"] / (sec * 1e3)
+            pl.close()
+            del b, f, o
+            torch.cuda.empty_cache()
+        per_config["fp8_kv"] = fp8
         # shared-prefix batch: cascade plan (attn_plan_shared) against the same batch planned
         # without groups; algorithmic bytes count the shared keys once in both
         for name in W.SHARED_CONFIG_NAMES:

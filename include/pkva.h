@@ -59,6 +59,11 @@ enum pkva_mask_kind {
     PKVA_TREE = 1      /* verify: committed prefix + ancestors-or-self in the draft tree */
 };
 
+enum pkva_kv_dtype {
+    PKVA_KV_BF16 = 0,      /* bf16 caches (attn_run)                                       */
+    PKVA_KV_FP8_E4M3 = 1   /* FP8 E4M3 codes with one scale per KV head (attn_run_fp8)     */
+};
+
 enum pkva_status {
     PKVA_OK = 0,
     PKVA_EINVAL = -1,        /* bad argument (message says which)                        */
@@ -141,6 +146,45 @@ PKVA_API int attn_plan_shared(pkva_plan_t* out_plan, int num_seqs, const int32_t
               int num_pages, const int32_t* mask_kind, const int32_t* parents,
               int num_q_heads, int num_kv_heads, int head_dim, int page_size, float sm_scale,
               const int32_t* prefix_group, const int32_t* prefix_len, int num_groups);
+
+/*
+ * attn_plan_kv — attn_plan with the caches' element format: PKVA_KV_BF16 (the same as
+ * attn_plan) or PKVA_KV_FP8_E4M3 (run with attn_run_fp8).
+ *
+ * Cites: Arctic Inference review page, section 3 comments (the KV cache is held in the
+ * quantization formats the system supports; FP8 is named beside FP16). FP8 halves the
+ * bytes of the bandwidth-bound decode/verify path.
+ *
+ * An FP8 plan runs every sequence as decode/verify tasks (prefill chunks too: no
+ * tensor-core prefill tasks) and cannot be used with attn_run, attn_run_host or
+ * attn_run_append. Other arguments and errors as attn_plan; PKVA_EINVAL for an unknown
+ * kv_dtype, PKVA_EUNSUPPORTED with PKVA_DECODE_BODY=fma.
+ */
+PKVA_API int attn_plan_kv(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq_lens,
+              const int32_t* query_lens, const int32_t* block_table, int bt_stride,
+              int num_pages, const int32_t* mask_kind, const int32_t* parents,
+              int num_q_heads, int num_kv_heads, int head_dim, int page_size, float sm_scale,
+              int kv_dtype);
+
+/*
+ * attn_run_fp8 — attn_run over FP8 E4M3 caches (a plan made with PKVA_KV_FP8_E4M3).
+ *
+ *   q          device bf16 [sum T_s, Hq, D] (as attn_run; |q| must stay in f16's range,
+ *              the kernels compute in f16 with fp32 accumulation).
+ *   k_cache    device uint8 [num_pages, Hkv, page_size, D]: E4M3 codes, the same layout
+ *              as the bf16 cache.
+ *   v_cache_t  device uint8 [num_pages, Hkv, D, page_size]: E4M3 codes, each (page, KV
+ *              head) block TRANSPOSED (head-dim rows of page_size keys).
+ *   k_scale,
+ *   v_scale    device float32 [Hkv]: the value of a code c of KV head h is e4m3(c) * scale[h]
+ *              (E4M3: sign, 4 exponent bits with bias 7, 3 mantissa bits, no infinities,
+ *              S.1111.111 is NaN).
+ *   out        device bf16 [sum T_s, Hq, D].
+ * Codes in slots past a sequence's end may be anything (NaN codes included). Errors as
+ * attn_run; PKVA_EINVAL if the plan is not an FP8 plan or a scale pointer is NULL.
+ */
+PKVA_API int attn_run_fp8(pkva_plan_t plan, const void* q, const void* k_cache, const void* v_cache_t,
+                 const float* k_scale, const float* v_scale, void* out, void* stream);
 
 /*
  * attn_run — compute the batch's attention on `stream` (asynchronous).

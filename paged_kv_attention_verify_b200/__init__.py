@@ -27,11 +27,13 @@ TREE = 1
 PKVA_OK = 0
 STATUS_NAMES = {0: "PKVA_OK", -1: "PKVA_EINVAL", -2: "PKVA_EUNSUPPORTED", -3: "PKVA_ECUDA",
                 -4: "PKVA_ENOMEM", -5: "PKVA_EDEVICE"}
+KV_BF16 = 0
+KV_FP8_E4M3 = 1
 DEVERR_BAD_PAGE = 0x1
 DEVERR_TIMEOUT = 0x2
 
 # every entry point that include/pkva.h declares
-EXPORTED = ["attn_plan", "attn_plan_shared", "attn_run", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_destroy",
+EXPORTED = ["attn_plan", "attn_plan_shared", "attn_plan_kv", "attn_run", "attn_run_fp8", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_destroy",
             "attn_last_error", "attn_plan_get_info", "attn_plan_inspect", "attn_run_static",
             "pkva_selftest_wait_timeout"]
 
@@ -76,6 +78,8 @@ def lib() -> ctypes.CDLL:
                             ctypes.c_int, _i32p, _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                             ctypes.c_int, ctypes.c_float]
     L.attn_plan_shared.argtypes = L.attn_plan.argtypes + [_i32p, _i32p, ctypes.c_int]
+    L.attn_plan_kv.argtypes = L.attn_plan.argtypes + [ctypes.c_int]
+    L.attn_run_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
     L.attn_run.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp]
     L.attn_run_append.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
     L.attn_run_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp]
@@ -93,7 +97,7 @@ def lib() -> ctypes.CDLL:
                                   _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                   ctypes.c_float, _vp, _vp, _vp, _vp, _vp]
     L.pkva_selftest_wait_timeout.argtypes = [ctypes.c_longlong, _i32p]
-    for name in ("attn_plan", "attn_plan_shared", "attn_run", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_get_info",
+    for name in ("attn_plan", "attn_plan_shared", "attn_plan_kv", "attn_run_fp8", "attn_run", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_get_info",
                  "attn_plan_inspect", "attn_run_static", "pkva_selftest_wait_timeout"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -128,9 +132,9 @@ class Plan:
                  num_q_heads: int, num_kv_heads: int, head_dim: int, num_pages: int,
                  page_size: int = 16, sm_scale: Optional[float] = None,
                  prefix_group: Optional[Sequence[int]] = None,
-                 prefix_len: Optional[Sequence[int]] = None):
+                 prefix_len: Optional[Sequence[int]] = None, kv_fp8: bool = False):
         """``attn_plan``; with ``prefix_group`` / ``prefix_len`` (shared-prefix groups),
-        ``attn_plan_shared``."""
+        ``attn_plan_shared``; with ``kv_fp8``, ``attn_plan_kv`` for FP8 E4M3 caches."""
         import torch
         self._handle = None
         sl, ql, mk = _i32(seq_lens), _i32(query_lens), _i32(mask_kind)
@@ -153,7 +157,12 @@ class Plan:
         args = (ctypes.byref(h), len(sl), _ptr(sl), _ptr(ql), bt_ptr, bt_stride, num_pages, _ptr(mk),
                 _ptr(par), num_q_heads, num_kv_heads, head_dim, page_size,
                 float(sm_scale) if sm_scale else 0.0)
-        if prefix_group is None:
+        self.kv_fp8 = kv_fp8
+        if kv_fp8:
+            if prefix_group is not None:
+                raise ValueError("shared-prefix groups are not supported with FP8 caches")
+            _check(lib().attn_plan_kv(*args, KV_FP8_E4M3))
+        elif prefix_group is None:
             _check(lib().attn_plan(*args))
         else:
             pg, pl = _i32(prefix_group), _i32(prefix_len if prefix_len is not None else [])
@@ -197,6 +206,25 @@ class Plan:
         _check(lib().attn_run_append(self._handle, q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(),
                                      k_cache.data_ptr(), v_cache.data_ptr(), out.data_ptr(),
                                      _stream_handle(stream)))
+        return out
+
+    def run_fp8(self, q, k_cache, v_cache_t, k_scale, v_scale, out=None, stream=None):
+        """``attn_run_fp8``: E4M3 codes (uint8) in ``k_cache`` [pages, Hkv, 16, D] and, each
+        page block transposed, ``v_cache_t`` [pages, Hkv, D, 16]; float32 scales [Hkv]."""
+        import torch
+        if out is None:
+            out = torch.empty_like(q)
+        D, Hq, Hkv = self.head_dim, self.num_q_heads, self.num_kv_heads
+        checks = (("q", q, (self.total_q, Hq, D), torch.bfloat16), ("out", out, (self.total_q, Hq, D), torch.bfloat16),
+                  ("k_cache", k_cache, (self.num_pages, Hkv, self.page_size, D), torch.uint8),
+                  ("v_cache_t", v_cache_t, (self.num_pages, Hkv, D, self.page_size), torch.uint8),
+                  ("k_scale", k_scale, (Hkv,), torch.float32), ("v_scale", v_scale, (Hkv,), torch.float32))
+        for name, t, shape, dt in checks:
+            if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != dt or tuple(t.shape) != shape \
+                    or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous {dt} CUDA tensor {shape}")
+        _check(lib().attn_run_fp8(self._handle, q.data_ptr(), k_cache.data_ptr(), v_cache_t.data_ptr(),
+                                  k_scale.data_ptr(), v_scale.data_ptr(), out.data_ptr(), _stream_handle(stream)))
         return out
 
     def run_host(self, q_host, k_cache, v_cache, out_host, stream=None):
@@ -282,12 +310,14 @@ def selftest_wait_timeout(limit_ns: int = 20_000_000) -> int:
     return int(err.value)
 
 
-def plan_for_batch(batch, sm_scale: Optional[float] = None, shared: bool = True) -> Plan:
+def plan_for_batch(batch, sm_scale: Optional[float] = None, shared: bool = True, kv_fp8: bool = False) -> Plan:
     """Plan a ``workloads.Batch`` (a convenience for tests and the benchmark); a batch with
-    shared-prefix groups is planned with them unless ``shared`` is False."""
-    groups = getattr(batch, "prefix_group", None) if shared else None
+    shared-prefix groups is planned with them unless ``shared`` is False; ``kv_fp8`` plans
+    for FP8 caches."""
+    groups = getattr(batch, "prefix_group", None) if shared and not kv_fp8 else None
     return Plan(batch.seq_lens, batch.query_lens, batch.block_table, batch.mask_kinds,
                 batch.parents_flat, num_q_heads=batch.num_q_heads, num_kv_heads=batch.num_kv_heads,
                 head_dim=batch.head_dim, num_pages=batch.k_cache.shape[0],
                 page_size=batch.page_size, sm_scale=sm_scale,
-                prefix_group=groups, prefix_len=batch.prefix_len if groups is not None else None)
+                prefix_group=groups, prefix_len=batch.prefix_len if groups is not None else None,
+                kv_fp8=kv_fp8)

@@ -68,6 +68,31 @@ static bool encode_cache_map(CUtensorMap* map, const void* base, int num_pages, 
     return r == CUDA_SUCCESS;
 }
 
+// FP8 caches: K as a 2-D byte tensor [num_pages * Hkv * 16 rows, D] with one page block
+// per box (128-byte swizzle at D = 128, 64-byte at D = 64); V, transposed per page block, as
+// [num_pages * Hkv * D rows, 16] with one D x 16 box per block, unswizzled.
+static bool encode_fp8_maps(CUtensorMap* mk, CUtensorMap* mv, const void* k, const void* vt, int num_pages, int Hkv,
+                            int D) {
+    auto fn = tensor_map_encoder();
+    if (!fn) return false;
+    cuuint32_t estr[2] = {1, 1};
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)num_pages * Hkv * kPageSize};
+        cuuint64_t strides[1] = {(cuuint64_t)D};
+        cuuint32_t box[2] = {(cuuint32_t)D, (cuuint32_t)kPageSize};
+        if (fn(mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(k), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    cuuint64_t dims[2] = {(cuuint64_t)kPageSize, (cuuint64_t)num_pages * Hkv * D};
+    cuuint64_t strides[1] = {(cuuint64_t)kPageSize};
+    cuuint32_t box[2] = {(cuuint32_t)kPageSize, (cuuint32_t)D};
+    return fn(mv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(vt), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // q viewed as the 3-D bf16 tensor [sum T][Hq][D]; one box is 128 tokens x 64 columns of
 // one head, stored with the 128-byte swizzle (the prefill kernel's A operand layout). The
 // new tokens' K and V ([sum T][Hkv][D]) use the same view with Hkv heads. Cascade tasks
@@ -105,6 +130,7 @@ struct pkva_plan {
     int num_sms = 0;
     int decode_ctas = 0;
     bool decode_mma = true;
+    bool kv_fp8 = false;                    // caches are FP8 E4M3 codes (attn_run_fp8)
     const int32_t* block_table = nullptr;
     pkva::SeqInfo* d_seqs = nullptr;
     pkva::DecodeWork* d_dwork = nullptr;
@@ -160,7 +186,8 @@ static void free_plan(pkva_plan* p) {
 
 extern "C" const char* attn_last_error(void) { return g_last_error.c_str(); }
 
-static int plan_create(pkva_plan_t* out_plan, PlanArgs a, const int32_t* block_table, const char* who) {
+static int plan_create(pkva_plan_t* out_plan, PlanArgs a, const int32_t* block_table, const char* who,
+                       bool kv_fp8 = false) {
     const std::string name(who);
     if (!out_plan) {
         set_last_error(name + ": out_plan is NULL");
@@ -201,6 +228,7 @@ static int plan_create(pkva_plan_t* out_plan, PlanArgs a, const int32_t* block_t
     p->num_sms = sms;
     p->block_table = block_table;
     p->decode_mma = decode_body_is_mma();
+    p->kv_fp8 = kv_fp8;
 
     // Decode tasks are balanced over slots of four page-streaming warps: the unified kernel
     // runs one block per SM holding three decode tasks, the stand-alone CUDA-core kernel its
@@ -226,6 +254,11 @@ static int plan_create(pkva_plan_t* out_plan, PlanArgs a, const int32_t* block_t
         free_plan(p);
         set_last_error(name + ": " + err);
         return rc;
+    }
+    if (kv_fp8 && !p->decode_mma) {
+        free_plan(p);
+        set_last_error(name + ": FP8 caches need the tensor-core decode body (PKVA_DECODE_BODY=fma)");
+        return PKVA_EUNSUPPORTED;
     }
     if (!p->decode_mma && !p->hp.cwork.empty()) {
         free_plan(p);
@@ -287,6 +320,23 @@ extern "C" int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq
     return plan_create(out_plan, a, block_table, "attn_plan");
 }
 
+extern "C" int attn_plan_kv(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq_lens, const int32_t* query_lens,
+                            const int32_t* block_table, int bt_stride, int num_pages, const int32_t* mask_kind,
+                            const int32_t* parents, int num_q_heads, int num_kv_heads, int head_dim, int page_size,
+                            float sm_scale, int kv_dtype) {
+    if (kv_dtype != PKVA_KV_BF16 && kv_dtype != PKVA_KV_FP8_E4M3) {
+        set_last_error("attn_plan_kv: kv_dtype must be PKVA_KV_BF16 or PKVA_KV_FP8_E4M3");
+        if (out_plan) *out_plan = nullptr;
+        return PKVA_EINVAL;
+    }
+    PlanArgs a{num_seqs, seq_lens, query_lens, bt_stride, num_pages, mask_kind, parents, num_q_heads,
+               num_kv_heads, head_dim, page_size, sm_scale, 1, 1};
+    const bool fp8 = kv_dtype == PKVA_KV_FP8_E4M3;
+    a.use_prefill_kernel = !fp8;     // FP8 caches: every sequence runs as decode/verify tasks
+    a.kv_elem_bytes = fp8 ? 1 : 2;
+    return plan_create(out_plan, a, block_table, "attn_plan_kv", fp8);
+}
+
 extern "C" int attn_plan_shared(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq_lens,
                                 const int32_t* query_lens, const int32_t* block_table, int bt_stride, int num_pages,
                                 const int32_t* mask_kind, const int32_t* parents, int num_q_heads, int num_kv_heads,
@@ -334,7 +384,8 @@ extern "C" int attn_plan_get_info(pkva_plan_t plan, pkva_plan_info* info) {
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 static int run_impl(pkva_plan_t plan, const void* q, const void* k_new, const void* v_new, const void* k_cache,
-                    const void* v_cache, void* out, void* stream, const char* who) {
+                    const void* v_cache, void* out, void* stream, const char* who, const float* k_scale = nullptr,
+                    const float* v_scale = nullptr, bool fp8 = false) {
     const std::string name(who);
     if (!plan) {
         set_last_error(name + ": plan is NULL");
@@ -342,7 +393,16 @@ static int run_impl(pkva_plan_t plan, const void* q, const void* k_new, const vo
     }
     const HostPlan& hp = plan->hp;
     const bool append = k_new != nullptr || v_new != nullptr;
+    if (fp8 != plan->kv_fp8) {
+        set_last_error(name + (plan->kv_fp8 ? ": the plan is for FP8 caches (use attn_run_fp8)"
+                                            : ": the plan is for bf16 caches (plan with attn_plan_kv for FP8)"));
+        return PKVA_EINVAL;
+    }
     if (hp.num_seqs == 0) return PKVA_OK;
+    if (fp8 && (!k_scale || !v_scale)) {
+        set_last_error(name + ": k_scale / v_scale is NULL");
+        return PKVA_EINVAL;
+    }
     if (!q || !k_cache || !v_cache || !out || (append && (!k_new || !v_new))) {
         set_last_error(name + ": NULL tensor pointer");
         return PKVA_EINVAL;
@@ -357,6 +417,14 @@ static int run_impl(pkva_plan_t plan, const void* q, const void* k_new, const vo
         return PKVA_EUNSUPPORTED;
     }
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (fp8 && (plan->tm_k != k_cache || plan->tm_v != v_cache)) {
+        if (!encode_fp8_maps(&plan->tmK, &plan->tmV, k_cache, v_cache, hp.num_pages, hp.Hkv, hp.D)) {
+            set_last_error(name + ": cuTensorMapEncodeTiled failed for the FP8 caches");
+            return PKVA_ECUDA;
+        }
+        plan->tm_k = k_cache;
+        plan->tm_v = v_cache;
+    }
     if (plan->tm_k != k_cache) {
         if (!encode_cache_map(&plan->tmK, k_cache, hp.num_pages, hp.Hkv, hp.D)) {
             set_last_error(name + ": cuTensorMapEncodeTiled failed for k_cache");
@@ -439,6 +507,8 @@ static int run_impl(pkva_plan_t plan, const void* q, const void* k_new, const vo
     dp.G = hp.G;
     dp.num_pages = hp.num_pages;
     dp.scale_log2 = pp.scale_log2;
+    dp.k_scale = k_scale;
+    dp.v_scale = v_scale;
     if (append) {
         pp.append = dp.append = 1;
         pp.k_new = dp.k_new = static_cast<const __nv_bfloat16*>(k_new);
@@ -459,7 +529,7 @@ static int run_impl(pkva_plan_t plan, const void* q, const void* k_new, const vo
         ap.num_blocks = (int32_t)hp.order.size();
         ap.num_decode = (int32_t)hp.dwork.size();
         e = launch_attn(ap, hp.D, hp.decode_rows, has_prefill, plan->tmQ, plan->tmK, plan->tmV, tmKn, tmVn,
-                        plan->tmQc, st);
+                        plan->tmQc, st, fp8);
     } else {
         // comparison mode: decode tasks on the CUDA-core kernel, prefill tasks after them
         e = launch_decode(dp, (int)hp.dwork.size(), hp.D, hp.decode_rows, false, plan->tmK, plan->tmV, st);
@@ -486,7 +556,17 @@ extern "C" int attn_run_append(pkva_plan_t plan, const void* q, const void* k_ne
         set_last_error("attn_run_append: k_new / v_new is NULL");
         return PKVA_EINVAL;
     }
+    if (plan && plan->kv_fp8) {
+        set_last_error("attn_run_append: not supported on FP8 caches");
+        return PKVA_EUNSUPPORTED;
+    }
     return run_impl(plan, q, k_new, v_new, k_cache, v_cache, out, stream, "attn_run_append");
+}
+
+extern "C" int attn_run_fp8(pkva_plan_t plan, const void* q, const void* k_cache, const void* v_cache_t,
+                            const float* k_scale, const float* v_scale, void* out, void* stream) {
+    return run_impl(plan, q, nullptr, nullptr, k_cache, v_cache_t, out, stream, "attn_run_fp8", k_scale, v_scale,
+                    true);
 }
 
 extern "C" int attn_run_host(pkva_plan_t plan, const void* q_host, const void* k_cache, const void* v_cache,

@@ -33,33 +33,35 @@ constexpr int kDecWarps = 4;                      // page-streaming warps per de
 static_assert(kAttnThreads >= pre::kPThreadsAppend, "block too small for a prefill task");
 static_assert(kAttnThreads == kDecTasksPerBlock * 128, "one 128-thread group per decode task");
 
-template <int D>
+template <int D, bool FP8 = false>
 struct AttnNS {
-    static constexpr int value = D == 64 ? 4 : 2;  // decode stages per warp
+    // decode stages per warp: 16 KB of pages in flight per warp in every form
+    static constexpr int value = (D == 64 ? 4 : 2) * (FP8 ? 2 : 1);
 };
 
-template <int D, int NT>
+template <int D, int NT, bool FP8 = false>
 struct AttnSmem {
-    using DC = dec::DecodeCfg<D, NT * 8, false, kDecWarps, AttnNS<D>::value>;
+    using DC = dec::DecodeCfg<D, NT * 8, false, kDecWarps, AttnNS<D, FP8>::value, FP8 ? 1 : 2>;
     static constexpr int GROUP_BYTES = (DC::BYTES + 1023) / 1024 * 1024;    // one decode task
     static constexpr int DEC_BYTES = kDecTasksPerBlock * GROUP_BYTES;
-    static constexpr int TASK_BYTES = (D == 128 && pre::kSmemBytes > DEC_BYTES) ? pre::kSmemBytes : DEC_BYTES;
+    static constexpr int TASK_BYTES = (D == 128 && !FP8 && pre::kSmemBytes > DEC_BYTES) ? pre::kSmemBytes : DEC_BYTES;
     static constexpr int OFF_SCHED = TASK_BYTES;  // the TMEM address of a tensor-core block
     static constexpr int BYTES = TASK_BYTES + 64;
     static constexpr int ALLOC = BYTES + 1008;    // room to align to 1024
     static_assert(ALLOC <= 227 * 1024, "shared memory");
 };
 
-template <int D, int NT>
+// FP8: decode/verify tasks only (a plan over FP8 caches has no tensor-core tasks).
+template <int D, int NT, bool FP8>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKn,
             const __grid_constant__ CUtensorMap tmVn, const __grid_constant__ CUtensorMap tmQc) {
-    using S = AttnSmem<D, NT>;
+    using S = AttnSmem<D, NT, FP8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int e = p.order[blockIdx.x];
-    if constexpr (D == 128) {
+    if constexpr (D == 128 && !FP8) {
         if (e >= 0) {
             // tensor-core task: 512 TMEM columns for the block (one block per SM)
             uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + S::OFF_SCHED);
@@ -86,19 +88,21 @@ attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const _
     const int task = (-1 - e) * kDecTasksPerBlock + g;
     if (task >= p.num_decode) return;
     const dec::Group grp{(int)threadIdx.x & 127, 128, 1 + g};
-    dec::decode_mma_task<D, NT, kDecWarps, AttnNS<D>::value>(grp, p.dec, task, tmK, tmV, sm + g * S::GROUP_BYTES);
+    dec::decode_mma_task<D, NT, kDecWarps, AttnNS<D, FP8>::value, FP8>(grp, p.dec, task, tmK, tmV,
+                                                                    sm + g * S::GROUP_BYTES);
 }
 
-template <int D, int NT>
+template <int D, int NT, bool FP8>
 cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                      const CUtensorMap& tmKn, const CUtensorMap& tmVn, const CUtensorMap& tmQc,
                      cudaStream_t stream) {
-    using S = AttnSmem<D, NT>;
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::ALLOC);
+    using S = AttnSmem<D, NT, FP8>;
+    cudaError_t e =
+        cudaFuncSetAttribute(attn_kernel<D, NT, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::ALLOC);
     if (e != cudaSuccess) return e;
     const int grid = p.num_blocks;
     if (grid == 0) return cudaSuccess;
-    attn_kernel<D, NT><<<grid, kAttnThreads, S::ALLOC, stream>>>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc);
+    attn_kernel<D, NT, FP8><<<grid, kAttnThreads, S::ALLOC, stream>>>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc);
     return cudaGetLastError();
 }
 
@@ -106,13 +110,24 @@ template <int D, int NT>
 int ctas_t() {
     using S = AttnSmem<D, NT>;
     int n = 0;
-    if (cudaFuncSetAttribute(attn_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::ALLOC) !=
+    if (cudaFuncSetAttribute(attn_kernel<D, NT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::ALLOC) !=
         cudaSuccess)
         return 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_kernel<D, NT>, kAttnThreads, S::ALLOC) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_kernel<D, NT, false>, kAttnThreads, S::ALLOC) !=
         cudaSuccess)
         return 0;
     return n;
+}
+
+template <bool FP8>
+cudaError_t launch_kv(const AttnParams& p, int D, int rows, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                      const CUtensorMap& tmV, const CUtensorMap& tmKn, const CUtensorMap& tmVn,
+                      const CUtensorMap& tmQc, cudaStream_t stream) {
+    if (D == 64)
+        return rows <= 8 ? launch_t<64, 1, FP8>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
+                         : launch_t<64, 2, FP8>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
+    return rows <= 8 ? launch_t<128, 1, FP8>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
+                     : launch_t<128, 2, FP8>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
 }
 
 }  // namespace
@@ -125,14 +140,10 @@ int attn_ctas_per_sm(int D, int rows) {
 
 cudaError_t launch_attn(const AttnParams& p, int D, int rows, bool has_prefill, const CUtensorMap& tmQ,
                         const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKn,
-                        const CUtensorMap& tmVn, const CUtensorMap& tmQc, cudaStream_t stream) {
-    if (D == 64) {
-        if (has_prefill) return cudaErrorInvalidValue;   // prefill and cascade tasks need head_dim 128
-        return rows <= 8 ? launch_t<64, 1>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
-                         : launch_t<64, 2>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
-    }
-    return rows <= 8 ? launch_t<128, 1>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
-                     : launch_t<128, 2>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
+                        const CUtensorMap& tmVn, const CUtensorMap& tmQc, cudaStream_t stream, bool fp8) {
+    if ((D == 64 || fp8) && has_prefill) return cudaErrorInvalidValue;   // tensor-core tasks: bf16, head_dim 128
+    return fp8 ? launch_kv<true>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
+               : launch_kv<false>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
 }
 
 }  // namespace pkva

@@ -35,11 +35,11 @@ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
 // Shared-memory map of one task. NR = rows the launch is compiled for; QF = whether the
 // CUDA-core body's staged Q and P buffers are present; NW = page-streaming warps; NS =
-// stages per warp.
-template <int D, int NR, bool QF, int NW, int NS_>
+// stages per warp; EB = bytes per cached K/V element (2 bf16, 1 FP8).
+template <int D, int NR, bool QF, int NW, int NS_, int EB = 2>
 struct DecodeCfg {
     static constexpr int NS = NS_;
-    static constexpr int PAGE_BYTES = kPageSize * D * 2;
+    static constexpr int PAGE_BYTES = kPageSize * D * EB;
     static constexpr int STAGE_BYTES = 2 * PAGE_BYTES;              // K page + V page
     static constexpr int HALF = D / 2;                              // columns per lane half
     static constexpr int QROW = D + 8;                              // floats per staged Q row
@@ -124,27 +124,39 @@ __device__ __forceinline__ void task_setup(const Group& grp, const DecodeParams&
 }
 
 // Load page #i of this warp's stream (lane 0 only); ph is its physical page, -1 for none.
-template <int D, int NS, int STAGE_BYTES, int PAGE_BYTES>
+// bf16: K and V as 16 x 64 boxes (128-byte swizzle). FP8: the K page as one 16 x D-byte box
+// (128- or 64-byte swizzle) and the transposed V page as one D x 16-byte box.
+template <int D, int NS, int STAGE_BYTES, int PAGE_BYTES, bool FP8 = false>
 __device__ __forceinline__ void issue_page_at(const DecodeParams& p, const DecodeWork& w, int ph, uint8_t* ring,
                                               uint64_t* bar, int i, const CUtensorMap* tmK, const CUtensorMap* tmV) {
     const int stage = i % NS;
-    const int row = ph >= 0 ? (ph * p.Hkv + w.kv_head) * kPageSize : -kPageSize;
+    const int blk = ph >= 0 ? ph * p.Hkv + w.kv_head : -1;       // (page, KV head) block; -1 reads zeros
     uint8_t* dst = ring + stage * STAGE_BYTES;
     mbar_arrive_expect_tx(&bar[stage], STAGE_BYTES);
+    if constexpr (FP8) {
+        tma_load_2d(dst, tmK, &bar[stage], 0, blk * kPageSize);
+        tma_load_2d(dst + PAGE_BYTES, tmV, &bar[stage], 0, blk * D);
+    } else {
 #pragma unroll
-    for (int b = 0; b < D / 64; ++b) {
-        tma_load_2d(dst + b * kBoxBytes, tmK, &bar[stage], b * 64, row);
-        tma_load_2d(dst + PAGE_BYTES + b * kBoxBytes, tmV, &bar[stage], b * 64, row);
+        for (int b = 0; b < D / 64; ++b) {
+            tma_load_2d(dst + b * kBoxBytes, tmK, &bar[stage], b * 64, blk * kPageSize);
+            tma_load_2d(dst + PAGE_BYTES + b * kBoxBytes, tmV, &bar[stage], b * 64, blk * kPageSize);
+        }
     }
 }
 
 // Load page #i of this warp's stream from the staged block-table slice (lane 0 only).
-template <int D, int NS, int STAGE_BYTES, int PAGE_BYTES, int NW>
+template <int D, int NS, int STAGE_BYTES, int PAGE_BYTES, int NW, bool FP8 = false>
 __device__ __forceinline__ void issue_page(const DecodeParams& p, const DecodeWork& w, const int* bts,
                                            uint8_t* ring, uint64_t* bar, int warp, int i,
                                            const CUtensorMap* tmK, const CUtensorMap* tmV) {
-    issue_page_at<D, NS, STAGE_BYTES, PAGE_BYTES>(p, w, bts[warp + NW * i], ring, bar, i, tmK, tmV);
+    issue_page_at<D, NS, STAGE_BYTES, PAGE_BYTES, FP8>(p, w, bts[warp + NW * i], ring, bar, i, tmK, tmV);
 }
+
+// FP8 page body: the M row m of the K operand (and of S^T) holds key sigma(m) of the page,
+// so that after the in-register transpose of P its k slots line up with the keys the
+// transposed V operand delivers (four consecutive keys per lane, see decode_mma_task).
+__device__ __forceinline__ int fp8_key_of_row(int m) { return ((m & 7) >> 1) * 4 + (m >> 3) * 2 + (m & 1); }
 
 // Merge the four warps' (max, sum, unnormalised output) held in cm/cl/co, then either
 // write the rows (whole unit) or a split partial; the last split of a unit merges all
@@ -211,11 +223,23 @@ __device__ __forceinline__ void merge_and_store(const Group& grp, const DecodePa
 // =====================================================================================
 // One decode/verify task on the tensor-core page body. Every thread of the block calls it;
 // warps [0, NW) stream pages, any further warps only take part in the block barriers.
-template <int D, int NT, int NW, int NS>
+//
+// FP8 (E4M3 codes, one scale per KV head): the same tiles in f16 (every E4M3 value is an
+// f16 value, and bf16 Q converts exactly in f16's normal range). ldmatrix reads the codes
+// as 16-bit pairs, so a lane holds four consecutive bytes of a row where the bf16 layout
+// would give it two pairs eight apart; the k slots of both operands are permuted alike:
+//   QK^T: k slots (2t, 2t+1) and (2t+8, 2t+9) of a 16-column step take head-dim columns
+//         (4t, 4t+1) and (4t+2, 4t+3); Q is loaded (or staged) in that order;
+//   PV:   V is cached transposed per page ([D][16] bytes), so its rows are head-dim
+//         columns and a lane holds keys 4t..4t+3; S^T's M rows are permuted
+//         (fp8_key_of_row) so that after the transpose of P its k slots (2t, 2t+1) and
+//         (2t+8, 2t+9) are exactly keys (4t, 4t+1) and (4t+2, 4t+3).
+// The K scale folds into the softmax scale and the V scale into the output.
+template <int D, int NT, int NW, int NS, bool FP8 = false>
 __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodeParams& p, int task,
                                                 const CUtensorMap& tmK, const CUtensorMap& tmV, uint8_t* sm) {
     constexpr int NR = NT * 8;
-    using C = DecodeCfg<D, NR, false, NW, NS>;
+    using C = DecodeCfg<D, NR, false, NW, NS, FP8 ? 1 : 2>;
     constexpr int KS = D / 16;                    // k-steps of QK^T; d-tiles of PV
 
     const int tid = grp.tid, warp = tid >> 5, lane = tid & 31;
@@ -249,7 +273,7 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
         for (int i = 0; i < C::NS && i < n_my; ++i) {
             int ph = btrow[warp + NW * i];
             if (ph < 0 || ph >= p.num_pages) ph = -1;     // flagged by the slice staging below
-            issue_page_at<D, C::NS, C::STAGE_BYTES, C::PAGE_BYTES>(p, w, ph, ring, bar, i, &tmK, &tmV);
+            issue_page_at<D, C::NS, C::STAGE_BYTES, C::PAGE_BYTES, FP8>(p, w, ph, ring, bar, i, &tmK, &tmV);
         }
     }
     task_setup<NR, C::NS, NW>(grp, p, w, si, bts, rlim, ranc, rout, bars, flag, &tmK, &tmV, false);
@@ -260,12 +284,53 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
     constexpr int QREG = C::QB ? 1 : KS;
     uint32_t qf[NT][QREG][2];
     uint8_t* qs = sm + C::OFF_QB;
-    if constexpr (C::QB) {
+    if constexpr (C::QB && FP8) {
+        // f16, each 16-column group stored as columns 0,1,4,5,8,9,12,13, 2,3,6,7,10,11,14,15
+        for (int idx = tid; idx < NR * (D / 16); idx += grp.n) {
+            const int r = idx / (D / 16), j = idx - r * (D / 16);
+            uint32_t lo[4] = {0u, 0u, 0u, 0u}, hi[4] = {0u, 0u, 0u, 0u};
+            if (r < R) {
+                const uint4* src = reinterpret_cast<const uint4*>(p.q + (int64_t)q_row_index(p, si, w, r) * D + j * 16);
+                const uint4 a = src[0], b = src[1];
+                const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};   // bf16 pairs (2t', 2t'+1)
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    float x0, x1, x2, x3;
+                    bf16x2_to_f32(wv[2 * t], x0, x1);
+                    bf16x2_to_f32(wv[2 * t + 1], x2, x3);
+                    lo[t] = pack_f16x2(x0, x1);          // columns 4t, 4t+1
+                    hi[t] = pack_f16x2(x2, x3);          // columns 4t+2, 4t+3
+                }
+            }
+            *reinterpret_cast<uint4*>(qs + r * (D * 2) + (((2 * j) ^ (r & 7)) << 4)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            *reinterpret_cast<uint4*>(qs + r * (D * 2) + (((2 * j + 1) ^ (r & 7)) << 4)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        }
+    } else if constexpr (C::QB) {
         for (int idx = tid; idx < NR * (D / 8); idx += grp.n) {
             const int r = idx / (D / 8), c = idx - r * (D / 8);
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
             if (r < R) v = *reinterpret_cast<const uint4*>(p.q + (int64_t)q_row_index(p, si, w, r) * D + c * 8);
             *reinterpret_cast<uint4*>(qs + r * (D * 2) + ((c ^ (r & 7)) << 4)) = v;
+        }
+    } else if constexpr (FP8) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int r = nt * 8 + g;
+            if (r < R) {
+                const __nv_bfloat16* qp = p.q + (int64_t)q_row_index(p, si, w, r) * D + 4 * t4;
+#pragma unroll
+                for (int ks = 0; ks < QREG; ++ks) {
+                    const uint2 v = *reinterpret_cast<const uint2*>(qp + ks * 16);
+                    float x0, x1, x2, x3;
+                    bf16x2_to_f32(v.x, x0, x1);
+                    bf16x2_to_f32(v.y, x2, x3);
+                    qf[nt][ks][0] = pack_f16x2(x0, x1);
+                    qf[nt][ks][1] = pack_f16x2(x2, x3);
+                }
+            } else {
+#pragma unroll
+                for (int ks = 0; ks < QREG; ++ks) qf[nt][ks][0] = qf[nt][ks][1] = 0u;
+            }
         }
     } else {
 #pragma unroll
@@ -319,154 +384,354 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
     const int mi = lane >> 3, mr = lane & 7;
     const int k_key = mr + (mi & 1) * 8, k_chunk = mi >> 1;          // K: A operand, keys on M
     const int v_key = mr + (mi >> 1) * 8, v_chunk = mi & 1;          // V: A operand of V^T (trans)
+    const int k8_key = fp8_key_of_row(mr + 8 * (mi & 1)), k8_chunk = mi >> 1;   // FP8 K rows
+    const int v8_row = 8 * (mi & 1) + mr + 16 * (mi >> 1);           // FP8 V^T: head-dim row in a pair of d-tiles
+    const float sl2 = FP8 ? p.scale_log2 * p.k_scale[w.kv_head] : p.scale_log2;
     bool ok = true;
     int waited = 0;
 
-    for (int i = 0; i < n_my; ++i) {
-        const int stage = i % C::NS;
-        const bool got = mbar_wait_bounded(&bar[stage], (i / C::NS) & 1, p.err, PKVA_DEVERR_TIMEOUT);
-        waited = i + 1;
-        if (__any_sync(0xffffffffu, !got)) {
-            ok = false;
-            break;
-        }
-        uint8_t* Ks = ring + stage * C::STAGE_BYTES;
-        uint8_t* Vs = Ks + C::PAGE_BYTES;
-        const int kbase = (w.page_begin + warp + NW * i) * kPageSize;
-        if (p.append && kbase + kPageSize > prefix && kbase < si.seq_len) {
-            // fused append: the new tokens' rows come from the dense input, not the cache
-            const int r0 = max(prefix - kbase, 0), r1 = min(si.seq_len - kbase, kPageSize);
-            patch_page_rows<D>(Ks, Vs, p.k_new, p.v_new, si, p.Hkv, w.kv_head, r0, r1, kbase + r0 - prefix, lane);
-            __syncwarp();
-        }
-
-        // -- S^T = K Q^T (16 keys x 8 rows per n-tile) ------------------------------------
-        float s[NT][4];
+    if constexpr (FP8) {
+        // FP8 pages are half the bytes of bf16 ones, so a warp takes two pages (two stages) per
+        // iteration: their tiles are independent until the shared max, which halves the
+        // dependent chains per byte.
+        for (int i = 0; i < n_my; i += 2) {
+            const bool two = i + 1 < n_my;               // the pair's second page exists
+            bool got = mbar_wait_bounded(&bar[i % C::NS], (i / C::NS) & 1, p.err, PKVA_DEVERR_TIMEOUT);
+            if (two && got) got = mbar_wait_bounded(&bar[(i + 1) % C::NS], ((i + 1) / C::NS) & 1, p.err,
+                                                    PKVA_DEVERR_TIMEOUT);
+            waited = i + (two ? 2 : 1);
+            if (__any_sync(0xffffffffu, !got)) {
+                ok = false;
+                break;
+            }
+            int kbase[2];
+            uint8_t* Kp[2];
+            uint8_t* Vp[2];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+            for (int pp = 0; pp < 2; ++pp) {
+                kbase[pp] = (w.page_begin + warp + NW * (i + pp)) * kPageSize;
+                Kp[pp] = ring + ((i + pp) % C::NS) * C::STAGE_BYTES;
+                Vp[pp] = Kp[pp] + C::PAGE_BYTES;
+            }
+            // -- S^T = K Q^T for both pages ------------------------------------------------
+            float s[2][NT][4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
-        if constexpr (C::QB) {
+            for (int pp = 0; pp < 2; ++pp)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) s[pp][nt][e] = 0.f;
 #pragma unroll
             for (int k2 = 0; k2 < KS; k2 += 2) {
-                uint32_t qb[NT][4];              // b fragments of k-steps k2 and k2 + 1
+                uint32_t qb[NT][4];                      // b fragments of k-steps k2 and k2 + 1
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    const int qr = nt * 8 + (lane & 7), qc = 2 * k2 + (lane >> 3);
-                    ldmatrix_x4(qb[nt], qs + qr * (D * 2) + ((qc ^ (qr & 7)) << 4));
-                }
-#pragma unroll
-                for (int kk = 0; kk < 2; ++kk) {
-                    const int cg = (k2 + kk) * 2 + k_chunk;
-                    uint32_t a[4];
-                    ldmatrix_x4(a, Ks + (cg >> 3) * kBoxBytes + k_key * 128 + (((cg & 7) ^ (k_key & 7)) << 4));
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a, &qb[nt][2 * kk]);
-                }
-            }
-        } else {
-#pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
-                const int cg = ks * 2 + k_chunk;
-                uint32_t a[4];
-                ldmatrix_x4(a, Ks + (cg >> 3) * kBoxBytes + k_key * 128 + (((cg & 7) ^ (k_key & 7)) << 4));
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a, qf[nt][ks]);
-            }
-        }
-
-        // -- mask and per-row (column) max over the page's 16 keys ------------------------
-        const bool page_all = (kbase + kPageSize - 1) <= min_lim;
-        float cmax[NT][2];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int kpos = kbase + g + 8 * h;
-                    float v = s[nt][2 * h + e] * p.scale_log2;
-                    if (!page_all) {
-                        bool allow = kpos <= lim[nt][e];
-                        if (!allow && kpos >= prefix && kpos < si.seq_len)
-                            allow = (anc[nt][e] >> (kpos - prefix)) & 1ull;
-                        v = allow ? v : -INFINITY;
+                    if constexpr (C::QB) {
+                        const int qr = nt * 8 + (lane & 7), qc = 2 * k2 + (lane >> 3);
+                        ldmatrix_x4(qb[nt], qs + qr * (D * 2) + ((qc ^ (qr & 7)) << 4));
+                    } else {
+                        qb[nt][0] = qf[nt][k2][0];
+                        qb[nt][1] = qf[nt][k2][1];
+                        qb[nt][2] = qf[nt][k2 + 1][0];
+                        qb[nt][3] = qf[nt][k2 + 1][1];
                     }
-                    s[nt][2 * h + e] = v;
                 }
-                float mx = fmaxf(s[nt][e], s[nt][2 + e]);
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                cmax[nt][e] = mx;
+                // codes of keys sigma(g), sigma(g+8), head-dim bytes [16 k, 16 k + 16) for
+                // k = k2, k2 + 1 (K page: rows of D bytes, 128- or 64-byte swizzle)
+                const int kc = k2 + k8_chunk;
+                const int sw = D == 128 ? (kc ^ (k8_key & 7)) : (kc ^ ((k8_key >> 1) & 3));
+#pragma unroll
+                for (int pp = 0; pp < 2; ++pp) {
+                    if (pp == 1 && !two) break;
+                    uint32_t r[4];
+                    ldmatrix_x4(r, Kp[pp] + k8_key * D + (sw << 4));
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk) {
+                        const uint32_t a[4] = {e4m3x2_to_f16x2(r[2 * kk]), e4m3x2_to_f16x2(r[2 * kk + 1]),
+                                               e4m3x2_to_f16x2(r[2 * kk] >> 16),
+                                               e4m3x2_to_f16x2(r[2 * kk + 1] >> 16)};
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) mma_f16_16816(s[pp][nt], a, &qb[nt][2 * kk]);
+                    }
+                }
             }
-        // -- lazy rescale: only when some row's max passed its reference by the slack ------
-        bool need = false;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e)
-                need |= cmax[nt][e] > mref[nt][e] + kRescaleSlack ||
-                        (mref[nt][e] == -INFINITY && cmax[nt][e] != -INFINITY);
-        if (__any_sync(0xffffffffu, need)) {
+            // -- mask and per-row (column) max over the pair's 32 keys -----------------------
+            float cmax[NT][2];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const float mnew = fmaxf(mref[nt][e], cmax[nt][e]);
-                    if (mnew != mref[nt][e]) {
-                        const float alpha = mref[nt][e] == -INFINITY ? 0.f : exp2f(mref[nt][e] - mnew);
-                        mref[nt][e] = mnew;
-                        lsum[nt][e] *= alpha;
+                    float mx = -INFINITY;
 #pragma unroll
-                        for (int dt = 0; dt < KS; ++dt) {
-                            o[dt][nt][e] *= alpha;
-                            o[dt][nt][2 + e] *= alpha;
+                    for (int pp = 0; pp < 2; ++pp) {
+                        const bool page_all = (kbase[pp] + kPageSize - 1) <= min_lim;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int kpos = kbase[pp] + fp8_key_of_row(g + 8 * h);
+                            float v = s[pp][nt][2 * h + e] * sl2;
+                            if (pp == 1 && !two) {
+                                v = -INFINITY;
+                            } else if (!page_all) {
+                                bool allow = kpos <= lim[nt][e];
+                                if (!allow && kpos >= prefix && kpos < si.seq_len)
+                                    allow = (anc[nt][e] >> (kpos - prefix)) & 1ull;
+                                v = allow ? v : -INFINITY;
+                            }
+                            s[pp][nt][2 * h + e] = v;
+                            mx = fmaxf(mx, v);
                         }
                     }
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                    cmax[nt][e] = mx;
                 }
-        }
-        // -- P = exp2(S - ref), row sums, P^T as the B operand (transpose in registers) -----
-        uint32_t pb[NT][2];
+            // -- lazy rescale: only when some row's max passed its reference by the slack ----
+            bool need = false;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            float pv[4];
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const float ref = mref[nt][e] == -INFINITY ? 0.f : mref[nt][e];
-                pv[e] = exp2f(s[nt][e] - ref);
-                pv[2 + e] = exp2f(s[nt][2 + e] - ref);
-                lsum[nt][e] += pv[e] + pv[2 + e];
+                for (int e = 0; e < 2; ++e)
+                    need |= cmax[nt][e] > mref[nt][e] + kRescaleSlack ||
+                            (mref[nt][e] == -INFINITY && cmax[nt][e] != -INFINITY);
+            if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const float mnew = fmaxf(mref[nt][e], cmax[nt][e]);
+                        if (mnew != mref[nt][e]) {
+                            const float alpha = mref[nt][e] == -INFINITY ? 0.f : exp2f(mref[nt][e] - mnew);
+                            mref[nt][e] = mnew;
+                            lsum[nt][e] *= alpha;
+#pragma unroll
+                            for (int dt = 0; dt < KS; ++dt) {
+                                o[dt][nt][e] *= alpha;
+                                o[dt][nt][2 + e] *= alpha;
+                            }
+                        }
+                    }
             }
-            pb[nt][0] = movmatrix_trans(pack_bf16x2(pv[0], pv[1]));   // keys 0..7
-            pb[nt][1] = movmatrix_trans(pack_bf16x2(pv[2], pv[3]));   // keys 8..15
-        }
-        // slots past the sequence's end hold stale cache data: zero those V rows so that
-        // P = 0 times a non-finite value cannot reach the accumulators
-        const int nvalid = si.seq_len - kbase;
-        if (nvalid < kPageSize) {
-            for (int idx = lane; idx < (kPageSize - nvalid) * (D / 8); idx += 32) {
-                const int row = nvalid + idx / (D / 8);
-                const int cg = idx % (D / 8);
-                *reinterpret_cast<uint4*>(Vs + (cg >> 3) * kBoxBytes + row * 128 + (cg & 7) * 16) =
-                    make_uint4(0u, 0u, 0u, 0u);
+            // -- P = exp2(S - ref) in f16, row sums, P^T by an in-register transpose ----------
+            uint32_t pb[2][NT][2];
+#pragma unroll
+            for (int pp = 0; pp < 2; ++pp)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    float pv[4];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const float ref = mref[nt][e] == -INFINITY ? 0.f : mref[nt][e];
+                        pv[e] = exp2f(s[pp][nt][e] - ref);
+                        pv[2 + e] = exp2f(s[pp][nt][2 + e] - ref);
+                        lsum[nt][e] += pv[e] + pv[2 + e];
+                    }
+                    pb[pp][nt][0] = movmatrix_trans(pack_f16x2(pv[0], pv[1]));   // M rows 0..7
+                    pb[pp][nt][1] = movmatrix_trans(pack_f16x2(pv[2], pv[3]));   // M rows 8..15
+                }
+            // slots past the sequence's end hold stale codes (NaN among them): zero those V
+            // bytes so that P = 0 times a non-finite value cannot reach the accumulators. In a
+            // transposed page, byte j of each 16-byte head-dim row is key j.
+#pragma unroll
+            for (int pp = 0; pp < 2; ++pp) {
+                if (pp == 1 && !two) break;
+                const int nvalid = si.seq_len - kbase[pp];
+                if (nvalid < kPageSize) {
+                    for (int d = lane; d < D; d += 32) {
+                        uint4* rowp = reinterpret_cast<uint4*>(Vp[pp] + d * kPageSize);
+                        uint4 v = *rowp;
+                        uint32_t* wv = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const int keep = min(max(nvalid - 4 * q4, 0), 4);   // bytes of this word to keep
+                            wv[q4] &= keep >= 4 ? 0xffffffffu : ((1u << (8 * keep)) - 1u);
+                        }
+                        *rowp = v;
+                    }
+                    __syncwarp();
+                }
+            }
+            // -- O^T += V^T P^T for both pages ----------------------------------------------
+#pragma unroll
+            for (int d2 = 0; d2 < KS; d2 += 2) {
+#pragma unroll
+                for (int pp = 0; pp < 2; ++pp) {
+                    if (pp == 1 && !two) break;
+                    // head-dim rows 16 d2 + (0..31) of the transposed page, 16 key bytes each
+                    uint32_t r[4];
+                    ldmatrix_x4(r, Vp[pp] + (16 * d2 + v8_row) * kPageSize);
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk) {
+                        const uint32_t a[4] = {e4m3x2_to_f16x2(r[2 * kk]), e4m3x2_to_f16x2(r[2 * kk + 1]),
+                                               e4m3x2_to_f16x2(r[2 * kk] >> 16),
+                                               e4m3x2_to_f16x2(r[2 * kk + 1] >> 16)};
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) mma_f16_16816(o[d2 + kk][nt], a, pb[pp][nt]);
+                    }
+                }
             }
             __syncwarp();
-        }
-        // -- O^T += V^T P^T -----------------------------------------------------------------
+            if (lane == 0) {
+                fence_proxy_async_smem();
 #pragma unroll
-        for (int dt = 0; dt < KS; ++dt) {
-            const int cg = dt * 2 + v_chunk;
-            uint32_t a[4];
-            ldmatrix_x4_trans(a, Vs + (cg >> 3) * kBoxBytes + v_key * 128 + (((cg & 7) ^ (v_key & 7)) << 4));
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[dt][nt], a, pb[nt]);
+                for (int pp = 0; pp < 2; ++pp)
+                    if ((pp == 0 || two) && i + pp + C::NS < n_my)
+                        issue_page<D, C::NS, C::STAGE_BYTES, C::PAGE_BYTES, NW, FP8>(p, w, bts, ring, bar, warp,
+                                                                                  i + pp + C::NS, &tmK, &tmV);
+            }
         }
-        __syncwarp();
-        if (lane == 0 && i + C::NS < n_my) {
-            fence_proxy_async_smem();
-            issue_page<D, C::NS, C::STAGE_BYTES, C::PAGE_BYTES, NW>(p, w, bts, ring, bar, warp, i + C::NS, &tmK,
-                                                                 &tmV);
+    } else {
+        for (int i = 0; i < n_my; ++i) {
+            const int stage = i % C::NS;
+            const bool got = mbar_wait_bounded(&bar[stage], (i / C::NS) & 1, p.err, PKVA_DEVERR_TIMEOUT);
+            waited = i + 1;
+            if (__any_sync(0xffffffffu, !got)) {
+                ok = false;
+                break;
+            }
+            uint8_t* Ks = ring + stage * C::STAGE_BYTES;
+            uint8_t* Vs = Ks + C::PAGE_BYTES;
+            const int kbase = (w.page_begin + warp + NW * i) * kPageSize;
+            if constexpr (!FP8) {
+                if (p.append && kbase + kPageSize > prefix && kbase < si.seq_len) {
+                    // fused append: the new tokens' rows come from the dense input, not the cache
+                    const int r0 = max(prefix - kbase, 0), r1 = min(si.seq_len - kbase, kPageSize);
+                    patch_page_rows<D>(Ks, Vs, p.k_new, p.v_new, si, p.Hkv, w.kv_head, r0, r1, kbase + r0 - prefix,
+                                       lane);
+                    __syncwarp();
+                }
+            }
+
+            // -- S^T = K Q^T (16 keys x 8 rows per n-tile) ------------------------------------
+            float s[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
+            if constexpr (C::QB) {
+#pragma unroll
+                for (int k2 = 0; k2 < KS; k2 += 2) {
+                    uint32_t qb[NT][4];              // b fragments of k-steps k2 and k2 + 1
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const int qr = nt * 8 + (lane & 7), qc = 2 * k2 + (lane >> 3);
+                        ldmatrix_x4(qb[nt], qs + qr * (D * 2) + ((qc ^ (qr & 7)) << 4));
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk) {
+                        const int cg = (k2 + kk) * 2 + k_chunk;
+                        uint32_t a[4];
+                        ldmatrix_x4(a, Ks + (cg >> 3) * kBoxBytes + k_key * 128 + (((cg & 7) ^ (k_key & 7)) << 4));
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a, &qb[nt][2 * kk]);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int ks = 0; ks < KS; ++ks) {
+                    const int cg = ks * 2 + k_chunk;
+                    uint32_t a[4];
+                    ldmatrix_x4(a, Ks + (cg >> 3) * kBoxBytes + k_key * 128 + (((cg & 7) ^ (k_key & 7)) << 4));
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a, qf[nt][ks]);
+                }
+            }
+
+            // -- mask and per-row (column) max over the page's 16 keys ------------------------
+            const bool page_all = (kbase + kPageSize - 1) <= min_lim;
+            float cmax[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int kpos = kbase + g + 8 * h;
+                        float v = s[nt][2 * h + e] * sl2;
+                        if (!page_all) {
+                            bool allow = kpos <= lim[nt][e];
+                            if (!allow && kpos >= prefix && kpos < si.seq_len)
+                                allow = (anc[nt][e] >> (kpos - prefix)) & 1ull;
+                            v = allow ? v : -INFINITY;
+                        }
+                        s[nt][2 * h + e] = v;
+                    }
+                    float mx = fmaxf(s[nt][e], s[nt][2 + e]);
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                    cmax[nt][e] = mx;
+                }
+            // -- lazy rescale: only when some row's max passed its reference by the slack ------
+            bool need = false;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+                    need |= cmax[nt][e] > mref[nt][e] + kRescaleSlack ||
+                            (mref[nt][e] == -INFINITY && cmax[nt][e] != -INFINITY);
+            if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const float mnew = fmaxf(mref[nt][e], cmax[nt][e]);
+                        if (mnew != mref[nt][e]) {
+                            const float alpha = mref[nt][e] == -INFINITY ? 0.f : exp2f(mref[nt][e] - mnew);
+                            mref[nt][e] = mnew;
+                            lsum[nt][e] *= alpha;
+#pragma unroll
+                            for (int dt = 0; dt < KS; ++dt) {
+                                o[dt][nt][e] *= alpha;
+                                o[dt][nt][2 + e] *= alpha;
+                            }
+                        }
+                    }
+            }
+            // -- P = exp2(S - ref), row sums, P^T as the B operand (transpose in registers) -----
+            uint32_t pb[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                float pv[4];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float ref = mref[nt][e] == -INFINITY ? 0.f : mref[nt][e];
+                    pv[e] = exp2f(s[nt][e] - ref);
+                    pv[2 + e] = exp2f(s[nt][2 + e] - ref);
+                    lsum[nt][e] += pv[e] + pv[2 + e];
+                }
+                pb[nt][0] = movmatrix_trans(pack_bf16x2(pv[0], pv[1]));   // keys 0..7
+                pb[nt][1] = movmatrix_trans(pack_bf16x2(pv[2], pv[3]));   // keys 8..15
+            }
+            // slots past the sequence's end hold stale cache data: zero those V rows so that
+            // P = 0 times a non-finite value cannot reach the accumulators
+            const int nvalid = si.seq_len - kbase;
+            if (nvalid < kPageSize) {
+                for (int idx = lane; idx < (kPageSize - nvalid) * (D / 8); idx += 32) {
+                    const int row = nvalid + idx / (D / 8);
+                    const int cg = idx % (D / 8);
+                    *reinterpret_cast<uint4*>(Vs + (cg >> 3) * kBoxBytes + row * 128 + (cg & 7) * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+                __syncwarp();
+            }
+            // -- O^T += V^T P^T -----------------------------------------------------------------
+            {
+#pragma unroll
+                for (int dt = 0; dt < KS; ++dt) {
+                    const int cg = dt * 2 + v_chunk;
+                    uint32_t a[4];
+                    ldmatrix_x4_trans(a, Vs + (cg >> 3) * kBoxBytes + v_key * 128 + (((cg & 7) ^ (v_key & 7)) << 4));
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[dt][nt], a, pb[nt]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0 && i + C::NS < n_my) {
+                fence_proxy_async_smem();
+                issue_page<D, C::NS, C::STAGE_BYTES, C::PAGE_BYTES, NW, FP8>(p, w, bts, ring, bar, warp, i + C::NS,
+                                                                          &tmK, &tmV);
+            }
         }
     }
     if (!ok) {
@@ -477,6 +742,15 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
     __syncwarp();
     if (warp < NW && lane == 0)                    // every phase of this warp's stages is complete
         for (int i = 0; i < C::NS; ++i) mbar_inval(&bar[i]);
+    if constexpr (FP8) {                           // the V scale of this KV head
+        const float vs = p.v_scale[w.kv_head];
+#pragma unroll
+        for (int dt = 0; dt < KS; ++dt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) o[dt][nt][e] *= vs;
+    }
     // row sums over the 16 keys: lanes with the same t4 hold the column
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
@@ -517,7 +791,7 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
     }
     grp.sync();
     merge_and_store<D, NR, NW>(grp, p, w, cm, cl, co, rout, flag);
-    if (p.append && w.row_begin == 0 && w.split <= 0)   // one task per (sequence, KV head)
+    if (!FP8 && p.append && w.row_begin == 0 && w.split <= 0)   // one task per (sequence, KV head)
         append_rows<D>(p.k_new, p.v_new, p.k_cache, p.v_cache, p.block_table, p.bt_stride, p.num_pages, p.Hkv,
                        p.err, si, w.seq, w.kv_head, 0, si.query_len, tid, grp.n);
 }

@@ -136,6 +136,7 @@ struct PlanArgs {
     int num_sms;
     int ctas_per_sm;
     bool use_prefill_kernel = true;       // false: every sequence goes to the decode kernel
+    int kv_elem_bytes = 2;                // bytes per cached K/V element (2 bf16, 1 FP8)
     // shared-prefix groups (may be NULL / 0): prefix_group[s] in {-1} U [0, num_groups),
     // members of a group consecutive in the batch, prefix_len[g] keys shared (page multiple)
     const int32_t* prefix_group = nullptr;

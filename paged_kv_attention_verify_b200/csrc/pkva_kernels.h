@@ -31,6 +31,9 @@ struct DecodeParams {
     const __nv_bfloat16* v_new = nullptr;
     __nv_bfloat16* k_cache = nullptr;      // written at the new tokens' slots
     __nv_bfloat16* v_cache = nullptr;
+    // FP8 (E4M3) caches: one float scale per KV head for K and for V
+    const float* k_scale = nullptr;
+    const float* v_scale = nullptr;
 };
 
 struct PrefillParams {
@@ -80,9 +83,11 @@ int attn_ctas_per_sm(int D, int rows);
 // tmKn/tmVn view k_new/v_new like tmQ ({64, 1, 128} boxes); read only when p.pre.append.
 // tmQc views q in boxes of {64 columns, G heads, floor(128 / G) tokens}; read only by
 // cascade tasks.
+// fp8: the caches are E4M3 codes (tmK over [pages*Hkv*16][D] bytes, tmV over the transposed
+// [pages*Hkv*D][16] bytes) and the launch has decode/verify tasks only.
 cudaError_t launch_attn(const AttnParams& p, int D, int rows, bool has_prefill, const CUtensorMap& tmQ,
                         const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKn,
-                        const CUtensorMap& tmVn, const CUtensorMap& tmQc, cudaStream_t stream);
+                        const CUtensorMap& tmVn, const CUtensorMap& tmQc, cudaStream_t stream, bool fp8 = false);
 
 // Resident CTAs per SM of the decode kernel compiled for (D, rows); 0 if unsupported.
 // `mma` selects the tensor-core page body, otherwise the CUDA-core one.

@@ -107,7 +107,7 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
             return fail(err, PKVA_EUNSUPPORTED, "too many query rows");
 
         // algorithmic work: every K and V element once; 4*D*Hq flops per allowed pair
-        p.kv_bytes += (int64_t)L * a.Hkv * a.D * 2 /*K,V*/ * 2 /*bf16*/;
+        p.kv_bytes += (int64_t)L * a.Hkv * a.D * 2 /*K,V*/ * a.kv_elem_bytes;
         int64_t pairs = (int64_t)T * (L - T);
         if (mk == PKVA_CAUSAL) {
             pairs += (int64_t)T * (T + 1) / 2;
@@ -237,7 +237,7 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
         for (int s = 0; s < a.num_seqs; ++s) {
             if (!on_cascade[s]) continue;
             const int g = grp_of[s];
-            const int64_t per_key = (int64_t)a.Hkv * a.D * 2 * 2;
+            const int64_t per_key = (int64_t)a.Hkv * a.D * 2 * a.kv_elem_bytes;
             p.kv_bytes -= (int64_t)a.prefix_len[g] * per_key;
             if (!counted[g]) p.kv_bytes += (int64_t)a.prefix_len[g] * per_key;
             counted[g] = 1;

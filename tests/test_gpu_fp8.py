@@ -1,0 +1,114 @@
+"""GPU parity of the FP8 (E4M3) KV cache path (attn_plan_kv + attn_run_fp8) against the
+float64 oracle over the decoded codes (oracle.dequantize_kv: code value x per-head scale).
+
+The kernels decode every code exactly and compute in f16 with fp32 accumulation, so the
+same tolerance as the bf16 path applies (max abs <= 2e-2, mean abs <= 2e-3). Codes in the
+slots past each sequence's end are random bytes, NaN codes included.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_attention_verify_b200 as pk
+import workloads as W
+from _util import assert_close, np64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def fp8_oracle_rows(b, f, seq_ids=None, token_picker=None):
+    seq_ids = range(len(b.seqs)) if seq_ids is None else seq_ids
+    qoff, kvoff = b.q_offsets(), b.kv_offsets()
+    ks, vs = f.k_scale.cpu().numpy(), f.v_scale.cpu().numpy()
+    rows, exp = [], []
+    for s in seq_ids:
+        sp = b.seqs[s]
+        toks = list(range(sp.query_len)) if token_picker is None else token_picker(sp)
+        o = kvoff[s]
+        k = oracle.dequantize_kv(f.k_codes[o:o + sp.seq_len].cpu().numpy(), ks)
+        v = oracle.dequantize_kv(f.v_codes[o:o + sp.seq_len].cpu().numpy(), vs)
+        q = np64(b.seq_q(s)[toks])
+        exp.append(oracle.attend_rows(q, k, v, sp.seq_len, sp.query_len, toks, sp.mask_kind,
+                                      sp.parents or None, oracle.default_scale(b.head_dim)))
+        rows.extend(qoff[s] + t for t in toks)
+    return rows, np.concatenate(exp, axis=0)
+
+
+def run_fp8(b, f):
+    plan = pk.plan_for_batch(b, kv_fp8=True)
+    assert plan.info()["num_prefill_items"] == 0
+    out = plan.run_fp8(b.q, f.k_cache, f.v_cache_t, f.k_scale, f.v_scale)
+    assert plan.check() == 0
+    return out, plan
+
+
+SMALL = [
+    dict(seed=31, Hq=8, Hkv=2, d=64, max_ctx=80, max_q=9),
+    dict(seed=32, Hq=8, Hkv=2, d=128, max_ctx=300, max_q=20),
+    dict(seed=33, Hq=28, Hkv=4, d=128, max_ctx=500, max_q=6, tree_frac=0.6),
+    dict(seed=34, Hq=16, Hkv=16, d=128, max_ctx=200, max_q=33),
+    dict(seed=35, Hq=32, Hkv=2, d=64, max_ctx=700, max_q=5, tree_frac=0.5),
+    dict(seed=36, Hq=4, Hkv=1, d=128, max_ctx=40, max_q=64, tree_frac=0.5, max_draft=64),
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: f"seed{c['seed']}_H{c['Hq']}x{c['Hkv']}_d{c['d']}")
+def test_fp8_small_batches_all_rows(cfg):
+    cfg = dict(cfg)
+    b = W.random_small(cfg.pop("seed"), device=DEV, bt_extra=2, **cfg)
+    f = W.fp8_kv(b)
+    out, plan = run_fp8(b, f)
+    rows, exp = fp8_oracle_rows(b, f)
+    assert_close(out[rows], exp, "fp8 small batch")
+    plan.close()
+
+
+def test_fp8_prefill_chunk_runs_as_decode_tasks():
+    seqs = [W.SeqSpec(300, 300, W.CAUSAL, []), W.SeqSpec(133 + 200, 200, W.CAUSAL, []),
+            W.SeqSpec(900, 1, W.CAUSAL, [])]
+    b = W.build_batch("fp8_prefill", seqs, 16, 2, 128, seed=37, device=DEV)
+    f = W.fp8_kv(b)
+    out, plan = run_fp8(b, f)
+    rows, exp = fp8_oracle_rows(b, f)
+    assert_close(out[rows], exp, "fp8 prefill chunks")
+    plan.close()
+
+
+def _sample(sp):
+    return sorted({0, sp.query_len // 2, sp.query_len - 1})
+
+
+@pytest.mark.parametrize("name", ["llama3_8b_decode", "long_ctx_split", "qwen2_7b_unified"])
+def test_fp8_configs_full_size(name):
+    b = W.make_config(name, device=DEV)
+    f = W.fp8_kv(b)
+    out, plan = run_fp8(b, f)
+    seq_ids = list(range(0, len(b.seqs), max(1, len(b.seqs) // 12)))
+    rows, exp = fp8_oracle_rows(b, f, seq_ids=seq_ids, token_picker=_sample)
+    assert_close(out[rows], exp, f"fp8 {name}")
+    # the FP8 plan reads half the bytes of the bf16 one
+    bf = pk.plan_for_batch(b)
+    assert plan.info()["kv_bytes"] * 2 == bf.info()["kv_bytes"]
+    bf.close()
+    plan.close()
+
+
+def test_fp8_plan_and_run_mismatches_are_rejected():
+    b = W.random_small(38, num_seqs=2, d=64, device=DEV)
+    f = W.fp8_kv(b)
+    p8 = pk.plan_for_batch(b, kv_fp8=True)
+    with pytest.raises(pk.PkvaError) as ei:
+        p8.run(b.q, b.k_cache, b.v_cache)
+    assert ei.value.code == -1
+    pb = pk.plan_for_batch(b)
+    with pytest.raises(pk.PkvaError) as ei:
+        pb.run_fp8(b.q, f.k_cache, f.v_cache_t, f.k_scale, f.v_scale)
+    assert ei.value.code == -1
+    L = pk.lib()
+    rc = L.attn_run_fp8(p8._handle, b.q.data_ptr(), f.k_cache.data_ptr(), f.v_cache_t.data_ptr(), None,
+                        f.v_scale.data_ptr(), b.q.data_ptr(), None)
+    assert rc == -1
+    p8.close()
+    pb.close()

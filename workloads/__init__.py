@@ -397,6 +397,59 @@ def new_token_kv(batch: Batch):
     return batch.k_cache[pg, :, sl].contiguous(), batch.v_cache[pg, :, sl].contiguous()
 
 
+@dataclasses.dataclass
+class Fp8KV:
+    """A batch's K/V as FP8 (E4M3) codes with one scale per KV head.
+
+    k_codes, v_codes  [sum L, Hkv, d] uint8, contiguous per sequence (what the oracle
+                      decodes); k_scale, v_scale [Hkv] float32;
+    k_cache           [num_pages, Hkv, page_size, d] uint8 (the batch's paging);
+    v_cache_t         [num_pages, Hkv, d, page_size] uint8: each page block transposed,
+                      the layout the FP8 kernels read V in.
+    Unused slots past a sequence's end hold random bytes (NaN codes included)."""
+    k_codes: torch.Tensor
+    v_codes: torch.Tensor
+    k_scale: torch.Tensor
+    v_scale: torch.Tensor
+    k_cache: torch.Tensor
+    v_cache_t: torch.Tensor
+
+
+def fp8_kv(batch: Batch, seed: int = 0) -> Fp8KV:
+    """Quantise a batch's K/V to FP8 E4M3 per KV head (scale = max |x| / 448 over the head;
+    round to nearest with torch's float8_e4m3fn conversion) and lay the codes out paged.
+    Inputs only: the oracle decodes the codes itself."""
+    if batch.k is None:
+        raise ValueError("fp8_kv needs the batch's contiguous K/V")
+    dev = batch.k.device
+    P = batch.page_size
+
+    def quant(x):
+        amax = x.float().abs().amax(dim=(0, 2)).clamp_min(1e-30)          # [Hkv]
+        scale = amax / 448.0
+        codes = (x.float() / scale[None, :, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+        return codes, scale.to(torch.float32)
+
+    kc, ks = quant(batch.k)
+    vc, vs = quant(batch.v)
+    gen = torch.Generator(device=dev).manual_seed(seed + 4242)
+    num_pages, Hkv, _, d = batch.k_cache.shape
+    k_cache = torch.randint(0, 256, (num_pages, Hkv, P, d), generator=gen, device=dev, dtype=torch.int32).to(torch.uint8)
+    v_cache = torch.randint(0, 256, (num_pages, Hkv, P, d), generator=gen, device=dev, dtype=torch.int32).to(torch.uint8)
+    bt = batch.block_table.cpu()
+    pages, slots = [], []
+    for i, sp in enumerate(batch.seqs):
+        pos = torch.arange(sp.seq_len)
+        pages.append(bt[i, pos // P].long())
+        slots.append(pos % P)
+    pg = torch.cat(pages).to(dev)
+    sl = torch.cat(slots).to(dev)
+    k_cache[pg, :, sl] = kc
+    v_cache[pg, :, sl] = vc
+    return Fp8KV(k_codes=kc, v_codes=vc, k_scale=ks, v_scale=vs, k_cache=k_cache,
+                 v_cache_t=v_cache.transpose(2, 3).contiguous())
+
+
 def make_config(name: str, device="cpu", seed: Optional[int] = None,
                 keep_contiguous: bool = True, max_seqs: Optional[int] = None) -> Batch:
     """One of the five named batches, seeded by its index unless ``seed`` is given.
