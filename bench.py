@@ -194,13 +194,17 @@ def run_reference(args):
     return 0
 
 
-def time_steps(plan, batch, out, steps, warmup, stream, ws=1, clk=None):
-    """Device time of `steps` consecutive attn_run calls (one kernel launch each), bracketed
-    by a barrier and a synchronize on both sides. Returns (per-step ms list, total ms)."""
+def time_steps(plan, batch, out, steps, warmup, stream, ws=1, clk=None, run=None):
+    """Device time of `steps` consecutive attn_run calls (one kernel launch each; `run`
+    replaces the call), bracketed by a barrier and a synchronize on both sides. Returns
+    (per-step ms list, total ms)."""
     import torch
     import torch.distributed as dist
+    if run is None:
+        def run():
+            plan.run(batch.q, batch.k_cache, batch.v_cache, out, stream)
     for _ in range(warmup):
-        plan.run(batch.q, batch.k_cache, batch.v_cache, out, stream)
+        run()
     if plan.check(stream) != 0:
         raise RuntimeError("device error during warm-up")
     torch.cuda.synchronize()
@@ -213,7 +217,7 @@ def time_steps(plan, batch, out, steps, warmup, stream, ws=1, clk=None):
         torch.cuda.synchronize()
         ev[0].record(stream)
         for i in range(steps):
-            plan.run(batch.q, batch.k_cache, batch.v_cache, out, stream)
+            run()
             ev[i + 1].record(stream)
         torch.cuda.synchronize()
         if ws > 1:
@@ -295,12 +299,22 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
 
     batch = W.make_config(args.config, device=dev, max_seqs=args.seqs)
-    plan = pk.plan_for_batch(batch)
-    info = plan.info()
     out = torch.empty_like(batch.q)
+    run = None
+    if args.kv_fp8:
+        # the same batch over FP8 (E4M3) caches: attn_plan_kv + attn_run_fp8
+        f8 = W.fp8_kv(batch)
+        plan = pk.plan_for_batch(batch, kv_fp8=True)
+
+        def run():
+            plan.run_fp8(batch.q, f8.k_cache, f8.v_cache_t, f8.k_scale, f8.v_scale, out, stream)
+        args.no_e2e = args.no_append = True
+    else:
+        plan = pk.plan_for_batch(batch)
+    info = plan.info()
 
     clk = ClockSampler(dev.index)
-    per, elapsed_ms = time_steps(plan, batch, out, args.steps, args.warmup, stream, ws, clk)
+    per, elapsed_ms = time_steps(plan, batch, out, args.steps, args.warmup, stream, ws, clk, run)
     elapsed_ms = max_over_ranks(elapsed_ms, dev)
 
     # end to end through the C ABI with host buffers (pinned), copies inside the region
@@ -328,7 +342,8 @@ def run_ours(args):
     kv_gbs = info["kv_bytes"] / avg_launch_s / 1e9
     tflops = info["attn_flops"] / avg_launch_s / 1e12
     io_bytes = tokens * batch.num_q_heads * batch.head_dim * 2
-    workload = f"{args.config}" + (f" (first {args.seqs} sequences)" if args.seqs else "")
+    workload = f"{args.config}" + (f" (first {args.seqs} sequences)" if args.seqs else "") + \
+        (" over FP8 E4M3 caches" if args.kv_fp8 else "")
     rl = roofline(info, avg_launch_s, peaks)
     rl.update({"traffic": kernel_traffic(workload), "kernel": "attn_kernel",
                "peak_source": peaks["source"],
@@ -448,7 +463,8 @@ def run_ours(args):
         result = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 q/out, fp8-e4m3 KV" if args.kv_fp8 else "bf16",
+            "data": "synthetic",
             "config": {"workload": f"{workload}: {WORKLOADS[args.config]}",
                        "query_tokens_per_step": tokens, "kv_bytes_per_step": info["kv_bytes"],
                        "attn_flops_per_step": info["attn_flops"],
@@ -482,6 +498,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
     ap.add_argument("--no-append", action="store_true", help="skip the fused KV-append measurement")
+    ap.add_argument("--kv-fp8", action="store_true",
+                    help="time the workload over FP8 E4M3 caches (attn_run_fp8; no e2e or append pass)")
     ap.add_argument("--no-other-configs", action="store_true",
                     help="skip the per-config table of the other benchmark batches")
     ap.add_argument("--other-steps", type=int, default=50)

@@ -70,7 +70,7 @@ static bool encode_cache_map(CUtensorMap* map, const void* base, int num_pages, 
 
 // FP8 caches: K as a 2-D byte tensor [num_pages * Hkv * 16 rows, D] with one page block
 // per box (128-byte swizzle at D = 128, 64-byte at D = 64); V, transposed per page block, as
-// [num_pages * Hkv * D rows, 16] with one D x 16 box per block, unswizzled.
+// [num_pages * Hkv * D/8 rows, 128] with one block (D/8 rows) per box, unswizzled.
 static bool encode_fp8_maps(CUtensorMap* mk, CUtensorMap* mv, const void* k, const void* vt, int num_pages, int Hkv,
                             int D) {
     auto fn = tensor_map_encoder();
@@ -85,9 +85,11 @@ static bool encode_fp8_maps(CUtensorMap* mk, CUtensorMap* mv, const void* k, con
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return false;
     }
-    cuuint64_t dims[2] = {(cuuint64_t)kPageSize, (cuuint64_t)num_pages * Hkv * D};
-    cuuint64_t strides[1] = {(cuuint64_t)kPageSize};
-    cuuint32_t box[2] = {(cuuint32_t)kPageSize, (cuuint32_t)D};
+    // a transposed page block is D * 16 contiguous bytes: viewed as rows of 128 bytes so that
+    // one box is D/8 wide rows (a 16-byte-wide box would take the copy engine 8x the rows)
+    cuuint64_t dims[2] = {128, (cuuint64_t)num_pages * Hkv * (D / 8)};
+    cuuint64_t strides[1] = {128};
+    cuuint32_t box[2] = {128, (cuuint32_t)(D / 8)};
     return fn(mv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(vt), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;

@@ -125,7 +125,7 @@ __device__ __forceinline__ void task_setup(const Group& grp, const DecodeParams&
 
 // Load page #i of this warp's stream (lane 0 only); ph is its physical page, -1 for none.
 // bf16: K and V as 16 x 64 boxes (128-byte swizzle). FP8: the K page as one 16 x D-byte box
-// (128- or 64-byte swizzle) and the transposed V page as one D x 16-byte box.
+// (128- or 64-byte swizzle) and the transposed V page as one box of D/8 rows of 128 bytes.
 template <int D, int NS, int STAGE_BYTES, int PAGE_BYTES, bool FP8 = false>
 __device__ __forceinline__ void issue_page_at(const DecodeParams& p, const DecodeWork& w, int ph, uint8_t* ring,
                                               uint64_t* bar, int i, const CUtensorMap* tmK, const CUtensorMap* tmV) {
@@ -135,7 +135,7 @@ __device__ __forceinline__ void issue_page_at(const DecodeParams& p, const Decod
     mbar_arrive_expect_tx(&bar[stage], STAGE_BYTES);
     if constexpr (FP8) {
         tma_load_2d(dst, tmK, &bar[stage], 0, blk * kPageSize);
-        tma_load_2d(dst + PAGE_BYTES, tmV, &bar[stage], 0, blk * D);
+        tma_load_2d(dst + PAGE_BYTES, tmV, &bar[stage], 0, blk * (D / 8));
     } else {
 #pragma unroll
         for (int b = 0; b < D / 64; ++b) {
@@ -447,9 +447,9 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
                     ldmatrix_x4(r, Kp[pp] + k8_key * D + (sw << 4));
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk) {
-                        const uint32_t a[4] = {e4m3x2_to_f16x2(r[2 * kk]), e4m3x2_to_f16x2(r[2 * kk + 1]),
-                                               e4m3x2_to_f16x2(r[2 * kk] >> 16),
-                                               e4m3x2_to_f16x2(r[2 * kk + 1] >> 16)};
+                        uint32_t a[4];
+                        e4m3x4_to_f16x2x2(r[2 * kk], a[0], a[2]);
+                        e4m3x4_to_f16x2x2(r[2 * kk + 1], a[1], a[3]);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) mma_f16_16816(s[pp][nt], a, &qb[nt][2 * kk]);
                     }
@@ -562,9 +562,9 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
                     ldmatrix_x4(r, Vp[pp] + (16 * d2 + v8_row) * kPageSize);
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk) {
-                        const uint32_t a[4] = {e4m3x2_to_f16x2(r[2 * kk]), e4m3x2_to_f16x2(r[2 * kk + 1]),
-                                               e4m3x2_to_f16x2(r[2 * kk] >> 16),
-                                               e4m3x2_to_f16x2(r[2 * kk + 1] >> 16)};
+                        uint32_t a[4];
+                        e4m3x4_to_f16x2x2(r[2 * kk], a[0], a[2]);
+                        e4m3x4_to_f16x2x2(r[2 * kk + 1], a[1], a[3]);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) mma_f16_16816(o[d2 + kk][nt], a, pb[pp][nt]);
                     }

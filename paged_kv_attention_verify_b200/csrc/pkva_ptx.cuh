@@ -4,7 +4,6 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
-#include <cuda_fp8.h>
 #include <stdint.h>
 
 namespace pkva {
@@ -203,11 +202,15 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Two FP8 E4M3 codes (the low byte is the first) to f16x2, exactly (every E4M3 value is an
-// f16 value); the low byte's value lands in the low half.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two_codes & 0xffffu), __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+// Four FP8 E4M3 codes (byte 0 first) to two f16x2, exactly (every E4M3 value is an f16
+// value): bytes 0, 1 -> lo (byte 0 in the low half), bytes 2, 3 -> hi.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t codes, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 l, h;\n\t"
+        "mov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(codes));
 }
 
 // D += A B on tensor cores, warp-wide: m16n8k16, f16 A and B, fp32 accumulators (same
