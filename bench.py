@@ -299,6 +299,16 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
 
     batch = W.make_config(args.config, device=dev, max_seqs=args.seqs)
+    job_tokens = None
+    parallelism = f"replicas x{ws}" if ws > 1 else "single GPU"
+    if args.shard == "heads" and ws > 1:
+        # strong scaling: the one batch split over the ranks (KV-head groups x sequence
+        # subsets, no exchange inside attention); every rank builds it from the same seed
+        from paged_kv_attention_verify_b200 import shard as S
+        job_tokens = batch.total_q
+        parallelism = "kv-head/sequence shards tp%d x sp%d" % S.shard_layout(ws, batch.num_kv_heads)
+        batch = W.shard_batch(batch, rank, ws)
+        torch.cuda.empty_cache()
     out = torch.empty_like(batch.q)
     run = None
     if args.kv_fp8:
@@ -336,8 +346,12 @@ def run_ours(args):
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
 
     tokens = batch.total_q
-    value = job_throughput(tokens, args.steps, elapsed_ms, ws)
-    e2e_value = job_throughput(tokens, args.steps, e2e_ms, ws) if e2e_ms else None
+    if job_tokens is not None:       # the ranks share one batch: its tokens over the slowest rank's time
+        value = job_tokens * args.steps / (elapsed_ms * 1e-3)
+        e2e_value = job_tokens * args.steps / (e2e_ms * 1e-3) if e2e_ms else None
+    else:
+        value = job_throughput(tokens, args.steps, elapsed_ms, ws)
+        e2e_value = job_throughput(tokens, args.steps, e2e_ms, ws) if e2e_ms else None
     avg_launch_s = (sum(per) / len(per)) * 1e-3
     kv_gbs = info["kv_bytes"] / avg_launch_s / 1e9
     tflops = info["attn_flops"] / avg_launch_s / 1e12
@@ -463,13 +477,14 @@ def run_ours(args):
         result = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 q/out, fp8-e4m3 KV" if args.kv_fp8 else "bf16",
+            "scaling": "strong" if job_tokens is not None else "weak", "vs_baseline": None,
+            "dtype": "bf16 q/out, fp8-e4m3 KV" if args.kv_fp8 else "bf16",
             "data": "synthetic",
             "config": {"workload": f"{workload}: {WORKLOADS[args.config]}",
                        "query_tokens_per_step": tokens, "kv_bytes_per_step": info["kv_bytes"],
                        "attn_flops_per_step": info["attn_flops"],
                        "l2": "inputs larger than L2 (KV cache read each step exceeds 126 MB)",
-                       "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+                       "parallelism": parallelism},
             "kv_gbs": kv_gbs, "kv_frac_of_hbm": kv_gbs / peaks["hbm_gbs"], "prefill_tflops": tflops,
             "roofline": rl,
             "cpu_baseline": cpu,
@@ -498,6 +513,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
     ap.add_argument("--no-append", action="store_true", help="skip the fused KV-append measurement")
+    ap.add_argument("--shard", choices=["replica", "heads"], default="replica",
+                    help="with N > 1: every rank runs the whole batch (replica, weak scaling) or the batch "
+                         "is split over the ranks by KV heads and sequences (heads, strong scaling)")
     ap.add_argument("--kv-fp8", action="store_true",
                     help="time the workload over FP8 E4M3 caches (attn_run_fp8; no e2e or append pass)")
     ap.add_argument("--no-other-configs", action="store_true",

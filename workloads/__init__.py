@@ -450,6 +450,31 @@ def fp8_kv(batch: Batch, seed: int = 0) -> Fp8KV:
                  v_cache_t=v_cache.transpose(2, 3).contiguous())
 
 
+def shard_batch(batch: Batch, rank: int, world: int) -> Batch:
+    """The part of ``batch`` one of ``world`` GPUs holds (paged_kv_attention_verify_b200.shard):
+    its KV heads' cache and queries for its sequences. The page pool keeps its size (the
+    block table still addresses it); only the sequences' rows are taken."""
+    from paged_kv_attention_verify_b200 import shard as S
+    tp_rank, sp_rank, tp, sp = S.shard_coords(rank, world, batch.num_kv_heads)
+    kv0, kv1, q0, q1 = S.head_range(tp_rank, tp, batch.num_q_heads, batch.num_kv_heads)
+    seqs = S.sequence_subset(len(batch.seqs), sp_rank, sp)
+    qo, ko = batch.q_offsets(), batch.kv_offsets()
+    empty = torch.zeros(0, dtype=torch.long)
+    qrows = torch.cat([empty] + [torch.arange(qo[s], qo[s] + batch.seqs[s].query_len) for s in seqs]).to(batch.q.device)
+    k = v = None
+    if batch.k is not None:
+        krows = torch.cat([empty] + [torch.arange(ko[s], ko[s] + batch.seqs[s].seq_len) for s in seqs]).to(batch.k.device)
+        k = batch.k[krows, kv0:kv1].contiguous()
+        v = batch.v[krows, kv0:kv1].contiguous()
+    return Batch(name=f"{batch.name}[rank {rank}/{world}]", num_q_heads=q1 - q0, num_kv_heads=kv1 - kv0,
+                 head_dim=batch.head_dim, page_size=batch.page_size, seqs=[batch.seqs[s] for s in seqs],
+                 q=batch.q[qrows, q0:q1].contiguous(), k=k, v=v,
+                 k_cache=batch.k_cache[:, kv0:kv1].contiguous(), v_cache=batch.v_cache[:, kv0:kv1].contiguous(),
+                 block_table=batch.block_table[torch.tensor(seqs, dtype=torch.long,
+                                                            device=batch.block_table.device)].contiguous(),
+                 page_perm=batch.page_perm, seed=batch.seed, outlier_frac=batch.outlier_frac)
+
+
 def make_config(name: str, device="cpu", seed: Optional[int] = None,
                 keep_contiguous: bool = True, max_seqs: Optional[int] = None) -> Batch:
     """One of the five named batches, seeded by its index unless ``seed`` is given.
