@@ -206,10 +206,14 @@ PKVA_API int attn_run(pkva_plan_t plan, const void* q, const void* k_cache, cons
  * attn_run_host — attn_run with q and out in HOST memory (the end-to-end call).
  *
  * Copies q (host, [sum T_s, Hq, D] bf16) to a plan-owned device buffer, runs, and copies
- * the result back to out (host), all on `stream`; returns after enqueueing. The caller
- * synchronizes the stream before reading `out`. Pinned host memory makes the copies
- * asynchronous; pageable memory works but the copies then block. The caches stay in
- * device memory (they are the resident KV state).
+ * the result back to out (host); returns after enqueueing. The copy of q runs on a stream
+ * of the plan's own, into one of two staging buffers used alternately, so that it overlaps
+ * the previous call's attention and copy out; the attention (after that copy) and the copy
+ * out run on `stream`, so `out` is complete when `stream` has reached this call (the
+ * caller synchronizes `stream` before reading `out`); q_host must stay unchanged until then
+ * too. Pinned host memory makes the copies asynchronous; pageable memory
+ * works but the copies then block. The caches stay in device memory (they are the resident
+ * KV state).
  */
 PKVA_API int attn_run_host(pkva_plan_t plan, const void* q_host, const void* k_cache,
                   const void* v_cache, void* out_host, void* stream);

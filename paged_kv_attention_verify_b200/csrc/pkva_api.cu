@@ -147,8 +147,12 @@ struct pkva_plan {
     float* d_part_ml = nullptr;
     int32_t* d_counters = nullptr;
     int32_t* d_err = nullptr;
-    void* d_qstage = nullptr;
+    void* d_qstage[2] = {nullptr, nullptr};     // attn_run_host: q staging, used alternately
     void* d_ostage = nullptr;
+    cudaStream_t copy_in = nullptr;              // attn_run_host: the copies of q to the device
+    cudaEvent_t ev_q_in[2] = {nullptr, nullptr};
+    cudaEvent_t ev_q_used[2] = {nullptr, nullptr};
+    int host_parity = 0;
     CUtensorMap tmK, tmV;
     const void* tm_k = nullptr;
     const void* tm_v = nullptr;
@@ -181,8 +185,13 @@ static void free_plan(pkva_plan* p) {
     cudaFree(p->d_part_ml);
     cudaFree(p->d_counters);
     cudaFree(p->d_err);
-    cudaFree(p->d_qstage);
+    for (int b = 0; b < 2; ++b) {
+        cudaFree(p->d_qstage[b]);
+        if (p->ev_q_in[b]) cudaEventDestroy(p->ev_q_in[b]);
+        if (p->ev_q_used[b]) cudaEventDestroy(p->ev_q_used[b]);
+    }
     cudaFree(p->d_ostage);
+    if (p->copy_in) cudaStreamDestroy(p->copy_in);
     delete p;
 }
 
@@ -584,15 +593,31 @@ extern "C" int attn_run_host(pkva_plan_t plan, const void* q_host, const void* k
         return PKVA_EINVAL;
     }
     const size_t bytes = (size_t)hp.total_q * hp.Hq * hp.D * 2;
-    if (!plan->d_qstage) {
-        PKVA_CUDA(cudaMalloc(&plan->d_qstage, bytes), "cudaMalloc(q staging)");
+    if (!plan->d_ostage) {
+        for (int b = 0; b < 2; ++b) {
+            PKVA_CUDA(cudaMalloc(&plan->d_qstage[b], bytes), "cudaMalloc(q staging)");
+            PKVA_CUDA(cudaEventCreateWithFlags(&plan->ev_q_in[b], cudaEventDisableTiming), "cudaEventCreate");
+            PKVA_CUDA(cudaEventCreateWithFlags(&plan->ev_q_used[b], cudaEventDisableTiming), "cudaEventCreate");
+        }
+        PKVA_CUDA(cudaStreamCreateWithFlags(&plan->copy_in, cudaStreamNonBlocking), "cudaStreamCreate");
         PKVA_CUDA(cudaMalloc(&plan->d_ostage, bytes), "cudaMalloc(out staging)");
-        plan->scratch_bytes += 2 * (int64_t)bytes;
+        plan->scratch_bytes += 3 * (int64_t)bytes;
     }
+    // q goes in on the plan's own copy stream, into the staging buffer the run before the
+    // last one used, so that it overlaps the previous run's attention and copy out; the
+    // attention waits for it, and the attention and the copy out stay on `stream`, so the
+    // result is complete when `stream` reaches this point
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    PKVA_CUDA(cudaMemcpyAsync(plan->d_qstage, q_host, bytes, cudaMemcpyHostToDevice, st), "copy q to device");
-    const int rc = attn_run(plan, plan->d_qstage, k_cache, v_cache, plan->d_ostage, stream);
+    const int b = plan->host_parity;
+    plan->host_parity ^= 1;
+    PKVA_CUDA(cudaStreamWaitEvent(plan->copy_in, plan->ev_q_used[b], 0), "order q staging reuse");
+    PKVA_CUDA(cudaMemcpyAsync(plan->d_qstage[b], q_host, bytes, cudaMemcpyHostToDevice, plan->copy_in),
+              "copy q to device");
+    PKVA_CUDA(cudaEventRecord(plan->ev_q_in[b], plan->copy_in), "record q copy");
+    PKVA_CUDA(cudaStreamWaitEvent(st, plan->ev_q_in[b], 0), "order attention after q copy");
+    const int rc = attn_run(plan, plan->d_qstage[b], k_cache, v_cache, plan->d_ostage, stream);
     if (rc != PKVA_OK) return rc;
+    PKVA_CUDA(cudaEventRecord(plan->ev_q_used[b], st), "record q use");
     PKVA_CUDA(cudaMemcpyAsync(out_host, plan->d_ostage, bytes, cudaMemcpyDeviceToHost, st), "copy out to host");
     return PKVA_OK;
 }

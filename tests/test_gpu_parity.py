@@ -131,6 +131,25 @@ def test_run_host_matches_run():
     assert torch.equal(o_host, o_dev.cpu())
 
 
+def test_run_host_back_to_back_calls():
+    """Successive host calls alternate staging buffers and overlap the next copy of q with
+    the previous attention; each output must still match its own q (prefill tasks included,
+    so the q tensor map changes between calls)."""
+    seqs = [W.SeqSpec(300, 200, W.CAUSAL, []), W.SeqSpec(90, 1, W.CAUSAL, []), W.SeqSpec(45, 4, W.TREE, [-1, 0, 0, 1])]
+    b = W.build_batch("host_calls", seqs, 16, 2, 128, seed=44, device=DEV)
+    plan = pk.plan_for_batch(b)
+    qs = [(b.q.float() * f).to(torch.bfloat16) for f in (1.0, -0.5, 2.0, 0.25, 1.5)]
+    refs = [plan.run(q, b.k_cache, b.v_cache).cpu() for q in qs]
+    q_hosts = [q.cpu().pin_memory() for q in qs]
+    o_hosts = [torch.empty(q.shape, dtype=torch.bfloat16).pin_memory() for q in qs]
+    for qh, oh in zip(q_hosts, o_hosts):
+        plan.run_host(qh, b.k_cache, b.v_cache, oh)
+    torch.cuda.current_stream().synchronize()
+    assert plan.check() == 0
+    for i, (oh, ref) in enumerate(zip(o_hosts, refs)):
+        assert torch.equal(oh, ref), i
+
+
 def test_run_rejects_misaligned_pointer():
     b = W.make_config("tiny_decode", device=DEV)
     plan = pk.plan_for_batch(b)
