@@ -136,7 +136,7 @@ PKVA_API int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq_l
  * The output is the same as attn_plan's on the same batch (up to rounding). Members that
  * run as decode/verify tasks get their shared keys from cascade tasks: the stacked (token,
  * head) rows of a run of members, floor(128 / (Hq/Hkv)) tokens x all heads of one KV head
- * per tensor-core tile, against the shared keys in chunks of 1024; each member then merges
+ * per tensor-core tile, against the shared keys in chunks of 2048; each member then merges
  * those partial results with its own keys' (split-KV combine). Members that run as prefill
  * tasks (causal chunks of >= 64 tokens) read their whole prefix as before. Needs head_dim
  * 128 when any prefix_len > 0 (else PKVA_EUNSUPPORTED). Errors as attn_plan.

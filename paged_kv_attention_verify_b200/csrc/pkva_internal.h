@@ -18,7 +18,7 @@ constexpr int kPrefillTileN = 128;     // keys per prefill KV tile (8 pages)
 constexpr int kDecTasksPerBlock = 3;   // decode tasks side by side in one block of the unified kernel
 constexpr int kPrefillMinTokens = 64;  // causal sequences with at least this many new tokens
                                        // (and head_dim 128) run on the tensor-core prefill kernel
-constexpr int kCascadeTilesPerTask = 8; // shared-prefix KV tiles (128 keys) per cascade task
+constexpr int kCascadeTilesPerTask = 16; // shared-prefix KV tiles (128 keys) per cascade task
 
 // Per-sequence record (the "Token-Table" row of the batch).
 struct SeqInfo {

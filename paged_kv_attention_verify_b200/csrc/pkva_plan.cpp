@@ -256,7 +256,10 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
     for (size_t ui = 0; ui < units.size(); ++ui) {
         const Unit& u = units[ui];
         const int own = u.pages - u.pstart;
-        const int ns = (int)((own + target - 1) / target);
+        // nearest whole number of target-sized tasks (rounding up made near-target units two
+        // half-size tasks), never more pages per task than the staged block-table slice holds
+        const int ns = std::max<int>(std::max<int>(1, (int)((own + target / 2) / target)),
+                                     (own + kDecodeMaxPages - 1) / kDecodeMaxPages);
         unit_ns[ui] = ns;
         int unit_id = -1;
         if (ns > 1 || u.cs > 0) {

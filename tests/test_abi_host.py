@@ -197,8 +197,8 @@ def test_planner_covers_shared_prefix_config():
     items = _shared_inspect(b)
     _coverage(b, items, b.prefix_group, b.prefix_len)
     casc = [it for it in items if it["kind"] == 2]
-    # 4 groups x 8 KV heads x (32 members' 48 query tokens / 64 tokens per task) x 4 chunks
-    assert len(casc) == 4 * 8 * 1 * 4
+    # 4 groups x 8 KV heads x one task of 64 tokens x 2 chunks of 2048 shared keys
+    assert len(casc) == 4 * 8 * 1 * 2
 
 
 @pytest.mark.parametrize("groups, lens, code", [

@@ -49,7 +49,7 @@ def test_shared_prefix_config_full_size():
     b = W.make_shared_config("llama3_8b_shared_prefix", device=DEV)
     plan = pk.plan_for_batch(b)
     info = plan.info()
-    assert info["num_cascade_items"] == 4 * 8 * 4
+    assert info["num_cascade_items"] == 4 * 8 * 2
     out = plan.run(b.q, b.k_cache, b.v_cache)
     assert plan.check() == 0
     seq_ids = list(range(0, len(b.seqs), 5))
