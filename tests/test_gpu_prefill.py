@@ -19,6 +19,8 @@ CASES = [
     (500, 300, 28, 4),
     (129, 129, 16, 16),
     (1000, 513, 64, 8),
+    (128, 256, 8, 2),          # prefix and chunk aligned with the 128-key tiles
+    (16, 1536, 32, 8),         # six 256-token tasks per head
 ]
 
 
@@ -76,3 +78,36 @@ def test_prefill_matches_decode_body_on_same_rows(monkeypatch):
     torch.cuda.synchronize()
     d = (o_step[0].float() - o_full[T - 1].float()).abs().max().item()
     assert d <= 2e-2
+
+
+def test_chunk_below_the_prefill_threshold_runs_as_decode_tasks():
+    """63 new tokens (threshold 64) and head_dim 64 chunks go to the warp-level body."""
+    for prefix, T, d in ((255, 63, 128), (40, 300, 64)):
+        b = W.build_batch("below", [W.SeqSpec(prefix + T, T, W.CAUSAL, [])], 16, 4, d, seed=T + d, device=DEV)
+        plan = pk.plan_for_batch(b)
+        assert plan.info()["num_prefill_items"] == 0
+        out = plan.run(b.q, b.k_cache, b.v_cache)
+        assert plan.check() == 0
+        rows, exp = oracle_rows(b)
+        assert_close(out[rows], exp, f"prefix {prefix} T {T} d {d}")
+        plan.close()
+
+
+def test_explicit_softmax_scale():
+    """A scale other than 1/sqrt(d) on both bodies (the oracle takes the same scale)."""
+    import numpy as np
+    import oracle
+    from _util import np64
+    seqs = [W.SeqSpec(300, 100, W.CAUSAL, []), W.SeqSpec(200, 1, W.CAUSAL, []),
+            W.SeqSpec(60, 4, W.TREE, [-1, 0, 1, 0])]
+    b = W.build_batch("scale", seqs, 8, 2, 128, seed=9, device=DEV)
+    plan = pk.plan_for_batch(b, sm_scale=0.03)
+    out = plan.run(b.q, b.k_cache, b.v_cache)
+    assert plan.check() == 0
+    qo = b.q_offsets()
+    for s, sp in enumerate(seqs):
+        k, v = b.seq_kv(s)
+        exp = oracle.attend_rows(np64(b.seq_q(s)), np64(k), np64(v), sp.seq_len, sp.query_len,
+                                 list(range(sp.query_len)), sp.mask_kind, sp.parents or None, 0.03)
+        assert_close(out[qo[s]:qo[s] + sp.query_len], exp, f"scale 0.03, seq {s}")
+    plan.close()
