@@ -270,3 +270,40 @@ def dequantize_kv(codes: np.ndarray, scale_per_head: np.ndarray) -> np.ndarray:
     value = e4m3_decode(code) * scale[head]."""
     s = np.asarray(scale_per_head, dtype=np.float64)
     return e4m3_decode(codes) * s[None, :, None]
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """FP8 E4M3 code (uint8) of each value, rounded to the nearest representable value with
+    ties to the even mantissa, magnitudes beyond the largest finite value (448) clamped to
+    it, NaN to the NaN code 0x7F; the sign of a zero is kept.
+
+    Reading: quantising a value into an E4M3 cache rounds to nearest-even and saturates
+    (the format has no infinities); the value quantised is float32(x) / float32(scale),
+    the division correctly rounded in float32 (the caller does that division).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros(x.shape, dtype=np.uint8)
+    for idx, v in np.ndenumerate(x):
+        if np.isnan(v):
+            out[idx] = 0x7F
+            continue
+        sign = 0x80 if np.signbit(v) else 0x00
+        a = abs(v)
+        if a >= 448.0:
+            out[idx] = sign | 0x7E
+            continue
+        if a < 2.0 ** -6:                              # subnormal binade: quantum 2^-9
+            m = int(np.rint(a / 2.0 ** -9))            # ties to even (exact in float64)
+            out[idx] = sign | m                        # m = 8 is the smallest normal, 0x08
+            continue
+        e = int(np.floor(np.log2(a)))
+        if 2.0 ** e > a:                               # guard against log2 rounding
+            e -= 1
+        elif 2.0 ** (e + 1) <= a:
+            e += 1
+        m = int(np.rint(a / 2.0 ** (e - 3)))           # 8 .. 16
+        if m == 16:
+            e, m = e + 1, 8
+        code = ((e + 7) << 3) | (m - 8)
+        out[idx] = sign | min(code, 0x7E)              # 480 would round past 448: clamp
+    return out

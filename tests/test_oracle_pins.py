@@ -255,10 +255,31 @@ def pin10_e4m3_codes():
     assert deq[0, 0, 0] == 0.5 and deq[0, 1, 0] == 3.0 and deq[1, 1, 0] == -6.0
 
 
+def pin11_e4m3_encode():
+    """Rounding into E4M3: every finite code round-trips; halfway values go to the even
+    mantissa; values past 448 clamp; the subnormal binade has quantum 2^-9; and the
+    encoding agrees with torch's float8_e4m3fn conversion (a library special case) on a
+    dense grid of values below 448."""
+    enc, dec = oracle.e4m3_encode, oracle.e4m3_decode
+    finite = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.int64)
+    assert np.array_equal(enc(dec(finite)), finite.astype(np.uint8))
+    # halfway between 1.0 (0x38, even) and 1.125 (0x39): to 0x38; between 1.125 and 1.25: to 0x3A
+    assert enc(np.array([1.0625]))[0] == 0x38 and enc(np.array([1.1875]))[0] == 0x3A
+    assert enc(np.array([1.0624]))[0] == 0x38 and enc(np.array([1.0626]))[0] == 0x39
+    assert enc(np.array([448.0, 449.0, 1e6, -500.0])).tolist() == [0x7E, 0x7E, 0x7E, 0xFE]
+    assert enc(np.array([2.0 ** -10, 1.5 * 2.0 ** -9, 2.0 ** -11]))[:].tolist() == [0x00, 0x02, 0x00]
+    assert enc(np.array([np.nan]))[0] == 0x7F
+    assert enc(np.array([-0.0]))[0] == 0x80
+    import torch
+    grid = np.concatenate([np.linspace(-447.9, 447.9, 20001), np.linspace(-0.05, 0.05, 20001)]).astype(np.float32)
+    ref = torch.from_numpy(grid).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(enc(grid), ref)
+
+
 PINS = [pin1_rows_sum_to_one, pin2_single_key, pin3_identical_keys_give_mean,
         pin4_chain_tree_is_causal, pin5_decode_steps_match_prefill,
         pin6_page_permutation_invariance, pin7_brute_force, pin8_sdpa, pin9_split_merge,
-        pin10_e4m3_codes]
+        pin10_e4m3_codes, pin11_e4m3_encode]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -407,11 +428,26 @@ def _mut_dequant_wrong_head(orig):
     return {"dequantize_kv": dequantize_kv}
 
 
+def _mut_e4m3_round_half_up(orig):
+    def e4m3_encode(x):
+        x = np.asarray(x, np.float64)
+        return orig.e4m3_encode(np.nextafter(x, np.sign(x) * np.inf))     # ties pushed away from zero
+    return {"e4m3_encode": e4m3_encode}
+
+
+def _mut_e4m3_no_saturation(orig):
+    def e4m3_encode(x):
+        c = orig.e4m3_encode(x)
+        big = np.abs(np.asarray(x, np.float64)) > 464.0
+        return np.where(big, (c & 0x80) | 0x7F, c).astype(np.uint8)      # overflow to NaN
+    return {"e4m3_encode": e4m3_encode}
+
+
 MUTANTS = [_mut_gqa_modulo, _mut_causal_excludes_diagonal, _mut_tree_self_only,
            _mut_tree_parent_not_ancestors, _mut_no_max_subtraction_scale,
            _mut_top_left_causal, _mut_transposed_value, _mut_merge_unweighted,
            _mut_e4m3_bias_8, _mut_e4m3_no_subnormals, _mut_e4m3_ieee_style_inf,
-           _mut_dequant_wrong_head]
+           _mut_dequant_wrong_head, _mut_e4m3_round_half_up, _mut_e4m3_no_saturation]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS, ids=lambda f: f.__name__)
