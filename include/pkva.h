@@ -157,7 +157,7 @@ PKVA_API int attn_plan_shared(pkva_plan_t* out_plan, int num_seqs, const int32_t
  *
  * An FP8 plan runs every sequence as decode/verify tasks (prefill chunks too: no
  * tensor-core prefill tasks) and cannot be used with attn_run, attn_run_host or
- * attn_run_append. Other arguments and errors as attn_plan; PKVA_EINVAL for an unknown
+ * attn_run_append (attn_run_fp8_append appends into FP8 caches). Other arguments and errors as attn_plan; PKVA_EINVAL for an unknown
  * kv_dtype, PKVA_EUNSUPPORTED with PKVA_DECODE_BODY=fma.
  */
 PKVA_API int attn_plan_kv(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq_lens,
@@ -185,6 +185,22 @@ PKVA_API int attn_plan_kv(pkva_plan_t* out_plan, int num_seqs, const int32_t* se
  */
 PKVA_API int attn_run_fp8(pkva_plan_t plan, const void* q, const void* k_cache, const void* v_cache_t,
                  const float* k_scale, const float* v_scale, void* out, void* stream);
+
+/*
+ * attn_run_fp8_append — attn_run_append over FP8 E4M3 caches: writes the new tokens' codes
+ * into k_cache / v_cache_t and computes the batch's attention, in one launch on `stream`.
+ *
+ *   k_new, v_new  device bf16 [sum T_s, Hkv, D] (as attn_run_append).
+ *   other arguments as attn_run_fp8 (k_cache and v_cache_t are written at the new tokens'
+ *   slots only; v_cache_t transposed per page block).
+ * A new value x of KV head h becomes the code E4M3(float32(x) / scale[h]): the division
+ * correctly rounded in float32, the conversion to nearest with ties to even, saturating at
+ * +-448. The attention reads the same codes (the kernels quantise once per use with the same
+ * operation). Errors as attn_run_append and attn_run_fp8.
+ */
+PKVA_API int attn_run_fp8_append(pkva_plan_t plan, const void* q, const void* k_new, const void* v_new,
+                        void* k_cache, void* v_cache_t, const float* k_scale, const float* v_scale,
+                        void* out, void* stream);
 
 /*
  * attn_run — compute the batch's attention on `stream` (asynchronous).

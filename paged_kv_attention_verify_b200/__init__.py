@@ -33,7 +33,7 @@ DEVERR_BAD_PAGE = 0x1
 DEVERR_TIMEOUT = 0x2
 
 # every entry point that include/pkva.h declares
-EXPORTED = ["attn_plan", "attn_plan_shared", "attn_plan_kv", "attn_run", "attn_run_fp8", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_destroy",
+EXPORTED = ["attn_plan", "attn_plan_shared", "attn_plan_kv", "attn_run", "attn_run_fp8", "attn_run_fp8_append", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_destroy",
             "attn_last_error", "attn_plan_get_info", "attn_plan_inspect", "attn_run_static",
             "pkva_selftest_wait_timeout"]
 
@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
     L.attn_plan_shared.argtypes = L.attn_plan.argtypes + [_i32p, _i32p, ctypes.c_int]
     L.attn_plan_kv.argtypes = L.attn_plan.argtypes + [ctypes.c_int]
     L.attn_run_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+    L.attn_run_fp8_append.argtypes = [_vp] * 10
     L.attn_run.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp]
     L.attn_run_append.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
     L.attn_run_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp]
@@ -97,7 +98,7 @@ def lib() -> ctypes.CDLL:
                                   _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                   ctypes.c_float, _vp, _vp, _vp, _vp, _vp]
     L.pkva_selftest_wait_timeout.argtypes = [ctypes.c_longlong, _i32p]
-    for name in ("attn_plan", "attn_plan_shared", "attn_plan_kv", "attn_run_fp8", "attn_run", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_get_info",
+    for name in ("attn_plan", "attn_plan_shared", "attn_plan_kv", "attn_run_fp8", "attn_run_fp8_append", "attn_run", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_get_info",
                  "attn_plan_inspect", "attn_run_static", "pkva_selftest_wait_timeout"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -208,7 +209,7 @@ class Plan:
                                      _stream_handle(stream)))
         return out
 
-    def run_fp8(self, q, k_cache, v_cache_t, k_scale, v_scale, out=None, stream=None):
+    def run_fp8(self, q, k_cache, v_cache_t, k_scale, v_scale, out=None, stream=None, _new=None):
         """``attn_run_fp8``: E4M3 codes (uint8) in ``k_cache`` [pages, Hkv, 16, D] and, each
         page block transposed, ``v_cache_t`` [pages, Hkv, D, 16]; float32 scales [Hkv]."""
         import torch
@@ -223,8 +224,27 @@ class Plan:
             if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != dt or tuple(t.shape) != shape \
                     or not t.is_contiguous():
                 raise ValueError(f"{name} must be a contiguous {dt} CUDA tensor {shape}")
-        _check(lib().attn_run_fp8(self._handle, q.data_ptr(), k_cache.data_ptr(), v_cache_t.data_ptr(),
-                                  k_scale.data_ptr(), v_scale.data_ptr(), out.data_ptr(), _stream_handle(stream)))
+        if _new is None:
+            _check(lib().attn_run_fp8(self._handle, q.data_ptr(), k_cache.data_ptr(), v_cache_t.data_ptr(),
+                                      k_scale.data_ptr(), v_scale.data_ptr(), out.data_ptr(), _stream_handle(stream)))
+        else:
+            _check(lib().attn_run_fp8_append(self._handle, q.data_ptr(), _new[0].data_ptr(), _new[1].data_ptr(),
+                                             k_cache.data_ptr(), v_cache_t.data_ptr(), k_scale.data_ptr(),
+                                             v_scale.data_ptr(), out.data_ptr(), _stream_handle(stream)))
+        return out
+
+    def run_fp8_append(self, q, k_new, v_new, k_cache, v_cache_t, k_scale, v_scale, out=None, stream=None):
+        """``attn_run_fp8_append``: quantise the new tokens' K/V (bf16 [sum T, Hkv, D]) into the
+        FP8 caches at their slots and compute the attention, in one launch."""
+        import torch
+        if out is None:
+            out = torch.empty_like(q)
+        shape = (self.total_q, self.num_kv_heads, self.head_dim)
+        for name, t in (("k_new", k_new), ("v_new", v_new)):
+            if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.bfloat16 \
+                    or tuple(t.shape) != shape or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor {shape}")
+        self.run_fp8(q, k_cache, v_cache_t, k_scale, v_scale, out=out, stream=stream, _new=(k_new, v_new))
         return out
 
     def run_host(self, q_host, k_cache, v_cache, out_host, stream=None):

@@ -568,8 +568,8 @@ extern "C" int attn_run_append(pkva_plan_t plan, const void* q, const void* k_ne
         return PKVA_EINVAL;
     }
     if (plan && plan->kv_fp8) {
-        set_last_error("attn_run_append: not supported on FP8 caches");
-        return PKVA_EUNSUPPORTED;
+        set_last_error("attn_run_append: the plan is for FP8 caches (use attn_run_fp8_append)");
+        return PKVA_EINVAL;
     }
     return run_impl(plan, q, k_new, v_new, k_cache, v_cache, out, stream, "attn_run_append");
 }
@@ -577,6 +577,17 @@ extern "C" int attn_run_append(pkva_plan_t plan, const void* q, const void* k_ne
 extern "C" int attn_run_fp8(pkva_plan_t plan, const void* q, const void* k_cache, const void* v_cache_t,
                             const float* k_scale, const float* v_scale, void* out, void* stream) {
     return run_impl(plan, q, nullptr, nullptr, k_cache, v_cache_t, out, stream, "attn_run_fp8", k_scale, v_scale,
+                    true);
+}
+
+extern "C" int attn_run_fp8_append(pkva_plan_t plan, const void* q, const void* k_new, const void* v_new,
+                                   void* k_cache, void* v_cache_t, const float* k_scale, const float* v_scale,
+                                   void* out, void* stream) {
+    if (plan && plan->hp.num_seqs > 0 && (!k_new || !v_new)) {
+        set_last_error("attn_run_fp8_append: k_new / v_new is NULL");
+        return PKVA_EINVAL;
+    }
+    return run_impl(plan, q, k_new, v_new, k_cache, v_cache_t, out, stream, "attn_run_fp8_append", k_scale, v_scale,
                     true);
 }
 

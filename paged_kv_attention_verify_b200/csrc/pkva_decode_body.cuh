@@ -413,6 +413,20 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
                 Kp[pp] = ring + ((i + pp) % C::NS) * C::STAGE_BYTES;
                 Vp[pp] = Kp[pp] + C::PAGE_BYTES;
             }
+            if (p.append) {
+                // fused append: the new tokens' rows are the dense input's codes, not the cache's
+#pragma unroll
+                for (int pp = 0; pp < 2; ++pp) {
+                    if (pp == 1 && !two) break;
+                    if (kbase[pp] + kPageSize > prefix && kbase[pp] < si.seq_len) {
+                        const int r0 = max(prefix - kbase[pp], 0), r1 = min(si.seq_len - kbase[pp], kPageSize);
+                        patch_page_rows_fp8<D>(Kp[pp], Vp[pp], p.k_new, p.v_new, si, p.Hkv, w.kv_head, r0, r1,
+                                               kbase[pp] + r0 - prefix, lane, p.k_scale[w.kv_head],
+                                               p.v_scale[w.kv_head]);
+                    }
+                }
+                __syncwarp();
+            }
             // -- S^T = K Q^T for both pages ------------------------------------------------
             float s[2][NT][4];
 #pragma unroll
@@ -791,9 +805,16 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
     }
     grp.sync();
     merge_and_store<D, NR, NW>(grp, p, w, cm, cl, co, rout, flag);
-    if (!FP8 && p.append && w.row_begin == 0 && w.split <= 0)   // one task per (sequence, KV head)
-        append_rows<D>(p.k_new, p.v_new, p.k_cache, p.v_cache, p.block_table, p.bt_stride, p.num_pages, p.Hkv,
-                       p.err, si, w.seq, w.kv_head, 0, si.query_len, tid, grp.n);
+    if (p.append && w.row_begin == 0 && w.split <= 0) {          // one task per (sequence, KV head)
+        if constexpr (FP8)
+            append_rows_fp8<D>(p.k_new, p.v_new, reinterpret_cast<uint8_t*>(p.k_cache),
+                               reinterpret_cast<uint8_t*>(p.v_cache), p.block_table, p.bt_stride, p.num_pages, p.Hkv,
+                               p.err, si, w.seq, w.kv_head, 0, si.query_len, tid, grp.n, p.k_scale[w.kv_head],
+                               p.v_scale[w.kv_head]);
+        else
+            append_rows<D>(p.k_new, p.v_new, p.k_cache, p.v_cache, p.block_table, p.bt_stride, p.num_pages, p.Hkv,
+                           p.err, si, w.seq, w.kv_head, 0, si.query_len, tid, grp.n);
+    }
 }
 
 // =====================================================================================

@@ -56,8 +56,7 @@ constexpr int kOffBar = kOffV + kNV * kTileBytes;
 // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2], p_full[2], o_ready[2], mma_done,
 // v_fix
 constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 2 + 2 + 2 + 1 + 1;
-constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
-constexpr int kOffFlag = kOffTmemSlot + 16;
+constexpr int kOffFlag = kOffBar + kNumBars * 8;         // the task's abort flag
 constexpr int kSmemBytes = kOffFlag + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1008;
 constexpr uint32_t kTmemCols = 512;
@@ -468,7 +467,7 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
                 const float x0 = fmaf(__uint_as_float(sr[2 * c]), p.scale_log2, -ref);
                 const float x1 = fmaf(__uint_as_float(sr[2 * c + 1]), p.scale_log2, -ref);
                 float p0, p1;
-                if (kExp2PolyEvery > 0 && c % kExp2PolyEvery == 0) {
+                if (kExp2PolyEvery > 0 && c % (kExp2PolyEvery > 0 ? kExp2PolyEvery : 1) == 0) {
                     const float2 e = exp2_poly2(make_float2(x0, x1));
                     p0 = e.x;
                     p1 = e.y;

@@ -213,6 +213,14 @@ __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t codes, uint32_t& lo, 
         : "r"(codes));
 }
 
+// Two floats to two FP8 E4M3 codes, rounded to nearest even and saturating at +-448 (NaN
+// stays NaN); `lo`'s code in the low byte.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 // D += A B on tensor cores, warp-wide: m16n8k16, f16 A and B, fp32 accumulators (same
 // fragment layout as the bf16 form).
 __device__ __forceinline__ void mma_f16_16816(float d[4], const uint32_t a[4], const uint32_t b[2]) {

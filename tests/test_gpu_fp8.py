@@ -112,3 +112,52 @@ def test_fp8_plan_and_run_mismatches_are_rejected():
     assert rc == -1
     p8.close()
     pb.close()
+
+
+def _fp8_append_case(b):
+    """Append into FP8 caches: the new tokens' slots start as NaN codes; afterwards they hold
+    E4M3(float32(x) / scale) of the dense input (oracle.e4m3_encode, bit for bit) and every
+    other byte is unchanged; the output matches the oracle over those codes."""
+    f = W.fp8_kv(b)
+    k_new, v_new = W.new_token_kv(b)
+    pg, sl = W.new_token_slots(b)
+    ks, vs = f.k_scale.cpu().numpy(), f.v_scale.cpu().numpy()
+    k_enc = oracle.e4m3_encode((k_new.float().cpu().numpy() / ks[None, :, None]).astype(np.float32))
+    v_enc = oracle.e4m3_encode((v_new.float().cpu().numpy() / vs[None, :, None]).astype(np.float32))
+    exp_k, exp_vt = f.k_cache.clone(), f.v_cache_t.clone()
+    exp_k[pg, :, sl] = torch.from_numpy(k_enc).to(DEV)
+    exp_vt[pg, :, :, sl] = torch.from_numpy(v_enc).to(DEV)
+    kc, vct = f.k_cache.clone(), f.v_cache_t.clone()
+    kc[pg, :, sl] = 0x7F
+    vct[pg, :, :, sl] = 0x7F
+    plan = pk.plan_for_batch(b, kv_fp8=True)
+    out = plan.run_fp8_append(b.q, k_new, v_new, kc, vct, f.k_scale, f.v_scale)
+    assert plan.check() == 0
+    assert torch.equal(kc, exp_k), "k_cache codes after append"
+    assert torch.equal(vct, exp_vt), "v_cache_t codes after append"
+    # the oracle over the codes the caches now hold (the contiguous codes with the new ones)
+    kc_codes, vc_codes = f.k_codes.clone(), f.v_codes.clone()
+    kvo, qo = b.kv_offsets(), b.q_offsets()
+    for s, sp in enumerate(b.seqs):
+        T, L = sp.query_len, sp.seq_len
+        kc_codes[kvo[s] + L - T:kvo[s] + L] = torch.from_numpy(k_enc[qo[s]:qo[s] + T]).to(DEV)
+        vc_codes[kvo[s] + L - T:kvo[s] + L] = torch.from_numpy(v_enc[qo[s]:qo[s] + T]).to(DEV)
+    f.k_codes, f.v_codes = kc_codes, vc_codes
+    rows, exp = fp8_oracle_rows(b, f)
+    assert_close(out[rows], exp, "fp8 append output")
+    plan.close()
+
+
+@pytest.mark.parametrize("seed, d", [(51, 64), (52, 128)])
+def test_fp8_append_small(seed, d):
+    b = W.random_small(seed, num_seqs=6, Hq=16, Hkv=4, d=d, max_ctx=300, max_q=40, tree_frac=0.4, device=DEV)
+    _fp8_append_case(b)
+
+
+def test_fp8_append_rejects_bf16_paths():
+    b = W.random_small(53, num_seqs=2, d=64, device=DEV)
+    k_new, v_new = W.new_token_kv(b)
+    p8 = pk.plan_for_batch(b, kv_fp8=True)
+    with pytest.raises(pk.PkvaError):
+        p8.run_append(b.q, k_new, v_new, b.k_cache, b.v_cache)
+    p8.close()
