@@ -265,6 +265,25 @@ PKVA_API int attn_run_append(pkva_plan_t plan, const void* q, const void* k_new,
                     void* k_cache, void* v_cache, void* out, void* stream);
 
 /*
+ * attn_run_host_async — attn_run_host with the copy out on a stream of the plan's own, so
+ * that successive calls pipeline fully: the copy in of call i+1, the attention of call i+1
+ * and the copy out of call i overlap. Two out staging buffers are used alternately; the
+ * attention waits until the copy out of two calls before has drained its buffer.
+ * `out_host` (and `q_host`, until the copy in has run) belongs to the library until
+ * `stream` has passed an attn_host_wait(plan, stream) issued after this call: synchronize
+ * `stream` after that wait before reading `out_host`. Errors as attn_run_host.
+ */
+PKVA_API int attn_run_host_async(pkva_plan_t plan, const void* q_host, const void* k_cache,
+                        const void* v_cache, void* out_host, void* stream);
+
+/*
+ * attn_host_wait — make `stream` wait (on the device; the call does not block) for every
+ * copy out that attn_run_host_async has issued for this plan so far. Returns PKVA_OK,
+ * PKVA_EINVAL (NULL plan) or PKVA_ECUDA.
+ */
+PKVA_API int attn_host_wait(pkva_plan_t plan, void* stream);
+
+/*
  * attn_check — synchronize `stream`, read and clear the plan's device error word.
  * Returns PKVA_OK, PKVA_EDEVICE (bits in *device_error if not NULL) or PKVA_ECUDA.
  */

@@ -33,7 +33,8 @@ DEVERR_BAD_PAGE = 0x1
 DEVERR_TIMEOUT = 0x2
 
 # every entry point that include/pkva.h declares
-EXPORTED = ["attn_plan", "attn_plan_shared", "attn_plan_kv", "attn_run", "attn_run_fp8", "attn_run_fp8_append", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_destroy",
+EXPORTED = ["attn_plan", "attn_plan_shared", "attn_plan_kv", "attn_run", "attn_run_fp8", "attn_run_fp8_append",
+            "attn_run_host_async", "attn_host_wait", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_destroy",
             "attn_last_error", "attn_plan_get_info", "attn_plan_inspect", "attn_run_static",
             "pkva_selftest_wait_timeout"]
 
@@ -84,6 +85,8 @@ def lib() -> ctypes.CDLL:
     L.attn_run.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp]
     L.attn_run_append.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
     L.attn_run_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp]
+    L.attn_run_host_async.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp]
+    L.attn_host_wait.argtypes = [_vp, _vp]
     L.attn_check.argtypes = [_vp, _vp, _i32p]
     L.attn_plan_destroy.argtypes = [_vp]
     L.attn_plan_destroy.restype = None
@@ -98,7 +101,8 @@ def lib() -> ctypes.CDLL:
                                   _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                   ctypes.c_float, _vp, _vp, _vp, _vp, _vp]
     L.pkva_selftest_wait_timeout.argtypes = [ctypes.c_longlong, _i32p]
-    for name in ("attn_plan", "attn_plan_shared", "attn_plan_kv", "attn_run_fp8", "attn_run_fp8_append", "attn_run", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_get_info",
+    for name in ("attn_plan", "attn_plan_shared", "attn_plan_kv", "attn_run_fp8", "attn_run_fp8_append",
+                 "attn_run_host_async", "attn_host_wait", "attn_run", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_get_info",
                  "attn_plan_inspect", "attn_run_static", "pkva_selftest_wait_timeout"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -258,6 +262,23 @@ class Plan:
         _check(lib().attn_run_host(self._handle, q_host.data_ptr(), k_cache.data_ptr(),
                                    v_cache.data_ptr(), out_host.data_ptr(), _stream_handle(stream)))
         return out_host
+
+    def run_host_async(self, q_host, k_cache, v_cache, out_host, stream=None):
+        """``attn_run_host_async``: as ``run_host`` with the copy out on the plan's own stream;
+        ``out_host`` is complete once ``stream`` has passed ``host_wait`` (then synchronize)."""
+        import torch
+        for name, t in (("q_host", q_host), ("out_host", out_host)):
+            if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or \
+                    tuple(t.shape) != (self.total_q, self.num_q_heads, self.head_dim):
+                raise ValueError(f"{name} must be a contiguous bf16 host tensor "
+                                 f"[{self.total_q}, {self.num_q_heads}, {self.head_dim}]")
+        _check(lib().attn_run_host_async(self._handle, q_host.data_ptr(), k_cache.data_ptr(),
+                                         v_cache.data_ptr(), out_host.data_ptr(), _stream_handle(stream)))
+        return out_host
+
+    def host_wait(self, stream=None):
+        """``attn_host_wait``: order ``stream`` after every copy out issued so far."""
+        _check(lib().attn_host_wait(self._handle, _stream_handle(stream)))
 
     def check(self, stream=None) -> int:
         """Synchronize and return the device error bits (0 if none); raises on CUDA errors."""

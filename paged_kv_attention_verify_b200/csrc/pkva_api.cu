@@ -153,6 +153,9 @@ struct pkva_plan {
     cudaEvent_t ev_q_in[2] = {nullptr, nullptr};
     cudaEvent_t ev_q_used[2] = {nullptr, nullptr};
     int host_parity = 0;
+    void* d_ostage_a[2] = {nullptr, nullptr};    // attn_run_host_async: out staging, used alternately
+    cudaStream_t copy_out = nullptr;             // attn_run_host_async: the copies of out to the host
+    cudaEvent_t ev_out_done[2] = {nullptr, nullptr};
     CUtensorMap tmK, tmV;
     const void* tm_k = nullptr;
     const void* tm_v = nullptr;
@@ -192,6 +195,11 @@ static void free_plan(pkva_plan* p) {
     }
     cudaFree(p->d_ostage);
     if (p->copy_in) cudaStreamDestroy(p->copy_in);
+    for (int b = 0; b < 2; ++b) {
+        cudaFree(p->d_ostage_a[b]);
+        if (p->ev_out_done[b]) cudaEventDestroy(p->ev_out_done[b]);
+    }
+    if (p->copy_out) cudaStreamDestroy(p->copy_out);
     delete p;
 }
 
@@ -591,33 +599,53 @@ extern "C" int attn_run_fp8_append(pkva_plan_t plan, const void* q, const void* 
                     true);
 }
 
-extern "C" int attn_run_host(pkva_plan_t plan, const void* q_host, const void* k_cache, const void* v_cache,
-                             void* out_host, void* stream) {
+// The host entries' staging: two q buffers (copied in on the plan's own stream), and either
+// one out buffer (attn_run_host) or two (attn_run_host_async, copied out on a second stream).
+static int host_staging(pkva_plan_t plan, size_t bytes, bool async, const char* who) {
+    const std::string name(who);
+    if (!plan->copy_in) {
+        for (int b = 0; b < 2; ++b) {
+            PKVA_CUDA(cudaMalloc(&plan->d_qstage[b], bytes), (name + ": cudaMalloc(q staging)").c_str());
+            PKVA_CUDA(cudaEventCreateWithFlags(&plan->ev_q_in[b], cudaEventDisableTiming), "cudaEventCreate");
+            PKVA_CUDA(cudaEventCreateWithFlags(&plan->ev_q_used[b], cudaEventDisableTiming), "cudaEventCreate");
+        }
+        PKVA_CUDA(cudaStreamCreateWithFlags(&plan->copy_in, cudaStreamNonBlocking), "cudaStreamCreate");
+        plan->scratch_bytes += 2 * (int64_t)bytes;
+    }
+    if (!async && !plan->d_ostage) {
+        PKVA_CUDA(cudaMalloc(&plan->d_ostage, bytes), (name + ": cudaMalloc(out staging)").c_str());
+        plan->scratch_bytes += (int64_t)bytes;
+    }
+    if (async && !plan->copy_out) {
+        for (int b = 0; b < 2; ++b) {
+            PKVA_CUDA(cudaMalloc(&plan->d_ostage_a[b], bytes), (name + ": cudaMalloc(out staging)").c_str());
+            PKVA_CUDA(cudaEventCreateWithFlags(&plan->ev_out_done[b], cudaEventDisableTiming), "cudaEventCreate");
+        }
+        PKVA_CUDA(cudaStreamCreateWithFlags(&plan->copy_out, cudaStreamNonBlocking), "cudaStreamCreate");
+        plan->scratch_bytes += 2 * (int64_t)bytes;
+    }
+    return PKVA_OK;
+}
+
+static int run_host_impl(pkva_plan_t plan, const void* q_host, const void* k_cache, const void* v_cache,
+                         void* out_host, void* stream, bool async, const char* who) {
+    const std::string name(who);
     if (!plan) {
-        set_last_error("attn_run_host: plan is NULL");
+        set_last_error(name + ": plan is NULL");
         return PKVA_EINVAL;
     }
     const HostPlan& hp = plan->hp;
     if (hp.num_seqs == 0) return PKVA_OK;
     if (!q_host || !out_host) {
-        set_last_error("attn_run_host: NULL host pointer");
+        set_last_error(name + ": NULL host pointer");
         return PKVA_EINVAL;
     }
     const size_t bytes = (size_t)hp.total_q * hp.Hq * hp.D * 2;
-    if (!plan->d_ostage) {
-        for (int b = 0; b < 2; ++b) {
-            PKVA_CUDA(cudaMalloc(&plan->d_qstage[b], bytes), "cudaMalloc(q staging)");
-            PKVA_CUDA(cudaEventCreateWithFlags(&plan->ev_q_in[b], cudaEventDisableTiming), "cudaEventCreate");
-            PKVA_CUDA(cudaEventCreateWithFlags(&plan->ev_q_used[b], cudaEventDisableTiming), "cudaEventCreate");
-        }
-        PKVA_CUDA(cudaStreamCreateWithFlags(&plan->copy_in, cudaStreamNonBlocking), "cudaStreamCreate");
-        PKVA_CUDA(cudaMalloc(&plan->d_ostage, bytes), "cudaMalloc(out staging)");
-        plan->scratch_bytes += 3 * (int64_t)bytes;
-    }
-    // q goes in on the plan's own copy stream, into the staging buffer the run before the
-    // last one used, so that it overlaps the previous run's attention and copy out; the
-    // attention waits for it, and the attention and the copy out stay on `stream`, so the
-    // result is complete when `stream` reaches this point
+    const int rc0 = host_staging(plan, bytes, async, who);
+    if (rc0 != PKVA_OK) return rc0;
+    // q goes in on the plan's own copy stream, into the staging buffer the call before the
+    // last one used, so that it overlaps the previous call's attention and copy out; the
+    // attention (on `stream`) waits for it
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int b = plan->host_parity;
     plan->host_parity ^= 1;
@@ -626,10 +654,46 @@ extern "C" int attn_run_host(pkva_plan_t plan, const void* q_host, const void* k
               "copy q to device");
     PKVA_CUDA(cudaEventRecord(plan->ev_q_in[b], plan->copy_in), "record q copy");
     PKVA_CUDA(cudaStreamWaitEvent(st, plan->ev_q_in[b], 0), "order attention after q copy");
-    const int rc = attn_run(plan, plan->d_qstage[b], k_cache, v_cache, plan->d_ostage, stream);
+    void* ostage = plan->d_ostage;
+    if (async) {
+        // the out buffer is free once the copy out of the call before the last one is done
+        ostage = plan->d_ostage_a[b];
+        PKVA_CUDA(cudaStreamWaitEvent(st, plan->ev_out_done[b], 0), "order out staging reuse");
+    }
+    const int rc = attn_run(plan, plan->d_qstage[b], k_cache, v_cache, ostage, stream);
     if (rc != PKVA_OK) return rc;
-    PKVA_CUDA(cudaEventRecord(plan->ev_q_used[b], st), "record q use");
-    PKVA_CUDA(cudaMemcpyAsync(out_host, plan->d_ostage, bytes, cudaMemcpyDeviceToHost, st), "copy out to host");
+    PKVA_CUDA(cudaEventRecord(plan->ev_q_used[b], st), "record attention done");
+    if (!async) {
+        // the copy out stays on `stream`: the result is complete when `stream` reaches here
+        PKVA_CUDA(cudaMemcpyAsync(out_host, ostage, bytes, cudaMemcpyDeviceToHost, st), "copy out to host");
+        return PKVA_OK;
+    }
+    // the copy out on the plan's second stream, overlapping the next call's attention
+    PKVA_CUDA(cudaStreamWaitEvent(plan->copy_out, plan->ev_q_used[b], 0), "order copy out after attention");
+    PKVA_CUDA(cudaMemcpyAsync(out_host, ostage, bytes, cudaMemcpyDeviceToHost, plan->copy_out), "copy out to host");
+    PKVA_CUDA(cudaEventRecord(plan->ev_out_done[b], plan->copy_out), "record copy out");
+    return PKVA_OK;
+}
+
+extern "C" int attn_run_host(pkva_plan_t plan, const void* q_host, const void* k_cache, const void* v_cache,
+                             void* out_host, void* stream) {
+    return run_host_impl(plan, q_host, k_cache, v_cache, out_host, stream, false, "attn_run_host");
+}
+
+extern "C" int attn_run_host_async(pkva_plan_t plan, const void* q_host, const void* k_cache, const void* v_cache,
+                                   void* out_host, void* stream) {
+    return run_host_impl(plan, q_host, k_cache, v_cache, out_host, stream, true, "attn_run_host_async");
+}
+
+extern "C" int attn_host_wait(pkva_plan_t plan, void* stream) {
+    if (!plan) {
+        set_last_error("attn_host_wait: plan is NULL");
+        return PKVA_EINVAL;
+    }
+    if (!plan->copy_out) return PKVA_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    for (int b = 0; b < 2; ++b)
+        PKVA_CUDA(cudaStreamWaitEvent(st, plan->ev_out_done[b], 0), "attn_host_wait: order after copies out");
     return PKVA_OK;
 }
 

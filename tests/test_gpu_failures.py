@@ -34,6 +34,31 @@ def test_bad_block_table_entry_is_reported_not_faulted(T):
     assert plan.check() == 0                         # attn_check cleared the word
 
 
+def test_bad_block_table_entry_fp8_and_cascade():
+    """The same report on the FP8 path and on a shared-prefix (cascade) plan."""
+    seqs = [W.SeqSpec(600, 1, W.CAUSAL, []), W.SeqSpec(400, 1, W.CAUSAL, [])]
+    b = W.build_batch("bad8", seqs, 8, 2, 128, seed=5, device="cuda")
+    f = W.fp8_kv(b)
+    bt = b.block_table.clone()
+    bt[0, 3] = -7                                   # negative: out of range too
+    plan = pk.Plan(b.seq_lens, b.query_lens, bt, b.mask_kinds, None, num_q_heads=8, num_kv_heads=2,
+                   head_dim=128, num_pages=b.k_cache.shape[0], kv_fp8=True)
+    out = plan.run_fp8(b.q, f.k_cache, f.v_cache_t, f.k_scale, f.v_scale)
+    assert plan.check() & pk.DEVERR_BAD_PAGE
+    assert torch.isfinite(out.float()).all()
+    plan.close()
+    sb = W.random_shared_small(6, 16, 4, device="cuda")
+    bt = sb.block_table.clone()
+    bt[0, 1] = sb.k_cache.shape[0]                  # a shared page of group 0, seen by its cascade tasks
+    plan = pk.Plan(sb.seq_lens, sb.query_lens, bt, sb.mask_kinds, sb.parents_flat, num_q_heads=16,
+                   num_kv_heads=4, head_dim=128, num_pages=sb.k_cache.shape[0],
+                   prefix_group=sb.prefix_group, prefix_len=sb.prefix_len)
+    out = plan.run(sb.q, sb.k_cache, sb.v_cache)
+    assert plan.check() & pk.DEVERR_BAD_PAGE
+    assert torch.isfinite(out.float()).all()
+    plan.close()
+
+
 def test_bounded_wait_gives_up_with_timeout_bit():
     assert pk.selftest_wait_timeout(20_000_000) == pk.DEVERR_TIMEOUT
     # the context is still usable afterwards

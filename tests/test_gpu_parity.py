@@ -150,6 +150,26 @@ def test_run_host_back_to_back_calls():
         assert torch.equal(oh, ref), i
 
 
+def test_run_host_async_pipelined_calls():
+    """attn_run_host_async: copies out on the plan's own stream, two out buffers; after
+    host_wait and a synchronize every output matches its own q."""
+    seqs = [W.SeqSpec(300, 200, W.CAUSAL, []), W.SeqSpec(90, 1, W.CAUSAL, []), W.SeqSpec(45, 4, W.TREE, [-1, 0, 0, 1])]
+    b = W.build_batch("host_async", seqs, 16, 2, 128, seed=45, device=DEV)
+    plan = pk.plan_for_batch(b)
+    qs = [(b.q.float() * f).to(torch.bfloat16) for f in (1.0, -0.5, 2.0, 0.25, 1.5, -1.0)]
+    refs = [plan.run(q, b.k_cache, b.v_cache).cpu() for q in qs]
+    q_hosts = [q.cpu().pin_memory() for q in qs]
+    o_hosts = [torch.empty(q.shape, dtype=torch.bfloat16).pin_memory() for q in qs]
+    stream = torch.cuda.current_stream()
+    for qh, oh in zip(q_hosts, o_hosts):
+        plan.run_host_async(qh, b.k_cache, b.v_cache, oh, stream)
+    plan.host_wait(stream)
+    stream.synchronize()
+    assert plan.check() == 0
+    for i, (oh, ref) in enumerate(zip(o_hosts, refs)):
+        assert torch.equal(oh, ref), i
+
+
 def test_run_rejects_misaligned_pointer():
     b = W.make_config("tiny_decode", device=DEV)
     plan = pk.plan_for_batch(b)
