@@ -21,7 +21,7 @@ namespace pkva {
 namespace {
 
 constexpr int kMinSplitPages = 8;      // never split a unit into tasks below 128 keys
-constexpr int kTasksPerSlot = 3;       // aim for ~3 tasks per CTA slot before splitting stops
+constexpr int kTasksPerSlot = 1;       // split long units down to about one task per CTA slot
 
 int fail(std::string* err, int code, const char* fmt, long a = 0, long b = 0, long c = 0) {
     char buf[256];
