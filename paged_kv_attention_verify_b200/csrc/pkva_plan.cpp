@@ -247,8 +247,17 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
     if (units.empty()) p.decode_rows = 4;
 
     // -- split long units so the grid has ~kTasksPerSlot tasks per CTA slot -------------
-    const int64_t slots = (int64_t)a.num_sms * a.ctas_per_sm;
-    int64_t target = (total_pages + slots * kTasksPerSlot - 1) / (slots * kTasksPerSlot);
+    // When the per-task page cap forces more than one task per slot over FP8 caches, the
+    // target is set so that the tasks fill whole waves of slots: the FP8 body converts
+    // codes at about twice the instructions per byte, so a last wave only partly filled
+    // leaves HBM idle. The bf16 body keeps HBM busy with a partial last wave, and there
+    // the fewer, longer tasks measured faster.
+    const int64_t per_wave = (int64_t)a.num_sms * a.ctas_per_sm * kTasksPerSlot;
+    const int64_t waves =
+        a.kv_elem_bytes == 1 ? std::max<int64_t>(1, (total_pages + per_wave * kDecodeMaxPages - 1) /
+                                                        (per_wave * kDecodeMaxPages))
+                             : 1;
+    int64_t target = (total_pages + per_wave * waves - 1) / (per_wave * waves);
     target = std::max<int64_t>(target, kMinSplitPages);
     target = std::min<int64_t>(target, kDecodeMaxPages);
     std::vector<int> unit_id_of(units.size(), -1);
