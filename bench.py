@@ -246,6 +246,25 @@ def time_fn(fn, steps, warmup, stream):
     return [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
 
 
+def time_flushed(fn, steps, warmup, stream, flush):
+    """Per-step device times (ms) of `steps` calls of fn, each bracketed by its own pair of
+    events, with `flush` (a write larger than L2) run before each bracket: for inputs that
+    would otherwise stay in L2 from one step to the next."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for e0, e1 in ev:
+        flush()
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return [e0.elapsed_time(e1) for e0, e1 in ev]
+
+
 def roofline(info, seconds, peaks, sustained=False):
     """The binding resource of one launch and how close the launch comes to it.
 
@@ -396,6 +415,43 @@ def run_ours(args):
                   "gbs": (info["kv_bytes"] + 2 * new_bytes) / sf / 1e9,
                   "what": "algorithmic bytes: cache K/V read once + new K/V read and written"}
         del k_new, v_new, pg, sl
+    # the batch's classes (prefill chunks, decode steps, verify trees) each timed alone over
+    # the same caches, L2 flushed before every launch: where the unified launch's time goes
+    # and what running the classes in one launch saves against three launches
+    per_class = None
+    if ws == 1 and not args.kv_fp8 and not args.no_other_configs:
+        parts = W.class_batches(batch)
+        if len(parts) > 1:
+            per_class = {}
+            # the flush writes 512 MB, then reads another 512 MB so that the written lines
+            # leave L2 before the timed launch (dirty lines would be written back during it)
+            flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+            sweep_buf = torch.zeros(128 << 20, dtype=torch.float32, device=dev)
+
+            def flush():
+                flush_buf.fill_(1)
+                sweep_buf.sum()
+            for cls, b in parts.items():
+                pl = pk.plan_for_batch(b)
+                inf = pl.info()
+                o = torch.empty_like(b.q)
+
+                def step(pl=pl, b=b, o=o):
+                    pl.run(b.q, b.k_cache, b.v_cache, o, stream)
+                ps = time_flushed(step, args.other_steps, args.warmup, stream, flush)
+                if pl.check(stream) != 0:
+                    raise RuntimeError("device error in the per-class measurement")
+                sec = sum(ps) / len(ps) * 1e-3
+                per_class[cls] = {"sequences": len(b.seqs), "query_tokens": b.total_q,
+                                  "ms_per_launch": sec * 1e3, "kv_gbs": inf["kv_bytes"] / sec / 1e9,
+                                  "attn_tflops": inf["attn_flops"] / sec / 1e12,
+                                  "roofline": roofline(inf, sec, peaks)}
+                pl.close()
+                del b, o
+            per_class["sum_of_class_launches_ms"] = sum(v["ms_per_launch"] for v in per_class.values())
+            per_class["unified_launch_ms"] = avg_launch_s * 1e3
+            del flush_buf, sweep_buf, parts
+            torch.cuda.empty_cache()
     plan.close()
     del batch, out
 
@@ -499,7 +555,7 @@ def run_ours(args):
             "plan": {k: info[k] for k in ("num_decode_items", "num_prefill_items", "num_split_units",
                                           "decode_rows")},
             "per_config": per_config,
-            "append": append,
+            "append": append, "per_class": per_class,
         }
         print(json.dumps(result))
     if ws > 1:

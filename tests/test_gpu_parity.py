@@ -203,3 +203,24 @@ def test_full_size_config_sampled(name):
     assert_close(out[rows], exp, name)
     # every output row is finite
     assert torch.isfinite(out.float()).all()
+
+
+def test_unified_batch_classes_alone():
+    """Each class of the unified Qwen2-7B-shaped batch (prefill chunks, decode steps, verify
+    trees) planned and run alone over the shared caches, as the benchmark times them."""
+    b = W.make_config("qwen2_7b_unified", device=DEV)
+    parts = W.class_batches(b)
+    assert sorted(parts) == ["decode", "prefill", "verify"]
+    for cls, p in parts.items():
+        out, plan = run_batch(p)
+        info = plan.info()
+        if cls == "prefill":
+            assert info["num_prefill_items"] > 0 and info["num_decode_items"] == 0
+        else:
+            assert info["num_prefill_items"] == 0 and info["num_decode_items"] > 0
+        n = len(p.seqs)
+        seq_ids = sorted({0, n // 2, n - 1})
+        picker = (lambda sp: [0, 1, 255, 256, sp.query_len - 1]) if cls == "prefill" else None
+        rows, exp = oracle_rows(p, seq_ids, picker)
+        assert_close(out[rows], exp, f"qwen2_7b_unified[{cls}]")
+        plan.close()

@@ -475,6 +475,43 @@ def shard_batch(batch: Batch, rank: int, world: int) -> Batch:
                  page_perm=batch.page_perm, seed=batch.seed, outlier_frac=batch.outlier_frac)
 
 
+SEQUENCE_CLASSES = ("prefill", "decode", "verify")
+
+
+def seq_class(spec: SeqSpec) -> str:
+    """prefill: a causal chunk of several new tokens; decode: one new token; verify: a draft tree."""
+    if spec.mask_kind == TREE:
+        return "verify"
+    return "decode" if spec.query_len == 1 else "prefill"
+
+
+def class_batches(batch: Batch) -> dict:
+    """The batch's sequences split by class (prefill / decode / verify): each part keeps the
+    same page pool, caches and query values, and takes only its sequences' query rows and
+    block-table rows. Classes with no sequence are left out."""
+    qo = batch.q_offsets()
+    parts = {}
+    for cls in SEQUENCE_CLASSES:
+        seqs = [i for i, sp in enumerate(batch.seqs) if seq_class(sp) == cls]
+        if not seqs:
+            continue
+        qrows = torch.cat([torch.arange(qo[i], qo[i] + batch.seqs[i].query_len) for i in seqs]).to(batch.q.device)
+        k = v = None
+        if batch.k is not None:
+            ko = batch.kv_offsets()
+            krows = torch.cat([torch.arange(ko[i], ko[i] + batch.seqs[i].seq_len) for i in seqs]).to(batch.k.device)
+            k, v = batch.k[krows], batch.v[krows]
+        sel = torch.tensor(seqs, dtype=torch.long, device=batch.block_table.device)
+        parts[cls] = Batch(name=f"{batch.name}[{cls}]", num_q_heads=batch.num_q_heads,
+                           num_kv_heads=batch.num_kv_heads, head_dim=batch.head_dim,
+                           page_size=batch.page_size, seqs=[batch.seqs[i] for i in seqs],
+                           q=batch.q[qrows].contiguous(), k=k, v=v,
+                           k_cache=batch.k_cache, v_cache=batch.v_cache,
+                           block_table=batch.block_table[sel].contiguous(),
+                           page_perm=batch.page_perm, seed=batch.seed, outlier_frac=batch.outlier_frac)
+    return parts
+
+
 def make_config(name: str, device="cpu", seed: Optional[int] = None,
                 keep_contiguous: bool = True, max_seqs: Optional[int] = None) -> Batch:
     """One of the five named batches, seeded by its index unless ``seed`` is given.
