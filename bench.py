@@ -474,10 +474,11 @@ def run_ours(args):
             pl.close()
             del b, o
             torch.cuda.empty_cache()
-        # FP8 (E4M3) caches: the same batches through attn_plan_kv / attn_run_fp8 (every
-        # sequence as decode/verify tasks; algorithmic bytes are the FP8 bytes)
+        # FP8 (E4M3) caches: the same batches through attn_plan_kv / attn_run_fp8 (decode and
+        # verify tasks on the codes, tensor-core tasks on bf16 staging copies made in the same
+        # step; algorithmic bytes are the FP8 bytes)
         fp8 = {}
-        for name in ("llama3_8b_decode", "long_ctx_split", "qwen2_7b_unified"):
+        for name in ("llama3_8b_decode", "long_ctx_split", "qwen2_7b_unified", "llama33_70b_prefill"):
             b = W.make_config(name, device=dev)
             f = W.fp8_kv(b)
             b.k = b.v = None
@@ -550,7 +551,8 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
                     "d2h_bytes_per_step": io_bytes},
-            "gpu_launches": args.steps,
+            # FP8 plans with tensor-core tasks stage their pages in a launch of its own
+            "gpu_launches": args.steps * (2 if args.kv_fp8 and info["num_prefill_items"] > 0 else 1),
             "clocks": clk.summary(),
             "plan": {k: info[k] for k in ("num_decode_items", "num_prefill_items", "num_split_units",
                                           "decode_rows")},

@@ -155,9 +155,13 @@ PKVA_API int attn_plan_shared(pkva_plan_t* out_plan, int num_seqs, const int32_t
  * quantization formats the system supports; FP8 is named beside FP16). FP8 halves the
  * bytes of the bandwidth-bound decode/verify path.
  *
- * An FP8 plan runs every sequence as decode/verify tasks (prefill chunks too: no
- * tensor-core prefill tasks) and cannot be used with attn_run, attn_run_host or
- * attn_run_append (attn_run_fp8_append appends into FP8 caches). Other arguments and errors as attn_plan; PKVA_EINVAL for an unknown
+ * An FP8 plan splits the batch as attn_plan does. Its decode/verify tasks read the E4M3
+ * pages directly; its tensor-core (prefill) tasks, head_dim 128 only, read bf16 copies of
+ * their sequences' pages (the codes' exact values), which each run stages first in a second
+ * launch on the same stream. The plan owns that staging memory: 2 x 2 bytes x Hkv x
+ * page_size x D per page of every such sequence (counted in scratch_bytes). It cannot be
+ * used with attn_run, attn_run_host or attn_run_append (attn_run_fp8_append appends into
+ * FP8 caches). Other arguments and errors as attn_plan; PKVA_EINVAL for an unknown
  * kv_dtype, PKVA_EUNSUPPORTED with PKVA_DECODE_BODY=fma.
  */
 PKVA_API int attn_plan_kv(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq_lens,
@@ -169,8 +173,9 @@ PKVA_API int attn_plan_kv(pkva_plan_t* out_plan, int num_seqs, const int32_t* se
 /*
  * attn_run_fp8 — attn_run over FP8 E4M3 caches (a plan made with PKVA_KV_FP8_E4M3).
  *
- *   q          device bf16 [sum T_s, Hq, D] (as attn_run; |q| must stay in f16's range,
- *              the kernels compute in f16 with fp32 accumulation).
+ *   q          device bf16 [sum T_s, Hq, D] (as attn_run; |q| must stay in f16's range:
+ *              the decode/verify tasks compute in f16 with fp32 accumulation, the
+ *              tensor-core tasks in bf16 with fp32 accumulation).
  *   k_cache    device uint8 [num_pages, Hkv, page_size, D]: E4M3 codes, the same layout
  *              as the bf16 cache.
  *   v_cache_t  device uint8 [num_pages, Hkv, D, page_size]: E4M3 codes, each (page, KV
@@ -180,7 +185,8 @@ PKVA_API int attn_plan_kv(pkva_plan_t* out_plan, int num_seqs, const int32_t* se
  *              (E4M3: sign, 4 exponent bits with bias 7, 3 mantissa bits, no infinities,
  *              S.1111.111 is NaN).
  *   out        device bf16 [sum T_s, Hq, D].
- * Codes in slots past a sequence's end may be anything (NaN codes included). Errors as
+ * Codes in slots past a sequence's end may be anything (NaN codes included). One launch,
+ * or two when the plan has tensor-core tasks (the staging copy, then attention). Errors as
  * attn_run; PKVA_EINVAL if the plan is not an FP8 plan or a scale pointer is NULL.
  */
 PKVA_API int attn_run_fp8(pkva_plan_t plan, const void* q, const void* k_cache, const void* v_cache_t,
@@ -188,7 +194,8 @@ PKVA_API int attn_run_fp8(pkva_plan_t plan, const void* q, const void* k_cache, 
 
 /*
  * attn_run_fp8_append — attn_run_append over FP8 E4M3 caches: writes the new tokens' codes
- * into k_cache / v_cache_t and computes the batch's attention, in one launch on `stream`.
+ * into k_cache / v_cache_t and computes the batch's attention on `stream` (one launch; with
+ * tensor-core tasks the staging launch before it writes their sequences' new codes).
  *
  *   k_new, v_new  device bf16 [sum T_s, Hkv, D] (as attn_run_append).
  *   other arguments as attn_run_fp8 (k_cache and v_cache_t are written at the new tokens'

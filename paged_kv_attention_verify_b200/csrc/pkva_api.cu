@@ -167,6 +167,13 @@ struct pkva_plan {
     pkva::CascadeWork* d_cwork = nullptr;
     int32_t* d_crowmap = nullptr;
     int32_t* d_cunits = nullptr;
+    // FP8 caches: bf16 staging pages of the tensor-core sequences, their block table and
+    // source list, and the cache maps over them
+    __nv_bfloat16* d_stage_k = nullptr;
+    __nv_bfloat16* d_stage_v = nullptr;
+    int32_t* d_stage_bt = nullptr;
+    int32_t* d_stage_src = nullptr;
+    CUtensorMap tmSK, tmSV;
     int64_t scratch_bytes = 0;
 };
 
@@ -183,6 +190,10 @@ static void free_plan(pkva_plan* p) {
     cudaFree(p->d_cwork);
     cudaFree(p->d_crowmap);
     cudaFree(p->d_cunits);
+    cudaFree(p->d_stage_k);
+    cudaFree(p->d_stage_v);
+    cudaFree(p->d_stage_bt);
+    cudaFree(p->d_stage_src);
     cudaFree(p->d_anc);
     cudaFree(p->d_part_o);
     cudaFree(p->d_part_ml);
@@ -324,6 +335,19 @@ static int plan_create(pkva_plan_t* out_plan, PlanArgs a, const int32_t* block_t
                         "cudaMalloc(split partials)"));
     PKVA_TRY(alloc_zero((void**)&p->d_counters, hp.units.size() * sizeof(int32_t), "cudaMalloc(split counters)"));
     PKVA_TRY(alloc_zero((void**)&p->d_err, sizeof(int32_t), "cudaMalloc(error word)"));
+    if (hp.num_stage_pages > 0) {
+        PKVA_TRY(upload(&p->d_stage_bt, hp.stage_bt, &p->scratch_bytes));
+        PKVA_TRY(upload(&p->d_stage_src, hp.stage_src, &p->scratch_bytes));
+        const size_t bytes = (size_t)hp.num_stage_pages * hp.Hkv * kPageSize * hp.D * sizeof(__nv_bfloat16);
+        PKVA_TRY(alloc_zero((void**)&p->d_stage_k, bytes, "cudaMalloc(FP8 staging pages)"));
+        PKVA_TRY(alloc_zero((void**)&p->d_stage_v, bytes, "cudaMalloc(FP8 staging pages)"));
+        if (!encode_cache_map(&p->tmSK, p->d_stage_k, hp.num_stage_pages, hp.Hkv, hp.D) ||
+            !encode_cache_map(&p->tmSV, p->d_stage_v, hp.num_stage_pages, hp.Hkv, hp.D)) {
+            free_plan(p);
+            set_last_error(name + ": cuTensorMapEncodeTiled failed for the FP8 staging pages");
+            return PKVA_ECUDA;
+        }
+    }
 #undef PKVA_TRY
     set_last_error("");
     *out_plan = p;
@@ -351,7 +375,7 @@ extern "C" int attn_plan_kv(pkva_plan_t* out_plan, int num_seqs, const int32_t* 
     PlanArgs a{num_seqs, seq_lens, query_lens, bt_stride, num_pages, mask_kind, parents, num_q_heads,
                num_kv_heads, head_dim, page_size, sm_scale, 1, 1};
     const bool fp8 = kv_dtype == PKVA_KV_FP8_E4M3;
-    a.use_prefill_kernel = !fp8;     // FP8 caches: every sequence runs as decode/verify tasks
+    a.use_prefill_kernel = true;     // FP8 caches: tensor-core tasks read bf16 staging copies of their pages
     a.kv_elem_bytes = fp8 ? 1 : 2;
     return plan_create(out_plan, a, block_table, "attn_plan_kv", fp8);
 }
@@ -473,14 +497,14 @@ static int run_impl(pkva_plan_t plan, const void* q, const void* k_new, const vo
         }
         plan->tm_q = q;
     }
-    if (has_prefill && append && plan->tm_kn != k_new) {
+    if (has_prefill && append && !fp8 && plan->tm_kn != k_new) {
         if (!encode_q_map(&plan->tmKn, k_new, hp.total_q, hp.Hkv, hp.D)) {
             set_last_error(name + ": cuTensorMapEncodeTiled failed for k_new");
             return PKVA_ECUDA;
         }
         plan->tm_kn = k_new;
     }
-    if (has_prefill && append && plan->tm_vn != v_new) {
+    if (has_prefill && append && !fp8 && plan->tm_vn != v_new) {
         if (!encode_q_map(&plan->tmVn, v_new, hp.total_q, hp.Hkv, hp.D)) {
             set_last_error(name + ": cuTensorMapEncodeTiled failed for v_new");
             return PKVA_ECUDA;
@@ -529,19 +553,57 @@ static int run_impl(pkva_plan_t plan, const void* q, const void* k_new, const vo
     dp.k_scale = k_scale;
     dp.v_scale = v_scale;
     if (append) {
-        pp.append = dp.append = 1;
-        pp.k_new = dp.k_new = static_cast<const __nv_bfloat16*>(k_new);
-        pp.v_new = dp.v_new = static_cast<const __nv_bfloat16*>(v_new);
+        dp.append = 1;
+        dp.k_new = static_cast<const __nv_bfloat16*>(k_new);
+        dp.v_new = static_cast<const __nv_bfloat16*>(v_new);
         // the cache is written only at the new tokens' slots, which no task reads
-        pp.k_cache = dp.k_cache = static_cast<__nv_bfloat16*>(const_cast<void*>(k_cache));
-        pp.v_cache = dp.v_cache = static_cast<__nv_bfloat16*>(const_cast<void*>(v_cache));
+        dp.k_cache = static_cast<__nv_bfloat16*>(const_cast<void*>(k_cache));
+        dp.v_cache = static_cast<__nv_bfloat16*>(const_cast<void*>(v_cache));
+        if (!fp8) {                    // (over FP8 caches the staging pass appends for the tensor-core tasks)
+            pp.append = 1;
+            pp.k_new = dp.k_new;
+            pp.v_new = dp.v_new;
+            pp.k_cache = dp.k_cache;
+            pp.v_cache = dp.v_cache;
+        }
+    }
+    cudaError_t e;
+    if (fp8 && hp.num_stage_pages > 0) {
+        // FP8 caches: stage the tensor-core sequences' pages as bf16, then the tasks read
+        // those through the staging block table, with the caller's scales
+        StageParams sp;
+        sp.src = plan->d_stage_src;
+        sp.n = hp.num_stage_pages;
+        sp.block_table = plan->block_table;
+        sp.bt_stride = hp.bt_stride;
+        sp.num_pages = hp.num_pages;
+        sp.Hkv = hp.Hkv;
+        sp.seqs = plan->d_seqs;
+        sp.k_codes = static_cast<uint8_t*>(const_cast<void*>(k_cache));
+        sp.v_codes_t = static_cast<uint8_t*>(const_cast<void*>(v_cache));
+        sp.stage_k = plan->d_stage_k;
+        sp.stage_v = plan->d_stage_v;
+        sp.err = plan->d_err;
+        if (append) {
+            sp.append = 1;
+            sp.k_new = dp.k_new;
+            sp.v_new = dp.v_new;
+        }
+        sp.k_scale = k_scale;
+        sp.v_scale = v_scale;
+        e = launch_stage_fp8(sp, st);
+        if (e != cudaSuccess) return cuda_fail(e, (name + ": staging launch").c_str());
+        pp.block_table = plan->d_stage_bt;
+        pp.bt_stride = hp.stage_stride;
+        pp.num_pages = hp.num_stage_pages;
+        pp.k_scale = k_scale;
+        pp.v_scale = v_scale;
     }
     AttnParams ap;
     ap.pre = pp;
     ap.dec = dp;
-    const CUtensorMap& tmKn = append ? plan->tmKn : plan->tmQ;
-    const CUtensorMap& tmVn = append ? plan->tmVn : plan->tmQ;
-    cudaError_t e;
+    const CUtensorMap& tmKn = fp8 ? plan->tmSK : append ? plan->tmKn : plan->tmQ;
+    const CUtensorMap& tmVn = fp8 ? plan->tmSV : append ? plan->tmVn : plan->tmQ;
     if (plan->decode_mma) {
         // the whole batch in one launch
         ap.order = plan->d_order;

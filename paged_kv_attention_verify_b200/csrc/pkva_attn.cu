@@ -44,14 +44,14 @@ struct AttnSmem {
     using DC = dec::DecodeCfg<D, NT * 8, false, kDecWarps, AttnNS<D, FP8>::value, FP8 ? 1 : 2>;
     static constexpr int GROUP_BYTES = (DC::BYTES + 1023) / 1024 * 1024;    // one decode task
     static constexpr int DEC_BYTES = kDecTasksPerBlock * GROUP_BYTES;
-    static constexpr int TASK_BYTES = (D == 128 && !FP8 && pre::kSmemBytes > DEC_BYTES) ? pre::kSmemBytes : DEC_BYTES;
+    static constexpr int TASK_BYTES = (D == 128 && pre::kSmemBytes > DEC_BYTES) ? pre::kSmemBytes : DEC_BYTES;
     static constexpr int OFF_SCHED = TASK_BYTES;  // the TMEM address of a tensor-core block
     static constexpr int BYTES = TASK_BYTES + 64;
     static constexpr int ALLOC = BYTES + 1008;    // room to align to 1024
     static_assert(ALLOC <= 227 * 1024, "shared memory");
 };
 
-// FP8: decode/verify tasks only (a plan over FP8 caches has no tensor-core tasks).
+// FP8: decode/verify tasks read the E4M3 pages; tensor-core tasks read their bf16 staging copies.
 template <int D, int NT, bool FP8>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -61,7 +61,7 @@ attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const _
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int e = p.order[blockIdx.x];
-    if constexpr (D == 128 && !FP8) {
+    if constexpr (D == 128) {
         if (e >= 0) {
             // tensor-core task: 512 TMEM columns for the block (one block per SM)
             uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + S::OFF_SCHED);
@@ -74,7 +74,8 @@ attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const _
             __syncthreads();
             tc_fence_after();
             const uint32_t tmem = *tmem_slot;
-            pre::prefill_task(p.pre, e, tmQ, tmK, tmV, tmKn, tmVn, tmQc, tmem, sm);
+            // over FP8 caches the tensor-core tasks read the bf16 staging pages (tmKn / tmVn)
+            pre::prefill_task(p.pre, e, tmQ, FP8 ? tmKn : tmK, FP8 ? tmVn : tmV, tmKn, tmVn, tmQc, tmem, sm);
             tc_fence_before();
             __syncthreads();
             tc_fence_after();
@@ -141,7 +142,7 @@ int attn_ctas_per_sm(int D, int rows) {
 cudaError_t launch_attn(const AttnParams& p, int D, int rows, bool has_prefill, const CUtensorMap& tmQ,
                         const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKn,
                         const CUtensorMap& tmVn, const CUtensorMap& tmQc, cudaStream_t stream, bool fp8) {
-    if ((D == 64 || fp8) && has_prefill) return cudaErrorInvalidValue;   // tensor-core tasks: bf16, head_dim 128
+    if (D == 64 && has_prefill) return cudaErrorInvalidValue;   // tensor-core tasks: head_dim 128
     return fp8 ? launch_kv<true>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
                : launch_kv<false>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
 }

@@ -119,6 +119,14 @@ struct HostPlan {
     std::vector<int32_t> crowmap;
     std::vector<int32_t> cunits;
     int cascade_tok = 0;                  // tokens per cascade tile: floor(128 / G)
+    // FP8 caches: the pages of the tensor-core (prefill) sequences are staged as bf16 before
+    // the attention launch. Staging page n holds (sequence stage_src[2n], logical page
+    // stage_src[2n+1]); stage_bt [num_seqs][stage_stride] maps a prefill sequence's logical
+    // pages to staging pages (-1 elsewhere).
+    std::vector<int32_t> stage_src;
+    std::vector<int32_t> stage_bt;
+    int stage_stride = 0;
+    int num_stage_pages = 0;
     int64_t kv_bytes = 0;
     int64_t attn_flops = 0;
 };

@@ -61,7 +61,37 @@ struct PrefillParams {
     float* part_o = nullptr;
     float* part_ml = nullptr;
     int32_t* counters = nullptr;
+    // FP8 caches: the tasks read bf16 copies of the codes (block_table / num_pages address
+    // the staging pages); the K scale of the task's KV head multiplies the softmax scale and
+    // the V scale the output
+    const float* k_scale = nullptr;
+    const float* v_scale = nullptr;
 };
+
+// FP8 caches: copy the pages of the tensor-core sequences to bf16 staging pages (the codes'
+// exact values, unscaled), one block per staging page and all KV heads. Slots past the
+// sequence's end become zeros. With append, the new tokens' codes are computed from
+// k_new / v_new, written into the FP8 caches and staged.
+struct StageParams {
+    const int32_t* src;          // [n][2]: (sequence, logical page)
+    int32_t n;                   // staging pages
+    const int32_t* block_table;  // the caller's [B, bt_stride]
+    int32_t bt_stride;
+    int32_t num_pages;           // the caller's page pool
+    int32_t Hkv;
+    const SeqInfo* seqs;
+    uint8_t* k_codes;            // [pages, Hkv, 16, 128]
+    uint8_t* v_codes_t;          // [pages, Hkv, 128, 16]
+    __nv_bfloat16* stage_k;      // [n, Hkv, 16, 128]
+    __nv_bfloat16* stage_v;
+    int32_t* err;
+    int32_t append = 0;
+    const __nv_bfloat16* k_new = nullptr;   // [sum T, Hkv, 128]
+    const __nv_bfloat16* v_new = nullptr;
+    const float* k_scale = nullptr;
+    const float* v_scale = nullptr;
+};
+cudaError_t launch_stage_fp8(const StageParams& p, cudaStream_t stream);
 
 // Everything one launch of the unified attention kernel needs.
 // One entry of `order` per block: e >= 0 runs tensor-core task e (a prefill task, or
@@ -84,7 +114,8 @@ int attn_ctas_per_sm(int D, int rows);
 // tmQc views q in boxes of {64 columns, G heads, floor(128 / G) tokens}; read only by
 // cascade tasks.
 // fp8: the caches are E4M3 codes (tmK over [pages*Hkv*16][D] bytes, tmV over the transposed
-// [pages*Hkv*D][16] bytes) and the launch has decode/verify tasks only.
+// [pages*Hkv*D][16] bytes, read by decode/verify tasks); tensor-core tasks then read the bf16
+// staging pages through tmKn / tmVn (cache maps, 16 x 64 boxes), and p.pre.append is 0.
 cudaError_t launch_attn(const AttnParams& p, int D, int rows, bool has_prefill, const CUtensorMap& tmQ,
                         const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKn,
                         const CUtensorMap& tmVn, const CUtensorMap& tmQc, cudaStream_t stream, bool fp8 = false);

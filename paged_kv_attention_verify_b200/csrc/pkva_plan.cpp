@@ -196,6 +196,35 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
         });
     }
 
+    // FP8 caches: the tensor-core tasks read a bf16 copy of their sequences' pages
+    if (a.kv_elem_bytes == 1) {
+        int stride = 0, n = 0;
+        for (int s = 0; s < a.num_seqs; ++s)
+            if (on_prefill[s]) {
+                const int pages = (p.seqs[s].seq_len + kPageSize - 1) / kPageSize;
+                stride = std::max(stride, pages);
+                n += pages;
+            }
+        if ((int64_t)n * a.Hkv * kPageSize >= (int64_t(1) << 31))
+            return fail(err, PKVA_EUNSUPPORTED, "FP8 prefill staging too large: %ld pages", n);
+        if (n > 0) {
+            p.stage_stride = stride;
+            p.num_stage_pages = n;
+            p.stage_bt.assign((size_t)a.num_seqs * stride, -1);
+            p.stage_src.reserve(2 * (size_t)n);
+            int next = 0;
+            for (int s = 0; s < a.num_seqs; ++s) {
+                if (!on_prefill[s]) continue;
+                const int pages = (p.seqs[s].seq_len + kPageSize - 1) / kPageSize;
+                for (int lp = 0; lp < pages; ++lp) {
+                    p.stage_bt[(size_t)s * stride + lp] = next++;
+                    p.stage_src.push_back(s);
+                    p.stage_src.push_back(lp);
+                }
+            }
+        }
+    }
+
     // -- decode/verify units: (seq, kv head, chunk of packed rows) --------------------
     // A sequence of a shared-prefix group leaves its first prefix_len keys to the cascade
     // tasks: its units start at that page, and always merge partials.

@@ -413,6 +413,9 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         const int lim_first_b = w.tok0 + b * kPrefillTileM, lim_b = tok;
         const int lim_first_a = cascade || append ? key_limit - 1 : prefix + lim_first_b;
         const int lim_a = cascade || append ? key_limit - 1 : (row_in_task < w.ntok ? prefix + tok : 0x7fffffff);
+        // FP8 caches: the tiles hold the codes' values, so the K scale of this KV head joins
+        // the softmax scale (and the V scale the output, below)
+        const float sl2 = p.k_scale ? p.scale_log2 * p.k_scale[kvh] : p.scale_log2;
         float m_ref = -INFINITY, l_sum = 0.f;
         bool alive = true;
         // every break below is taken by the whole warp (tcgen05.ld/st are warp-collective)
@@ -445,7 +448,7 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
             for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
 #pragma unroll
             for (int i = 0; i < 4; ++i) mx8[i] = fmaxf(mx8[i], mx8[i + 4]);
-            const float m_tile = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])) * p.scale_log2;
+            const float m_tile = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])) * sl2;
             bool need = false;
             float m_new = m_ref;
             if (j == 0) {
@@ -464,8 +467,8 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
             // P in place: pair c goes to word c (already consumed), then out to S_b[0, 64)
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
-                const float x0 = fmaf(__uint_as_float(sr[2 * c]), p.scale_log2, -ref);
-                const float x1 = fmaf(__uint_as_float(sr[2 * c + 1]), p.scale_log2, -ref);
+                const float x0 = fmaf(__uint_as_float(sr[2 * c]), sl2, -ref);
+                const float x1 = fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -ref);
                 float p0, p1;
                 if (kExp2PolyEvery > 0 && c % (kExp2PolyEvery > 0 ? kExp2PolyEvery : 1) == 0) {
                     const float2 e = exp2_poly2(make_float2(x0, x1));
@@ -563,7 +566,8 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         else if (nb > 0 && alive && __all_sync(0xffffffffu, wait_or_abort(&B.o_ready[b], 0, p.err, abort_flag))) {
             tc_fence_after();
             const bool real_row = row_in_task < w.ntok;
-            const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+            float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+            if (p.v_scale) inv *= p.v_scale[kvh];
             __nv_bfloat16* dst = p.out + ((int64_t)(si.q_start + tok) * p.Hq + w.q_head) * kD;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {

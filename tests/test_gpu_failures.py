@@ -34,9 +34,10 @@ def test_bad_block_table_entry_is_reported_not_faulted(T):
     assert plan.check() == 0                         # attn_check cleared the word
 
 
-def test_bad_block_table_entry_fp8_and_cascade():
+@pytest.mark.parametrize("T", [1, 300])            # FP8: a decode task, or the bf16 staging pass
+def test_bad_block_table_entry_fp8_and_cascade(T):
     """The same report on the FP8 path and on a shared-prefix (cascade) plan."""
-    seqs = [W.SeqSpec(600, 1, W.CAUSAL, []), W.SeqSpec(400, 1, W.CAUSAL, [])]
+    seqs = [W.SeqSpec(600, T, W.CAUSAL, []), W.SeqSpec(400, 1, W.CAUSAL, [])]
     b = W.build_batch("bad8", seqs, 8, 2, 128, seed=5, device="cuda")
     f = W.fp8_kv(b)
     bt = b.block_table.clone()

@@ -1,9 +1,11 @@
 """GPU parity of the FP8 (E4M3) KV cache path (attn_plan_kv + attn_run_fp8) against the
 float64 oracle over the decoded codes (oracle.dequantize_kv: code value x per-head scale).
 
-The kernels decode every code exactly and compute in f16 with fp32 accumulation, so the
-same tolerance as the bf16 path applies (max abs <= 2e-2, mean abs <= 2e-3). Codes in the
-slots past each sequence's end are random bytes, NaN codes included.
+The decode/verify tasks decode every code exactly and compute in f16 with fp32
+accumulation; the tensor-core (prefill) tasks read exact bf16 copies of the codes staged
+before the launch and apply the scales in fp32. So the same tolerance as the bf16 path
+applies (max abs <= 2e-2, mean abs <= 2e-3). Codes in the slots past each sequence's end
+are random bytes, NaN codes included.
 """
 import numpy as np
 import pytest
@@ -38,7 +40,6 @@ def fp8_oracle_rows(b, f, seq_ids=None, token_picker=None):
 
 def run_fp8(b, f):
     plan = pk.plan_for_batch(b, kv_fp8=True)
-    assert plan.info()["num_prefill_items"] == 0
     out = plan.run_fp8(b.q, f.k_cache, f.v_cache_t, f.k_scale, f.v_scale)
     assert plan.check() == 0
     return out, plan
@@ -65,14 +66,23 @@ def test_fp8_small_batches_all_rows(cfg):
     plan.close()
 
 
-def test_fp8_prefill_chunk_runs_as_decode_tasks():
+def test_fp8_prefill_chunks_run_on_tensor_cores():
+    """Long causal chunks over FP8 caches run as tensor-core tasks on bf16 staging copies:
+    no prefix, a prefix that ends inside a page, a multi-tile chunk on a long prefix, and a
+    decode step beside them. Every row against the oracle."""
     seqs = [W.SeqSpec(300, 300, W.CAUSAL, []), W.SeqSpec(133 + 200, 200, W.CAUSAL, []),
-            W.SeqSpec(900, 1, W.CAUSAL, [])]
+            W.SeqSpec(1500 + 384, 384, W.CAUSAL, []), W.SeqSpec(900, 1, W.CAUSAL, [])]
     b = W.build_batch("fp8_prefill", seqs, 16, 2, 128, seed=37, device=DEV)
     f = W.fp8_kv(b)
     out, plan = run_fp8(b, f)
+    info = plan.info()
+    assert info["num_prefill_items"] > 0 and info["num_decode_items"] > 0
     rows, exp = fp8_oracle_rows(b, f)
     assert_close(out[rows], exp, "fp8 prefill chunks")
+    # the same batch again (staging pages rewritten, nothing carried over)
+    out2 = plan.run_fp8(b.q, f.k_cache, f.v_cache_t, f.k_scale, f.v_scale)
+    assert plan.check() == 0
+    assert torch.equal(out, out2)
     plan.close()
 
 
@@ -80,7 +90,7 @@ def _sample(sp):
     return sorted({0, sp.query_len // 2, sp.query_len - 1})
 
 
-@pytest.mark.parametrize("name", ["llama3_8b_decode", "long_ctx_split", "qwen2_7b_unified"])
+@pytest.mark.parametrize("name", ["llama3_8b_decode", "long_ctx_split", "qwen2_7b_unified", "llama33_70b_prefill"])
 def test_fp8_configs_full_size(name):
     b = W.make_config(name, device=DEV)
     f = W.fp8_kv(b)
@@ -114,7 +124,7 @@ def test_fp8_plan_and_run_mismatches_are_rejected():
     pb.close()
 
 
-def _fp8_append_case(b):
+def _fp8_append_case(b, expect_prefill=False):
     """Append into FP8 caches: the new tokens' slots start as NaN codes; afterwards they hold
     E4M3(float32(x) / scale) of the dense input (oracle.e4m3_encode, bit for bit) and every
     other byte is unchanged; the output matches the oracle over those codes."""
@@ -131,6 +141,8 @@ def _fp8_append_case(b):
     kc[pg, :, sl] = 0x7F
     vct[pg, :, :, sl] = 0x7F
     plan = pk.plan_for_batch(b, kv_fp8=True)
+    if expect_prefill:
+        assert plan.info()["num_prefill_items"] > 0
     out = plan.run_fp8_append(b.q, k_new, v_new, kc, vct, f.k_scale, f.v_scale)
     assert plan.check() == 0
     assert torch.equal(kc, exp_k), "k_cache codes after append"
@@ -152,6 +164,16 @@ def _fp8_append_case(b):
 def test_fp8_append_small(seed, d):
     b = W.random_small(seed, num_seqs=6, Hq=16, Hkv=4, d=d, max_ctx=300, max_q=40, tree_frac=0.4, device=DEV)
     _fp8_append_case(b)
+
+
+def test_fp8_append_with_prefill_chunks():
+    """Append over FP8 caches when long chunks run as tensor-core tasks: the staging pass
+    writes those sequences' new codes into the caches, the decode tasks write theirs."""
+    seqs = [W.SeqSpec(200, 200, W.CAUSAL, []), W.SeqSpec(77 + 150, 150, W.CAUSAL, []),
+            W.SeqSpec(640, 1, W.CAUSAL, []), W.SeqSpec(400 + 5, 5, W.TREE, [-1, 0, 0, 1, 2]),
+            W.SeqSpec(1024 + 256, 256, W.CAUSAL, [])]
+    b = W.build_batch("fp8_append_prefill", seqs, 16, 4, 128, seed=54, device=DEV)
+    _fp8_append_case(b, expect_prefill=True)
 
 
 def test_fp8_append_rejects_bf16_paths():
