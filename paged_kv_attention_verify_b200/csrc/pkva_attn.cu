@@ -39,12 +39,14 @@ struct AttnNS {
     static constexpr int value = (D == 64 ? 4 : 2) * (FP8 ? 2 : 1);
 };
 
-template <int D, int NT, bool FP8 = false>
+// TC: the kernel can run tensor-core tasks (head_dim 128 only). FP8 launches without any
+// tensor-core task use the TC = false kernel: smaller code for the decode-only plans.
+template <int D, int NT, bool FP8 = false, bool TC = true>
 struct AttnSmem {
     using DC = dec::DecodeCfg<D, NT * 8, false, kDecWarps, AttnNS<D, FP8>::value, FP8 ? 1 : 2>;
     static constexpr int GROUP_BYTES = (DC::BYTES + 1023) / 1024 * 1024;    // one decode task
     static constexpr int DEC_BYTES = kDecTasksPerBlock * GROUP_BYTES;
-    static constexpr int TASK_BYTES = (D == 128 && pre::kSmemBytes > DEC_BYTES) ? pre::kSmemBytes : DEC_BYTES;
+    static constexpr int TASK_BYTES = (D == 128 && TC && pre::kSmemBytes > DEC_BYTES) ? pre::kSmemBytes : DEC_BYTES;
     static constexpr int OFF_SCHED = TASK_BYTES;  // the TMEM address of a tensor-core block
     static constexpr int BYTES = TASK_BYTES + 64;
     static constexpr int ALLOC = BYTES + 1008;    // room to align to 1024
@@ -52,16 +54,16 @@ struct AttnSmem {
 };
 
 // FP8: decode/verify tasks read the E4M3 pages; tensor-core tasks read their bf16 staging copies.
-template <int D, int NT, bool FP8>
+template <int D, int NT, bool FP8, bool TC>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKn,
             const __grid_constant__ CUtensorMap tmVn, const __grid_constant__ CUtensorMap tmQc) {
-    using S = AttnSmem<D, NT, FP8>;
+    using S = AttnSmem<D, NT, FP8, TC>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int e = p.order[blockIdx.x];
-    if constexpr (D == 128) {
+    if constexpr (D == 128 && TC) {
         if (e >= 0) {
             // tensor-core task: 512 TMEM columns for the block (one block per SM)
             uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + S::OFF_SCHED);
@@ -93,42 +95,43 @@ attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const _
                                                                     sm + g * S::GROUP_BYTES);
 }
 
-template <int D, int NT, bool FP8>
+template <int D, int NT, bool FP8, bool TC>
 cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                      const CUtensorMap& tmKn, const CUtensorMap& tmVn, const CUtensorMap& tmQc,
                      cudaStream_t stream) {
-    using S = AttnSmem<D, NT, FP8>;
+    using S = AttnSmem<D, NT, FP8, TC>;
     cudaError_t e =
-        cudaFuncSetAttribute(attn_kernel<D, NT, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::ALLOC);
+        cudaFuncSetAttribute(attn_kernel<D, NT, FP8, TC>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::ALLOC);
     if (e != cudaSuccess) return e;
     const int grid = p.num_blocks;
     if (grid == 0) return cudaSuccess;
-    attn_kernel<D, NT, FP8><<<grid, kAttnThreads, S::ALLOC, stream>>>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc);
+    attn_kernel<D, NT, FP8, TC><<<grid, kAttnThreads, S::ALLOC, stream>>>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc);
     return cudaGetLastError();
 }
 
 template <int D, int NT>
 int ctas_t() {
-    using S = AttnSmem<D, NT>;
+    constexpr bool TC = D == 128;
+    using S = AttnSmem<D, NT, false, TC>;
     int n = 0;
-    if (cudaFuncSetAttribute(attn_kernel<D, NT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::ALLOC) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(attn_kernel<D, NT, false, TC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             S::ALLOC) != cudaSuccess)
         return 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_kernel<D, NT, false>, kAttnThreads, S::ALLOC) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_kernel<D, NT, false, TC>, kAttnThreads, S::ALLOC) !=
         cudaSuccess)
         return 0;
     return n;
 }
 
-template <bool FP8>
+template <bool FP8, bool TC>
 cudaError_t launch_kv(const AttnParams& p, int D, int rows, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                       const CUtensorMap& tmV, const CUtensorMap& tmKn, const CUtensorMap& tmVn,
                       const CUtensorMap& tmQc, cudaStream_t stream) {
     if (D == 64)
-        return rows <= 8 ? launch_t<64, 1, FP8>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
-                         : launch_t<64, 2, FP8>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
-    return rows <= 8 ? launch_t<128, 1, FP8>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
-                     : launch_t<128, 2, FP8>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
+        return rows <= 8 ? launch_t<64, 1, FP8, false>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
+                         : launch_t<64, 2, FP8, false>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
+    return rows <= 8 ? launch_t<128, 1, FP8, TC>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
+                     : launch_t<128, 2, FP8, TC>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
 }
 
 }  // namespace
@@ -143,8 +146,9 @@ cudaError_t launch_attn(const AttnParams& p, int D, int rows, bool has_prefill, 
                         const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKn,
                         const CUtensorMap& tmVn, const CUtensorMap& tmQc, cudaStream_t stream, bool fp8) {
     if (D == 64 && has_prefill) return cudaErrorInvalidValue;   // tensor-core tasks: head_dim 128
-    return fp8 ? launch_kv<true>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
-               : launch_kv<false>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
+    if (!fp8) return launch_kv<false, true>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
+    return has_prefill ? launch_kv<true, true>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
+                       : launch_kv<true, false>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
 }
 
 }  // namespace pkva
