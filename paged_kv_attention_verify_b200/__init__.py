@@ -239,7 +239,8 @@ class Plan:
 
     def run_fp8_append(self, q, k_new, v_new, k_cache, v_cache_t, k_scale, v_scale, out=None, stream=None):
         """``attn_run_fp8_append``: quantise the new tokens' K/V (bf16 [sum T, Hkv, D]) into the
-        FP8 caches at their slots and compute the attention, in one launch."""
+        FP8 caches at their slots and compute the attention (one launch; with tensor-core
+        tasks, the staging launch before it appends their sequences' rows)."""
         import torch
         if out is None:
             out = torch.empty_like(q)
