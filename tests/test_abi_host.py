@@ -219,3 +219,22 @@ def test_shared_prefix_needs_head_dim_128():
         pk.inspect([40, 60], [1, 1], [0, 0], num_q_heads=8, num_kv_heads=2, head_dim=64,
                    num_pages=12, bt_stride=4, prefix_group=[0, 0], prefix_len=[32])
     assert ei.value.code == -2
+
+
+@pytest.mark.parametrize("num_sms, ctas", [(1, 1), (4, 3), (148, 3)])
+def test_decode_tasks_never_exceed_the_staged_block_table_slice(num_sms, ctas):
+    """A decode/verify task stages its block-table entries in shared memory (1024 of them), so
+    no task may span more pages, whatever the number of CTA slots the split targets."""
+    lens = [200_000, 131_072, 16_385, 1024 * 16 + 1, 17]
+    items = pk.inspect(lens, [1, 1, 1, 1, 1], [0] * 5, num_q_heads=16, num_kv_heads=2, head_dim=128,
+                       num_pages=sum((L + 15) // 16 for L in lens), bt_stride=(max(lens) + 15) // 16,
+                       num_sms=num_sms, ctas_per_sm=ctas)
+    assert items and all(it["kind"] == 0 for it in items)
+    for it in items:
+        assert (it["key_end"] + 15) // 16 - it["key_begin"] // 16 <= 1024
+    # every (sequence, KV head) still covers all its keys
+    for s, L in enumerate(lens):
+        for h in range(2):
+            spans = sorted((it["key_begin"], it["key_end"]) for it in items if it["seq"] == s and it["kv_head"] == h)
+            assert spans[0][0] == 0 and spans[-1][1] == L
+            assert all(a[1] == b[0] for a, b in zip(spans[:-1], spans[1:]))
