@@ -1,5 +1,5 @@
 // Fused paged-KV append: writing the new tokens' K/V into their cache slots inside the
-// attention launch (survey section 8, next row 1).
+// attention launch.
 //
 // Attention tasks never read these writes: a decode/verify task patches the new tokens'
 // rows into its shared-memory copy of each page from the dense input, and a prefill task

@@ -65,28 +65,6 @@ constexpr float kRescaleSlack = 8.f;
 constexpr int kWarpKProd = 8, kWarpMma = 9, kWarpVProd = 10;
 constexpr bool kSpinOnS = true;    // softmax warps poll S without suspending
 
-// 2^x on the FMA pipe: 2^x = 2^n * p(f), n = round(x), f = x - n in [-1/2, 1/2], p the cubic
-// interpolating 2^f at the Chebyshev nodes of [-1/2, 1/2] (max relative error 1.0e-4, below
-// the 2^-9 rounding of bf16 P). Coefficients from csrc/exp2_poly_fit.py. Moving one pair of
-// columns in four off the special-function unit made this kernel slower on B200 (its
-// softmax is bound by issue and latency, not by that unit), so kExp2PolyEvery = 0 (off).
-constexpr float kExp2C0 = 0.99992454f, kExp2C1 = 0.69313675f, kExp2C2 = 0.24263948f, kExp2C3 = 0.055838283f;
-constexpr int kExp2PolyEvery = 0;
-
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-    x.x = fmaxf(x.x, -126.f);                               // 2^-126: no exponent wrap-around
-    x.y = fmaxf(x.y, -126.f);
-    const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));      // 1.5 * 2^23: round
-    const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-    float2 q = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
-    q = __ffma2_rn(q, f, make_float2(kExp2C1, kExp2C1));
-    q = __ffma2_rn(q, f, make_float2(kExp2C0, kExp2C0));
-    // n sits in the low mantissa bits of t; shifted by 23 it is the exponent increment
-    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
-                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
-}
-
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);   // Q, K both K-major
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);    // P from TMEM, V MN-major
 
@@ -469,15 +447,8 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
             for (int c = 0; c < 64; ++c) {
                 const float x0 = fmaf(__uint_as_float(sr[2 * c]), sl2, -ref);
                 const float x1 = fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -ref);
-                float p0, p1;
-                if (kExp2PolyEvery > 0 && c % (kExp2PolyEvery > 0 ? kExp2PolyEvery : 1) == 0) {
-                    const float2 e = exp2_poly2(make_float2(x0, x1));
-                    p0 = e.x;
-                    p1 = e.y;
-                } else {
-                    p0 = exp2f(x0);
-                    p1 = exp2f(x1);
-                }
+                const float p0 = exp2f(x0);
+                const float p1 = exp2f(x1);
                 ls4[c & 3] += p0 + p1;
                 sr[c] = pack_bf16x2(p0, p1);
             }

@@ -1,5 +1,7 @@
-"""Regression check of the oracle against its stored outputs on the tiny decode batch
-(see tests/golden/README.md: a fixture written by a script that calls only the oracle)."""
+"""Regression check of the oracle against its stored outputs on the tiny decode batch.
+
+The fixture was written by tests/golden/make_golden.py, which calls only the oracle: it
+detects later changes to the oracle's results, it does not pin the oracle."""
 import json
 import os
 import sys
