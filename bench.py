@@ -55,7 +55,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, index: int, period_s: float = 0.02):
+    def __init__(self, index: int, period_s: float = 0.0005):
         self.samples, self.reasons = [], set()
         self.max_mhz = None
         self._stop = threading.Event()
@@ -73,7 +73,8 @@ class ClockSampler:
 
     def _run(self):
         nv = self._nv
-        while not self._stop.is_set():
+        stop = self._stop
+        while not stop.is_set():
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
                 r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
@@ -85,7 +86,9 @@ class ClockSampler:
             time.sleep(self.period)
 
     def __enter__(self):
+        """Start sampling (again): samples of every entered region accumulate."""
         if self._ok:
+            self._stop = threading.Event()
             self._t = threading.Thread(target=self._run, daemon=True)
             self._t.start()
         return self
@@ -167,12 +170,28 @@ class OracleRunner:
                 f"all {len(self.data)} sequences")
 
 
+def workload_name(args):
+    """The workload as both arms name it (the GPU arm's batch options included)."""
+    return f"{args.config}" + (f" (first {args.seqs} sequences)" if args.seqs else "") + \
+        (f" (seed {args.seed})" if args.seed is not None else "") + \
+        (" over FP8 E4M3 caches" if args.kv_fp8 else "")
+
+
+def parallelism_text(args, ws, num_kv_heads):
+    if ws <= 1:
+        return "single GPU"
+    if args.shard == "heads":
+        from paged_kv_attention_verify_b200 import shard as S
+        return "kv-head/sequence shards tp%d x sp%d" % S.shard_layout(ws, num_kv_heads)
+    return f"replicas x{ws}"
+
+
 def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
         return 0
     import workloads as W
-    batch = W.make_config(args.config, device="cpu")
+    batch = W.make_config(args.config, device="cpu", seed=args.seed)
     runner = OracleRunner(batch)
     step_s = args.ref_seconds / (args.warmup + args.steps)
     for _ in range(args.warmup):
@@ -186,10 +205,13 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": f"{args.config}: {WORKLOADS[args.config]}"},
+            "data": "synthetic",
+            "config": workload_config(args.config, batch, workload_name(args),
+                                      parallelism_text(args, ws, batch.num_kv_heads)),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": runner.threads, "kind": "oracle",
                              "sample": "each step: " + runner.sample_text()},
-            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "source": source_identity()}
     print(json.dumps(line))
     return 0
 
@@ -290,6 +312,57 @@ def roofline(info, seconds, peaks, sustained=False):
             "frac": ach / tf_peak, "frac_of_spec_2250": ach / 2250.0}
 
 
+def source_identity():
+    """The git commit of the checkout (None where the tree carries no .git, as on a copied
+    tree) and a SHA-256 over the library's kernel and planner sources."""
+    import glob
+    import hashlib
+    import subprocess
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "paged_kv_attention_verify_b200", "csrc", "*"))):
+        if f.endswith((".cu", ".cuh", ".h", ".cpp")):
+            h.update(open(f, "rb").read())
+    try:
+        sha = subprocess.run(["git", "-C", ROOT, "rev-parse", "HEAD"], capture_output=True, text=True,
+                             timeout=10).stdout.strip() or None
+    except Exception:
+        sha = None
+    return {"git_sha": sha, "source_sha256": h.hexdigest()}
+
+
+def workload_config(name, batch, workload_text, parallelism):
+    """The ``config`` object of a bench line; both arms print the same one."""
+    return {"workload": f"{workload_text}: {WORKLOADS[name]}",
+            "query_tokens_per_step": batch.total_q,
+            "kv_bytes_per_step": batch_kv_bytes(batch),
+            "attn_flops_per_step": batch_attn_flops(batch),
+            "l2": "inputs larger than L2 (KV cache read each step exceeds 126 MB)",
+            "parallelism": parallelism}
+
+
+def batch_kv_bytes(batch):
+    """Algorithmic K+V bytes of one pass: every cached element of every sequence once."""
+    return sum(sp.seq_len for sp in batch.seqs) * batch.num_kv_heads * batch.head_dim * 2 * 2
+
+
+def batch_attn_flops(batch):
+    """Algorithmic attention flops: 4 * D * Hq per allowed (query, key) pair."""
+    pairs = 0
+    for sp in batch.seqs:
+        T, L = sp.query_len, sp.seq_len
+        pairs += T * (L - T)
+        if sp.mask_kind == 0:
+            pairs += T * (T + 1) // 2
+        else:
+            for i in range(T):                      # a node sees itself and its ancestors
+                a, n = i, 0
+                while a >= 0:
+                    n += 1
+                    a = sp.parents[a]
+                pairs += n
+    return pairs * batch.num_q_heads * 4 * batch.head_dim
+
+
 def kernel_traffic(workload):
     """DRAM bytes per launch of the attention kernel from the committed ncu summary, if it
     was taken on this workload and on the current kernel sources (else None)."""
@@ -324,15 +397,14 @@ def run_ours(args):
     peaks = load_peaks()
     stream = torch.cuda.current_stream()
 
-    batch = W.make_config(args.config, device=dev, max_seqs=args.seqs)
+    batch = W.make_config(args.config, device=dev, max_seqs=args.seqs, seed=args.seed)
     job_tokens = None
-    parallelism = f"replicas x{ws}" if ws > 1 else "single GPU"
+    parallelism = parallelism_text(args, ws, batch.num_kv_heads)
+    config = workload_config(args.config, batch, workload_name(args), parallelism)
     if args.shard == "heads" and ws > 1:
         # strong scaling: the one batch split over the ranks (KV-head groups x sequence
         # subsets, no exchange inside attention); every rank builds it from the same seed
-        from paged_kv_attention_verify_b200 import shard as S
         job_tokens = batch.total_q
-        parallelism = "kv-head/sequence shards tp%d x sp%d" % S.shard_layout(ws, batch.num_kv_heads)
         batch = W.shard_batch(batch, rank, ws)
         torch.cuda.empty_cache()
     out = torch.empty_like(batch.q)
@@ -367,12 +439,13 @@ def run_ours(args):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if ws > 1:
             dist.barrier()
-        e0.record(stream)
-        for _ in range(args.steps):
-            plan.run_host_async(q_host, batch.k_cache, batch.v_cache, o_host, stream)
-        plan.host_wait(stream)
-        e1.record(stream)
-        torch.cuda.synchronize()
+        with clk:                                  # clocks of this timed region join the line's
+            e0.record(stream)
+            for _ in range(args.steps):
+                plan.run_host_async(q_host, batch.k_cache, batch.v_cache, o_host, stream)
+            plan.host_wait(stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
 
     tokens = batch.total_q
@@ -386,8 +459,7 @@ def run_ours(args):
     kv_gbs = info["kv_bytes"] / avg_launch_s / 1e9
     tflops = info["attn_flops"] / avg_launch_s / 1e12
     io_bytes = tokens * batch.num_q_heads * batch.head_dim * 2
-    workload = f"{args.config}" + (f" (first {args.seqs} sequences)" if args.seqs else "") + \
-        (" over FP8 E4M3 caches" if args.kv_fp8 else "")
+    workload = workload_name(args)
     rl = roofline(info, avg_launch_s, peaks)
     rl.update({"traffic": kernel_traffic(workload), "kernel": "attn_kernel",
                "peak_source": peaks["source"],
@@ -512,7 +584,7 @@ def run_ours(args):
         # shared-prefix batch: cascade plan (attn_plan_shared) against the same batch planned
         # without groups; algorithmic bytes count the shared keys once in both
         for name in W.SHARED_CONFIG_NAMES:
-            b = W.make_shared_config(name, device=dev, keep_contiguous=False)
+            b = W.make_shared_config(name, device=dev)
             o = torch.empty_like(b.q)
             res = {}
             for tag, shared in (("cascade", True), ("no_cascade", False)):
@@ -529,14 +601,32 @@ def run_ours(args):
                 pl.close()
             res["kv_bytes_unique"] = kv_unique
             res["speedup"] = res["no_cascade"]["ms_per_launch"] / res["cascade"]["ms_per_launch"]
+            # the same groups over FP8 caches (attn_plan_shared_kv + attn_run_fp8: the cascade
+            # tasks read bf16 copies of the shared pages staged in the same step)
+            f = W.fp8_kv(b)
+            pl = pk.plan_for_batch(b, kv_fp8=True)
+            inf = pl.info()
+
+            def step8(pl=pl, b=b, f=f, o=o):
+                pl.run_fp8(b.q, f.k_cache, f.v_cache_t, f.k_scale, f.v_scale, o, stream)
+
+            ps = time_fn(step8, args.other_steps, args.warmup, stream)
+            if pl.check(stream) != 0:
+                raise RuntimeError("device error in the FP8 shared-prefix measurement")
+            sec = sum(ps) / len(ps) * 1e-3
+            res["cascade_fp8"] = {"ms_per_launch": sec * 1e3, "ms_median": _median(ps),
+                                  "tokens_per_s": b.total_q / sec, "kv_bytes_fp8": inf["kv_bytes"],
+                                  "roofline": roofline(inf, sec, peaks),
+                                  "speedup_vs_bf16_cascade": res["cascade"]["ms_per_launch"] / (sec * 1e3)}
+            pl.close()
             per_config[name] = res
-            del b, o
+            del b, o, f
             torch.cuda.empty_cache()
 
     if rank == 0:
         cpu = None
         if ws == 1 and not args.no_cpu_baseline:
-            b = W.make_config(args.config, device=dev, max_seqs=args.seqs)
+            b = W.make_config(args.config, device=dev, max_seqs=args.seqs, seed=args.seed)
             runner = OracleRunner(b)
             tk, sec = runner.run(args.cpu_seconds)
             cpu = {"value": tk / sec, "unit": "tokens/s", "cores": runner.threads, "kind": "oracle",
@@ -548,11 +638,7 @@ def run_ours(args):
             "scaling": "strong" if job_tokens is not None else "weak", "vs_baseline": None,
             "dtype": "bf16 q/out, fp8-e4m3 KV" if args.kv_fp8 else "bf16",
             "data": "synthetic",
-            "config": {"workload": f"{workload}: {WORKLOADS[args.config]}",
-                       "query_tokens_per_step": tokens, "kv_bytes_per_step": info["kv_bytes"],
-                       "attn_flops_per_step": info["attn_flops"],
-                       "l2": "inputs larger than L2 (KV cache read each step exceeds 126 MB)",
-                       "parallelism": parallelism},
+            "config": config,
             "kv_gbs": kv_gbs, "kv_frac_of_hbm": kv_gbs / peaks["hbm_gbs"], "prefill_tflops": tflops,
             "roofline": rl,
             "cpu_baseline": cpu,
@@ -562,7 +648,8 @@ def run_ours(args):
             "gpu_launches": args.steps * (2 if args.kv_fp8 and info["num_prefill_items"] > 0 else 1),
             "clocks": clk.summary(),
             "plan": {k: info[k] for k in ("num_decode_items", "num_prefill_items", "num_split_units",
-                                          "decode_rows")},
+                                          "decode_rows", "kv_bytes", "attn_flops")},
+            "source": source_identity(),
             "per_config": per_config,
             "append": append, "per_class": per_class,
         }
@@ -596,6 +683,8 @@ def main():
                     help="host time for the oracle baseline line of our arm")
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="total host time the reference arm spreads over warm-up + steps")
+    ap.add_argument("--seed", type=int, default=None,
+                    help="seed of the workload draw (default: the config's index, as the tests use)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -171,6 +171,29 @@ PKVA_API int attn_plan_kv(pkva_plan_t* out_plan, int num_seqs, const int32_t* se
               int kv_dtype);
 
 /*
+ * attn_plan_shared_kv — attn_plan_shared with the caches' element format (kv_dtype as in
+ * attn_plan_kv): shared-prefix groups over FP8 E4M3 caches (run with attn_run_fp8 /
+ * attn_run_fp8_append), or over bf16 caches (the same as attn_plan_shared).
+ *
+ * Cites: XY-Serve verdict page, pith_inferences[0] (attention reusing a cached prefix) and
+ * the Arctic Inference review page, section 3 comments (quantised KV formats): the two
+ * together, a shared prefix held once in an FP8 cache.
+ *
+ * Over FP8 caches the cascade tasks (tensor cores) read bf16 copies of the group's shared
+ * pages, staged once per run by the staging launch together with the pages of the prefill
+ * sequences, through the block-table row of the run's first member; the K scale of the KV
+ * head joins the softmax scale and the V scale the partial outputs, and the members'
+ * decode/verify tasks read their own keys' E4M3 pages. The plan owns the staging memory
+ * (2 x 2 bytes x Hkv x page_size x D per staged page; counted in scratch_bytes). Arguments
+ * and errors as attn_plan_shared, plus PKVA_EINVAL for an unknown kv_dtype.
+ */
+PKVA_API int attn_plan_shared_kv(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq_lens,
+              const int32_t* query_lens, const int32_t* block_table, int bt_stride,
+              int num_pages, const int32_t* mask_kind, const int32_t* parents,
+              int num_q_heads, int num_kv_heads, int head_dim, int page_size, float sm_scale,
+              const int32_t* prefix_group, const int32_t* prefix_len, int num_groups, int kv_dtype);
+
+/*
  * attn_run_fp8 — attn_run over FP8 E4M3 caches (a plan made with PKVA_KV_FP8_E4M3).
  *
  *   q          device bf16 [sum T_s, Hq, D] (as attn_run; |q| must stay in f16's range:
@@ -324,9 +347,13 @@ PKVA_API const char* attn_last_error(void);
  * device address; make that first call before any stream capture. Every call shares the
  * one array, which keeps the last call's contents (the call clears the parts that must
  * start at zero), so calls that overlap on the GPU (on different streams, or from
- * different threads) race: serialize them. Device-side error bits (a block-table entry
- * out of range) are not reported by this call. The task tables are copied from host
- * memory with cudaMemcpyAsync, which may wait for `stream` before returning.
+ * different threads) race: serialize them. Device-side errors are not reported by this
+ * call: neither a block-table entry out of range (its page reads as zeros) nor a bounded
+ * device wait that gave up (the output is then incomplete) comes back to the caller; use
+ * attn_plan / attn_run / attn_check where those must be seen. q, k_cache, v_cache, out and
+ * block_table must be device memory of the current device (PKVA_EINVAL otherwise). The
+ * task tables are copied from host memory with cudaMemcpyAsync, which may wait for
+ * `stream` before returning.
  */
 PKVA_API int attn_run_static(int num_seqs, const int32_t* seq_lens, const int32_t* query_lens,
                              const int32_t* block_table, int bt_stride, int num_pages,

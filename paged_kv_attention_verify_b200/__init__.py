@@ -33,7 +33,7 @@ DEVERR_BAD_PAGE = 0x1
 DEVERR_TIMEOUT = 0x2
 
 # every entry point that include/pkva.h declares
-EXPORTED = ["attn_plan", "attn_plan_shared", "attn_plan_kv", "attn_run", "attn_run_fp8", "attn_run_fp8_append",
+EXPORTED = ["attn_plan", "attn_plan_shared", "attn_plan_kv", "attn_plan_shared_kv", "attn_run", "attn_run_fp8", "attn_run_fp8_append",
             "attn_run_host_async", "attn_host_wait", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_destroy",
             "attn_last_error", "attn_plan_get_info", "attn_plan_inspect", "attn_run_static",
             "pkva_selftest_wait_timeout"]
@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
                             ctypes.c_int, ctypes.c_float]
     L.attn_plan_shared.argtypes = L.attn_plan.argtypes + [_i32p, _i32p, ctypes.c_int]
     L.attn_plan_kv.argtypes = L.attn_plan.argtypes + [ctypes.c_int]
+    L.attn_plan_shared_kv.argtypes = L.attn_plan_shared.argtypes + [ctypes.c_int]
     L.attn_run_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
     L.attn_run_fp8_append.argtypes = [_vp] * 10
     L.attn_run.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp]
@@ -101,7 +102,7 @@ def lib() -> ctypes.CDLL:
                                   _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                   ctypes.c_float, _vp, _vp, _vp, _vp, _vp]
     L.pkva_selftest_wait_timeout.argtypes = [ctypes.c_longlong, _i32p]
-    for name in ("attn_plan", "attn_plan_shared", "attn_plan_kv", "attn_run_fp8", "attn_run_fp8_append",
+    for name in ("attn_plan", "attn_plan_shared", "attn_plan_kv", "attn_plan_shared_kv", "attn_run_fp8", "attn_run_fp8_append",
                  "attn_run_host_async", "attn_host_wait", "attn_run", "attn_run_append", "attn_run_host", "attn_check", "attn_plan_get_info",
                  "attn_plan_inspect", "attn_run_static", "pkva_selftest_wait_timeout"):
         getattr(L, name).restype = ctypes.c_int
@@ -129,6 +130,40 @@ def _stream_handle(stream) -> Optional[int]:
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
+def _host_arrays(seq_lens, query_lens, mask_kind, parents):
+    """The per-sequence host arrays as int32 buffers, one entry per sequence each."""
+    sl, ql, mk = _i32(seq_lens), _i32(query_lens), _i32(mask_kind)
+    par = _i32(parents if parents is not None else [])
+    if len(sl) != len(ql) or len(sl) != len(mk):
+        raise ValueError("seq_lens, query_lens and mask_kind must have one entry per sequence")
+    return sl, ql, mk, par
+
+
+def _block_table_arg(block_table, num_seqs: int):
+    """(device pointer, bt_stride) of a contiguous int32 CUDA block table [num_seqs, stride]."""
+    import torch
+    if not num_seqs:
+        return None, 0
+    if not (isinstance(block_table, torch.Tensor) and block_table.is_cuda
+            and block_table.dtype == torch.int32 and block_table.dim() == 2
+            and block_table.is_contiguous() and block_table.shape[0] == num_seqs):
+        raise ValueError("block_table must be a contiguous int32 CUDA tensor [num_seqs, bt_stride]")
+    return block_table.data_ptr(), block_table.shape[1]
+
+
+def _check_bf16_tensors(q, k_cache, v_cache, out, total_q, Hq, Hkv, D, num_pages, page_size):
+    """q / out bf16 [total_q, Hq, D] and the caches bf16 [num_pages, Hkv, page_size, D], all
+    contiguous CUDA tensors."""
+    import torch
+    for name, t, shape in (("q", q, (total_q, Hq, D)), ("out", out, (total_q, Hq, D)),
+                           ("k_cache", k_cache, (num_pages, Hkv, page_size, D)),
+                           ("v_cache", v_cache, (num_pages, Hkv, page_size, D))):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be a bf16 CUDA tensor")
+        if tuple(t.shape) != shape or not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous with shape {shape}, got {tuple(t.shape)}")
+
+
 class Plan:
     """A planned batch (``attn_plan``); run it any number of times with ``run``."""
 
@@ -139,21 +174,11 @@ class Plan:
                  prefix_group: Optional[Sequence[int]] = None,
                  prefix_len: Optional[Sequence[int]] = None, kv_fp8: bool = False):
         """``attn_plan``; with ``prefix_group`` / ``prefix_len`` (shared-prefix groups),
-        ``attn_plan_shared``; with ``kv_fp8``, ``attn_plan_kv`` for FP8 E4M3 caches."""
-        import torch
+        ``attn_plan_shared``; with ``kv_fp8``, ``attn_plan_kv`` (or ``attn_plan_shared_kv``
+        with groups) for FP8 E4M3 caches."""
         self._handle = None
-        sl, ql, mk = _i32(seq_lens), _i32(query_lens), _i32(mask_kind)
-        par = _i32(parents if parents is not None else [])
-        if len(sl) != len(ql) or len(sl) != len(mk):
-            raise ValueError("seq_lens, query_lens and mask_kind must have one entry per sequence")
-        if len(sl):
-            if not (isinstance(block_table, torch.Tensor) and block_table.is_cuda
-                    and block_table.dtype == torch.int32 and block_table.dim() == 2
-                    and block_table.is_contiguous() and block_table.shape[0] == len(sl)):
-                raise ValueError("block_table must be a contiguous int32 CUDA tensor [num_seqs, bt_stride]")
-            bt_ptr, bt_stride = block_table.data_ptr(), block_table.shape[1]
-        else:
-            bt_ptr, bt_stride = None, 0
+        sl, ql, mk, par = _host_arrays(seq_lens, query_lens, mask_kind, parents)
+        bt_ptr, bt_stride = _block_table_arg(block_table, len(sl))
         self.block_table = block_table          # keep the caller's table alive with the plan
         self.num_q_heads, self.num_kv_heads, self.head_dim = num_q_heads, num_kv_heads, head_dim
         self.num_pages, self.page_size = num_pages, page_size
@@ -163,28 +188,22 @@ class Plan:
                 _ptr(par), num_q_heads, num_kv_heads, head_dim, page_size,
                 float(sm_scale) if sm_scale else 0.0)
         self.kv_fp8 = kv_fp8
-        if kv_fp8:
-            if prefix_group is not None:
-                raise ValueError("shared-prefix groups are not supported with FP8 caches")
-            _check(lib().attn_plan_kv(*args, KV_FP8_E4M3))
-        elif prefix_group is None:
-            _check(lib().attn_plan(*args))
+        if prefix_group is None:
+            _check(lib().attn_plan_kv(*args, KV_FP8_E4M3) if kv_fp8 else lib().attn_plan(*args))
         else:
             pg, pl = _i32(prefix_group), _i32(prefix_len if prefix_len is not None else [])
-            _check(lib().attn_plan_shared(*args, _ptr(pg), _ptr(pl), len(pl)))
+            if len(pg) != len(sl):
+                raise ValueError("prefix_group must have one entry per sequence")
+            if kv_fp8:
+                _check(lib().attn_plan_shared_kv(*args, _ptr(pg), _ptr(pl), len(pl), KV_FP8_E4M3))
+            else:
+                _check(lib().attn_plan_shared(*args, _ptr(pg), _ptr(pl), len(pl)))
         self._handle = h
 
     # -- marshalling checks (shapes, dtypes, devices) ---------------------------------
     def _check_tensors(self, q, k_cache, v_cache, out):
-        import torch
-        D, Hq, Hkv = self.head_dim, self.num_q_heads, self.num_kv_heads
-        for name, t, shape in (("q", q, (self.total_q, Hq, D)), ("out", out, (self.total_q, Hq, D)),
-                               ("k_cache", k_cache, (self.num_pages, Hkv, self.page_size, D)),
-                               ("v_cache", v_cache, (self.num_pages, Hkv, self.page_size, D))):
-            if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.bfloat16:
-                raise ValueError(f"{name} must be a bf16 CUDA tensor")
-            if tuple(t.shape) != shape or not t.is_contiguous():
-                raise ValueError(f"{name} must be contiguous with shape {shape}, got {tuple(t.shape)}")
+        _check_bf16_tensors(q, k_cache, v_cache, out, self.total_q, self.num_q_heads, self.num_kv_heads,
+                            self.head_dim, self.num_pages, self.page_size)
 
     def run(self, q, k_cache, v_cache, out=None, stream=None):
         """out = attention(q, paged K/V); asynchronous on ``stream`` (default: current)."""
@@ -333,11 +352,22 @@ def run_static(seq_lens, query_lens, block_table, mask_kind, parents, q, k_cache
     For callers that cannot allocate where they need attention; ``out`` must be
     allocated by the caller beforehand. The library keeps the call's tables and split
     scratch in a fixed array it reserves per GPU, so overlapping calls race (serialize
-    them), and batches beyond that array's limits raise PKVA_EUNSUPPORTED."""
-    sl, ql, mk = _i32(seq_lens), _i32(query_lens), _i32(mask_kind)
-    par = _i32(parents if parents is not None else [])
-    bt_stride = block_table.shape[1] if len(sl) else 0
-    _check(lib().attn_run_static(len(sl), _ptr(sl), _ptr(ql), block_table.data_ptr() if len(sl) else None,
+    them), and batches beyond that array's limits raise PKVA_EUNSUPPORTED.
+
+    Every tensor must be on the current CUDA device: the call reaches the scratch of that
+    device and launches there."""
+    import torch
+    sl, ql, mk, par = _host_arrays(seq_lens, query_lens, mask_kind, parents)
+    bt_ptr, bt_stride = _block_table_arg(block_table, len(sl))
+    total_q = int(ql.sum()) if len(ql) else 0
+    _check_bf16_tensors(q, k_cache, v_cache, out, total_q, num_q_heads, num_kv_heads, head_dim, num_pages,
+                        page_size)
+    dev = torch.cuda.current_device()
+    for name, t in (("block_table", block_table), ("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
+                    ("out", out)):
+        if (name != "block_table" or len(sl)) and t.device.index != dev:
+            raise ValueError(f"{name} is on {t.device}, not on the current device cuda:{dev}")
+    _check(lib().attn_run_static(len(sl), _ptr(sl), _ptr(ql), bt_ptr,
                                  bt_stride, num_pages, _ptr(mk), _ptr(par), num_q_heads, num_kv_heads,
                                  head_dim, page_size, float(sm_scale) if sm_scale else 0.0,
                                  q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), out.data_ptr(),
@@ -356,7 +386,7 @@ def plan_for_batch(batch, sm_scale: Optional[float] = None, shared: bool = True,
     """Plan a ``workloads.Batch`` (a convenience for tests and the benchmark); a batch with
     shared-prefix groups is planned with them unless ``shared`` is False; ``kv_fp8`` plans
     for FP8 caches."""
-    groups = getattr(batch, "prefix_group", None) if shared and not kv_fp8 else None
+    groups = getattr(batch, "prefix_group", None) if shared else None
     return Plan(batch.seq_lens, batch.query_lens, batch.block_table, batch.mask_kinds,
                 batch.parents_flat, num_q_heads=batch.num_q_heads, num_kv_heads=batch.num_kv_heads,
                 head_dim=batch.head_dim, num_pages=batch.k_cache.shape[0],

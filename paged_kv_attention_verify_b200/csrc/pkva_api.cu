@@ -13,6 +13,8 @@
 #include <new>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "pkva.h"
 #include "pkva_internal.h"
 #include "pkva_kernels.h"
@@ -20,6 +22,15 @@
 namespace pkva {
 
 static thread_local std::string g_last_error;
+
+// A named NVTX range over one host call (planning, a run), visible on a profiler timeline;
+// without a profiler attached the push and pop do nothing.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 void set_last_error(const std::string& msg) { g_last_error = msg; }
 
@@ -218,6 +229,7 @@ extern "C" const char* attn_last_error(void) { return g_last_error.c_str(); }
 
 static int plan_create(pkva_plan_t* out_plan, PlanArgs a, const int32_t* block_table, const char* who,
                        bool kv_fp8 = false) {
+    NvtxRange range(who);
     const std::string name(who);
     if (!out_plan) {
         set_last_error(name + ": out_plan is NULL");
@@ -225,6 +237,8 @@ static int plan_create(pkva_plan_t* out_plan, PlanArgs a, const int32_t* block_t
     }
     *out_plan = nullptr;
     const int num_seqs = a.num_seqs, head_dim = a.D;
+    // row-split tasks run in the unified kernel only (not on the CUDA-core comparison body)
+    a.wide_tasks = decode_body_is_mma();
     if (num_seqs > 0 && !block_table) {
         set_last_error(name + ": block_table is NULL");
         return PKVA_EINVAL;
@@ -393,6 +407,27 @@ extern "C" int attn_plan_shared(pkva_plan_t* out_plan, int num_seqs, const int32
     return plan_create(out_plan, a, block_table, "attn_plan_shared");
 }
 
+extern "C" int attn_plan_shared_kv(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq_lens,
+                                   const int32_t* query_lens, const int32_t* block_table, int bt_stride,
+                                   int num_pages, const int32_t* mask_kind, const int32_t* parents,
+                                   int num_q_heads, int num_kv_heads, int head_dim, int page_size, float sm_scale,
+                                   const int32_t* prefix_group, const int32_t* prefix_len, int num_groups,
+                                   int kv_dtype) {
+    if (kv_dtype != PKVA_KV_BF16 && kv_dtype != PKVA_KV_FP8_E4M3) {
+        set_last_error("attn_plan_shared_kv: kv_dtype must be PKVA_KV_BF16 or PKVA_KV_FP8_E4M3");
+        if (out_plan) *out_plan = nullptr;
+        return PKVA_EINVAL;
+    }
+    PlanArgs a{num_seqs, seq_lens, query_lens, bt_stride, num_pages, mask_kind, parents, num_q_heads,
+               num_kv_heads, head_dim, page_size, sm_scale, 1, 1};
+    a.prefix_group = prefix_group;
+    a.prefix_len = prefix_len;
+    a.num_groups = num_groups;
+    const bool fp8 = kv_dtype == PKVA_KV_FP8_E4M3;
+    a.kv_elem_bytes = fp8 ? 1 : 2;
+    return plan_create(out_plan, a, block_table, "attn_plan_shared_kv", fp8);
+}
+
 extern "C" void attn_plan_destroy(pkva_plan_t plan) {
     if (!plan) return;
     const int dev = plan->device;
@@ -429,6 +464,7 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 static int run_impl(pkva_plan_t plan, const void* q, const void* k_new, const void* v_new, const void* k_cache,
                     const void* v_cache, void* out, void* stream, const char* who, const float* k_scale = nullptr,
                     const float* v_scale = nullptr, bool fp8 = false) {
+    NvtxRange range(who);
     const std::string name(who);
     if (!plan) {
         set_last_error(name + ": plan is NULL");
@@ -691,6 +727,7 @@ static int host_staging(pkva_plan_t plan, size_t bytes, bool async, const char* 
 
 static int run_host_impl(pkva_plan_t plan, const void* q_host, const void* k_cache, const void* v_cache,
                          void* out_host, void* stream, bool async, const char* who) {
+    NvtxRange range(who);
     const std::string name(who);
     if (!plan) {
         set_last_error(name + ": plan is NULL");

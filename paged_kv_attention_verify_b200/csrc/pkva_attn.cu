@@ -3,12 +3,14 @@
 // The planner's task list is one grid: shared-prefix (cascade) tasks first, then prefill
 // tasks and decode/verify tasks, each heaviest first, merged in proportion. A block whose
 // entry is a tensor-core task runs it with all its warps (TMEM, tcgen05.mma, four warp
-// roles); any other block runs three decode/verify tasks side by side, each on four
-// page-streaming warps with its own third of shared memory and its own named barrier
-// (warp-level tensor-core page body). Both kinds use the same 384-thread block and the
-// same dynamic shared memory (one block per SM), so the hardware block scheduler deals the
-// mixed work out as one longest-task-first schedule and decode blocks fill the SMs as
-// prefill blocks finish.
+// roles); any other block runs three decode/verify tasks side by side, each on four warps
+// with its own third of shared memory and its own named barrier (warp-level tensor-core
+// page body): a task of at most 16 packed rows streams every fourth page on each warp; a
+// wider one (a draft tree times the GQA group) is row-split, three warps owning 16 rows
+// each and the fourth streaming every page once. Both kinds use the same 384-thread block
+// and the same dynamic shared memory (one block per SM), so the hardware block scheduler
+// deals the mixed work out as one longest-task-first schedule and decode blocks fill the
+// SMs as prefill blocks finish.
 //
 // (A persistent variant, blocks pulling tasks from two global queues with each decode
 // group taking its next task on its own, measured 3-13 % slower on B200 and was dropped:
@@ -51,6 +53,9 @@ struct AttnSmem {
     static constexpr int BYTES = TASK_BYTES + 64;
     static constexpr int ALLOC = BYTES + 1008;    // room to align to 1024
     static_assert(ALLOC <= 227 * 1024, "shared memory");
+    // a row-split (wide) task takes one decode task's share: as many ring stages as fit
+    static constexpr int WIDE_NS = dec::wide_stages(D, GROUP_BYTES);
+    static_assert(dec::wide_bytes(D, WIDE_NS) <= GROUP_BYTES, "wide task");
 };
 
 // FP8: decode/verify tasks read the E4M3 pages; tensor-core tasks read their bf16 staging copies.
@@ -91,6 +96,13 @@ attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const _
     const int task = (-1 - e) * kDecTasksPerBlock + g;
     if (task >= p.num_decode) return;
     const dec::Group grp{(int)threadIdx.x & 127, 128, 1 + g};
+    if constexpr (!FP8) {
+        // more than 16 packed rows (a draft tree times the GQA group): one pass over the pages
+        if (p.dec.work[task].row_count > kDecodeRowsMax) {
+            dec::decode_wide_task<D, S::WIDE_NS>(grp, p.dec, task, tmK, tmV, sm + g * S::GROUP_BYTES);
+            return;
+        }
+    }
     dec::decode_mma_task<D, NT, kDecWarps, AttnNS<D, FP8>::value, FP8>(grp, p.dec, task, tmK, tmV,
                                                                     sm + g * S::GROUP_BYTES);
 }

@@ -158,6 +158,163 @@ __device__ __forceinline__ void issue_page(const DecodeParams& p, const DecodeWo
 // transposed V operand delivers (four consecutive keys per lane, see decode_mma_task).
 __device__ __forceinline__ int fp8_key_of_row(int m) { return ((m & 7) >> 1) * 4 + (m >> 3) * 2 + (m & 1); }
 
+// One bf16 page (16 keys) for the rows one warp holds (NT n-tiles of 8 rows): S^T = K Q^T,
+// the row masks, the lazily rescaled online softmax and O^T += V^T P^T. Ks / Vs: the page's
+// K and V (16 x 64 boxes, 128-byte swizzle); Q from qs (rows staged in shared memory, 16-byte
+// chunk c of row r at c ^ (r & 7)) when QB, else from the fragments in qf. Slots past the
+// sequence's end hold stale cache data: their V rows are zeroed in shared memory first
+// (every warp that reads the page writes the same zeros, so several may share it).
+template <int D, int NT, bool QB>
+__device__ __forceinline__ void bf16_page(const uint8_t* Ks, uint8_t* Vs, const uint8_t* qs,
+                                          const uint32_t (&qf)[NT][QB ? 1 : D / 16][2], int kbase, int prefix,
+                                          int seq_len, int min_lim, const int (&lim)[NT][2],
+                                          const uint64_t (&anc)[NT][2], float sl2, float (&o)[D / 16][NT][4],
+                                          float (&mref)[NT][2], float (&lsum)[NT][2]) {
+    constexpr int KS = D / 16;
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int mi = lane >> 3, mr = lane & 7;
+    const int k_key = mr + (mi & 1) * 8, k_chunk = mi >> 1;          // K: A operand, keys on M
+    const int v_key = mr + (mi >> 1) * 8, v_chunk = mi & 1;          // V: A operand of V^T (trans)
+    // -- S^T = K Q^T (16 keys x 8 rows per n-tile) ------------------------------------
+    // even and odd k-steps accumulate into separate tiles (two dependent MMA chains of half
+    // the length), added at the end
+    float s[NT][4], s2[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[nt][e] = s2[nt][e] = 0.f;
+    if constexpr (QB) {
+#pragma unroll
+        for (int k2 = 0; k2 < KS; k2 += 2) {
+            uint32_t qb[NT][4];              // b fragments of k-steps k2 and k2 + 1
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int qr = nt * 8 + (lane & 7), qc = 2 * k2 + (lane >> 3);
+                ldmatrix_x4(qb[nt], qs + qr * (D * 2) + ((qc ^ (qr & 7)) << 4));
+            }
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+                const int cg = (k2 + kk) * 2 + k_chunk;
+                uint32_t a[4];
+                ldmatrix_x4(a, Ks + (cg >> 3) * kBoxBytes + k_key * 128 + (((cg & 7) ^ (k_key & 7)) << 4));
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(kk ? s2[nt] : s[nt], a, &qb[nt][2 * kk]);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            const int cg = ks * 2 + k_chunk;
+            uint32_t a[4];
+            ldmatrix_x4(a, Ks + (cg >> 3) * kBoxBytes + k_key * 128 + (((cg & 7) ^ (k_key & 7)) << 4));
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816((ks & 1) ? s2[nt] : s[nt], a, qf[nt][ks]);
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[nt][e] += s2[nt][e];
+
+    // -- mask ---------------------------------------------------------------------------
+    const bool page_all = (kbase + kPageSize - 1) <= min_lim;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int kpos = kbase + g + 8 * h;
+                float v = s[nt][2 * h + e] * sl2;
+                if (!page_all) {
+                    bool allow = kpos <= lim[nt][e];
+                    if (!allow && kpos >= prefix && kpos < seq_len)
+                        allow = (anc[nt][e] >> (kpos - prefix)) & 1ull;
+                    v = allow ? v : -INFINITY;
+                }
+                s[nt][2 * h + e] = v;
+            }
+    // -- lazy rescale: only when some score passed its row's reference by the slack (or the
+    //    row has no reference yet). Each lane checks its own scores; the row max over the
+    //    page (shuffles across the lanes of a column) is taken only in that rare case.
+    bool need = false;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const float mx = fmaxf(s[nt][e], s[nt][2 + e]);
+            need |= mx > mref[nt][e] + kRescaleSlack || (mref[nt][e] == -INFINITY && mx != -INFINITY);
+        }
+    if (__any_sync(0xffffffffu, need)) {
+        float cmax[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float mx = fmaxf(s[nt][e], s[nt][2 + e]);
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                cmax[nt][e] = mx;
+            }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float mnew = fmaxf(mref[nt][e], cmax[nt][e]);
+                if (mnew != mref[nt][e]) {
+                    const float alpha = mref[nt][e] == -INFINITY ? 0.f : exp2f(mref[nt][e] - mnew);
+                    mref[nt][e] = mnew;
+                    lsum[nt][e] *= alpha;
+#pragma unroll
+                    for (int dt = 0; dt < KS; ++dt) {
+                        o[dt][nt][e] *= alpha;
+                        o[dt][nt][2 + e] *= alpha;
+                    }
+                }
+            }
+    }
+    // -- P = exp2(S - ref), row sums, P^T as the B operand (transpose in registers) -----
+    uint32_t pb[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        float pv[4];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const float ref = mref[nt][e] == -INFINITY ? 0.f : mref[nt][e];
+            pv[e] = exp2f(s[nt][e] - ref);
+            pv[2 + e] = exp2f(s[nt][2 + e] - ref);
+            lsum[nt][e] += pv[e] + pv[2 + e];
+        }
+        pb[nt][0] = movmatrix_trans(pack_bf16x2(pv[0], pv[1]));   // keys 0..7
+        pb[nt][1] = movmatrix_trans(pack_bf16x2(pv[2], pv[3]));   // keys 8..15
+    }
+    // slots past the sequence's end hold stale cache data: zero those V rows so that
+    // P = 0 times a non-finite value cannot reach the accumulators
+    const int nvalid = seq_len - kbase;
+    if (nvalid < kPageSize) {
+        for (int idx = lane; idx < (kPageSize - nvalid) * (D / 8); idx += 32) {
+            const int row = nvalid + idx / (D / 8);
+            const int cg = idx % (D / 8);
+            *reinterpret_cast<uint4*>(Vs + (cg >> 3) * kBoxBytes + row * 128 + (cg & 7) * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
+        __syncwarp();
+    }
+    // -- O^T += V^T P^T -----------------------------------------------------------------
+    {
+#pragma unroll
+        for (int dt = 0; dt < KS; ++dt) {
+            const int cg = dt * 2 + v_chunk;
+            uint32_t a[4];
+            ldmatrix_x4_trans(a, Vs + (cg >> 3) * kBoxBytes + v_key * 128 + (((cg & 7) ^ (v_key & 7)) << 4));
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[dt][nt], a, pb[nt]);
+        }
+    }
+}
+
 // Merge the four warps' (max, sum, unnormalised output) held in cm/cl/co, then either
 // write the rows (whole unit) or a split partial; the last split of a unit merges all
 // partials. Every thread of the CTA calls this.
@@ -469,8 +626,8 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
                     }
                 }
             }
-            // -- mask and per-row (column) max over the pair's 32 keys -----------------------
-            float cmax[NT][2];
+            // -- mask; this lane's max of each row over the pair's 32 keys ---------------------
+            float lmax[NT][2];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -495,20 +652,29 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
                             mx = fmaxf(mx, v);
                         }
                     }
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                    cmax[nt][e] = mx;
+                    lmax[nt][e] = mx;
                 }
-            // -- lazy rescale: only when some row's max passed its reference by the slack ----
+            // -- lazy rescale: only when some score passed its row's reference by the slack (or
+            //    the row has no reference yet); the row max (shuffles) only in that case --------
             bool need = false;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e)
-                    need |= cmax[nt][e] > mref[nt][e] + kRescaleSlack ||
-                            (mref[nt][e] == -INFINITY && cmax[nt][e] != -INFINITY);
+                    need |= lmax[nt][e] > mref[nt][e] + kRescaleSlack ||
+                            (mref[nt][e] == -INFINITY && lmax[nt][e] != -INFINITY);
             if (__any_sync(0xffffffffu, need)) {
+                float cmax[NT][2];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        float mx = lmax[nt][e];
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                        cmax[nt][e] = mx;
+                    }
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -616,130 +782,7 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
                 }
             }
 
-            // -- S^T = K Q^T (16 keys x 8 rows per n-tile) ------------------------------------
-            float s[NT][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
-            if constexpr (C::QB) {
-#pragma unroll
-                for (int k2 = 0; k2 < KS; k2 += 2) {
-                    uint32_t qb[NT][4];              // b fragments of k-steps k2 and k2 + 1
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const int qr = nt * 8 + (lane & 7), qc = 2 * k2 + (lane >> 3);
-                        ldmatrix_x4(qb[nt], qs + qr * (D * 2) + ((qc ^ (qr & 7)) << 4));
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < 2; ++kk) {
-                        const int cg = (k2 + kk) * 2 + k_chunk;
-                        uint32_t a[4];
-                        ldmatrix_x4(a, Ks + (cg >> 3) * kBoxBytes + k_key * 128 + (((cg & 7) ^ (k_key & 7)) << 4));
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a, &qb[nt][2 * kk]);
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int ks = 0; ks < KS; ++ks) {
-                    const int cg = ks * 2 + k_chunk;
-                    uint32_t a[4];
-                    ldmatrix_x4(a, Ks + (cg >> 3) * kBoxBytes + k_key * 128 + (((cg & 7) ^ (k_key & 7)) << 4));
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a, qf[nt][ks]);
-                }
-            }
-
-            // -- mask and per-row (column) max over the page's 16 keys ------------------------
-            const bool page_all = (kbase + kPageSize - 1) <= min_lim;
-            float cmax[NT][2];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int kpos = kbase + g + 8 * h;
-                        float v = s[nt][2 * h + e] * sl2;
-                        if (!page_all) {
-                            bool allow = kpos <= lim[nt][e];
-                            if (!allow && kpos >= prefix && kpos < si.seq_len)
-                                allow = (anc[nt][e] >> (kpos - prefix)) & 1ull;
-                            v = allow ? v : -INFINITY;
-                        }
-                        s[nt][2 * h + e] = v;
-                    }
-                    float mx = fmaxf(s[nt][e], s[nt][2 + e]);
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                    cmax[nt][e] = mx;
-                }
-            // -- lazy rescale: only when some row's max passed its reference by the slack ------
-            bool need = false;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e)
-                    need |= cmax[nt][e] > mref[nt][e] + kRescaleSlack ||
-                            (mref[nt][e] == -INFINITY && cmax[nt][e] != -INFINITY);
-            if (__any_sync(0xffffffffu, need)) {
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const float mnew = fmaxf(mref[nt][e], cmax[nt][e]);
-                        if (mnew != mref[nt][e]) {
-                            const float alpha = mref[nt][e] == -INFINITY ? 0.f : exp2f(mref[nt][e] - mnew);
-                            mref[nt][e] = mnew;
-                            lsum[nt][e] *= alpha;
-#pragma unroll
-                            for (int dt = 0; dt < KS; ++dt) {
-                                o[dt][nt][e] *= alpha;
-                                o[dt][nt][2 + e] *= alpha;
-                            }
-                        }
-                    }
-            }
-            // -- P = exp2(S - ref), row sums, P^T as the B operand (transpose in registers) -----
-            uint32_t pb[NT][2];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                float pv[4];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const float ref = mref[nt][e] == -INFINITY ? 0.f : mref[nt][e];
-                    pv[e] = exp2f(s[nt][e] - ref);
-                    pv[2 + e] = exp2f(s[nt][2 + e] - ref);
-                    lsum[nt][e] += pv[e] + pv[2 + e];
-                }
-                pb[nt][0] = movmatrix_trans(pack_bf16x2(pv[0], pv[1]));   // keys 0..7
-                pb[nt][1] = movmatrix_trans(pack_bf16x2(pv[2], pv[3]));   // keys 8..15
-            }
-            // slots past the sequence's end hold stale cache data: zero those V rows so that
-            // P = 0 times a non-finite value cannot reach the accumulators
-            const int nvalid = si.seq_len - kbase;
-            if (nvalid < kPageSize) {
-                for (int idx = lane; idx < (kPageSize - nvalid) * (D / 8); idx += 32) {
-                    const int row = nvalid + idx / (D / 8);
-                    const int cg = idx % (D / 8);
-                    *reinterpret_cast<uint4*>(Vs + (cg >> 3) * kBoxBytes + row * 128 + (cg & 7) * 16) =
-                        make_uint4(0u, 0u, 0u, 0u);
-                }
-                __syncwarp();
-            }
-            // -- O^T += V^T P^T -----------------------------------------------------------------
-            {
-#pragma unroll
-                for (int dt = 0; dt < KS; ++dt) {
-                    const int cg = dt * 2 + v_chunk;
-                    uint32_t a[4];
-                    ldmatrix_x4_trans(a, Vs + (cg >> 3) * kBoxBytes + v_key * 128 + (((cg & 7) ^ (v_key & 7)) << 4));
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[dt][nt], a, pb[nt]);
-                }
-            }
+            bf16_page<D, NT, C::QB>(Ks, Vs, qs, qf, kbase, prefix, si.seq_len, min_lim, lim, anc, sl2, o, mref, lsum);
             __syncwarp();
             if (lane == 0 && i + C::NS < n_my) {
                 fence_proxy_async_smem();
@@ -815,6 +858,314 @@ __device__ __forceinline__ void decode_mma_task(const Group& grp, const DecodePa
             append_rows<D>(p.k_new, p.v_new, p.k_cache, p.v_cache, p.block_table, p.bt_stride, p.num_pages, p.Hkv,
                            p.err, si, w.seq, w.kv_head, 0, si.query_len, tid, grp.n);
     }
+}
+
+// =====================================================================================
+// Row-split (wide) task: one pass over the pages for up to 48 packed rows.
+// =====================================================================================
+// A verify unit of a (sequence, KV head) has T draft tokens x G query heads packed rows
+// (5 x 7 = 35 on the Qwen2-7B shape), more than the 16 columns one warp's tiles hold. The
+// page-streaming task above would take such a unit as several 16-row tasks that each read
+// every page of the unit again. Here one task takes up to three 16-row chunks of the unit:
+// warp 3 streams each page once through a ring shared by the task (TMA, a full and an
+// empty mbarrier per stage), and warps 0..2 each run the page body for their own chunk on
+// every page, so no warp shares rows with another and nothing is combined across warps.
+// Every chunk keeps its own split unit (partial slots, arrival counter), so splits and
+// shared-prefix partials work per chunk as for the page-streaming task.
+constexpr int kWideChunks = 3;                           // consumer warps (16-row chunks)
+constexpr int kWideRows = kWideChunks * kDecodeRowsMax;  // rows one wide task holds
+constexpr int kWideProducer = 3;                         // the warp that issues the page loads
+
+// Shared-memory bytes of a wide task with `nsw` ring stages (the map of WideCfg).
+constexpr int wide_bytes(int D, int nsw) {
+    return align_up(align_up(align_up(nsw * 2 * kPageSize * D * 2 + kWideRows * 4, 8) + kWideRows * 12, 8) +
+                        2 * nsw * 8 + 48, 128) + kWideRows * D * 2;
+}
+
+// The most ring stages a wide task can have within `budget` bytes of shared memory.
+constexpr int wide_stages(int D, int budget) {
+    int n = 1;
+    while (n < 32 && wide_bytes(D, n + 1) <= budget) ++n;
+    return n;
+}
+
+template <int D, int NSW_>
+struct WideCfg {
+    static constexpr int NSW = NSW_;                      // ring stages (one page each)
+    static constexpr int PAGE_BYTES = kPageSize * D * 2;
+    static constexpr int STAGE_BYTES = 2 * PAGE_BYTES;    // K page + V page
+    static constexpr int RING = NSW * STAGE_BYTES;
+    static constexpr int OFF_LIM = RING;
+    static constexpr int OFF_ANC = align_up(OFF_LIM + kWideRows * 4, 8);
+    static constexpr int OFF_OUT = OFF_ANC + kWideRows * 8;
+    static constexpr int OFF_BAR = align_up(OFF_OUT + kWideRows * 4, 8);   // full[NSW], empty[NSW]
+    static constexpr int OFF_FLAG = OFF_BAR + 2 * NSW * 8;   // [0, 3) merge flags, [3] units to merge,
+                                                             // [4, 7) their ids, [8, 11) row offsets
+    static constexpr int OFF_Q = align_up(OFF_FLAG + 48, 128);
+    static constexpr int BYTES = OFF_Q + kWideRows * D * 2;
+    static_assert(kWideRows * (D + 2) * 4 <= RING, "end-of-task buffers must fit in the ring");
+    static_assert(BYTES == wide_bytes(D, NSW), "wide task map");
+};
+
+template <int D, int NSW>
+__device__ __forceinline__ void decode_wide_task(const Group& grp, const DecodeParams& p, int task,
+                                                 const CUtensorMap& tmK, const CUtensorMap& tmV, uint8_t* sm) {
+    using C = WideCfg<D, NSW>;
+    const int tid = grp.tid, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t4 = lane & 3;
+    const DecodeWork w = p.work[task];
+    const SeqInfo si = p.seqs[w.seq];
+    const int R = w.row_count;                               // 17 .. 48
+    const int nch = (R + kDecodeRowsMax - 1) / kDecodeRowsMax;
+    const int npg = w.page_end - w.page_begin;
+    const int prefix = si.seq_len - si.query_len;
+
+    int* rlim = reinterpret_cast<int*>(sm + C::OFF_LIM);
+    uint64_t* ranc = reinterpret_cast<uint64_t*>(sm + C::OFF_ANC);
+    int* rout = reinterpret_cast<int*>(sm + C::OFF_OUT);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
+    uint64_t* empty = full + NSW;
+    int* flag = reinterpret_cast<int*>(sm + C::OFF_FLAG);
+    uint8_t* qs = sm + C::OFF_Q;
+    uint8_t* ring = sm;
+
+    if (tid == 0) {
+        for (int i = 0; i < NSW; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], nch);
+        }
+        fence_mbar_init();
+        fence_proxy_async_smem();                 // the block's earlier generic accesses come first
+        for (int i = 0; i < 12; ++i) flag[i] = 0;
+    }
+    // per-row records: output row, causal limit, tree ancestor mask
+    for (int r = tid; r < kWideRows; r += grp.n) {
+        if (r < R) {
+            const int t = (w.row_begin + r) / p.G;
+            rout[r] = q_row_index(p, si, w, r);
+            rlim[r] = si.mask_kind == PKVA_CAUSAL ? prefix + t : prefix - 1;
+            ranc[r] = si.mask_kind == PKVA_CAUSAL ? 0ull : p.anc[si.anc_off + t];
+        } else {
+            rout[r] = -1;
+            rlim[r] = 0x7fffffff;
+            ranc[r] = 0ull;
+        }
+    }
+    // Q rows staged in shared memory (16-byte chunk c of row r at c ^ (r & 7)); missing rows zero
+    for (int idx = tid; idx < kWideRows * (D / 8); idx += grp.n) {
+        const int r = idx / (D / 8), c = idx - r * (D / 8);
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (r < R) v = *reinterpret_cast<const uint4*>(p.q + (int64_t)q_row_index(p, si, w, r) * D + c * 8);
+        *reinterpret_cast<uint4*>(qs + r * (D * 2) + ((c ^ (r & 7)) << 4)) = v;
+    }
+    grp.sync();
+
+    bool ok = true;
+    if (warp == kWideProducer) {
+        // ---- producer: every page once, in order; a stage is refilled once all chunks are done
+        //      with it. Block-table entries are read 32 at a time and handed out by shuffle.
+        if (lane == 0) {
+            prefetch_tensormap(&tmK);
+            prefetch_tensormap(&tmV);
+        }
+        const int32_t* btrow = p.block_table + (int64_t)w.seq * p.bt_stride + w.page_begin;
+        int issued = 0;
+        for (int base = 0; base < npg && ok; base += 32) {
+            int ph = -1;
+            if (base + lane < npg) {
+                ph = btrow[base + lane];
+                if (ph < 0 || ph >= p.num_pages) {
+                    atomicOr(p.err, PKVA_DEVERR_BAD_PAGE);
+                    ph = -1;                      // read from a fully out-of-bounds box: zeros
+                }
+            }
+            const int n = min(32, npg - base);
+            for (int j = 0; j < n; ++j) {
+                const int phj = __shfl_sync(0xffffffffu, ph, j);
+                const int i = base + j;
+                bool got = true;
+                if (lane == 0) {
+                    if (i >= NSW)
+                        got = mbar_wait_bounded(&empty[i % NSW], ((i / NSW) - 1) & 1, p.err, PKVA_DEVERR_TIMEOUT);
+                    if (got) {
+                        fence_proxy_async_smem();
+                        issue_page_at<D, NSW, C::STAGE_BYTES, C::PAGE_BYTES>(p, w, phj, ring, full, i, &tmK, &tmV);
+                    }
+                }
+                if (!__shfl_sync(0xffffffffu, got, 0)) {
+                    ok = false;
+                    break;
+                }
+                ++issued;
+            }
+        }
+        // every issued load has landed before the ring is reused (the consumers normally
+        // waited for all of them already)
+        if (lane == 0)
+            for (int i = max(0, issued - NSW); i < issued; ++i)
+                mbar_wait_bounded(&full[i % NSW], (i / NSW) & 1, p.err, PKVA_DEVERR_TIMEOUT);
+        __syncwarp();
+    }
+
+    // ---- consumers: warp c owns packed rows [16c, 16c + 16) of the task
+    constexpr int NT = 2;
+    constexpr int KS = D / 16;
+    float o[KS][NT][4];
+    float mref[NT][2], lsum[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            mref[nt][e] = -INFINITY;
+            lsum[nt][e] = 0.f;
+        }
+#pragma unroll
+        for (int dt = 0; dt < KS; ++dt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[dt][nt][i] = 0.f;
+    }
+    const bool consumer = warp < nch;
+    if (consumer) {
+        const int r0 = warp * kDecodeRowsMax;
+        int lim[NT][2];
+        uint64_t anc[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int c = r0 + nt * 8 + 2 * t4 + e;
+                lim[nt][e] = rlim[c];
+                anc[nt][e] = ranc[c];
+            }
+        int min_lim = 0x7fffffff;
+        for (int r = r0; r < min(R, r0 + kDecodeRowsMax); ++r) min_lim = min(min_lim, rlim[r]);
+        const uint8_t* qw = qs + r0 * (D * 2);
+        const uint32_t qf_unused[NT][1][2] = {};
+        const float sl2 = p.scale_log2;
+        for (int i = 0; i < npg; ++i) {
+            const int stage = i % NSW;
+            const bool got = mbar_wait_bounded(&full[stage], (i / NSW) & 1, p.err, PKVA_DEVERR_TIMEOUT);
+            if (__any_sync(0xffffffffu, !got)) {
+                ok = false;
+                break;
+            }
+            uint8_t* Ks = ring + stage * C::STAGE_BYTES;
+            uint8_t* Vs = Ks + C::PAGE_BYTES;
+            const int kbase = (w.page_begin + i) * kPageSize;
+            if (p.append && kbase + kPageSize > prefix && kbase < si.seq_len) {
+                // fused append: the new tokens' rows come from the dense input (each chunk's warp
+                // writes the same bytes, so the copies agree whichever lands last)
+                const int a0 = max(prefix - kbase, 0), a1 = min(si.seq_len - kbase, kPageSize);
+                patch_page_rows<D>(Ks, Vs, p.k_new, p.v_new, si, p.Hkv, w.kv_head, a0, a1, kbase + a0 - prefix,
+                                   lane);
+                __syncwarp();
+            }
+            bf16_page<D, NT, true>(Ks, Vs, qw, qf_unused, kbase, prefix, si.seq_len, min_lim, lim, anc, sl2, o,
+                                   mref, lsum);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+        }
+        // row sums over the 16 keys: lanes with the same t4 hold the column
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float l = lsum[nt][e];
+                l += __shfl_xor_sync(0xffffffffu, l, 4);
+                l += __shfl_xor_sync(0xffffffffu, l, 8);
+                l += __shfl_xor_sync(0xffffffffu, l, 16);
+                lsum[nt][e] = l;
+            }
+    }
+    grp.sync();                                     // every page consumed and every load landed
+    if (tid == 0)
+        for (int i = 0; i < NSW; ++i) {
+            mbar_inval(&full[i]);
+            mbar_inval(&empty[i]);
+        }
+
+    // ---- per-row state into shared memory (the ring is free now) --------------------
+    float* cm = reinterpret_cast<float*>(sm);       // [48]
+    float* cl = cm + kWideRows;                     // [48]
+    float* co = cl + kWideRows;                     // [48][D]
+    if (consumer) {
+        const int r0 = warp * kDecodeRowsMax;
+        if (g == 0) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int c = r0 + nt * 8 + 2 * t4 + e;
+                    cm[c] = mref[nt][e];
+                    cl[c] = lsum[nt][e];
+                }
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int dt = 0; dt < KS; ++dt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int c = r0 + nt * 8 + 2 * t4 + (i & 1);
+                    const int d = dt * 16 + g + 8 * (i >> 1);
+                    co[c * D + d] = o[dt][nt][i];
+                }
+    }
+    grp.sync();
+
+    // ---- rows out, or each chunk's partial into its unit's slot ----------------------
+    const bool split = w.unit >= 0;
+    for (int idx = tid; idx < R * (D / 2); idx += grp.n) {
+        const int r = idx / (D / 2);
+        const int c = (idx - r * (D / 2)) * 2;
+        const float2 v = *reinterpret_cast<const float2*>(co + r * D + c);
+        if (!split) {
+            const float L = cl[r];
+            const float inv = L > 0.f ? 1.f / L : 0.f;
+            *reinterpret_cast<__nv_bfloat162*>(p.out + (int64_t)rout[r] * D + c) =
+                __floats2bfloat162_rn(v.x * inv, v.y * inv);
+        } else {
+            const int ch = r / kDecodeRowsMax, rr = r - ch * kDecodeRowsMax;
+            const int slot = p.units[w.unit + ch].slot_base + w.split;
+            *reinterpret_cast<float2*>(p.part_o + ((int64_t)slot * kDecodeRowsMax + rr) * D + c) = v;
+            if (c == 0)
+                *reinterpret_cast<float2*>(p.part_ml + ((int64_t)slot * kDecodeRowsMax + rr) * 2) =
+                    make_float2(cm[r], cl[r]);
+        }
+    }
+    if (split) {
+        // ---- split-KV combine per chunk: the last task of a unit to finish merges it ------
+        __threadfence();
+        grp.sync();
+        if (tid < nch) {
+            const int u = w.unit + tid;
+            const int prev = atomicAdd(&p.counters[u], 1);
+            flag[tid] = (prev == p.units[u].arrivals - 1);
+            if (flag[tid]) p.counters[u] = 0;           // every arrival is in: ready for the next run
+        }
+        grp.sync();
+        if (tid == 0) {
+            int n = 0, rows = 0;
+            for (int ch = 0; ch < nch; ++ch)
+                if (flag[ch]) {
+                    flag[4 + n] = w.unit + ch;
+                    flag[8 + n] = rows;
+                    rows += p.units[w.unit + ch].row_count;
+                    ++n;
+                }
+            flag[3] = n;
+            flag[11] = rows;
+        }
+        grp.sync();
+        if (flag[3] > 0) {
+            __threadfence();
+            merge_units<D>(warp, grp.n >> 5, lane, flag + 4, flag + 8, flag[3], flag[11], p.units, p.part_o,
+                           p.part_ml, p.seqs, p.out, p.Hq, p.G);
+        }
+    }
+    if (p.append && w.row_begin == 0 && w.split <= 0)          // one task per (sequence, KV head)
+        append_rows<D>(p.k_new, p.v_new, p.k_cache, p.v_cache, p.block_table, p.bt_stride, p.num_pages, p.Hkv,
+                       p.err, si, w.seq, w.kv_head, 0, si.query_len, tid, grp.n);
 }
 
 // =====================================================================================

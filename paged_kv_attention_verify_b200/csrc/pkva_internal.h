@@ -11,6 +11,7 @@ namespace pkva {
 constexpr int kPageSize = 16;          // keys per page (the only page size supported)
 constexpr int kMaxTreeTokens = 64;     // draft tokens per TREE sequence (one 64-bit mask)
 constexpr int kDecodeRowsMax = 16;     // packed (token, head) rows per decode task
+constexpr int kWideRowsMax = 48;       // packed rows per row-split (wide) decode/verify task
 constexpr int kDecodeMaxPages = 1024;  // pages per decode task (block-table slice in smem)
 constexpr int kPrefillTileM = 128;     // query tokens per prefill tile (tcgen05 M)
 constexpr int kPrefillTaskTokens = 256; // query tokens per prefill task (two tiles, ping-pong)
@@ -38,7 +39,8 @@ struct DecodeWork {
     int32_t seq;
     int32_t kv_head;
     int32_t row_begin;   // packed row = token * group + head-in-group
-    int32_t row_count;   // <= kDecodeRowsMax
+    int32_t row_count;   // <= kDecodeRowsMax; up to kWideRowsMax for a row-split task, whose
+                         // 16-row chunks are split units unit, unit + 1, ... when split
     int32_t page_begin;  // logical pages of the sequence
     int32_t page_end;
     int32_t unit;        // split unit id, -1 when the task covers its whole unit
@@ -145,6 +147,10 @@ struct PlanArgs {
     int ctas_per_sm;
     bool use_prefill_kernel = true;       // false: every sequence goes to the decode kernel
     int kv_elem_bytes = 2;                // bytes per cached K/V element (2 bf16, 1 FP8)
+    // rows of a (sequence, KV head) beyond one 16-row task go to row-split tasks of up to
+    // 48 rows that read each page once (the unified kernel's bf16 decode/verify path); false:
+    // every task holds at most 16 rows (the stand-alone decode kernels)
+    bool wide_tasks = true;
     // shared-prefix groups (may be NULL / 0): prefix_group[s] in {-1} U [0, num_groups),
     // members of a group consecutive in the batch, prefix_len[g] keys shared (page multiple)
     const int32_t* prefix_group = nullptr;

@@ -22,6 +22,10 @@ namespace {
 
 constexpr int kMinSplitPages = 8;      // never split a unit into tasks below 128 keys
 constexpr int kTasksPerSlot = 1;       // split long units down to about one task per CTA slot
+// A row-split task's warps each run every page of the task, where a 16-row task's four warps
+// share its pages: it gets a quarter of the pages of a 16-row task, so that its warps' page
+// chains are as long as theirs.
+constexpr int kWideSplit = 4;
 
 int fail(std::string* err, int code, const char* fmt, long a = 0, long b = 0, long c = 0) {
     char buf[256];
@@ -196,40 +200,15 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
         });
     }
 
-    // FP8 caches: the tensor-core tasks read a bf16 copy of their sequences' pages
-    if (a.kv_elem_bytes == 1) {
-        int stride = 0, n = 0;
-        for (int s = 0; s < a.num_seqs; ++s)
-            if (on_prefill[s]) {
-                const int pages = (p.seqs[s].seq_len + kPageSize - 1) / kPageSize;
-                stride = std::max(stride, pages);
-                n += pages;
-            }
-        if ((int64_t)n * a.Hkv * kPageSize >= (int64_t(1) << 31))
-            return fail(err, PKVA_EUNSUPPORTED, "FP8 prefill staging too large: %ld pages", n);
-        if (n > 0) {
-            p.stage_stride = stride;
-            p.num_stage_pages = n;
-            p.stage_bt.assign((size_t)a.num_seqs * stride, -1);
-            p.stage_src.reserve(2 * (size_t)n);
-            int next = 0;
-            for (int s = 0; s < a.num_seqs; ++s) {
-                if (!on_prefill[s]) continue;
-                const int pages = (p.seqs[s].seq_len + kPageSize - 1) / kPageSize;
-                for (int lp = 0; lp < pages; ++lp) {
-                    p.stage_bt[(size_t)s * stride + lp] = next++;
-                    p.stage_src.push_back(s);
-                    p.stage_src.push_back(lp);
-                }
-            }
-        }
-    }
-
     // -- decode/verify units: (seq, kv head, chunk of packed rows) --------------------
     // A sequence of a shared-prefix group leaves its first prefix_len keys to the cascade
     // tasks: its units start at that page, and always merge partials.
-    struct Unit { int seq, kvh, rb, rc, pstart, pages, cs; };   // cs: cascade splits (0: none)
+    // cs: cascade splits (0: none). A row-split task covers several consecutive chunk units:
+    // its first (lead) unit has wrows = the task's rows, the others wrows = 0; a plain unit
+    // has wrows = rc. All chunks of a row-split task share its page range.
+    struct Unit { int seq, kvh, rb, rc, pstart, pages, cs, wrows; };
     std::vector<Unit> units;
+    const bool wide = a.wide_tasks && a.kv_elem_bytes == 2;
     std::vector<int> unit_base(a.num_seqs, -1);     // index of (s, head 0, chunk 0) in units
     std::vector<char> on_cascade(a.num_seqs, 0);
     int64_t total_pages = 0;
@@ -246,17 +225,28 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
         on_cascade[s] = g >= 0;
         p.seqs[s].shared_len = g >= 0 ? a.prefix_len[g] : 0;
         unit_base[s] = (int)units.size();
+        // keys past the last row's own position are masked for every row of a task (causal
+        // and tree alike), so the task never loads them
+        auto pages_to = [&](int last_row) {
+            const int kend = si.seq_len - si.query_len + last_row / p.G + 1;
+            return (kend + kPageSize - 1) / kPageSize;
+        };
         for (int h = 0; h < a.Hkv; ++h) {
-            for (int rb = 0; rb < rows; rb += kDecodeRowsMax) {
-                const int rc = std::min(kDecodeRowsMax, rows - rb);
-                const int t_last = (rb + rc - 1) / p.G;
-                // keys past the last row's own position are masked for every row of the
-                // chunk (causal and tree alike), so the task never loads them
-                const int kend = si.seq_len - si.query_len + t_last + 1;
-                const int pages = (kend + kPageSize - 1) / kPageSize;
-                units.push_back({s, h, rb, rc, pstart, pages, cs});
+            for (int tb = 0; tb < rows; tb += wide ? kWideRowsMax : kDecodeRowsMax) {
+                const int tr = std::min(wide ? kWideRowsMax : kDecodeRowsMax, rows - tb);
+                if (tr <= kDecodeRowsMax) {
+                    const int pages = pages_to(tb + tr - 1);
+                    units.push_back({s, h, tb, tr, pstart, pages, cs, tr});
+                    total_pages += pages - pstart;
+                    max_rc = std::max(max_rc, tr);
+                    continue;
+                }
+                // one row-split task: its 16-row chunks, the whole row range's pages
+                const int pages = pages_to(tb + tr - 1);
+                for (int rb = tb; rb < tb + tr; rb += kDecodeRowsMax)
+                    units.push_back({s, h, rb, std::min(kDecodeRowsMax, tb + tr - rb), pstart, pages, cs,
+                                     rb == tb ? tr : 0});
                 total_pages += pages - pstart;
-                max_rc = std::max(max_rc, rc);
             }
         }
     }
@@ -293,33 +283,41 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
     std::vector<int> unit_ns(units.size(), 0);
     for (size_t ui = 0; ui < units.size(); ++ui) {
         const Unit& u = units[ui];
+        if (u.wrows == 0) continue;           // a later chunk of a row-split task: done with its lead
         const int own = u.pages - u.pstart;
+        const int nchunks = (u.wrows + kDecodeRowsMax - 1) / kDecodeRowsMax;
         // nearest whole number of target-sized tasks (rounding up made near-target units two
         // half-size tasks), never more pages per task than the staged block-table slice holds
-        const int ns = std::max<int>(std::max<int>(1, (int)((own + target / 2) / target)),
+        const int64_t cost = nchunks > 1 ? (int64_t)own * kWideSplit : own;
+        const int ns = std::max<int>(std::max<int>(1, (int)((cost + target / 2) / target)),
                                      (own + kDecodeMaxPages - 1) / kDecodeMaxPages);
-        unit_ns[ui] = ns;
-        int unit_id = -1;
-        if (ns > 1 || u.cs > 0) {
-            unit_id = (int)p.units.size();
-            SplitUnit su{};
-            su.slot_base = p.num_slots;
-            su.num_splits = ns + u.cs;
-            su.arrivals = ns;                 // cascade tasks add theirs below
-            su.seq = u.seq;
-            su.kv_head = u.kvh;
-            su.row_begin = u.rb;
-            su.row_count = u.rc;
-            p.units.push_back(su);
-            p.num_slots += ns + u.cs;
+        int unit_id = -1;                     // the lead chunk's; chunk c has unit_id + c
+        for (int c = 0; c < nchunks; ++c) {
+            const Unit& uc = units[ui + c];
+            unit_ns[ui + c] = ns;
+            int id = -1;
+            if (ns > 1 || uc.cs > 0) {
+                id = (int)p.units.size();
+                SplitUnit su{};
+                su.slot_base = p.num_slots;
+                su.num_splits = ns + uc.cs;
+                su.arrivals = ns;             // cascade tasks add theirs below
+                su.seq = uc.seq;
+                su.kv_head = uc.kvh;
+                su.row_begin = uc.rb;
+                su.row_count = uc.rc;
+                p.units.push_back(su);
+                p.num_slots += ns + uc.cs;
+            }
+            unit_id_of[ui + c] = id;
+            if (c == 0) unit_id = id;
         }
-        unit_id_of[ui] = unit_id;
         for (int k = 0; k < ns; ++k) {
             DecodeWork w{};
             w.seq = u.seq;
             w.kv_head = u.kvh;
             w.row_begin = u.rb;
-            w.row_count = u.rc;
+            w.row_count = u.wrows;
             w.page_begin = u.pstart + (int)((int64_t)own * k / ns);
             w.page_end = u.pstart + (int)((int64_t)own * (k + 1) / ns);
             w.unit = unit_id;
@@ -396,9 +394,46 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
             s = e + 1;
         }
     }
+    // FP8 caches: the tensor-core tasks read a bf16 copy of the pages they use: all pages of
+    // a sequence that runs as prefill tasks, the shared pages of a cascade run's lead sequence
+    // (whose block-table row supplies the shared keys to its cascade tasks)
+    if (a.kv_elem_bytes == 1) {
+        std::vector<int> stage_pages(a.num_seqs, 0);
+        for (int s = 0; s < a.num_seqs; ++s)
+            if (on_prefill[s]) stage_pages[s] = (p.seqs[s].seq_len + kPageSize - 1) / kPageSize;
+        for (const CascadeWork& cw : p.cwork)
+            stage_pages[cw.lead_seq] = a.prefix_len[grp_of[cw.lead_seq]] / kPageSize;
+        int stride = 0;
+        int64_t n = 0;
+        for (int s = 0; s < a.num_seqs; ++s) {
+            stride = std::max(stride, stage_pages[s]);
+            n += stage_pages[s];
+        }
+        if (n * a.Hkv * kPageSize >= (int64_t(1) << 31))
+            return fail(err, PKVA_EUNSUPPORTED, "FP8 tensor-core staging too large: %ld pages", (long)n);
+        if (n > 0) {
+            p.stage_stride = stride;
+            p.num_stage_pages = (int)n;
+            p.stage_bt.assign((size_t)a.num_seqs * stride, -1);
+            p.stage_src.reserve(2 * (size_t)n);
+            int next = 0;
+            for (int s = 0; s < a.num_seqs; ++s) {
+                for (int lp = 0; lp < stage_pages[s]; ++lp) {
+                    p.stage_bt[(size_t)s * stride + lp] = next++;
+                    p.stage_src.push_back(s);
+                    p.stage_src.push_back(lp);
+                }
+            }
+        }
+    }
+
     // heaviest first; ties keep (seq, head, chunk) order so chunks of one head stay adjacent
-    std::stable_sort(p.dwork.begin(), p.dwork.end(), [](const DecodeWork& x, const DecodeWork& y) {
-        return (x.page_end - x.page_begin) > (y.page_end - y.page_begin);
+    // (a row-split task weighs its pages kWideSplit times: each of its warps runs every page)
+    auto task_cost = [](const DecodeWork& w) {
+        return (w.page_end - w.page_begin) * (w.row_count > kDecodeRowsMax ? kWideSplit : 1);
+    };
+    std::stable_sort(p.dwork.begin(), p.dwork.end(), [&](const DecodeWork& x, const DecodeWork& y) {
+        return task_cost(x) > task_cost(y);
     });
 
     // -- one launch order. Cascade tasks go first: few, long, and every unit of their rows

@@ -480,6 +480,8 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
             if (nb > 0 && alive && __all_sync(0xffffffffu, wait_or_abort(&B.o_ready[b], 0, p.err, abort_flag))) {
                 tc_fence_after();
                 float* dst = p.part_o + (int64_t)(part_idx < 0 ? 0 : part_idx) * kD;
+                // FP8 caches: the V scale of this KV head, as on every other partial
+                const float vsc = p.v_scale ? p.v_scale[kvh] : 1.f;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t ov[32];
@@ -489,8 +491,8 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
 #pragma unroll
                         for (int e = 0; e < 32; e += 4)
                             *reinterpret_cast<float4*>(dst + c * 32 + e) =
-                                make_float4(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1]),
-                                            __uint_as_float(ov[e + 2]), __uint_as_float(ov[e + 3]));
+                                make_float4(__uint_as_float(ov[e]) * vsc, __uint_as_float(ov[e + 1]) * vsc,
+                                            __uint_as_float(ov[e + 2]) * vsc, __uint_as_float(ov[e + 3]) * vsc);
                     }
                 }
                 if (real_row)

@@ -138,6 +138,7 @@ extern "C" int attn_run_static(int num_seqs, const int32_t* seq_lens, const int3
     PlanArgs a{num_seqs, seq_lens, query_lens, bt_stride, num_pages, mask_kind, parents, num_q_heads,
                num_kv_heads, head_dim, page_size, sm_scale, 1, 1};
     a.use_prefill_kernel = false;          // everything on the decode kernel (no TMEM, no extra tables)
+    a.wide_tasks = false;                  // tasks of at most 16 rows (the stand-alone decode kernel)
     HostPlan hp;
     std::string err;
     int rc = build_host_plan(a, &hp, &err);
@@ -155,6 +156,25 @@ extern "C" int attn_run_static(int num_seqs, const int32_t* seq_lens, const int3
     if (major != 10) {
         set_last_error("attn_run_static: this library is built for sm_100a (B200); the current device is not");
         return PKVA_EUNSUPPORTED;
+    }
+    // the kernel runs on the current device and reaches that device's scratch: every
+    // tensor must live there (a pointer to another GPU or to host memory is rejected)
+    {
+        const void* ptrs[5] = {block_table, q, k_cache, v_cache, out};
+        const char* names[5] = {"block_table", "q", "k_cache", "v_cache", "out"};
+        for (int i = 0; i < 5; ++i) {
+            cudaPointerAttributes at{};
+            if (cudaPointerGetAttributes(&at, ptrs[i]) != cudaSuccess) {
+                cudaGetLastError();
+                set_last_error(std::string("attn_run_static: cannot query the memory of ") + names[i]);
+                return PKVA_EINVAL;
+            }
+            if ((at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged) || at.device != dev) {
+                set_last_error(std::string("attn_run_static: ") + names[i] +
+                               " is not device memory of the current device");
+                return PKVA_EINVAL;
+            }
+        }
     }
     a.num_sms = sms;
     const bool mma = decode_body_is_mma();

@@ -97,8 +97,9 @@ def _coverage(batch, items, prefix_group=None, prefix_len=None):
                 assert prefix_group[s] == prefix_group[it["seq"]] >= 0
                 assert it["key_end"] <= prefix_len[prefix_group[s]]
                 rows += [(s, (tok - q_start[s]) * G + g) for g in range(G)]
-        else:
-            assert 1 <= it["row_count"] <= 16 and it["q_head"] == -1
+        else:                          # decode/verify: up to 16 rows, or a row-split task of up to 48
+            assert 1 <= it["row_count"] <= 48 and it["q_head"] == -1
+            assert it["row_count"] <= 16 or it["row_begin"] % 48 == 0
             rows = [(it["seq"], r) for r in range(it["row_begin"], it["row_begin"] + it["row_count"])]
         for s, r in rows:
             seen.setdefault((s, it["kv_head"], r), []).append((it["key_begin"], it["key_end"], it["kind"],
@@ -150,8 +151,11 @@ def test_planner_covers_configs(name):
     kinds = [it["kind"] for it in items]
     assert kinds == sorted(kinds, reverse=True)
     dec = [it for it in items if it["kind"] == 0]
-    pg = [(it["key_end"] + 15) // 16 - it["key_begin"] // 16 for it in dec]
-    assert pg == sorted(pg, reverse=True)
+    # heaviest first: pages, times 4 for a row-split task (more than 16 rows, every warp
+    # runs every page)
+    cost = [((it["key_end"] + 15) // 16 - it["key_begin"] // 16) * (4 if it["row_count"] > 16 else 1)
+            for it in dec]
+    assert cost == sorted(cost, reverse=True)
     assert all(it["key_end"] - it["key_begin"] <= 1024 * 16 for it in dec)
 
 
@@ -238,3 +242,57 @@ def test_decode_tasks_never_exceed_the_staged_block_table_slice(num_sms, ctas):
             spans = sorted((it["key_begin"], it["key_end"]) for it in items if it["seq"] == s and it["kv_head"] == h)
             assert spans[0][0] == 0 and spans[-1][1] == L
             assert all(a[1] == b[0] for a, b in zip(spans[:-1], spans[1:]))
+
+
+
+def _static_call(**over):
+    """run_static on a 2-sequence batch whose tensors live on the host (CPU)."""
+    import torch
+    a = dict(seq_lens=[40, 17], query_lens=[8, 1], block_table=torch.zeros(2, 4, dtype=torch.int32),
+             mask_kind=[W.CAUSAL, W.CAUSAL], parents=None,
+             q=torch.zeros(9, 8, 64, dtype=torch.bfloat16), k_cache=torch.zeros(8, 2, 16, 64, dtype=torch.bfloat16),
+             v_cache=torch.zeros(8, 2, 16, 64, dtype=torch.bfloat16), out=torch.zeros(9, 8, 64, dtype=torch.bfloat16),
+             num_q_heads=8, num_kv_heads=2, head_dim=64, num_pages=8)
+    a.update(over)
+    return pk.run_static(a.pop("seq_lens"), a.pop("query_lens"), a.pop("block_table"), a.pop("mask_kind"),
+                         a.pop("parents"), a.pop("q"), a.pop("k_cache"), a.pop("v_cache"), a.pop("out"), **a)
+
+
+def _bt(dtype="int32", shape=(2, 4)):
+    import torch
+    return torch.zeros(*shape, dtype=getattr(torch, dtype))
+
+
+@pytest.mark.parametrize("over, what", [
+    (dict(query_lens=[8]), "one entry per sequence"),
+    (dict(mask_kind=[W.CAUSAL]), "one entry per sequence"),
+    (dict(seq_lens=[40, 17, 5]), "one entry per sequence"),
+    (dict(block_table="host int32"), "block_table"),
+    (dict(block_table="host int64"), "block_table"),
+    (dict(block_table="numpy"), "block_table"),
+])
+def test_run_static_rejects_bad_host_arguments_before_the_call(over, what):
+    # the binding checks what the C side cannot see (array lengths, where and what the
+    # tensors are) and raises before it reaches the library, so no device is touched
+    bt = over.get("block_table")
+    if bt == "host int32":
+        over["block_table"] = _bt("int32")
+    elif bt == "host int64":
+        over["block_table"] = _bt("int64")
+    elif bt == "numpy":
+        over["block_table"] = np.zeros((2, 4), dtype=np.int32)
+    with pytest.raises(ValueError, match=what):
+        _static_call(**over)
+
+
+def test_verify_units_wider_than_16_rows_are_one_row_split_task():
+    """A draft tree of 5 tokens under a GQA group of 7 has 35 packed rows per KV head: one
+    task reads its pages once (no 16-row chunks re-reading them); a 64-token tree under the same
+    group (448 rows) becomes nine 48-row tasks and one 16-row task."""
+    items = pk.inspect([2000, 900], [5, 64], [W.TREE, W.TREE], [-1, 0, 0, 2, -1] + [-1] + list(range(63)),
+                       num_q_heads=28, num_kv_heads=4, head_dim=128, num_pages=200, bt_stride=125)
+    rows = sorted((it["seq"], it["kv_head"], it["row_begin"], it["row_count"]) for it in items if it["split"] <= 0)
+    assert [r for r in rows if r[0] == 0] == [(0, h, 0, 35) for h in range(4)]
+    big = [r[2:] for r in rows if r[0] == 1 and r[1] == 0]
+    assert big == [(0, 48), (48, 48), (96, 48), (144, 48), (192, 48), (240, 48), (288, 48), (336, 48),
+                   (384, 48), (432, 16)]

@@ -88,3 +88,26 @@ def test_reference_arm_prints_the_contract_line():
     assert e["value"] == d["value"] and e["unit"] == d["unit"]
     assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
     assert "workload" in d["config"]
+    # the same config object the GPU arm prints for this workload
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    b = W.make_config(bench.DEFAULT_CONFIG)
+    assert d["config"] == bench.workload_config(bench.DEFAULT_CONFIG, b, bench.DEFAULT_CONFIG, "single GPU")
+    assert d["source"]["source_sha256"]
+
+
+def test_bench_algorithmic_counts_match_the_oracle_masks():
+    """The bench's algorithmic flop count (4 * D * Hq per allowed query-key pair) against the
+    number of allowed pairs the oracle's masks give, on a batch with causal chunks and trees."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import oracle
+    import workloads as W
+    b = W.random_small(5, num_seqs=8, Hq=8, Hkv=2, d=64, max_ctx=60, max_q=20, tree_frac=0.5)
+    pairs = 0
+    for sp in b.seqs:
+        m = oracle.allowed_mask(sp.seq_len, sp.query_len, sp.mask_kind, sp.parents or None)
+        pairs += int(m.sum())
+    assert bench.batch_attn_flops(b) == pairs * b.num_q_heads * 4 * b.head_dim
+    assert bench.batch_kv_bytes(b) == sum(sp.seq_len for sp in b.seqs) * b.num_kv_heads * b.head_dim * 4

@@ -183,3 +183,39 @@ def test_fp8_append_rejects_bf16_paths():
     with pytest.raises(pk.PkvaError):
         p8.run_append(b.q, k_new, v_new, b.k_cache, b.v_cache)
     p8.close()
+
+
+@pytest.mark.parametrize("seed, heads", [(0, (16, 4)), (1, (28, 4)), (3, (64, 2)), (4, (32, 1))])
+def test_fp8_shared_prefix_small_all_rows(seed, heads):
+    """Shared-prefix groups over FP8 caches (attn_plan_shared_kv): the cascade tasks read bf16
+    copies of the shared pages, the members' own keys stay E4M3. Every row against the oracle
+    over the decoded codes; a second run is bitwise the same (arrival counters reset)."""
+    b = W.random_shared_small(seed, *heads, device=DEV)
+    f = W.fp8_kv(b)
+    plan = pk.plan_for_batch(b, kv_fp8=True)
+    assert plan.info()["num_cascade_items"] > 0
+    out = plan.run_fp8(b.q, f.k_cache, f.v_cache_t, f.k_scale, f.v_scale)
+    assert plan.check() == 0
+    rows, exp = fp8_oracle_rows(b, f)
+    assert_close(out[rows], exp, f"fp8 shared prefix seed {seed}")
+    again = plan.run_fp8(b.q, f.k_cache, f.v_cache_t, f.k_scale, f.v_scale)
+    assert plan.check() == 0
+    assert torch.equal(out, again)
+    plan.close()
+
+
+def test_fp8_shared_prefix_config_full_size():
+    b = W.make_shared_config("llama3_8b_shared_prefix", device=DEV)
+    f = W.fp8_kv(b)
+    plan = pk.plan_for_batch(b, kv_fp8=True)
+    assert plan.info()["num_cascade_items"] == 4 * 8 * 2
+    out = plan.run_fp8(b.q, f.k_cache, f.v_cache_t, f.k_scale, f.v_scale)
+    assert plan.check() == 0
+    rows, exp = fp8_oracle_rows(b, f, seq_ids=list(range(0, len(b.seqs), 5)),
+                                token_picker=lambda sp: sorted({0, sp.query_len - 1}))
+    assert_close(out[rows], exp, "fp8 llama3_8b_shared_prefix")
+    plan.close()
+
+
+def test_fp8_shared_prefix_with_fused_append():
+    _fp8_append_case(W.random_shared_small(5, 16, 4, device=DEV), expect_prefill=True)

@@ -184,21 +184,30 @@ FULL = ["llama3_8b_decode", "qwen2_7b_unified", "long_ctx_split", "llama33_70b_p
 
 @pytest.mark.parametrize("name", FULL)
 def test_full_size_config_sampled(name):
+    """The full-size batches in the launch configuration the benchmark times, against the
+    oracle on: every sequence of the 70B prefill batch at the tile and task boundaries
+    (tokens 0, 127 / 128, 255 / 256, 511 / 512 and the last), every sequence of the
+    long-context batch, 32 of the Llama-3-8B decode sequences, and on the unified batch every
+    prefill chunk at its boundaries, every verify tree and 32 decode sequences."""
     b = W.make_config(name, device=DEV)
     out, plan = run_batch(b)
     n = len(b.seqs)
+    picker = None
     if name == "llama33_70b_prefill":
-        seq_ids = [0, 5]
-        picker = lambda sp: [0, 1, 127, 128, 1000, sp.query_len - 1]
+        seq_ids = list(range(n))
+        picker = lambda sp: [0, 127, 128, 255, 256, 511, 512, sp.query_len - 1]
     elif name == "qwen2_7b_unified":
-        seq_ids = [0, 3, 4, 100, n - 32, n - 1]
-        picker = None
+        kinds = [W.seq_class(sp) for sp in b.seqs]
+        pre = [i for i, k in enumerate(kinds) if k == "prefill"]
+        ver = [i for i, k in enumerate(kinds) if k == "verify"]
+        dec = [i for i, k in enumerate(kinds) if k == "decode"]
+        rows, exp = oracle_rows(b, pre, lambda sp: [0, 127, 128, 255, 256, sp.query_len - 1])
+        assert_close(out[rows], exp, f"{name} prefill chunks")
+        seq_ids = ver + dec[::len(dec) // 32][:32]
     elif name == "long_ctx_split":
-        seq_ids = [0, 7, 15]
-        picker = None
+        seq_ids = list(range(n))
     else:
-        seq_ids = [0, 31, 64, 127]
-        picker = None
+        seq_ids = list(range(0, n, n // 32))[:32]
     rows, exp = oracle_rows(b, seq_ids, picker)
     assert_close(out[rows], exp, name)
     # every output row is finite
