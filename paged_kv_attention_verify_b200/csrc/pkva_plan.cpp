@@ -24,8 +24,10 @@ constexpr int kMinSplitPages = 8;      // never split a unit into tasks below 12
 constexpr int kTasksPerSlot = 1;       // split long units down to about one task per CTA slot
 // A row-split task's warps each run every page of the task, where a 16-row task's four warps
 // share its pages: it gets a quarter of the pages of a 16-row task, so that its warps' page
-// chains are as long as theirs.
+// chains are as long as theirs, but no fewer than kMinWidePages (a task's set-up and the
+// merge of its chunks' partials would outweigh shorter chains).
 constexpr int kWideSplit = 4;
+constexpr int kMinWidePages = 32;
 
 int fail(std::string* err, int code, const char* fmt, long a = 0, long b = 0, long c = 0) {
     char buf[256];
@@ -208,7 +210,25 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
     // has wrows = rc. All chunks of a row-split task share its page range.
     struct Unit { int seq, kvh, rb, rc, pstart, pages, cs, wrows; };
     std::vector<Unit> units;
-    const bool wide = a.wide_tasks && a.kv_elem_bytes == 2;
+    // Row-split tasks pay off for units of three or more 16-row chunks (each page then read
+    // once instead of three times) in a batch where such units are a minority of the
+    // decode/verify pages: there the other tasks keep the SMs busy while the row-split
+    // tasks' warps each run all of their pages; a batch made mostly of such units keeps the
+    // 16-row tasks, whose four warps share a unit's pages (measured on B200: a verify-only
+    // batch took 2.4x longer with row-split tasks, the mixed batch 9 % less time).
+    bool wide = a.wide_tasks && a.kv_elem_bytes == 2;
+    if (wide) {
+        int64_t wide_pages = 0, all_pages = 0;
+        for (int s = 0; s < a.num_seqs; ++s) {
+            if (on_prefill[s]) continue;
+            const SeqInfo& si = p.seqs[s];
+            const int64_t pg = (int64_t)(si.seq_len + kPageSize - 1) / kPageSize -
+                               (grp_of[s] >= 0 ? a.prefix_len[grp_of[s]] / kPageSize : 0);
+            all_pages += pg;
+            if (si.query_len * p.G > 2 * kDecodeRowsMax) wide_pages += pg;
+        }
+        wide = 2 * wide_pages <= all_pages;
+    }
     std::vector<int> unit_base(a.num_seqs, -1);     // index of (s, head 0, chunk 0) in units
     std::vector<char> on_cascade(a.num_seqs, 0);
     int64_t total_pages = 0;
@@ -234,11 +254,14 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
         for (int h = 0; h < a.Hkv; ++h) {
             for (int tb = 0; tb < rows; tb += wide ? kWideRowsMax : kDecodeRowsMax) {
                 const int tr = std::min(wide ? kWideRowsMax : kDecodeRowsMax, rows - tb);
-                if (tr <= kDecodeRowsMax) {
-                    const int pages = pages_to(tb + tr - 1);
-                    units.push_back({s, h, tb, tr, pstart, pages, cs, tr});
-                    total_pages += pages - pstart;
-                    max_rc = std::max(max_rc, tr);
+                if (tr <= 2 * kDecodeRowsMax) {          // one or two 16-row tasks
+                    for (int rb = tb; rb < tb + tr; rb += kDecodeRowsMax) {
+                        const int rc = std::min(kDecodeRowsMax, tb + tr - rb);
+                        const int pages = pages_to(rb + rc - 1);
+                        units.push_back({s, h, rb, rc, pstart, pages, cs, rc});
+                        total_pages += pages - pstart;
+                        max_rc = std::max(max_rc, rc);
+                    }
                     continue;
                 }
                 // one row-split task: its 16-row chunks, the whole row range's pages
@@ -288,8 +311,8 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
         const int nchunks = (u.wrows + kDecodeRowsMax - 1) / kDecodeRowsMax;
         // nearest whole number of target-sized tasks (rounding up made near-target units two
         // half-size tasks), never more pages per task than the staged block-table slice holds
-        const int64_t cost = nchunks > 1 ? (int64_t)own * kWideSplit : own;
-        const int ns = std::max<int>(std::max<int>(1, (int)((cost + target / 2) / target)),
+        const int64_t per_task = nchunks > 1 ? std::max<int64_t>(target / kWideSplit, kMinWidePages) : target;
+        const int ns = std::max<int>(std::max<int>(1, (int)((own + per_task / 2) / per_task)),
                                      (own + kDecodeMaxPages - 1) / kDecodeMaxPages);
         int unit_id = -1;                     // the lead chunk's; chunk c has unit_id + c
         for (int c = 0; c < nchunks; ++c) {

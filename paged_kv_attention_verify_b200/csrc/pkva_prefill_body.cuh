@@ -63,7 +63,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;
 constexpr float kRescaleSlack = 8.f;
 constexpr int kWarpKProd = 8, kWarpMma = 9, kWarpVProd = 10;
-constexpr bool kSpinOnS = true;    // softmax warps poll S without suspending
+constexpr bool kSpinOnS = false;   // softmax warps wait for S suspended (polling took issue slots from the other tile)
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);   // Q, K both K-major
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);    // P from TMEM, V MN-major

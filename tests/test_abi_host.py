@@ -285,14 +285,25 @@ def test_run_static_rejects_bad_host_arguments_before_the_call(over, what):
         _static_call(**over)
 
 
-def test_verify_units_wider_than_16_rows_are_one_row_split_task():
-    """A draft tree of 5 tokens under a GQA group of 7 has 35 packed rows per KV head: one
-    task reads its pages once (no 16-row chunks re-reading them); a 64-token tree under the same
-    group (448 rows) becomes nine 48-row tasks and one 16-row task."""
-    items = pk.inspect([2000, 900], [5, 64], [W.TREE, W.TREE], [-1, 0, 0, 2, -1] + [-1] + list(range(63)),
-                       num_q_heads=28, num_kv_heads=4, head_dim=128, num_pages=200, bt_stride=125)
+def test_verify_units_wider_than_32_rows_are_row_split_tasks_in_mixed_batches():
+    """In a batch of mostly decode steps, a draft tree of 5 tokens under a GQA group of 7 has
+    35 packed rows per KV head: one task reads its pages once (no 16-row chunks re-reading
+    them); a 64-token tree under the same group (448 rows) becomes nine 48-row tasks and one
+    16-row task; a tree of 20 rows stays two 16-row tasks. A batch made only of such trees
+    keeps 16-row tasks throughout."""
+    lens = [2000, 900, 700] + [3000] * 20
+    qlens = [5, 64, 3] + [1] * 20
+    kinds = [W.TREE, W.TREE, W.TREE] + [W.CAUSAL] * 20
+    parents = [-1, 0, 0, 2, -1] + [-1] + list(range(63)) + [-1, 0, 1]
+    pages = sum((L + 15) // 16 for L in lens)
+    items = pk.inspect(lens, qlens, kinds, parents, num_q_heads=28, num_kv_heads=4, head_dim=128,
+                       num_pages=pages, bt_stride=200)
     rows = sorted((it["seq"], it["kv_head"], it["row_begin"], it["row_count"]) for it in items if it["split"] <= 0)
     assert [r for r in rows if r[0] == 0] == [(0, h, 0, 35) for h in range(4)]
     big = [r[2:] for r in rows if r[0] == 1 and r[1] == 0]
     assert big == [(0, 48), (48, 48), (96, 48), (144, 48), (192, 48), (240, 48), (288, 48), (336, 48),
                    (384, 48), (432, 16)]
+    assert [r[2:] for r in rows if r[0] == 2 and r[1] == 0] == [(0, 16), (16, 5)]
+    only = pk.inspect(lens[:3], qlens[:3], kinds[:3], parents, num_q_heads=28, num_kv_heads=4, head_dim=128,
+                      num_pages=pages, bt_stride=200)
+    assert max(it["row_count"] for it in only) == 16

@@ -129,3 +129,20 @@ def test_append_argument_checks():
                            b.v_cache.data_ptr(), b.q.data_ptr(), None)
     assert rc == -1 and b"k_new" in L.attn_last_error()
     plan.close()
+
+
+def test_append_with_row_split_verify_tasks():
+    """A mixed batch whose verify trees (5 tokens x 7 heads = 35 packed rows per KV head) run
+    as row-split tasks, one of them split over its long context: the append patches the new
+    rows into the pages every consumer warp reads, and one task per (sequence, KV head) writes
+    the cache."""
+    gen = torch.Generator().manual_seed(8)
+    seqs = [W.SeqSpec(2500, 1, W.CAUSAL, []) for _ in range(6)] + \
+        [W.SeqSpec(9000 + 5, 5, W.TREE, W.random_tree(gen, 5)), W.SeqSpec(300 + 5, 5, W.TREE, W.random_tree(gen, 5))]
+    b = W.build_batch("append_row_split", seqs, 28, 4, 128, seed=81, device=DEV)
+    items = pk.inspect(b.seq_lens, b.query_lens, b.mask_kinds, b.parents_flat, num_q_heads=28, num_kv_heads=4,
+                       head_dim=128, num_pages=b.k_cache.shape[0], bt_stride=b.block_table.shape[1],
+                       num_sms=torch.cuda.get_device_properties(0).multi_processor_count, ctas_per_sm=3)
+    wide = [it for it in items if it["row_count"] > 16]
+    assert wide and any(it["num_splits"] > 1 for it in wide)
+    run_append_case(b, expect_identical=True)

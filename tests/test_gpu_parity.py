@@ -233,3 +233,27 @@ def test_unified_batch_classes_alone():
         rows, exp = oracle_rows(p, seq_ids, picker)
         assert_close(out[rows], exp, f"qwen2_7b_unified[{cls}]")
         plan.close()
+
+
+def test_row_split_verify_tasks_all_rows():
+    """Verify trees of 35 and 48 packed rows per KV head among decode steps run as row-split
+    tasks (one warp streams each page once, three own 16 rows each), split over long contexts
+    and not; trees of 80 and 96 rows (group 16) as a 48-row task plus 16-row or 48-row ones.
+    Every row against the oracle, and a second run is bitwise the same."""
+    gen = torch.Generator().manual_seed(9)
+    seqs = [W.SeqSpec(3000 + 7 * i, 1, W.CAUSAL, []) for i in range(8)] + \
+        [W.SeqSpec(12000 + 5, 5, W.TREE, W.random_tree(gen, 5)), W.SeqSpec(600 + 5, 5, W.TREE, W.random_tree(gen, 5)),
+         W.SeqSpec(37 + 6, 6, W.TREE, W.random_tree(gen, 6))]
+    for Hq, Hkv in ((28, 4), (32, 2)):        # 35 / 42 rows; 80 / 96 rows (48-row tasks plus 16-row ones)
+        b = W.build_batch("row_split", seqs, Hq, Hkv, 128, seed=91, device=DEV)
+        items = pk.inspect(b.seq_lens, b.query_lens, b.mask_kinds, b.parents_flat, num_q_heads=Hq,
+                           num_kv_heads=b.num_kv_heads, head_dim=128, num_pages=b.k_cache.shape[0],
+                           bt_stride=b.block_table.shape[1],
+                           num_sms=torch.cuda.get_device_properties(0).multi_processor_count, ctas_per_sm=3)
+        assert any(it["row_count"] > 16 for it in items)
+        out, plan = run_batch(b)
+        rows, exp = oracle_rows(b)
+        assert_close(out[rows], exp, f"row-split Hq={Hq} Hkv={Hkv}")
+        again = plan.run(b.q, b.k_cache, b.v_cache)
+        assert plan.check() == 0
+        assert torch.equal(out, again)
