@@ -46,6 +46,8 @@ struct AttnNS {
 template <int D, int NT, bool FP8 = false, bool TC = true>
 struct AttnSmem {
     using DC = dec::DecodeCfg<D, NT * 8, false, kDecWarps, AttnNS<D, FP8>::value, FP8 ? 1 : 2>;
+    static_assert(dec::DecodeCfg<D, 8, false, kDecWarps, AttnNS<D, FP8>::value, FP8 ? 1 : 2>::BYTES <= DC::BYTES,
+                  "one-n-tile tasks fit a task's share");
     static constexpr int GROUP_BYTES = (DC::BYTES + 1023) / 1024 * 1024;    // one decode task
     static constexpr int DEC_BYTES = kDecTasksPerBlock * GROUP_BYTES;
     static constexpr int TASK_BYTES = (D == 128 && TC && pre::kSmemBytes > DEC_BYTES) ? pre::kSmemBytes : DEC_BYTES;
@@ -100,6 +102,15 @@ attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const _
         // more than 16 packed rows (a draft tree times the GQA group): one pass over the pages
         if (p.dec.work[task].row_count > kDecodeRowsMax) {
             dec::decode_wide_task<D, S::WIDE_NS>(grp, p.dec, task, tmK, tmV, sm + g * S::GROUP_BYTES);
+            return;
+        }
+    }
+    if constexpr (NT == 2) {
+        // a launch compiled for 16-row tasks runs its tasks of at most 8 rows (decode steps
+        // beside 16-row verify chunks) on the one-n-tile body
+        if (p.dec.work[task].row_count <= 8) {
+            dec::decode_mma_task<D, 1, kDecWarps, AttnNS<D, FP8>::value, FP8>(grp, p.dec, task, tmK, tmV,
+                                                                           sm + g * S::GROUP_BYTES);
             return;
         }
     }
