@@ -14,7 +14,6 @@ constexpr int kDecodeRowsMax = 16;     // packed (token, head) rows per decode t
 constexpr int kWideRowsMax = 48;       // packed rows per row-split (wide) decode/verify task
 constexpr int kDecodeMaxPages = 1024;  // pages per decode task (block-table slice in smem)
 constexpr int kPrefillTileM = 128;     // query tokens per prefill tile (tcgen05 M)
-constexpr int kPrefillTaskTokens = 256; // query tokens per prefill task (two tiles, ping-pong)
 constexpr int kPrefillTileN = 128;     // keys per prefill KV tile (8 pages)
 constexpr int kDecTasksPerBlock = 3;   // decode tasks side by side in one block of the unified kernel
 constexpr int kPrefillMinTokens = 64;  // causal sequences with at least this many new tokens
@@ -48,14 +47,20 @@ struct DecodeWork {
 };
 static_assert(sizeof(DecodeWork) == 32, "DecodeWork layout");
 
-// One prefill task: up to 256 query tokens [tok0, tok0 + ntok) of one query head, as two
-// 128-token tiles; tile 0 needs KV tiles [0, kv_tiles0) of 128 keys, tile 1 [0, kv_tiles1)
-// (0 when the task has at most 128 tokens).
+// One prefill task: two tcgen05 query tiles of up to 128 tokens each, of query heads that
+// share one KV head: tile 0 holds tokens [tok0, tok0 + ntok0) of q_head, tile 1 tokens
+// [tok1, tok1 + ntok1) of q_head1 (ntok1 = 0: no tile 1). Usually the two tiles are two heads
+// of one token tile (they need the same KV tiles); a head left over in an odd group pairs
+// two consecutive token tiles of its own. Tile 0 needs KV tiles [0, kv_tiles0) of 128 keys,
+// tile 1 [0, kv_tiles1).
 struct PrefillWork {
     int32_t seq;
     int32_t q_head;
     int32_t tok0;
-    int32_t ntok;
+    int32_t ntok0;
+    int32_t q_head1;
+    int32_t tok1;
+    int32_t ntok1;
     int32_t kv_tiles0;
     int32_t kv_tiles1;
     // with a fused KV append, keys come from the cache for the committed prefix (tiles
@@ -63,8 +68,9 @@ struct PrefillWork {
     // chunk start): the tile counts of the two query tiles in that mode
     int32_t kv_tiles0_append;
     int32_t kv_tiles1_append;
+    int32_t pad;
 };
-static_assert(sizeof(PrefillWork) == 32, "PrefillWork layout");
+static_assert(sizeof(PrefillWork) == 48, "PrefillWork layout");
 
 // A (seq, kv_head, row chunk) whose keys are split over several tasks: where its partials
 // live, how many task arrivals complete it, and which output rows it owns (so that any

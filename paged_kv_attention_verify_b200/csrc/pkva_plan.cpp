@@ -170,33 +170,47 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
             if (si.mask_kind != PKVA_CAUSAL || si.query_len < kPrefillMinTokens) continue;
             on_prefill[s] = 1;
             const int prefix = si.seq_len - si.query_len;
-            for (int t0 = 0; t0 < si.query_len; t0 += kPrefillTaskTokens) {
-                const int ntok = std::min(kPrefillTaskTokens, si.query_len - t0);
-                // each tile needs keys up to its last row's own position (causal tile skipping)
-                const int n0tok = std::min(kPrefillTileM, ntok);
-                const int tiles0 = (prefix + t0 + n0tok + kPrefillTileN - 1) / kPrefillTileN;
-                const int tiles1 =
-                    ntok > kPrefillTileM ? (prefix + t0 + ntok + kPrefillTileN - 1) / kPrefillTileN : 0;
-                const int cache_tiles = (prefix + kPrefillTileN - 1) / kPrefillTileN;
-                const int tiles0_app = cache_tiles + (t0 + n0tok - 1) / kPrefillTileN + 1;
-                const int tiles1_app =
-                    ntok > kPrefillTileM ? cache_tiles + (t0 + ntok - 1) / kPrefillTileN + 1 : 0;
-                for (int h = 0; h < a.Hq; ++h) {
-                    PrefillWork pw{};
-                    pw.seq = s;
-                    pw.q_head = h;
-                    pw.tok0 = t0;
-                    pw.ntok = ntok;
-                    pw.kv_tiles0 = tiles0;
-                    pw.kv_tiles1 = tiles1;
-                    pw.kv_tiles0_append = tiles0_app;
-                    pw.kv_tiles1_append = tiles1_app;
-                    p.pwork.push_back(pw);
+            const int cache_tiles = (prefix + kPrefillTileN - 1) / kPrefillTileN;
+            const int ntt = (si.query_len + kPrefillTileM - 1) / kPrefillTileM;     // token tiles
+            auto ntok_of = [&](int tt) { return std::min(kPrefillTileM, si.query_len - tt * kPrefillTileM); };
+            // each tile needs keys up to its last row's own position (causal tile skipping)
+            auto tiles_of = [&](int tt) {
+                return (prefix + tt * kPrefillTileM + ntok_of(tt) + kPrefillTileN - 1) / kPrefillTileN;
+            };
+            auto tiles_app_of = [&](int tt) {
+                return cache_tiles + (tt * kPrefillTileM + ntok_of(tt) - 1) / kPrefillTileN + 1;
+            };
+            auto add = [&](int h0, int tt0, int h1, int tt1) {    // tt1 < 0: no tile 1
+                PrefillWork pw{};
+                pw.seq = s;
+                pw.q_head = h0;
+                pw.tok0 = tt0 * kPrefillTileM;
+                pw.ntok0 = ntok_of(tt0);
+                pw.kv_tiles0 = tiles_of(tt0);
+                pw.kv_tiles0_append = tiles_app_of(tt0);
+                if (tt1 >= 0) {
+                    pw.q_head1 = h1;
+                    pw.tok1 = tt1 * kPrefillTileM;
+                    pw.ntok1 = ntok_of(tt1);
+                    pw.kv_tiles1 = tiles_of(tt1);
+                    pw.kv_tiles1_append = tiles_app_of(tt1);
+                } else {                                   // an absent tile loads (unused) rows past tile 0
+                    pw.q_head1 = h0;
+                    pw.tok1 = pw.tok0 + kPrefillTileM;
                 }
-            }
+                p.pwork.push_back(pw);
+            };
+            // pairs of query heads of one KV head on the same token tile; in an odd group the
+            // last head pairs consecutive token tiles of its own
+            for (int tt = 0; tt < ntt; ++tt)
+                for (int kvh = 0; kvh < a.Hkv; ++kvh) {
+                    const int h0 = kvh * p.G;
+                    for (int i = 0; i + 1 < p.G; i += 2) add(h0 + i, tt, h0 + i + 1, tt);
+                    if ((p.G & 1) && (tt & 1) == 0) add(h0 + p.G - 1, tt, h0 + p.G - 1, tt + 1 < ntt ? tt + 1 : -1);
+                }
         }
-        // heaviest first; equal work keeps (seq, tile, head) order so that the query heads
-        // of one GQA group run side by side and share their K/V tiles through L2
+        // heaviest first; equal work keeps (seq, token tile, KV head) order so that the query
+        // heads of one GQA group run side by side and share their K/V tiles through L2
         std::stable_sort(p.pwork.begin(), p.pwork.end(), [](const PrefillWork& x, const PrefillWork& y) {
             return x.kv_tiles0 + x.kv_tiles1 > y.kv_tiles0 + y.kv_tiles1;
         });
@@ -506,7 +520,9 @@ extern "C" int attn_plan_inspect(int num_seqs, const int32_t* seq_lens, const in
         set_last_error(err);
         return rc;
     }
-    const int np = (int)hp.pwork.size();
+    // prefill tasks are listed one entry per query tile (a task holds one or two)
+    int np = 0;
+    for (const PrefillWork& w : hp.pwork) np += w.ntok1 > 0 ? 2 : 1;
     const int nc = (int)hp.cwork.size();
     const int n = np + nc + (int)hp.dwork.size();
     if (num_items) *num_items = n;
@@ -515,21 +531,24 @@ extern "C" int attn_plan_inspect(int num_seqs, const int32_t* seq_lens, const in
         set_last_error("attn_plan_inspect: max_items is smaller than the number of tasks");
         return PKVA_EINVAL;
     }
-    for (int i = 0; i < np; ++i) {      // prefill tasks first
-        const PrefillWork& w = hp.pwork[i];
+    int ip = 0;
+    for (const PrefillWork& w : hp.pwork) {      // prefill tiles first
         const SeqInfo& si = hp.seqs[w.seq];
-        pkva_work_desc d;
-        d.kind = 1;
-        d.seq = w.seq;
-        d.kv_head = w.q_head / hp.G;
-        d.q_head = w.q_head;
-        d.row_begin = w.tok0;
-        d.row_count = w.ntok;
-        d.key_begin = 0;
-        d.key_end = std::min(si.seq_len - si.query_len + w.tok0 + w.ntok, si.seq_len);
-        d.split = -1;
-        d.num_splits = 1;
-        items[i] = d;
+        for (int b = 0; b < (w.ntok1 > 0 ? 2 : 1); ++b) {
+            const int h = b ? w.q_head1 : w.q_head, t0 = b ? w.tok1 : w.tok0, nt = b ? w.ntok1 : w.ntok0;
+            pkva_work_desc d;
+            d.kind = 1;
+            d.seq = w.seq;
+            d.kv_head = h / hp.G;
+            d.q_head = h;
+            d.row_begin = t0;
+            d.row_count = nt;
+            d.key_begin = 0;
+            d.key_end = std::min(si.seq_len - si.query_len + t0 + nt, si.seq_len);
+            d.split = -1;
+            d.num_splits = 1;
+            items[ip++] = d;
+        }
     }
     for (int i = 0; i < nc; ++i) {      // then shared-prefix tasks
         const CascadeWork& w = hp.cwork[i];

@@ -2,10 +2,11 @@
 // (K-P): S = Q K^T and O += P V are tcgen05.mma BF16 tiles with fp32 accumulators in
 // tensor memory (TMEM).
 //
-// One CTA runs one task: up to 256 query tokens of one query head, as two 128-token tiles
-// (tcgen05 M = 128) that share every 128-key KV tile (8 pages, gathered by TMA through the
-// block table). KV tiles past a tile's last row are never loaded (causal tile skipping)
-// and only tiles that cross the diagonal are masked element by element.
+// One CTA runs one task: two 128-token query tiles (tcgen05 M = 128) of query heads that
+// share one KV head (two heads on the same tokens, or one head's two consecutive token
+// tiles), sharing every 128-key KV tile (8 pages, gathered by TMA through the block
+// table). KV tiles past a tile's last row are never loaded (causal tile skipping) and only
+// tiles that cross the diagonal are masked element by element.
 //
 // Warp roles (352 threads):
 //   warps 0-3, 4-7  two softmax warpgroups, one per query tile: thread r owns row r =
@@ -171,7 +172,7 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         cw = p.cwork[ci];
         w.seq = cw.lead_seq;
         w.tok0 = cw.tok0;
-        w.ntok = cw.ntok;
+        w.ntok0 = cw.ntok;
     } else {
         w = p.work[task];
     }
@@ -240,14 +241,13 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
                 prefetch_tensormap(&tmQ);
                 prefetch_tensormap(&tmK);
                 if (append) prefetch_tensormap(&tmKn);
-                const int qrow0 = si.q_start + w.tok0;
                 mbar_arrive_expect_tx(B.q_full, 2 * kTileBytes);
 #pragma unroll
                 for (int b = 0; b < 2; ++b)
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
                         tma_load_3d(sm + kOffQ + b * kTileBytes + h * kHalfBytes, &tmQ, B.q_full, h * 64,
-                                    w.q_head, qrow0 + b * kPrefillTileM);
+                                    b ? w.q_head1 : w.q_head, si.q_start + (b ? w.tok1 : w.tok0));
             } else {
                 prefetch_tensormap(&tmV);
                 if (append) prefetch_tensormap(&tmVn);
@@ -378,7 +378,11 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         const uint32_t s_addr = tmem + lane_off + kColS + b * 128;
         const uint32_t o_addr = tmem + lane_off + kColO + b * 128;
         const int row_in_task = b * kPrefillTileM + r;
-        const int tok = w.tok0 + row_in_task;
+        // this tile's query head and tokens (a cascade task's rows come from its row map)
+        const int qh = b ? w.q_head1 : w.q_head;
+        const int tok0_b = b ? w.tok1 : w.tok0;
+        const int ntok_b = b ? w.ntok1 : w.ntok0;
+        const int tok = tok0_b + r;
         // Per KV tile j: its first key kb and the last key this row (lim) and the tile's
         // first row (lim_first) may see. Tiles [0, na) are cache tiles j + jbase with limits
         // (lim_a, lim_first_a); append mode's new tiles j >= na are indexed from the chunk
@@ -388,9 +392,9 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         //           keys up to its own token index;
         //   cascade: every shared key (below key_limit) is visible.
         const int na = append ? nc : nmax;
-        const int lim_first_b = w.tok0 + b * kPrefillTileM, lim_b = tok;
+        const int lim_first_b = tok0_b, lim_b = tok;
         const int lim_first_a = cascade || append ? key_limit - 1 : prefix + lim_first_b;
-        const int lim_a = cascade || append ? key_limit - 1 : (row_in_task < w.ntok ? prefix + tok : 0x7fffffff);
+        const int lim_a = cascade || append ? key_limit - 1 : (r < ntok_b ? prefix + tok : 0x7fffffff);
         // FP8 caches: the tiles hold the codes' values, so the K scale of this KV head joins
         // the softmax scale (and the V scale the output, below)
         const float sl2 = p.k_scale ? p.scale_log2 * p.k_scale[kvh] : p.scale_log2;
@@ -538,10 +542,10 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         // ---- epilogue: O / l -> bf16 rows --------------------------------------------------
         else if (nb > 0 && alive && __all_sync(0xffffffffu, wait_or_abort(&B.o_ready[b], 0, p.err, abort_flag))) {
             tc_fence_after();
-            const bool real_row = row_in_task < w.ntok;
+            const bool real_row = r < ntok_b;
             float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
             if (p.v_scale) inv *= p.v_scale[kvh];
-            __nv_bfloat16* dst = p.out + ((int64_t)(si.q_start + tok) * p.Hq + w.q_head) * kD;
+            __nv_bfloat16* dst = p.out + ((int64_t)(si.q_start + tok) * p.Hq + qh) * kD;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t ov[32];
@@ -562,12 +566,16 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         }
     } else if (append) {
         // ------------------- warp 11: this task's share of the cache writes -------------------
-        // the G query-head tasks of one KV head and token range each write 1/G of its rows
-        const int gi = w.q_head % p.G;
-        const int t_begin = w.tok0 + (int)((int64_t)w.ntok * gi / p.G);
-        const int t_end = w.tok0 + (int)((int64_t)w.ntok * (gi + 1) / p.G);
-        append_rows<kD>(p.k_new, p.v_new, p.k_cache, p.v_cache, p.block_table, p.bt_stride, p.num_pages, p.Hkv,
-                        p.err, si, w.seq, kvh, t_begin, t_end, lane, 32);
+        // the G query tiles (one per head of the KV head) on a token tile each write 1/G of its
+        // rows; a task does the shares of both its tiles
+        for (int b = 0; b < 2; ++b) {
+            const int nt = b ? w.ntok1 : w.ntok0, t0 = b ? w.tok1 : w.tok0;
+            const int gi = (b ? w.q_head1 : w.q_head) % p.G;
+            const int t_begin = t0 + (int)((int64_t)nt * gi / p.G);
+            const int t_end = t0 + (int)((int64_t)nt * (gi + 1) / p.G);
+            append_rows<kD>(p.k_new, p.v_new, p.k_cache, p.v_cache, p.block_table, p.bt_stride, p.num_pages,
+                            p.Hkv, p.err, si, w.seq, kvh, t_begin, t_end, lane, 32);
+        }
     }
     // all roles done (the MMA thread waited for its last MMA): TMEM and shared memory are
     // free for the block's next task
