@@ -377,7 +377,7 @@ PKVA_API int pkva_selftest_wait_timeout(long long limit_ns, int32_t* device_erro
 typedef struct pkva_plan_info {
     int32_t num_seqs;
     int32_t num_decode_items;    /* decode/verify tile tasks (one block each)              */
-    int32_t num_prefill_items;   /* prefill tile tasks (one block each, 256 tokens, 1 head)  */
+    int32_t num_prefill_items;   /* prefill tasks (one block each: two 128-token tiles)       */
     int32_t num_split_units;     /* (seq, kv head, row chunk) units split over several CTAs */
     int32_t num_partial_slots;   /* split-KV partial results held in plan scratch           */
     int32_t decode_rows;         /* rows per decode task the launch is compiled for         */
@@ -392,7 +392,8 @@ PKVA_API int attn_plan_get_info(pkva_plan_t plan, pkva_plan_info* info);
 
 /* One tile task as the planner emitted it (host-side inspection only). */
 typedef struct pkva_work_desc {
-    int32_t kind;        /* 0 = decode/verify task, 1 = prefill task, 2 = shared-prefix     */
+    int32_t kind;        /* 0 = decode/verify task, 1 = one query tile of a prefill task,  */
+                         /* 2 = shared-prefix                                               */
                          /* (cascade) task: all heads of kv_head for q rows [row_begin,    */
                          /* row_begin + row_count) of consecutive group members, keys      */
                          /* [key_begin, key_end) of the shared prefix; split / num_splits  */
@@ -412,8 +413,9 @@ typedef struct pkva_work_desc {
 
 /*
  * attn_plan_inspect — run the planner on the host only (no device, nothing allocated on
- * it) and return its tile tasks grouped by kind: prefill tasks, then shared-prefix tasks,
- * then decode/verify tasks, each in the planner's order (heaviest first; the single launch
+ * it) and return its tile tasks grouped by kind: prefill tasks (one entry per query tile; a
+ * task holds two), then shared-prefix tasks, then decode/verify tasks (a row-split task of
+ * up to 48 packed rows is one entry), each in the planner's order (heaviest first; the single launch
  * interleaves the tensor-core and decode/verify lists in proportion, three decode/verify
  * tasks to a block). Arguments as attn_plan_shared (prefix_group / prefix_len may be NULL
  * with num_groups 0), plus:
