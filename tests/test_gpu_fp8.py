@@ -219,3 +219,37 @@ def test_fp8_shared_prefix_config_full_size():
 
 def test_fp8_shared_prefix_with_fused_append():
     _fp8_append_case(W.random_shared_small(5, 16, 4, device=DEV), expect_prefill=True)
+
+
+def _large_tree_seqs():
+    gen = torch.Generator().manual_seed(9)
+    return [W.SeqSpec(3000 + 7 * i, 1, W.CAUSAL, []) for i in range(8)] + \
+        [W.SeqSpec(12000 + 5, 5, W.TREE, W.random_tree(gen, 5)), W.SeqSpec(600 + 5, 5, W.TREE, W.random_tree(gen, 5)),
+         W.SeqSpec(37 + 6, 6, W.TREE, W.random_tree(gen, 6))]
+
+
+@pytest.mark.parametrize("Hq, Hkv, d", [(28, 4, 128), (32, 2, 128), (32, 2, 64)])
+def test_fp8_large_verify_trees_all_rows(Hq, Hkv, d):
+    """Verify trees of 35 to 96 packed rows per KV head among decode steps, over FP8 caches (the
+    planner keeps 16-row tasks there: row-split tasks measured slower over E4M3 pages). Every row
+    against the oracle over the codes, and a second run is bitwise the same."""
+    b = W.build_batch("large_trees_fp8", _large_tree_seqs(), Hq, Hkv, d, seed=92, device=DEV)
+    items = pk.inspect(b.seq_lens, b.query_lens, b.mask_kinds, b.parents_flat, num_q_heads=Hq,
+                       num_kv_heads=Hkv, head_dim=d, num_pages=b.k_cache.shape[0],
+                       bt_stride=b.block_table.shape[1],
+                       num_sms=torch.cuda.get_device_properties(0).multi_processor_count, ctas_per_sm=3)
+    assert any(it["row_count"] > 16 for it in items)
+    f = W.fp8_kv(b)
+    out, plan = run_fp8(b, f)
+    rows, exp = fp8_oracle_rows(b, f)
+    assert_close(out[rows], exp, f"fp8 large trees Hq={Hq} Hkv={Hkv} d={d}")
+    again = plan.run_fp8(b.q, f.k_cache, f.v_cache_t, f.k_scale, f.v_scale)
+    assert plan.check() == 0
+    assert torch.equal(out, again)
+    plan.close()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp8_append_with_large_verify_trees(d):
+    b = W.build_batch("large_trees_fp8_append", _large_tree_seqs(), 28, 4, d, seed=93, device=DEV)
+    _fp8_append_case(b)
