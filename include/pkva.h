@@ -397,7 +397,14 @@ typedef struct pkva_work_desc {
                          /* (cascade) task: all heads of kv_head for q rows [row_begin,    */
                          /* row_begin + row_count) of consecutive group members, keys      */
                          /* [key_begin, key_end) of the shared prefix; split / num_splits  */
-                         /* count the cascade chunks of the prefix only                    */
+                         /* count the cascade chunks of the prefix only. The same kind     */
+                         /* lists the tensor-core verify tasks: a verify tree (or causal   */
+                         /* chunk) of 17 to 128 packed rows per KV head, outside any       */
+                         /* caller group, with at least 512 keys runs as such tasks over   */
+                         /* all of its keys (masked), chunks of 16 KV tiles of 128 keys,   */
+                         /* and has no decode/verify task (head_dim 128, bf16 caches), in  */
+                         /* a batch where such sequences hold at most half of the          */
+                         /* decode/verify pages                                            */
     int32_t seq;         /* sequence index (cascade: the group's first member in the run)  */
     int32_t kv_head;     /* KV head whose keys and values the task reads                   */
     int32_t q_head;      /* prefill: the one query head; decode/verify: -1 (all heads of   */
@@ -413,8 +420,8 @@ typedef struct pkva_work_desc {
 
 /*
  * attn_plan_inspect — run the planner on the host only (no device, nothing allocated on
- * it) and return its tile tasks grouped by kind: prefill tasks (one entry per query tile; a
- * task holds two), then shared-prefix tasks, then decode/verify tasks (a row-split task of
+ * it) and return its tile tasks grouped by kind: shared-prefix tasks, then prefill tasks (one
+ * entry per query tile; a task holds two), then decode/verify tasks (a row-split task of
  * up to 48 packed rows is one entry), each in the planner's order (heaviest first; the single launch
  * interleaves the tensor-core and decode/verify lists in proportion, three decode/verify
  * tasks to a block). Arguments as attn_plan_shared (prefix_group / prefix_len may be NULL

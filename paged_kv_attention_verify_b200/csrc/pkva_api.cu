@@ -239,6 +239,7 @@ static int plan_create(pkva_plan_t* out_plan, PlanArgs a, const int32_t* block_t
     const int num_seqs = a.num_seqs, head_dim = a.D;
     // row-split tasks run in the unified kernel only (not on the CUDA-core comparison body)
     a.wide_tasks = decode_body_is_mma();
+    a.self_cascade = decode_body_is_mma();  // cascade tasks run in the unified kernel only
     if (num_seqs > 0 && !block_table) {
         set_last_error(name + ": block_table is NULL");
         return PKVA_EINVAL;
@@ -564,6 +565,7 @@ static int run_impl(pkva_plan_t plan, const void* q, const void* k_new, const vo
     pp.cwork = plan->d_cwork;
     pp.crowmap = plan->d_crowmap;
     pp.cunits = plan->d_cunits;
+    pp.anc = plan->d_anc;
     pp.units = plan->d_units;
     pp.part_o = plan->d_part_o;
     pp.part_ml = plan->d_part_ml;

@@ -41,7 +41,7 @@ struct AttnNS {
     static constexpr int value = (D == 64 ? 4 : 2) * (FP8 ? 2 : 1);
 };
 
-// TC: the kernel can run tensor-core tasks (head_dim 128 only). FP8 launches without any
+// TC: the kernel can run tensor-core tasks (head_dim 128 only). Launches without any
 // tensor-core task use the TC = false kernel: smaller code for the decode-only plans.
 template <int D, int NT, bool FP8 = false, bool TC = true>
 struct AttnSmem {
@@ -169,7 +169,10 @@ cudaError_t launch_attn(const AttnParams& p, int D, int rows, bool has_prefill, 
                         const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKn,
                         const CUtensorMap& tmVn, const CUtensorMap& tmQc, cudaStream_t stream, bool fp8) {
     if (D == 64 && has_prefill) return cudaErrorInvalidValue;   // tensor-core tasks: head_dim 128
-    if (!fp8) return launch_kv<false, true>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
+    // plans without tensor-core tasks launch the TC = false code (no prefill body in it)
+    if (!fp8)
+        return has_prefill ? launch_kv<false, true>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
+                           : launch_kv<false, false>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
     return has_prefill ? launch_kv<true, true>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
                        : launch_kv<true, false>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
 }

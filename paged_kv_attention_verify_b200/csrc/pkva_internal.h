@@ -19,6 +19,8 @@ constexpr int kDecTasksPerBlock = 3;   // decode tasks side by side in one block
 constexpr int kPrefillMinTokens = 64;  // causal sequences with at least this many new tokens
                                        // (and head_dim 128) run on the tensor-core prefill kernel
 constexpr int kCascadeTilesPerTask = 16; // shared-prefix KV tiles (128 keys) per cascade task
+constexpr int kOwnMinKeys = 512;         // keys from which a verify tree's rows run on the tensor cores
+constexpr int kOwnTilesPerTask = 16;     // KV tiles (128 keys) per tensor-core verify task
 
 // Per-sequence record (the "Token-Table" row of the batch).
 struct SeqInfo {
@@ -100,8 +102,13 @@ struct CascadeWork {
     int32_t tile_end;
     int32_t unit_off;    // into the cascade unit list
     int32_t unit_cnt;
+    int32_t own;         // 0: a shared prefix; 1: the rows of one sequence over a chunk of its
+                         // own keys [0, seq_len) with the tree / causal masks (tensor-core
+                         // verify task), partials to split slots; 2: as 1, over all of its
+                         // keys, writing the output rows itself
+    int32_t pad[3];
 };
-static_assert(sizeof(CascadeWork) == 32, "CascadeWork layout");
+static_assert(sizeof(CascadeWork) == 48, "CascadeWork layout");
 
 // Host-side result of planning, before anything is uploaded.
 struct HostPlan {
@@ -157,6 +164,9 @@ struct PlanArgs {
     // 48 rows that read each page once (the unified kernel's bf16 decode/verify path); false:
     // every task holds at most 16 rows (the stand-alone decode kernels)
     bool wide_tasks = true;
+    // verify trees / short causal chunks of 17 to 128 packed rows per KV head on the
+    // tensor cores (cascade-style tasks over their own keys); false: decode/verify tasks only
+    bool self_cascade = true;
     // shared-prefix groups (may be NULL / 0): prefix_group[s] in {-1} U [0, num_groups),
     // members of a group consecutive in the batch, prefix_len[g] keys shared (page multiple)
     const int32_t* prefix_group = nullptr;

@@ -57,6 +57,7 @@ struct PrefillParams {
     const CascadeWork* cwork = nullptr;
     const int32_t* crowmap = nullptr;    // [tasks][256]: partial index slot*16 + row, or -1
     const int32_t* cunits = nullptr;
+    const uint64_t* anc = nullptr;       // tree ancestor masks (tensor-core verify tasks)
     const SplitUnit* units = nullptr;
     float* part_o = nullptr;
     float* part_ml = nullptr;

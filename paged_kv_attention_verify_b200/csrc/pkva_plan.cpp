@@ -162,6 +162,10 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
         }
     }
 
+    // keys each group's cascade tasks cover
+    std::vector<int> glen;
+    for (int g = 0; g < (a.num_seqs > 0 ? a.num_groups : 0); ++g) glen.push_back(a.prefix_len[g]);
+
     // -- prefill tiles: long causal chunks go to the tensor-core prefill kernel ---------
     std::vector<char> on_prefill(a.num_seqs, 0);
     if (a.use_prefill_kernel && a.D == 128) {
@@ -216,6 +220,36 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
         });
     }
 
+    // -- verify trees (and short causal chunks) of 17 to 128 packed rows per KV head run
+    //    on the tensor cores: one cascade-style task per (sequence, KV head, chunk of
+    //    kOwnTilesPerTask KV tiles) holds all of the unit's rows in one query tile and reads
+    //    each key once for all of them (tree / causal masks on the tiles with the new tokens'
+    //    keys); its halves interleave the KV tiles so that the tensor cores and the softmax
+    //    overlap. bf16 caches only (FP8 would stage the whole sequence to bf16 first).
+    //    Like the row-split rule below, only in a batch where such units hold at most half of
+    //    the decode/verify pages: a tensor-core task takes a whole SM and streams its keys at
+    //    about 40 GB/s, so it pays beside decode blocks that keep HBM busy, while a batch of
+    //    such units alone ran faster as 16-row decode/verify tasks (measured on B200: the
+    //    Qwen2-7B verify class 0.0614 against 0.0655 ms, the unified batch 0.170 against
+    //    0.166 ms).
+    std::vector<char> on_own(a.num_seqs, 0);
+    if (a.self_cascade && a.use_prefill_kernel && a.D == 128 && a.kv_elem_bytes == 2 && p.G <= kPrefillTileM) {
+        int64_t own_pages = 0, all_pages = 0;
+        for (int s = 0; s < a.num_seqs; ++s) {
+            if (on_prefill[s]) continue;
+            const SeqInfo& si = p.seqs[s];
+            const int64_t pg = (int64_t)(si.seq_len + kPageSize - 1) / kPageSize -
+                               (grp_of[s] >= 0 ? glen[grp_of[s]] / kPageSize : 0);
+            all_pages += pg;
+            if (grp_of[s] >= 0 || si.query_len * p.G <= kDecodeRowsMax || si.query_len > kPrefillTileM / p.G ||
+                si.seq_len < kOwnMinKeys)
+                continue;
+            on_own[s] = 1;
+            own_pages += pg;
+        }
+        if (2 * own_pages > all_pages) std::fill(on_own.begin(), on_own.end(), 0);
+    }
+
     // -- decode/verify units: (seq, kv head, chunk of packed rows) --------------------
     // A sequence of a shared-prefix group leaves its first prefix_len keys to the cascade
     // tasks: its units start at that page, and always merge partials.
@@ -234,10 +268,10 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
     if (wide) {
         int64_t wide_pages = 0, all_pages = 0;
         for (int s = 0; s < a.num_seqs; ++s) {
-            if (on_prefill[s]) continue;
+            if (on_prefill[s] || on_own[s]) continue;
             const SeqInfo& si = p.seqs[s];
             const int64_t pg = (int64_t)(si.seq_len + kPageSize - 1) / kPageSize -
-                               (grp_of[s] >= 0 ? a.prefix_len[grp_of[s]] / kPageSize : 0);
+                               (grp_of[s] >= 0 ? glen[grp_of[s]] / kPageSize : 0);
             all_pages += pg;
             if (si.query_len * p.G > 2 * kDecodeRowsMax) wide_pages += pg;
         }
@@ -252,12 +286,26 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
         const SeqInfo& si = p.seqs[s];
         const int rows = si.query_len * p.G;
         const int g = grp_of[s];
-        const int pstart = g >= 0 ? a.prefix_len[g] / kPageSize : 0;
-        const int cs = g >= 0 ? (a.prefix_len[g] + kPrefillTileN * kCascadeTilesPerTask - 1) /
+        if (on_own[s]) {
+            // tensor-core rows: one unit per 16-row chunk (split slots for the KV chunks; none
+            // when one task covers all keys and writes the rows itself), no decode/verify task
+            const int tiles = (si.seq_len + kPrefillTileN - 1) / kPrefillTileN;
+            int cs = (tiles + kOwnTilesPerTask - 1) / kOwnTilesPerTask;
+            if (cs == 1) cs = 0;
+            unit_base[s] = (int)units.size();
+            for (int h = 0; h < a.Hkv; ++h)
+                for (int rb = 0; rb < rows; rb += kDecodeRowsMax) {
+                    const int rc = std::min(kDecodeRowsMax, rows - rb);
+                    units.push_back({s, h, rb, rc, 0, 0, cs, rc});
+                }
+            continue;
+        }
+        const int pstart = g >= 0 ? glen[g] / kPageSize : 0;
+        const int cs = g >= 0 ? (glen[g] + kPrefillTileN * kCascadeTilesPerTask - 1) /
                                     (kPrefillTileN * kCascadeTilesPerTask)
                               : 0;
         on_cascade[s] = g >= 0;
-        p.seqs[s].shared_len = g >= 0 ? a.prefix_len[g] : 0;
+        p.seqs[s].shared_len = g >= 0 ? glen[g] : 0;
         unit_base[s] = (int)units.size();
         // keys past the last row's own position are masked for every row of a task (causal
         // and tree alike), so the task never loads them
@@ -288,14 +336,14 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
         }
     }
     // algorithmic bytes: a shared prefix is one set of keys, counted once per group
-    if (a.num_groups > 0) {
-        std::vector<char> counted(a.num_groups, 0);
+    if (!glen.empty()) {
+        std::vector<char> counted(glen.size(), 0);
         for (int s = 0; s < a.num_seqs; ++s) {
             if (!on_cascade[s]) continue;
             const int g = grp_of[s];
             const int64_t per_key = (int64_t)a.Hkv * a.D * 2 * a.kv_elem_bytes;
-            p.kv_bytes -= (int64_t)a.prefix_len[g] * per_key;
-            if (!counted[g]) p.kv_bytes += (int64_t)a.prefix_len[g] * per_key;
+            p.kv_bytes -= (int64_t)glen[g] * per_key;
+            if (!counted[g]) p.kv_bytes += (int64_t)glen[g] * per_key;
             counted[g] = 1;
         }
     }
@@ -326,8 +374,9 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
         // nearest whole number of target-sized tasks (rounding up made near-target units two
         // half-size tasks), never more pages per task than the staged block-table slice holds
         const int64_t per_task = nchunks > 1 ? std::max<int64_t>(target / kWideSplit, kMinWidePages) : target;
-        const int ns = std::max<int>(std::max<int>(1, (int)((own + per_task / 2) / per_task)),
-                                     (own + kDecodeMaxPages - 1) / kDecodeMaxPages);
+        const int ns = on_own[u.seq] ? 0          // tensor-core rows: only cascade-style tasks
+                                     : std::max<int>(std::max<int>(1, (int)((own + per_task / 2) / per_task)),
+                                                     (own + kDecodeMaxPages - 1) / kDecodeMaxPages);
         int unit_id = -1;                     // the lead chunk's; chunk c has unit_id + c
         for (int c = 0; c < nchunks; ++c) {
             const Unit& uc = units[ui + c];
@@ -367,7 +416,7 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
     //    members (their q rows are contiguous), per KV head: tiles of floor(128 / G) tokens
     //    x G heads, two tiles per task, the prefix split into chunks of tiles ---------------
     p.cascade_tok = kPrefillTileM / p.G;
-    if (a.num_groups > 0) {
+    if (!glen.empty()) {
         const int TOK = p.cascade_tok;
         auto seq_of_token = [&](int tok) {
             int lo = 0, hi = a.num_seqs - 1;       // last s with q_start <= tok
@@ -385,7 +434,7 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
             while (e + 1 < a.num_seqs && on_cascade[e + 1] && grp_of[e + 1] == g) ++e;
             const int run_t0 = p.seqs[s].q_start;
             const int run_t1 = p.seqs[e].q_start + p.seqs[e].query_len;
-            const int tiles = (a.prefix_len[g] + kPrefillTileN - 1) / kPrefillTileN;
+            const int tiles = (glen[g] + kPrefillTileN - 1) / kPrefillTileN;
             const int cs = units[unit_base[s]].cs;
             for (int h = 0; h < a.Hkv; ++h) {
                 for (int t0 = run_t0; t0 < run_t1; t0 += 2 * TOK) {
@@ -431,6 +480,42 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
             s = e + 1;
         }
     }
+    // -- tensor-core verify tasks (see on_own): all of a unit's rows in tile 0, its KV tiles
+    //    split into chunks of kOwnTilesPerTask --------------------------------------------
+    for (int s = 0; s < a.num_seqs; ++s) {
+        if (!on_own[s]) continue;
+        const SeqInfo& si = p.seqs[s];
+        const int rows = si.query_len * p.G;
+        const int chunks = (rows + kDecodeRowsMax - 1) / kDecodeRowsMax;
+        const int tiles = (si.seq_len + kPrefillTileN - 1) / kPrefillTileN;
+        const int cs = std::max(1, units[unit_base[s]].cs);
+        const bool direct = units[unit_base[s]].cs == 0;       // one task: it writes the rows
+        for (int h = 0; h < a.Hkv; ++h) {
+            const int ub = unit_base[s] + h * chunks;
+            for (int k = 0; k < cs; ++k) {
+                CascadeWork cw{};
+                cw.lead_seq = s;
+                cw.kv_head = h;
+                cw.tok0 = si.q_start;
+                cw.ntok = si.query_len;
+                cw.tile_begin = (int)((int64_t)tiles * k / cs);
+                cw.tile_end = (int)((int64_t)tiles * (k + 1) / cs);
+                cw.unit_off = (int)p.cunits.size();
+                cw.unit_cnt = direct ? 0 : chunks;
+                cw.own = direct ? 2 : 1;
+                for (int c = 0; c < cw.unit_cnt; ++c) {
+                    p.cunits.push_back(unit_id_of[ub + c]);
+                    p.units[unit_id_of[ub + c]].arrivals += 1;
+                }
+                for (int r = 0; r < 2 * kPrefillTileM; ++r)
+                    p.crowmap.push_back(!direct && r < rows
+                                            ? (p.units[unit_id_of[ub + r / kDecodeRowsMax]].slot_base + k) *
+                                                      kDecodeRowsMax + r % kDecodeRowsMax
+                                            : -1);
+                p.cwork.push_back(cw);
+            }
+        }
+    }
     // FP8 caches: the tensor-core tasks read a bf16 copy of the pages they use: all pages of
     // a sequence that runs as prefill tasks, the shared pages of a cascade run's lead sequence
     // (whose block-table row supplies the shared keys to its cascade tasks)
@@ -439,7 +524,7 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
         for (int s = 0; s < a.num_seqs; ++s)
             if (on_prefill[s]) stage_pages[s] = (p.seqs[s].seq_len + kPageSize - 1) / kPageSize;
         for (const CascadeWork& cw : p.cwork)
-            stage_pages[cw.lead_seq] = a.prefix_len[grp_of[cw.lead_seq]] / kPageSize;
+            stage_pages[cw.lead_seq] = glen[grp_of[cw.lead_seq]] / kPageSize;
         int stride = 0;
         int64_t n = 0;
         for (int s = 0; s < a.num_seqs; ++s) {
@@ -473,22 +558,39 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
         return task_cost(x) > task_cost(y);
     });
 
-    // -- one launch order. Cascade tasks go first: few, long, and every unit of their rows
-    //    waits for them, so the units' own decode tasks tend to arrive last and do the
-    //    merges, spread over many blocks. Prefill and decode tasks each keep their
-    //    heaviest-first order; the two lists are merged in proportion, so prefill blocks
-    //    (tensor cores, latency) run beside decode blocks (HBM) from start to end instead of
-    //    one kind forming the tail. Decode tasks go three to a block, neighbours in the
-    //    sorted list.
-    for (size_t i = 0; i < p.cwork.size(); ++i) p.order.push_back((int32_t)(p.pwork.size() + i));
-    const int np = (int)p.pwork.size();
+    // -- one launch order. Shared-prefix cascade tasks go first: few, long, and every unit of
+    //    their rows waits for them, so the units' own decode tasks tend to arrive last and do
+    //    the merges, spread over many blocks. The other tensor-core tasks (prefill tiles and
+    //    tensor-core verify tasks, heaviest first by the KV tiles each query tile runs) and
+    //    the decode tasks (heaviest first) are merged in proportion, so tensor-core blocks
+    //    (latency) run beside decode blocks (HBM) from start to end instead of one kind
+    //    forming the tail. Decode tasks go three to a block, neighbours in the sorted list.
+    std::vector<int32_t> tc;                  // block entries of the tensor-core list
+    std::vector<int> tc_cost;
+    for (size_t i = 0; i < p.pwork.size(); ++i) {
+        tc.push_back((int32_t)i);
+        tc_cost.push_back(p.pwork[i].kv_tiles0 + p.pwork[i].kv_tiles1);
+    }
+    for (size_t i = 0; i < p.cwork.size(); ++i) {
+        const int32_t e = (int32_t)(p.pwork.size() + i);
+        if (!p.cwork[i].own) {
+            p.order.push_back(e);
+            continue;
+        }
+        tc.push_back(e);
+        tc_cost.push_back(p.cwork[i].tile_end - p.cwork[i].tile_begin);
+    }
+    std::vector<int> tci(tc.size());
+    for (size_t i = 0; i < tc.size(); ++i) tci[i] = (int)i;
+    std::stable_sort(tci.begin(), tci.end(), [&](int x, int y) { return tc_cost[x] > tc_cost[y]; });
+    const int np = (int)tc.size();
     const int nd = (int)((p.dwork.size() + kDecTasksPerBlock - 1) / kDecTasksPerBlock);
     int ip = 0, id = 0;
     while (ip < np || id < nd) {
         // take from the list that is further behind in its share of the launch
         const bool take_p = id >= nd || (ip < np && (int64_t)ip * nd <= (int64_t)id * np);
         if (take_p)
-            p.order.push_back(ip++);
+            p.order.push_back(tc[tci[ip++]]);
         else
             p.order.push_back(-1 - id++);
     }
@@ -531,8 +633,8 @@ extern "C" int attn_plan_inspect(int num_seqs, const int32_t* seq_lens, const in
         set_last_error("attn_plan_inspect: max_items is smaller than the number of tasks");
         return PKVA_EINVAL;
     }
-    int ip = 0;
-    for (const PrefillWork& w : hp.pwork) {      // prefill tiles first
+    int ip = nc;
+    for (const PrefillWork& w : hp.pwork) {      // prefill tiles after the cascade tasks
         const SeqInfo& si = hp.seqs[w.seq];
         for (int b = 0; b < (w.ntok1 > 0 ? 2 : 1); ++b) {
             const int h = b ? w.q_head1 : w.q_head, t0 = b ? w.tok1 : w.tok0, nt = b ? w.ntok1 : w.ntok0;
@@ -550,11 +652,14 @@ extern "C" int attn_plan_inspect(int num_seqs, const int32_t* seq_lens, const in
             items[ip++] = d;
         }
     }
-    for (int i = 0; i < nc; ++i) {      // then shared-prefix tasks
+    for (int i = 0; i < nc; ++i) {      // shared-prefix (cascade) tasks first, as in the launch
         const CascadeWork& w = hp.cwork[i];
-        const int P = a.prefix_len[a.prefix_group[w.lead_seq]];
+        // keys the task's unit covers: the shared prefix, or (tensor-core verify rows) the
+        // whole sequence
+        const int P = w.own ? hp.seqs[w.lead_seq].seq_len : hp.seqs[w.lead_seq].shared_len;
         const int tiles = (P + kPrefillTileN - 1) / kPrefillTileN;
-        const int cs = (P + kPrefillTileN * kCascadeTilesPerTask - 1) / (kPrefillTileN * kCascadeTilesPerTask);
+        const int cs = w.own ? (tiles + kOwnTilesPerTask - 1) / kOwnTilesPerTask
+                             : (P + kPrefillTileN * kCascadeTilesPerTask - 1) / (kPrefillTileN * kCascadeTilesPerTask);
         int k = 0;
         while (k < cs && (int)((int64_t)tiles * k / cs) != w.tile_begin) ++k;
         pkva_work_desc d;
@@ -568,7 +673,7 @@ extern "C" int attn_plan_inspect(int num_seqs, const int32_t* seq_lens, const in
         d.key_end = std::min(w.tile_end * kPrefillTileN, P);
         d.split = k;
         d.num_splits = cs;
-        items[np + i] = d;
+        items[i] = d;
     }
     for (int i = np + nc; i < n; ++i) {
         const DecodeWork& w = hp.dwork[i - np - nc];

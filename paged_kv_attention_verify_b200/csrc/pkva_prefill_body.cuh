@@ -23,6 +23,12 @@
 // columns [0,64) of S_b (bf16 pairs). Tensor-core operations of one issuing thread run in
 // issue order, so the next QK^T into S_b is issued right after the PV that reads P_b.
 //
+// The same body runs shared-prefix (cascade) tasks and tensor-core verify tasks: the packed
+// (token, head) rows of one KV head in a query tile, the KV tiles of a shared prefix or of
+// the sequence's own keys (tree / causal masks on the tiles that hold the new tokens' keys,
+// which fused append patches in from the dense input). With one query tile the two
+// warpgroups take alternate KV tiles and combine their halves at the end.
+//
 // Sources: XY-Serve (arXiv 2412.18106), verdict page — key_machinery (the attention
 // primitive is a matmul-softmax-matmul tile whose QK and SV products overlap the softmax),
 // core_discovery (chunked prefill on cached prefixes; fully masked tiles are skipped);
@@ -55,8 +61,8 @@ constexpr int kOffK = kOffQ + 2 * kTileBytes;
 constexpr int kOffV = kOffK + kNK * kTileBytes;
 constexpr int kOffBar = kOffV + kNV * kTileBytes;
 // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2], p_full[2], o_ready[2], mma_done,
-// v_fix
-constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 2 + 2 + 2 + 1 + 1;
+// v_fix, k_fix
+constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 2 + 2 + 2 + 1 + 1 + 1;
 constexpr int kOffFlag = kOffBar + kNumBars * 8;         // the task's abort flag
 constexpr int kSmemBytes = kOffFlag + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1008;
@@ -79,7 +85,8 @@ struct Bars {
     uint64_t* p_full;
     uint64_t* o_ready;
     uint64_t* mma_done;
-    uint64_t* v_fix;         // the V tile whose stale rows the producer zeroes first
+    uint64_t* v_fix;         // a V tile the producer patches before releasing it
+    uint64_t* k_fix;         // a K tile the producer patches before releasing it
 };
 
 __device__ __forceinline__ Bars bars_at(uint8_t* sm) {
@@ -95,6 +102,7 @@ __device__ __forceinline__ Bars bars_at(uint8_t* sm) {
     r.o_ready = r.p_full + 2;
     r.mma_done = r.o_ready + 2;
     r.v_fix = r.mma_done + 1;
+    r.k_fix = r.v_fix + 1;
     return r;
 }
 
@@ -159,6 +167,10 @@ __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, 
 // KV tiles are a chunk of the shared prefix (all keys visible to every row), and each row's
 // unnormalised output, max and sum go to the split slot its row-map entry names; the task
 // then counts one arrival on every unit it touched and merges those it completed.
+// A cascade task whose rows fit one query tile runs interleaved: both warpgroups hold the
+// same rows (Q loaded once), tile b takes the KV tiles j with j % 2 == b, so the tensor
+// cores run one half's PV and next QK^T while the other half's softmax runs, and the two
+// halves' (max, sum, output) are combined before the partial is written.
 __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, const CUtensorMap& tmQ,
                                              const CUtensorMap& tmK, const CUtensorMap& tmV,
                                              const CUtensorMap& tmKn, const CUtensorMap& tmVn,
@@ -181,16 +193,20 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffFlag);
     const bool append = p.append != 0 && !cascade;
     const int TOK = p.cascade_tok;                      // cascade: tokens per query tile
-    const int n0 = cascade ? cw.tile_end - cw.tile_begin : append ? w.kv_tiles0_append : w.kv_tiles0;
-    const int n1 = cascade ? (cw.ntok > TOK ? n0 : 0) : append ? w.kv_tiles1_append : w.kv_tiles1;
-    const int nmax = n0 > n1 ? n0 : n1;
+    const bool il = cascade && cw.ntok <= TOK;          // one query tile, KV tiles interleaved
+    const int ncas = cw.tile_end - cw.tile_begin;
+    const int n0 = il ? (ncas + 1) / 2 : cascade ? ncas : append ? w.kv_tiles0_append : w.kv_tiles0;
+    const int n1 = il ? ncas / 2 : cascade ? (cw.ntok > TOK ? ncas : 0) : append ? w.kv_tiles1_append : w.kv_tiles1;
+    const int nmax = il ? ncas : (n0 > n1 ? n0 : n1);   // KV tiles loaded, in order
     const int jbase = cascade ? cw.tile_begin : 0;     // first KV tile (of 128 keys) of the task
     const int kvh = cascade ? cw.kv_head : w.q_head / p.G;
     const int prefix = si.seq_len - si.query_len;
     const int nc = append ? (prefix + kPrefillTileN - 1) / kPrefillTileN : nmax;   // tiles read from the cache
     // cache keys that hold data: the shared prefix (cascade), the committed prefix
     // (append), the whole sequence (otherwise)
-    const int key_limit = cascade ? si.shared_len : append ? prefix : si.seq_len;
+    // own: a tensor-core verify task, the rows of one sequence over its own keys (masked)
+    const bool own = cascade && cw.own != 0;
+    const int key_limit = own ? si.seq_len : cascade ? si.shared_len : append ? prefix : si.seq_len;
 
     if (tid == 0) {
         mbar_init(B.q_full, 1);
@@ -209,6 +225,7 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         }
         mbar_init(B.mma_done, 1);
         mbar_init(B.v_fix, 1);
+        mbar_init(B.k_fix, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -218,21 +235,22 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
 
     if (warp == kWarpKProd || warp == kWarpVProd) {
         // ------------------ TMA producers: warp 8 loads Q and K, warp 10 loads V ------------
+        // lane 0 issues the loads; the whole warp patches a tile before releasing it
+        const bool is_k = warp == kWarpKProd;
+        const int32_t* btrow = p.block_table + (int64_t)w.seq * p.bt_stride;
+        // the cache page holding key_limit has stale rows from key_limit on (when it is
+        // not page-aligned): the V tile with that page is zeroed there before its PV
+        const int fix_tile = (key_limit % kPageSize) ? key_limit / kPageSize / 8 - jbase : -1;
         if (lane == 0) {
             fence_proxy_async_smem();              // the previous task's generic accesses come first
-            const bool is_k = warp == kWarpKProd;
-            const int32_t* btrow = p.block_table + (int64_t)w.seq * p.bt_stride;
-            // the cache page holding key_limit has stale rows from key_limit on (when it is
-            // not page-aligned): the V tile with that page is zeroed there before its PV
-            const int fix_tile = (key_limit % kPageSize) ? key_limit / kPageSize / 8 - jbase : -1;
             if (is_k && cascade) {
                 // G heads x TOK tokens per tile: rows (token, head) in the tile's first
                 // G * TOK rows, the same 128-byte rows as a one-head box
                 prefetch_tensormap(&tmQc);
                 prefetch_tensormap(&tmK);
-                mbar_arrive_expect_tx(B.q_full, 4u * (uint32_t)(p.G * TOK) * 128u);
-#pragma unroll
-                for (int b = 0; b < 2; ++b)
+                const int nq = il ? 1 : 2;                 // interleaved: both halves read Q tile 0
+                mbar_arrive_expect_tx(B.q_full, 2u * (uint32_t)nq * (uint32_t)(p.G * TOK) * 128u);
+                for (int b = 0; b < nq; ++b)
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
                         tma_load_3d(sm + kOffQ + b * kTileBytes + h * kHalfBytes, &tmQc, B.q_full, h * 64,
@@ -252,83 +270,143 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
                 prefetch_tensormap(&tmV);
                 if (append) prefetch_tensormap(&tmVn);
             }
-            const int NSt = is_k ? kNK : kNV;
-            uint64_t* full = is_k ? B.k_full : B.v_full;
-            uint64_t* empty = is_k ? B.k_empty : B.v_empty;
-            uint8_t* base = sm + (is_k ? kOffK : kOffV);
-            for (int j = 0; j < nmax; ++j) {
-                const int st = j % NSt;
-                if (j >= NSt && !wait_or_abort(&empty[st], ((j / NSt) - 1) & 1, p.err, abort_flag)) break;
-                uint8_t* dst = base + st * kTileBytes;
-                if (j >= nc) {
-                    // new tokens [128 (j - nc), +128) of the chunk, straight from the input
+        }
+        const int NSt = is_k ? kNK : kNV;
+        uint64_t* full = is_k ? B.k_full : B.v_full;
+        uint64_t* empty = is_k ? B.k_empty : B.v_empty;
+        uint64_t* fixbar = is_k ? B.k_fix : B.v_fix;
+        uint8_t* base = sm + (is_k ? kOffK : kOffV);
+        int nfix = 0;                                  // phases of fixbar used
+        for (int j = 0; j < nmax; ++j) {
+            const int st = j % NSt;
+            if (j >= NSt &&
+                !__all_sync(0xffffffffu, wait_or_abort(&empty[st], ((j / NSt) - 1) & 1, p.err, abort_flag)))
+                break;
+            uint8_t* dst = base + st * kTileBytes;
+            if (j >= nc) {
+                // new tokens [128 (j - nc), +128) of the chunk, straight from the input
+                if (lane == 0) {
                     const int row0 = si.q_start + (j - nc) * kPrefillTileN;
                     mbar_arrive_expect_tx(&full[st], kTileBytes);
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
                         tma_load_3d(dst + h * kHalfBytes, is_k ? &tmKn : &tmVn, &full[st], h * 64, kvh, row0);
-                    continue;
                 }
-                int rows[8];
-                tile_rows(p, btrow, key_limit, kvh, jbase + j, rows);
-                if (is_k || j != fix_tile) {
-                    load_tile(dst, is_k ? &tmK : &tmV, &full[st], rows);
-                    continue;
-                }
-                load_tile(dst, &tmV, B.v_fix, rows);
-                if (!wait_or_abort(B.v_fix, 0, p.err, abort_flag)) break;
-                const int pg = (key_limit / kPageSize) % 8;
-                for (int r = key_limit % kPageSize; r < kPageSize; ++r)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-#pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            *reinterpret_cast<uint4*>(dst + h * kHalfBytes + (pg * kPageSize + r) * 128 + c * 16) =
-                                make_uint4(0u, 0u, 0u, 0u);
-                fence_proxy_async_smem();
-                mbar_arrive(&full[st]);
+                continue;
             }
-            // drain: the last stages' release arrives (from tcgen05.commit) must have landed
-            // before the task ends and its barriers are invalidated and reused
-            for (int j = nmax > NSt ? nmax - NSt : 0; j < nmax; ++j)
-                if (!wait_or_abort(&empty[j % NSt], (j / NSt) & 1, p.err, abort_flag)) break;
+            int rows[8];
+            tile_rows(p, btrow, key_limit, kvh, jbase + j, rows);
+            // a tensor-core verify task under fused append: the new tokens' keys are not in
+            // the cache yet, their rows come from the dense input
+            const int kb = (jbase + j) * kPrefillTileN;
+            const bool patch = own && p.append && kb + kPrefillTileN > prefix && kb < si.seq_len;
+            const bool zero = !is_k && j == fix_tile;
+            if (!patch && !zero) {
+                if (lane == 0) load_tile(dst, is_k ? &tmK : &tmV, &full[st], rows);
+                continue;
+            }
+            if (lane == 0) load_tile(dst, is_k ? &tmK : &tmV, fixbar, rows);
+            if (!__all_sync(0xffffffffu, wait_or_abort(fixbar, nfix & 1, p.err, abort_flag))) break;
+            ++nfix;
+            if (patch) {
+                const int k0 = max(prefix, kb), k1 = min(si.seq_len, kb + kPrefillTileN);
+                const __nv_bfloat16* src = is_k ? p.k_new : p.v_new;
+                for (int idx = lane; idx < (k1 - k0) * 16; idx += 32) {
+                    const int key = k0 + (idx >> 4), c = idx & 15, r = key - kb;   // chunk c: half c / 8
+                    const uint4 v = *reinterpret_cast<const uint4*>(
+                        src + ((int64_t)(si.q_start + key - prefix) * p.Hkv + kvh) * kD + c * 8);
+                    *reinterpret_cast<uint4*>(dst + (c >> 3) * kHalfBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
+                }
+            }
+            if (zero) {
+                const int pg = (key_limit / kPageSize) % 8, r0 = key_limit % kPageSize;
+                for (int idx = lane; idx < (kPageSize - r0) * 16; idx += 32) {
+                    const int r = r0 + (idx >> 4), c = idx & 15;
+                    *reinterpret_cast<uint4*>(dst + (c >> 3) * kHalfBytes + (pg * kPageSize + r) * 128 + (c & 7) * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+            fence_proxy_async_smem();                  // every lane's writes, before the MMAs read them
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full[st]);
         }
+        // drain: the last stages' release arrives (from tcgen05.commit) must have landed
+        // before the task ends and its barriers are invalidated and reused
+        for (int j = nmax > NSt ? nmax - NSt : 0; j < nmax; ++j)
+            if (!__all_sync(0xffffffffu, wait_or_abort(&empty[j % NSt], (j / NSt) & 1, p.err, abort_flag))) break;
     } else if (warp == kWarpMma) {
         // ------------------------------ MMA issuer -------------------------------------------
         if (lane == 0) {
             const uint32_t q_base = smem_addr(sm + kOffQ);
             const uint32_t k_base = smem_addr(sm + kOffK);
             const uint32_t v_base = smem_addr(sm + kOffV);
-            auto issue_qk = [&](int b, int j) {           // S_b = Q_b K_j^T
+            auto issue_qk = [&](int b, int j) {           // S_b = Q_b K_j^T (interleaved: Q_0)
                 const int st = j % kNK;
                 const uint32_t d = tmem + kColS + b * 128;
+                const uint32_t qt = q_base + (il ? 0 : b) * kTileBytes;
 #pragma unroll
                 for (int ks = 0; ks < kD / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * kHalfBytes + (ks & 3) * 32;
-                    const uint64_t ad = smem_desc_sw128(q_base + b * kTileBytes + off, 16, 1024);
+                    const uint64_t ad = smem_desc_sw128(qt + off, 16, 1024);
                     const uint64_t bd = smem_desc_sw128(k_base + st * kTileBytes + off, 16, 1024);
                     tc_mma_ss(d, ad, bd, kIdescQK, ks > 0);
                 }
                 tc_commit(&B.s_full[b]);
             };
-            auto issue_pv = [&](int b, int j) {           // O_b += P_b V_j
+            auto issue_pv = [&](int b, int j, bool acc) {   // O_b (+)= P_b V_j
                 const int st = j % kNV;
                 const uint32_t pcol = tmem + kColS + b * 128;
 #pragma unroll
                 for (int ks = 0; ks < kPrefillTileN / 16; ++ks) {
                     const uint64_t bd = smem_desc_sw128(v_base + st * kTileBytes + ks * 2048, kHalfBytes, 1024);
-                    tc_mma_ts(tmem + kColO + b * 128, pcol + ks * 8, bd, kIdescPV, (j > 0 || ks > 0) ? 1u : 0u);
+                    tc_mma_ts(tmem + kColO + b * 128, pcol + ks * 8, bd, kIdescPV, (acc || ks > 0) ? 1u : 0u);
                 }
             };
             bool ok = wait_or_abort(B.q_full, 0, p.err, abort_flag) &&
                       wait_or_abort(&B.k_full[0], 0, p.err, abort_flag);
-            if (ok) {
+            if (ok && il) {
+                // interleaved: S_0 of KV tile 0 and S_1 of KV tile 1 first; then per KV tile j
+                // (half b = j % 2): PV of j, and QK^T of b's next tile j + 2
+                tc_fence_after();
+                issue_qk(0, 0);
+                tc_commit(&B.k_empty[0]);
+                if (n1 > 0) {
+                    ok = wait_or_abort(&B.k_full[1], 0, p.err, abort_flag);
+                    if (ok) {
+                        tc_fence_after();
+                        issue_qk(1, 1);
+                        tc_commit(&B.k_empty[1]);
+                    }
+                }
+                for (int j = 0; ok && j < nmax; ++j) {
+                    const int b = j & 1, i = j >> 1, vst = j % kNV;
+                    if (!wait_or_abort(&B.v_full[vst], (j / kNV) & 1, p.err, abort_flag) ||
+                        !spin_or_abort(&B.p_full[b], i & 1, p.err, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    issue_pv(b, j, i > 0);
+                    if (i == (b ? n1 : n0) - 1) tc_commit(&B.o_ready[b]);
+                    tc_commit(&B.v_empty[vst]);
+                    if (j + 2 < nmax) {
+                        const int kst = (j + 2) % kNK;
+                        if (!wait_or_abort(&B.k_full[kst], ((j + 2) / kNK) & 1, p.err, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        issue_qk(b, j + 2);
+                        tc_commit(&B.k_empty[kst]);
+                    }
+                }
+            } else if (ok) {
                 tc_fence_after();
                 if (n0 > 0) issue_qk(0, 0);
                 if (n1 > 0) issue_qk(1, 0);
                 tc_commit(&B.k_empty[0]);
             }
-            for (int j = 0; ok && j < nmax; ++j) {
+            for (int j = 0; ok && !il && j < nmax; ++j) {
                 const int vst = j % kNV;
                 bool vwaited = false, kwaited = false;
 #pragma unroll
@@ -347,7 +425,7 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
                         break;
                     }
                     tc_fence_after();
-                    issue_pv(b, j);
+                    issue_pv(b, j, j > 0);
                     if (j == nb - 1) tc_commit(&B.o_ready[b]);
                     if (j + 1 < nb) {
                         if (!kwaited) {
@@ -377,7 +455,7 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t s_addr = tmem + lane_off + kColS + b * 128;
         const uint32_t o_addr = tmem + lane_off + kColO + b * 128;
-        const int row_in_task = b * kPrefillTileM + r;
+        const int row_in_task = (il ? 0 : b) * kPrefillTileM + r;   // interleaved: tile 0's rows
         // this tile's query head and tokens (a cascade task's rows come from its row map)
         const int qh = b ? w.q_head1 : w.q_head;
         const int tok0_b = b ? w.tok1 : w.tok0;
@@ -413,14 +491,52 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
             for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
             tmem_wait_ld();
             const bool tile_a = j < na;
-            const int kb = tile_a ? (jbase + j) * kPrefillTileN : (j - na) * kPrefillTileN;
+            const int jj = il ? 2 * j + b : j;                 // this half's j-th KV tile
+            const int kb = tile_a ? (jbase + jj) * kPrefillTileN : (j - na) * kPrefillTileN;
             const int lim_j = tile_a ? lim_a : lim_b;
             const int lim_first_j = tile_a ? lim_first_a : lim_first_b;
-            if (kb + kPrefillTileN - 1 > lim_first_j) {        // tile crosses the diagonal
+            // masks as four 32-column words of visible columns, applied by one loop
+            uint32_t mw[4];
+            bool masked = false;
+            if (own) {
+                if (kb + kPrefillTileN > prefix) {             // the tile holds new tokens' keys
+                    // row r is packed row (token r / G, head r % G): every committed key is
+                    // visible, a new token's key only to its tree descendants (causal: to the
+                    // tokens from it on). Rows past the unit's take token T - 1's mask (unused).
+                    // (Read here, not kept across the loop: no registers taken from it.)
+                    const int own_t = min(r / p.G, si.query_len - 1);
+                    const bool own_tree = si.mask_kind == PKVA_TREE;
+                    const uint64_t own_anc = own_tree ? p.anc[si.anc_off + own_t] : 0ull;
+                    masked = true;
+                    const int pk = prefix - kb;                // columns below pk: committed keys
+#pragma unroll
+                    for (int wd = 0; wd < 4; ++wd) {
+                        const int lo = 32 * wd;
+                        if (own_tree) {                        // committed keys, then the row's ancestors
+                            uint32_t m = pk >= lo + 32 ? ~0u : (pk <= lo ? 0u : ((1u << (pk - lo)) - 1u));
+                            const int sh = lo - pk;            // bit i of the word is ancestor bit i + sh
+                            m |= sh >= 64 ? 0u : sh >= 0 ? (uint32_t)(own_anc >> sh)
+                                                         : (sh <= -32 ? 0u : (uint32_t)(own_anc << -sh));
+                            mw[wd] = m;
+                        } else {                               // causal: columns up to the row's own key
+                            const int v = pk + own_t - lo;
+                            mw[wd] = v >= 31 ? ~0u : (v < 0 ? 0u : ((2u << v) - 1u));
+                        }
+                    }
+                }
+            } else if (kb + kPrefillTileN - 1 > lim_first_j) {        // tile crosses the diagonal
+                masked = true;
                 const int vis = lim_j - kb;                        // columns <= vis are visible
 #pragma unroll
+                for (int wd = 0; wd < 4; ++wd) {
+                    const int v = vis - 32 * wd;
+                    mw[wd] = v >= 31 ? ~0u : (v < 0 ? 0u : ((2u << v) - 1u));
+                }
+            }
+            if (masked) {
+#pragma unroll
                 for (int c = 0; c < 128; ++c)
-                    if (c > vis) sr[c] = __float_as_uint(-INFINITY);
+                    if (!((mw[c >> 5] >> (c & 31)) & 1u)) sr[c] = __float_as_uint(-INFINITY);
             }
             // row max as eight independent chains (short dependency depth)
             float mx8[8];
@@ -481,7 +597,82 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
             // where this row's partial goes (slot * 16 + row in unit), or -1
             const int part_idx = p.crowmap[(int64_t)ci * 2 * kPrefillTileM + row_in_task];
             const bool real_row = part_idx >= 0;
-            if (nb > 0 && alive && __all_sync(0xffffffffu, wait_or_abort(&B.o_ready[b], 0, p.err, abort_flag))) {
+            if (il) {
+                // combine the halves: each warpgroup hands its (max, sum) over through Q tile
+                // 1's shared memory (never loaded in this mode), then writes half the columns
+                float* xch = reinterpret_cast<float*>(sm + kOffQ + kTileBytes);    // [2][128][2]
+                const bool mine = nb > 0 && alive;
+                xch[(b * kPrefillTileM + r) * 2] = mine ? m_ref : -INFINITY;
+                xch[(b * kPrefillTileM + r) * 2 + 1] = mine ? l_sum : 0.f;
+                asm volatile("bar.sync 1, 256;" ::: "memory");
+                const float m0 = xch[r * 2], l0 = xch[r * 2 + 1];
+                const float m1 = xch[(kPrefillTileM + r) * 2], l1 = xch[(kPrefillTileM + r) * 2 + 1];
+                const float M = fmaxf(m0, m1);
+                const float w0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M);
+                const float w1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M);
+                const bool waited = __all_sync(0xffffffffu, alive && !*abort_flag &&
+                                                                (n0 == 0 || wait_or_abort(&B.o_ready[0], 0, p.err, abort_flag)) &&
+                                                                (n1 == 0 || wait_or_abort(&B.o_ready[1], 0, p.err, abort_flag)));
+                if (waited && cw.own != 2) {
+                    tc_fence_after();
+                    float* dst = p.part_o + (int64_t)(part_idx < 0 ? 0 : part_idx) * kD;
+                    const float vsc = p.v_scale ? p.v_scale[kvh] : 1.f;
+                    const float f0 = w0 * vsc, f1 = w1 * vsc;
+                    const uint32_t o0 = tmem + lane_off + kColO, o1 = o0 + 128;
+#pragma unroll
+                    for (int c = 2 * b; c < 2 * b + 2; ++c) {
+                        uint32_t v0[32], v1[32];
+                        if (n0 > 0) tmem_ld32(o0 + c * 32, v0);
+                        if (n1 > 0) tmem_ld32(o1 + c * 32, v1);
+                        tmem_wait_ld();
+                        if (real_row) {
+#pragma unroll
+                            for (int e = 0; e < 32; e += 4) {
+                                float4 v;
+                                v.x = (n0 > 0 ? __uint_as_float(v0[e]) * f0 : 0.f) + (n1 > 0 ? __uint_as_float(v1[e]) * f1 : 0.f);
+                                v.y = (n0 > 0 ? __uint_as_float(v0[e + 1]) * f0 : 0.f) +
+                                      (n1 > 0 ? __uint_as_float(v1[e + 1]) * f1 : 0.f);
+                                v.z = (n0 > 0 ? __uint_as_float(v0[e + 2]) * f0 : 0.f) +
+                                      (n1 > 0 ? __uint_as_float(v1[e + 2]) * f1 : 0.f);
+                                v.w = (n0 > 0 ? __uint_as_float(v0[e + 3]) * f0 : 0.f) +
+                                      (n1 > 0 ? __uint_as_float(v1[e + 3]) * f1 : 0.f);
+                                *reinterpret_cast<float4*>(dst + c * 32 + e) = v;
+                            }
+                        }
+                    }
+                    if (real_row && b == 0)
+                        *reinterpret_cast<float2*>(p.part_ml + (int64_t)part_idx * 2) = make_float2(M, l0 * w0 + l1 * w1);
+                }
+                if (waited && cw.own == 2) {
+                    // one task over all of the sequence's keys: O / l straight to the row
+                    tc_fence_after();
+                    const bool real = r < cw.ntok * p.G;
+                    const float Lr = l0 * w0 + l1 * w1;
+                    const float inv = (Lr > 0.f ? 1.f / Lr : 0.f) * (p.v_scale ? p.v_scale[kvh] : 1.f);
+                    const float f0 = w0 * inv, f1 = w1 * inv;
+                    __nv_bfloat16* dst = p.out + ((int64_t)(si.q_start + r / p.G) * p.Hq + kvh * p.G + r % p.G) * kD;
+                    const uint32_t o0 = tmem + lane_off + kColO, o1 = o0 + 128;
+#pragma unroll
+                    for (int c = 2 * b; c < 2 * b + 2; ++c) {
+                        uint32_t v0[32], v1[32];
+                        if (n0 > 0) tmem_ld32(o0 + c * 32, v0);
+                        if (n1 > 0) tmem_ld32(o1 + c * 32, v1);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; e += 8) {
+                            float x[8];
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                x[q] = (n0 > 0 ? __uint_as_float(v0[e + q]) * f0 : 0.f) +
+                                       (n1 > 0 ? __uint_as_float(v1[e + q]) * f1 : 0.f);
+                            if (real)
+                                *reinterpret_cast<uint4*>(dst + c * 32 + e) =
+                                    make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                                               pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+                        }
+                    }
+                }
+            } else if (nb > 0 && alive && __all_sync(0xffffffffu, wait_or_abort(&B.o_ready[b], 0, p.err, abort_flag))) {
                 tc_fence_after();
                 float* dst = p.part_o + (int64_t)(part_idx < 0 ? 0 : part_idx) * kD;
                 // FP8 caches: the V scale of this KV head, as on every other partial
@@ -564,6 +755,14 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
                 }
             }
         }
+    } else if (own && p.append && warp == kPThreads / 32) {
+        // ------------------- warp 11: a tensor-core verify task's cache writes ----------------
+        // the task with the unit's last KV tiles writes the sequence's new rows of its KV head
+        // (no other task reads those cache slots: any task whose tiles hold them patches them
+        // from the dense input)
+        if (jbase + ncas == (si.seq_len + kPrefillTileN - 1) / kPrefillTileN)
+            append_rows<kD>(p.k_new, p.v_new, p.k_cache, p.v_cache, p.block_table, p.bt_stride, p.num_pages,
+                            p.Hkv, p.err, si, w.seq, kvh, 0, si.query_len, lane, 32);
     } else if (append) {
         // ------------------- warp 11: this task's share of the cache writes -------------------
         // the G query tiles (one per head of the KV head) on a token tile each write 1/G of its

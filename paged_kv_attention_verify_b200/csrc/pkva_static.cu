@@ -139,6 +139,7 @@ extern "C" int attn_run_static(int num_seqs, const int32_t* seq_lens, const int3
                num_kv_heads, head_dim, page_size, sm_scale, 1, 1};
     a.use_prefill_kernel = false;          // everything on the decode kernel (no TMEM, no extra tables)
     a.wide_tasks = false;                  // tasks of at most 16 rows (the stand-alone decode kernel)
+    a.self_cascade = false;                // no tensor-core tasks
     HostPlan hp;
     std::string err;
     int rc = build_host_plan(a, &hp, &err);

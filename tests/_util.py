@@ -4,6 +4,7 @@ import numpy as np
 import torch
 
 import oracle
+import workloads as W
 
 # tolerance of the bf16-in / fp32-accumulate / bf16-out path against the float64 oracle
 TOL_MAX_ABS = 2e-2
@@ -45,3 +46,19 @@ def assert_close(got, exp, what=""):
     assert np.isfinite(mx), f"{what}: non-finite output"
     assert mx <= TOL_MAX_ABS and mean <= TOL_MEAN_ABS, f"{what}: max abs {mx:.3e}, mean abs {mean:.3e}"
     return mx, mean
+
+
+def tc_verify_seqs():
+    """Decode steps beside verify trees and short causal chunks that run as tensor-core tasks
+    (16 query / 4 KV heads: 20 to 128 packed rows per KV head, at least 512 keys)."""
+    gen = torch.Generator().manual_seed(12)
+    return [W.SeqSpec(3000 + 7 * i, 1, W.CAUSAL, []) for i in range(6)] + [
+        W.SeqSpec(640 + 7, 7, W.TREE, W.random_tree(gen, 7)),       # new keys start a KV tile
+        W.SeqSpec(766 + 6, 6, W.TREE, W.random_tree(gen, 6)),       # new keys cross a tile boundary
+        W.SeqSpec(4100, 5, W.TREE, W.random_tree(gen, 5)),          # three chunks of 16 KV tiles
+        W.SeqSpec(1000 + 20, 20, W.CAUSAL, []),                     # a short causal chunk: 80 rows
+        W.SeqSpec(2500, 30, W.CAUSAL, []),                          # 120 rows
+        W.SeqSpec(513, 8, W.TREE, W.random_tree(gen, 8)),           # one key past the threshold
+        W.SeqSpec(128 * 5 + 1, 1, W.CAUSAL, []),
+        W.SeqSpec(600, 32, W.TREE, W.random_tree(gen, 32)),         # 128 rows: a full tile
+    ]

@@ -78,10 +78,38 @@ def test_attn_plan_validates_before_touching_the_device():
     L.attn_plan_destroy(None)
 
 
-def _coverage(batch, items, prefix_group=None, prefix_len=None):
+def _tc_verify_set(batch, head_dim=128, prefix_group=None, prefix_len=None):
+    """Sequences whose rows run as tensor-core verify tasks over all of their keys: outside any
+    caller group, 17 to 128 packed rows per KV head, at least 512 keys, and together at most
+    half of the decode/verify pages of the batch (otherwise none)."""
+    G = batch.num_q_heads // batch.num_kv_heads
+    cand, own_pages, all_pages = set(), 0, 0
+    for s, sp in enumerate(batch.seqs):
+        if sp.mask_kind == W.CAUSAL and sp.query_len >= 64:       # a prefill chunk
+            continue
+        grouped = prefix_group is not None and prefix_group[s] >= 0
+        pages = (sp.seq_len + 15) // 16 - (prefix_len[prefix_group[s]] // 16 if grouped else 0)
+        all_pages += pages
+        if head_dim == 128 and not grouped and 16 < sp.query_len * G and sp.query_len <= 128 // G and \
+                sp.seq_len >= 512:
+            cand.add(s)
+            own_pages += pages
+    return cand if 2 * own_pages <= all_pages else set()
+
+
+def _shared_keys(batch, s, prefix_group, prefix_len, head_dim=128):
+    """Keys of sequence s that cascade-kind tasks cover: its group's shared prefix, or all keys
+    of a tensor-core verify sequence (no decode/verify task)."""
+    if prefix_group is not None and prefix_group[s] >= 0:
+        return prefix_len[prefix_group[s]]
+    return batch.seqs[s].seq_len if s in _tc_verify_set(batch, head_dim, prefix_group, prefix_len) else 0
+
+
+def _coverage(batch, items, prefix_group=None, prefix_len=None, head_dim=128):
     """Every (seq, kv head, packed row) must see exactly the keys it needs, once."""
     G = batch.num_q_heads // batch.num_kv_heads
     q_start = np.cumsum([0] + [sp.query_len for sp in batch.seqs])
+    shared = [_shared_keys(batch, s, prefix_group, prefix_len, head_dim) for s in range(len(batch.seqs))]
     seen = {}
     for it in items:
         assert it["key_begin"] % 16 == 0 and it["key_end"] > it["key_begin"]
@@ -94,8 +122,11 @@ def _coverage(batch, items, prefix_group=None, prefix_len=None):
             rows = []
             for tok in range(it["row_begin"], it["row_begin"] + it["row_count"]):
                 s = int(np.searchsorted(q_start, tok, side="right") - 1)
-                assert prefix_group[s] == prefix_group[it["seq"]] >= 0
-                assert it["key_end"] <= prefix_len[prefix_group[s]]
+                if prefix_group is not None and prefix_group[s] >= 0:
+                    assert prefix_group[s] == prefix_group[it["seq"]]
+                else:                  # a single-sequence group of the planner's own
+                    assert s == it["seq"] and shared[s] > 0
+                assert it["key_end"] <= shared[s]
                 rows += [(s, (tok - q_start[s]) * G + g) for g in range(G)]
         else:                          # decode/verify: up to 16 rows, or a row-split task of up to 48
             assert 1 <= it["row_count"] <= 48 and it["q_head"] == -1
@@ -118,12 +149,16 @@ def _coverage(batch, items, prefix_group=None, prefix_len=None):
                 assert rngs[-1][1] <= sp.seq_len
                 casc = [x for x in rngs if x[2] == 2]
                 own = [x for x in rngs if x[2] != 2]
-                if casc:               # cascade chunks then the sequence's own splits
+                if casc and not own:   # tensor-core verify rows: cascade-kind chunks of all keys
+                    assert s in _tc_verify_set(batch, head_dim, prefix_group, prefix_len)
+                    assert all(x[4] == len(casc) for x in casc) and casc[-1][1] == sp.seq_len
+                    assert sorted(x[3] for x in casc) == list(range(len(casc)))
+                elif casc:             # cascade chunks then the sequence's own splits
                     assert all(x[4] == len(casc) for x in casc)
                     assert sorted(x[3] for x in casc) == list(range(len(casc)))
                     assert all(x[2] == 0 and x[4] == len(own) + len(casc) for x in own)
                     assert sorted(x[3] for x in own) == list(range(len(own)))
-                    assert casc[-1][1] == own[0][0] == prefix_len[prefix_group[s]]
+                    assert casc[-1][1] == own[0][0] == shared[s]
                 else:
                     n = rngs[0][4]
                     assert len(rngs) == n and sorted(x[3] for x in rngs) == (list(range(n)) if n > 1 else [-1])
@@ -146,8 +181,8 @@ def test_planner_covers_configs(name):
                        [s.mask_kind for s in b.seqs], [p for s in b.seqs for p in s.parents],
                        num_q_heads=Hq, num_kv_heads=Hkv, head_dim=d, num_pages=pages,
                        bt_stride=max((s.seq_len + 15) // 16 for s in b.seqs))
-    _coverage(b, items)
-    # launch order: prefill tasks, then decode/verify tasks, each heaviest first
+    _coverage(b, items, head_dim=d)
+    # listed as launched: cascade tasks, prefill tasks, then decode/verify tasks (heaviest first)
     kinds = [it["kind"] for it in items]
     assert kinds == sorted(kinds, reverse=True)
     dec = [it for it in items if it["kind"] == 0]
@@ -166,7 +201,7 @@ def test_planner_covers_random_batches(seed, d, max_q):
                        num_q_heads=b.num_q_heads, num_kv_heads=b.num_kv_heads, head_dim=b.head_dim,
                        num_pages=b.k_cache.shape[0], bt_stride=b.block_table.shape[1],
                        num_sms=4, ctas_per_sm=1)
-    _coverage(b, items)
+    _coverage(b, items, head_dim=d)
 
 
 def test_empty_batch_plans_to_nothing():
@@ -193,13 +228,13 @@ def test_planner_covers_shared_prefix_batches(seed, heads):
     b = W.random_shared_small(seed, *heads)
     items = _shared_inspect(b, num_sms=4, ctas_per_sm=1)
     assert any(it["kind"] == 2 for it in items)
-    _coverage(b, items, b.prefix_group, b.prefix_len)
+    _coverage(b, items, b.prefix_group, b.prefix_len, b.head_dim)
 
 
 def test_planner_covers_shared_prefix_config():
     b = W.make_shared_config("llama3_8b_shared_prefix")
     items = _shared_inspect(b)
-    _coverage(b, items, b.prefix_group, b.prefix_len)
+    _coverage(b, items, b.prefix_group, b.prefix_len, b.head_dim)
     casc = [it for it in items if it["kind"] == 2]
     # 4 groups x 8 KV heads x one task of 64 tokens x 2 chunks of 2048 shared keys
     assert len(casc) == 4 * 8 * 1 * 2
@@ -296,14 +331,48 @@ def test_verify_units_wider_than_32_rows_are_row_split_tasks_in_mixed_batches():
     kinds = [W.TREE, W.TREE, W.TREE] + [W.CAUSAL] * 20
     parents = [-1, 0, 0, 2, -1] + [-1] + list(range(63)) + [-1, 0, 1]
     pages = sum((L + 15) // 16 for L in lens)
-    items = pk.inspect(lens, qlens, kinds, parents, num_q_heads=28, num_kv_heads=4, head_dim=128,
+    items = pk.inspect(lens, qlens, kinds, parents, num_q_heads=28, num_kv_heads=4, head_dim=64,
                        num_pages=pages, bt_stride=200)
-    rows = sorted((it["seq"], it["kv_head"], it["row_begin"], it["row_count"]) for it in items if it["split"] <= 0)
+    rows = sorted((it["seq"], it["kv_head"], it["row_begin"], it["row_count"]) for it in items
+                  if it["kind"] == 0 and it["split"] <= 0)
     assert [r for r in rows if r[0] == 0] == [(0, h, 0, 35) for h in range(4)]
     big = [r[2:] for r in rows if r[0] == 1 and r[1] == 0]
     assert big == [(0, 48), (48, 48), (96, 48), (144, 48), (192, 48), (240, 48), (288, 48), (336, 48),
                    (384, 48), (432, 16)]
     assert [r[2:] for r in rows if r[0] == 2 and r[1] == 0] == [(0, 16), (16, 5)]
-    only = pk.inspect(lens[:3], qlens[:3], kinds[:3], parents, num_q_heads=28, num_kv_heads=4, head_dim=128,
+    only = pk.inspect(lens[:3], qlens[:3], kinds[:3], parents, num_q_heads=28, num_kv_heads=4, head_dim=64,
                       num_pages=pages, bt_stride=200)
-    assert max(it["row_count"] for it in only) == 16
+    assert max(it["row_count"] for it in only if it["kind"] == 0) == 16
+
+
+def test_verify_trees_run_as_tensor_core_tasks():
+    """Beside decode steps, a tree of 17 to 128 packed rows per KV head with at least 512 keys
+    runs as cascade-kind tensor-core tasks over all of its keys, one per KV head and chunk of
+    16 KV tiles (2048 keys), with no decode/verify task. A 64-token tree (448 rows), a tree of
+    16 rows or fewer, fewer than 512 keys, head_dim 64, and members of the caller's
+    shared-prefix groups keep the decode/verify path (a group member's shared prefix stays a
+    cascade task); so does every tree of a batch where such trees hold more than half of the
+    decode/verify pages."""
+    lens = [2000, 900, 700, 3000, 400, 5000] + [3000] * 10
+    qlens = [5, 64, 3, 2, 5, 5] + [1] * 10
+    kinds = [W.TREE] * 6 + [W.CAUSAL] * 10
+    parents = [-1, 0, 0, 2, -1] + [-1] + list(range(63)) + [-1, 0, 1] + [-1, 0] + [-1, 0, 0, 2, -1] + [-1, 0, 1, 1, 0]
+    pages = sum((L + 15) // 16 for L in lens)
+    kw = dict(num_q_heads=28, num_kv_heads=4, num_pages=pages, bt_stride=400)
+    items = pk.inspect(lens, qlens, kinds, parents, head_dim=128, **kw)
+    casc = sorted((it["seq"], it["kv_head"], it["key_begin"], it["key_end"], it["row_count"], it["split"],
+                   it["num_splits"]) for it in items if it["kind"] == 2)
+    split5 = [(0, 1664, 0), (1664, 3328, 1), (3328, 5000, 2)]      # 40 tiles in three chunks
+    assert casc == [(0, h, 0, 2000, 5, 0, 1) for h in range(4)] + [(2, h, 0, 700, 3, 0, 1) for h in range(4)] + \
+        [(5, h, kb, ke, 5, k, 3) for h in range(4) for kb, ke, k in split5]
+    assert not any(it["kind"] == 0 and it["seq"] in (0, 2, 5) for it in items)
+    assert {it["seq"] for it in items if it["kind"] == 0} == {1, 3, 4} | set(range(6, 16))
+    assert not any(it["kind"] == 2 for it in pk.inspect(lens, qlens, kinds, parents, head_dim=64, **kw))
+    grouped = pk.inspect(lens, qlens, kinds, parents, head_dim=128, prefix_group=[0] + [-1] * 15, prefix_len=[512],
+                         **kw)
+    assert sorted({(it["seq"], it["key_end"]) for it in grouped if it["kind"] == 2}) == \
+        [(0, 512), (2, 700), (5, 1664), (5, 3328), (5, 5000)]
+    assert min(it["key_begin"] for it in grouped if it["kind"] == 0 and it["seq"] == 0) == 512
+    # the trees alone: more than half of the pages, so all stay on the decode/verify path
+    alone = pk.inspect(lens[:6], qlens[:6], kinds[:6], parents, head_dim=128, **kw)
+    assert not any(it["kind"] == 2 for it in alone)

@@ -14,7 +14,7 @@ import torch
 
 import paged_kv_attention_verify_b200 as pk
 import workloads as W
-from _util import assert_close, oracle_rows
+from _util import assert_close, oracle_rows, tc_verify_seqs
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -135,14 +135,27 @@ def test_append_with_row_split_verify_tasks():
     """A mixed batch whose verify trees (5 tokens x 7 heads = 35 packed rows per KV head) run
     as row-split tasks, one of them split over its long context: the append patches the new
     rows into the pages every consumer warp reads, and one task per (sequence, KV head) writes
-    the cache."""
+    the cache. (head_dim 64: at 128 these trees run as tensor-core tasks, tested below.)"""
     gen = torch.Generator().manual_seed(8)
     seqs = [W.SeqSpec(2500, 1, W.CAUSAL, []) for _ in range(6)] + \
         [W.SeqSpec(9000 + 5, 5, W.TREE, W.random_tree(gen, 5)), W.SeqSpec(300 + 5, 5, W.TREE, W.random_tree(gen, 5))]
-    b = W.build_batch("append_row_split", seqs, 28, 4, 128, seed=81, device=DEV)
+    b = W.build_batch("append_row_split", seqs, 28, 4, 64, seed=81, device=DEV)
     items = pk.inspect(b.seq_lens, b.query_lens, b.mask_kinds, b.parents_flat, num_q_heads=28, num_kv_heads=4,
-                       head_dim=128, num_pages=b.k_cache.shape[0], bt_stride=b.block_table.shape[1],
+                       head_dim=64, num_pages=b.k_cache.shape[0], bt_stride=b.block_table.shape[1],
                        num_sms=torch.cuda.get_device_properties(0).multi_processor_count, ctas_per_sm=3)
     wide = [it for it in items if it["row_count"] > 16]
     assert wide and any(it["num_splits"] > 1 for it in wide)
+    run_append_case(b, expect_identical=True)
+
+
+def test_append_with_tensor_core_verify_tasks():
+    """Verify trees and short causal chunks of 20 to 120 packed rows per KV head run as
+    tensor-core tasks over their own keys: under fused append the producers patch the new
+    tokens' K / V rows (NaN in the cache beforehand) from the dense input into the tiles, the
+    task with the last KV tiles writes them into the cache, and the output is bitwise that of
+    attn_run over the appended cache."""
+    b = W.build_batch("append_tc_verify", tc_verify_seqs(), 16, 4, 128, seed=83, device=DEV)
+    plan = pk.plan_for_batch(b)
+    assert plan.info()["num_cascade_items"] > 0
+    plan.close()
     run_append_case(b, expect_identical=True)

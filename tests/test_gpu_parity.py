@@ -11,7 +11,7 @@ import torch
 
 import paged_kv_attention_verify_b200 as pk
 import workloads as W
-from _util import assert_close, oracle_rows
+from _util import assert_close, oracle_rows, tc_verify_seqs
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -235,6 +235,27 @@ def test_unified_batch_classes_alone():
         plan.close()
 
 
+@pytest.mark.parametrize("Hq, Hkv", [(16, 4), (28, 4), (32, 2)])
+def test_tensor_core_verify_tasks_all_rows(Hq, Hkv):
+    """Rows of 17 to 128 per KV head with at least 512 keys run as tensor-core tasks over their
+    own keys (one pass for all rows, the two warpgroups' halves of the KV tiles combined),
+    including KV chunks merged as split partials; every row against the oracle, and a second
+    run is bitwise the same. With 28 / 4 and 32 / 2 heads some units exceed 128 rows and stay
+    on the decode/verify path beside them."""
+    b = W.build_batch("tc_verify", tc_verify_seqs(), Hq, Hkv, 128, seed=94, device=DEV)
+    items = pk.inspect(b.seq_lens, b.query_lens, b.mask_kinds, b.parents_flat, num_q_heads=Hq,
+                       num_kv_heads=Hkv, head_dim=128, num_pages=b.k_cache.shape[0],
+                       bt_stride=b.block_table.shape[1],
+                       num_sms=torch.cuda.get_device_properties(0).multi_processor_count, ctas_per_sm=3)
+    assert any(it["kind"] == 2 for it in items)
+    out, plan = run_batch(b)
+    rows, exp = oracle_rows(b)
+    assert_close(out[rows], exp, f"tensor-core verify Hq={Hq} Hkv={Hkv}")
+    again = plan.run(b.q, b.k_cache, b.v_cache)
+    assert plan.check() == 0
+    assert torch.equal(out, again)
+
+
 def test_row_split_verify_tasks_all_rows():
     """Verify trees of 35 and 48 packed rows per KV head among decode steps run as row-split
     tasks (one warp streams each page once, three own 16 rows each), split over long contexts
@@ -245,9 +266,10 @@ def test_row_split_verify_tasks_all_rows():
         [W.SeqSpec(12000 + 5, 5, W.TREE, W.random_tree(gen, 5)), W.SeqSpec(600 + 5, 5, W.TREE, W.random_tree(gen, 5)),
          W.SeqSpec(37 + 6, 6, W.TREE, W.random_tree(gen, 6))]
     for Hq, Hkv in ((28, 4), (32, 2)):        # 35 / 42 rows; 80 / 96 rows (48-row tasks plus 16-row ones)
-        b = W.build_batch("row_split", seqs, Hq, Hkv, 128, seed=91, device=DEV)
+        # head_dim 64: at 128 the longer trees run as tensor-core tasks instead
+        b = W.build_batch("row_split", seqs, Hq, Hkv, 64, seed=91, device=DEV)
         items = pk.inspect(b.seq_lens, b.query_lens, b.mask_kinds, b.parents_flat, num_q_heads=Hq,
-                           num_kv_heads=b.num_kv_heads, head_dim=128, num_pages=b.k_cache.shape[0],
+                           num_kv_heads=b.num_kv_heads, head_dim=64, num_pages=b.k_cache.shape[0],
                            bt_stride=b.block_table.shape[1],
                            num_sms=torch.cuda.get_device_properties(0).multi_processor_count, ctas_per_sm=3)
         assert any(it["row_count"] > 16 for it in items)
