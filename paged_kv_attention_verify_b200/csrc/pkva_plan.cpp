@@ -564,7 +564,10 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
     //    tensor-core verify tasks, heaviest first by the KV tiles each query tile runs) and
     //    the decode tasks (heaviest first) are merged in proportion, so tensor-core blocks
     //    (latency) run beside decode blocks (HBM) from start to end instead of one kind
-    //    forming the tail. Decode tasks go three to a block, neighbours in the sorted list.
+    //    forming the tail; the tensor-core list runs 1.25x ahead of its share, so that its
+    //    long blocks are not the last to finish (measured on the Qwen2-7B-shaped unified
+    //    batch: 0.1638 against 0.166 ms in plain proportion; 1.75x ahead, 0.172 ms). Decode
+    //    tasks go three to a block, neighbours in the sorted list.
     std::vector<int32_t> tc;                  // block entries of the tensor-core list
     std::vector<int> tc_cost;
     for (size_t i = 0; i < p.pwork.size(); ++i) {
@@ -588,7 +591,7 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
     int ip = 0, id = 0;
     while (ip < np || id < nd) {
         // take from the list that is further behind in its share of the launch
-        const bool take_p = id >= nd || (ip < np && (int64_t)ip * nd <= (int64_t)id * np);
+        const bool take_p = id >= nd || (ip < np && (int64_t)ip * nd * 4 <= (int64_t)(id + 1) * np * 5);
         if (take_p)
             p.order.push_back(tc[tci[ip++]]);
         else
