@@ -62,3 +62,15 @@ def tc_verify_seqs():
         W.SeqSpec(128 * 5 + 1, 1, W.CAUSAL, []),
         W.SeqSpec(600, 32, W.TREE, W.random_tree(gen, 32)),         # 128 rows: a full tile
     ]
+
+
+def tc_verify_wide_seqs():
+    """Decode steps beside tensor-core verify units at their row limit (8 query / 4 KV heads:
+    64-node trees = 128 packed rows, a 63-token causal chunk = 126 rows, a 40-node chain)."""
+    gen = torch.Generator().manual_seed(21)
+    return [W.SeqSpec(2000 + 9 * i, 1, W.CAUSAL, []) for i in range(12)] + [
+        W.SeqSpec(700 + 64, 64, W.TREE, W.random_tree(gen, 64)),
+        W.SeqSpec(740 + 64, 64, W.TREE, W.random_tree(gen, 64)),       # new keys 740..803 cross 768
+        W.SeqSpec(4000 + 63, 63, W.CAUSAL, []),                         # 32 KV tiles: two chunks
+        W.SeqSpec(1000 + 40, 40, W.TREE, list(range(-1, 39))),          # a chain
+    ]

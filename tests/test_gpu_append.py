@@ -14,7 +14,7 @@ import torch
 
 import paged_kv_attention_verify_b200 as pk
 import workloads as W
-from _util import assert_close, oracle_rows, tc_verify_seqs
+from _util import assert_close, oracle_rows, tc_verify_seqs, tc_verify_wide_seqs
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -158,4 +158,12 @@ def test_append_with_tensor_core_verify_tasks():
     plan = pk.plan_for_batch(b)
     assert plan.info()["num_cascade_items"] > 0
     plan.close()
+    run_append_case(b, expect_identical=True)
+
+
+def test_append_with_tensor_core_verify_tasks_at_the_row_limit():
+    """As above with 128-row tensor-core verify tiles (64-node trees under a group of 2), new
+    keys across a KV-tile boundary and a causal chunk split into two KV chunks: the patched
+    rows span two tiles and the task that writes the cache is the unit's last."""
+    b = W.build_batch("append_tc_verify_wide", tc_verify_wide_seqs(), 8, 4, 128, seed=84, device=DEV)
     run_append_case(b, expect_identical=True)

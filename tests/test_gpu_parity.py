@@ -11,7 +11,7 @@ import torch
 
 import paged_kv_attention_verify_b200 as pk
 import workloads as W
-from _util import assert_close, oracle_rows, tc_verify_seqs
+from _util import assert_close, oracle_rows, tc_verify_seqs, tc_verify_wide_seqs
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -254,6 +254,24 @@ def test_tensor_core_verify_tasks_all_rows(Hq, Hkv):
     again = plan.run(b.q, b.k_cache, b.v_cache)
     assert plan.check() == 0
     assert torch.equal(out, again)
+
+
+def test_tensor_core_verify_tasks_wide_trees_and_chunks():
+    """Tensor-core verify tasks at their limits: 64-node trees under a group of 2 (128 packed
+    rows, ancestor bits across all four 32-column mask words), one with its new keys across a
+    KV-tile boundary, a 63-token causal chunk (126 rows) split into two chunks of 16 KV
+    tiles, and a 40-node chain; every row against the oracle."""
+    b = W.build_batch("tc_verify_wide", tc_verify_wide_seqs(), 8, 4, 128, seed=95, device=DEV)
+    items = pk.inspect(b.seq_lens, b.query_lens, b.mask_kinds, b.parents_flat, num_q_heads=8,
+                       num_kv_heads=4, head_dim=128, num_pages=b.k_cache.shape[0],
+                       bt_stride=b.block_table.shape[1],
+                       num_sms=torch.cuda.get_device_properties(0).multi_processor_count, ctas_per_sm=3)
+    assert {it["seq"] for it in items if it["kind"] == 2} == {12, 13, 14, 15}
+    assert any(it["kind"] == 2 and it["num_splits"] > 1 for it in items)
+    out, plan = run_batch(b)
+    rows, exp = oracle_rows(b)
+    assert_close(out[rows], exp, "tensor-core verify, 128-row tiles")
+    plan.close()
 
 
 def test_row_split_verify_tasks_all_rows():
