@@ -401,7 +401,7 @@ typedef struct pkva_work_desc {
                          /* lists the tensor-core verify tasks: a verify tree (or causal   */
                          /* chunk) of 17 to 128 packed rows per KV head, outside any       */
                          /* caller group, with at least 512 keys runs as such tasks over   */
-                         /* all of its keys (masked), chunks of 16 KV tiles of 128 keys,   */
+                         /* all of its keys (masked), chunks of 32 KV tiles of 128 keys,   */
                          /* and has no decode/verify task (head_dim 128, bf16 caches), in  */
                          /* a batch where such sequences hold at most half of the          */
                          /* decode/verify pages                                            */

@@ -20,7 +20,7 @@ constexpr int kPrefillMinTokens = 64;  // causal sequences with at least this ma
                                        // (and head_dim 128) run on the tensor-core prefill kernel
 constexpr int kCascadeTilesPerTask = 16; // shared-prefix KV tiles (128 keys) per cascade task
 constexpr int kOwnMinKeys = 512;         // keys from which a verify tree's rows run on the tensor cores
-constexpr int kOwnTilesPerTask = 16;     // KV tiles (128 keys) per tensor-core verify task
+constexpr int kOwnTilesPerTask = 32;     // KV tiles (128 keys) per tensor-core verify task
 
 // Per-sequence record (the "Token-Table" row of the batch).
 struct SeqInfo {

@@ -55,7 +55,7 @@ def tc_verify_seqs():
     return [W.SeqSpec(3000 + 7 * i, 1, W.CAUSAL, []) for i in range(6)] + [
         W.SeqSpec(640 + 7, 7, W.TREE, W.random_tree(gen, 7)),       # new keys start a KV tile
         W.SeqSpec(766 + 6, 6, W.TREE, W.random_tree(gen, 6)),       # new keys cross a tile boundary
-        W.SeqSpec(4100, 5, W.TREE, W.random_tree(gen, 5)),          # three chunks of 16 KV tiles
+        W.SeqSpec(4100, 5, W.TREE, W.random_tree(gen, 5)),          # two chunks of KV tiles
         W.SeqSpec(1000 + 20, 20, W.CAUSAL, []),                     # a short causal chunk: 80 rows
         W.SeqSpec(2500, 30, W.CAUSAL, []),                          # 120 rows
         W.SeqSpec(513, 8, W.TREE, W.random_tree(gen, 8)),           # one key past the threshold
@@ -71,6 +71,6 @@ def tc_verify_wide_seqs():
     return [W.SeqSpec(2000 + 9 * i, 1, W.CAUSAL, []) for i in range(12)] + [
         W.SeqSpec(700 + 64, 64, W.TREE, W.random_tree(gen, 64)),
         W.SeqSpec(740 + 64, 64, W.TREE, W.random_tree(gen, 64)),       # new keys 740..803 cross 768
-        W.SeqSpec(4000 + 63, 63, W.CAUSAL, []),                         # 32 KV tiles: two chunks
+        W.SeqSpec(4500 + 63, 63, W.CAUSAL, []),                         # 36 KV tiles: two chunks
         W.SeqSpec(1000 + 40, 40, W.TREE, list(range(-1, 39))),          # a chain
     ]

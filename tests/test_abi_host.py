@@ -348,7 +348,7 @@ def test_verify_units_wider_than_32_rows_are_row_split_tasks_in_mixed_batches():
 def test_verify_trees_run_as_tensor_core_tasks():
     """Beside decode steps, a tree of 17 to 128 packed rows per KV head with at least 512 keys
     runs as cascade-kind tensor-core tasks over all of its keys, one per KV head and chunk of
-    16 KV tiles (2048 keys), with no decode/verify task. A 64-token tree (448 rows), a tree of
+    32 KV tiles (4096 keys), with no decode/verify task. A 64-token tree (448 rows), a tree of
     16 rows or fewer, fewer than 512 keys, head_dim 64, and members of the caller's
     shared-prefix groups keep the decode/verify path (a group member's shared prefix stays a
     cascade task); so does every tree of a batch where such trees hold more than half of the
@@ -362,16 +362,16 @@ def test_verify_trees_run_as_tensor_core_tasks():
     items = pk.inspect(lens, qlens, kinds, parents, head_dim=128, **kw)
     casc = sorted((it["seq"], it["kv_head"], it["key_begin"], it["key_end"], it["row_count"], it["split"],
                    it["num_splits"]) for it in items if it["kind"] == 2)
-    split5 = [(0, 1664, 0), (1664, 3328, 1), (3328, 5000, 2)]      # 40 tiles in three chunks
+    split5 = [(0, 2560, 0), (2560, 5000, 1)]                      # 40 tiles in two chunks
     assert casc == [(0, h, 0, 2000, 5, 0, 1) for h in range(4)] + [(2, h, 0, 700, 3, 0, 1) for h in range(4)] + \
-        [(5, h, kb, ke, 5, k, 3) for h in range(4) for kb, ke, k in split5]
+        [(5, h, kb, ke, 5, k, 2) for h in range(4) for kb, ke, k in split5]
     assert not any(it["kind"] == 0 and it["seq"] in (0, 2, 5) for it in items)
     assert {it["seq"] for it in items if it["kind"] == 0} == {1, 3, 4} | set(range(6, 16))
     assert not any(it["kind"] == 2 for it in pk.inspect(lens, qlens, kinds, parents, head_dim=64, **kw))
     grouped = pk.inspect(lens, qlens, kinds, parents, head_dim=128, prefix_group=[0] + [-1] * 15, prefix_len=[512],
                          **kw)
     assert sorted({(it["seq"], it["key_end"]) for it in grouped if it["kind"] == 2}) == \
-        [(0, 512), (2, 700), (5, 1664), (5, 3328), (5, 5000)]
+        [(0, 512), (2, 700), (5, 2560), (5, 5000)]
     assert min(it["key_begin"] for it in grouped if it["kind"] == 0 and it["seq"] == 0) == 512
     # the trees alone: more than half of the pages, so all stay on the decode/verify path
     alone = pk.inspect(lens[:6], qlens[:6], kinds[:6], parents, head_dim=128, **kw)

@@ -259,8 +259,8 @@ def test_tensor_core_verify_tasks_all_rows(Hq, Hkv):
 def test_tensor_core_verify_tasks_wide_trees_and_chunks():
     """Tensor-core verify tasks at their limits: 64-node trees under a group of 2 (128 packed
     rows, ancestor bits across all four 32-column mask words), one with its new keys across a
-    KV-tile boundary, a 63-token causal chunk (126 rows) split into two chunks of 16 KV
-    tiles, and a 40-node chain; every row against the oracle."""
+    KV-tile boundary, a 63-token causal chunk (126 rows) split into two chunks of KV tiles,
+    and a 40-node chain; every row against the oracle."""
     b = W.build_batch("tc_verify_wide", tc_verify_wide_seqs(), 8, 4, 128, seed=95, device=DEV)
     items = pk.inspect(b.seq_lens, b.query_lens, b.mask_kinds, b.parents_flat, num_q_heads=8,
                        num_kv_heads=4, head_dim=128, num_pages=b.k_cache.shape[0],
