@@ -274,6 +274,24 @@ def test_tensor_core_verify_tasks_wide_trees_and_chunks():
     plan.close()
 
 
+@pytest.mark.parametrize("seed", range(200, 216))
+def test_random_mixed_batches_with_tensor_core_verify(seed):
+    """Random mixed batches at head_dim 128 (4 to 13 sequences, contexts up to 3000 keys,
+    trees of up to 32 nodes, causal chunks of up to 40 tokens, six head shapes): where verify
+    units qualify and are a minority of the pages they run as tensor-core verify tasks,
+    elsewhere on the decode/verify path. Every row against the oracle."""
+    g = torch.Generator().manual_seed(seed)
+    Hq, Hkv = [(8, 2), (16, 4), (28, 4), (32, 8), (8, 4), (32, 2)][seed % 6]
+    ns = int(torch.randint(4, 14, (1,), generator=g))
+    b = W.random_small(seed, num_seqs=ns, Hq=Hq, Hkv=Hkv, d=128,
+                       max_ctx=int(torch.randint(300, 3000, (1,), generator=g)),
+                       max_q=int(torch.randint(2, 40, (1,), generator=g)), tree_frac=0.6,
+                       max_draft=int(torch.randint(2, 33, (1,), generator=g)), device=DEV, bt_extra=1)
+    out, plan = run_batch(b)
+    rows, exp = oracle_rows(b)
+    assert_close(out[rows], exp, f"random mixed batch {seed}")
+
+
 def test_row_split_verify_tasks_all_rows():
     """Verify trees of 35 and 48 packed rows per KV head among decode steps run as row-split
     tasks (one warp streams each page once, three own 16 rows each), split over long contexts
