@@ -138,8 +138,10 @@ PKVA_API int attn_plan(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq_l
  * head) rows of a run of members, floor(128 / (Hq/Hkv)) tokens x all heads of one KV head
  * per tensor-core tile, against the shared keys in chunks of 2048; each member then merges
  * those partial results with its own keys' (split-KV combine). Members that run as prefill
- * tasks (causal chunks of >= 64 tokens) read their whole prefix as before. Needs head_dim
- * 128 when any prefix_len > 0 (else PKVA_EUNSUPPORTED). Errors as attn_plan.
+ * tasks (causal chunks of >= 64 tokens) read their whole prefix as before. Cascade and
+ * prefill tasks run at head_dim 64 and 128 over bf16 caches. Over FP8 caches
+ * (attn_plan_shared_kv), any prefix_len > 0 needs head_dim 128, else PKVA_EUNSUPPORTED.
+ * Errors as attn_plan.
  */
 PKVA_API int attn_plan_shared(pkva_plan_t* out_plan, int num_seqs, const int32_t* seq_lens,
               const int32_t* query_lens, const int32_t* block_table, int bt_stride,
@@ -156,7 +158,8 @@ PKVA_API int attn_plan_shared(pkva_plan_t* out_plan, int num_seqs, const int32_t
  * bytes of the bandwidth-bound decode/verify path.
  *
  * An FP8 plan splits the batch as attn_plan does. Its decode/verify tasks read the E4M3
- * pages directly; its tensor-core (prefill) tasks, head_dim 128 only, read bf16 copies of
+ * pages directly; its tensor-core (prefill) tasks, head_dim 128 only (at 64 the chunks run
+ * as decode/verify tasks), read bf16 copies of
  * their sequences' pages (the codes' exact values), which each run stages first in a second
  * launch on the same stream. The plan owns that staging memory: 2 x 2 bytes x Hkv x
  * page_size x D per page of every such sequence (counted in scratch_bytes). It cannot be

@@ -50,7 +50,8 @@ struct AttnSmem {
                   "one-n-tile tasks fit a task's share");
     static constexpr int GROUP_BYTES = (DC::BYTES + 1023) / 1024 * 1024;    // one decode task
     static constexpr int DEC_BYTES = kDecTasksPerBlock * GROUP_BYTES;
-    static constexpr int TASK_BYTES = (D == 128 && TC && pre::kSmemBytes > DEC_BYTES) ? pre::kSmemBytes : DEC_BYTES;
+    static constexpr int TASK_BYTES =
+        (TC && pre::Lay<D>::kSmemBytes > DEC_BYTES) ? pre::Lay<D>::kSmemBytes : DEC_BYTES;
     static constexpr int OFF_SCHED = TASK_BYTES;  // the TMEM address of a tensor-core block
     static constexpr int BYTES = TASK_BYTES + 64;
     static constexpr int ALLOC = BYTES + 1008;    // room to align to 1024
@@ -61,6 +62,7 @@ struct AttnSmem {
 };
 
 // FP8: decode/verify tasks read the E4M3 pages; tensor-core tasks read their bf16 staging copies.
+// Tensor-core tasks run at head_dim 128 and, over bf16 caches, 64.
 template <int D, int NT, bool FP8, bool TC>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -70,7 +72,7 @@ attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const _
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int e = p.order[blockIdx.x];
-    if constexpr (D == 128 && TC) {
+    if constexpr (TC) {
         if (e >= 0) {
             // tensor-core task: 512 TMEM columns for the block (one block per SM)
             uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + S::OFF_SCHED);
@@ -84,7 +86,7 @@ attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const _
             tc_fence_after();
             const uint32_t tmem = *tmem_slot;
             // over FP8 caches the tensor-core tasks read the bf16 staging pages (tmKn / tmVn)
-            pre::prefill_task(p.pre, e, tmQ, FP8 ? tmKn : tmK, FP8 ? tmVn : tmV, tmKn, tmVn, tmQc, tmem, sm);
+            pre::prefill_task<D>(p.pre, e, tmQ, FP8 ? tmKn : tmK, FP8 ? tmVn : tmV, tmKn, tmVn, tmQc, tmem, sm);
             tc_fence_before();
             __syncthreads();
             tc_fence_after();
@@ -92,7 +94,7 @@ attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const _
             return;
         }
     }
-    if (e >= 0) return;                          // (never planned: tensor-core tasks need head_dim 128)
+    if (e >= 0) return;                          // (never planned: a launch without tensor-core code)
     // decode block: warps 4g .. 4g+3 run task g of the block's three
     const int g = threadIdx.x >> 7;
     const int task = (-1 - e) * kDecTasksPerBlock + g;
@@ -134,7 +136,7 @@ cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tmQ, const CUtensor
 
 template <int D, int NT>
 int ctas_t() {
-    constexpr bool TC = D == 128;
+    constexpr bool TC = true;
     using S = AttnSmem<D, NT, false, TC>;
     int n = 0;
     if (cudaFuncSetAttribute(attn_kernel<D, NT, false, TC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -150,9 +152,13 @@ template <bool FP8, bool TC>
 cudaError_t launch_kv(const AttnParams& p, int D, int rows, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                       const CUtensorMap& tmV, const CUtensorMap& tmKn, const CUtensorMap& tmVn,
                       const CUtensorMap& tmQc, cudaStream_t stream) {
-    if (D == 64)
-        return rows <= 8 ? launch_t<64, 1, FP8, false>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
-                         : launch_t<64, 2, FP8, false>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
+    if (D == 64) {
+        // head_dim 64 tensor-core tasks run over bf16 caches only (the FP8 staging copies are
+        // head_dim 128)
+        constexpr bool TC64 = TC && !FP8;
+        return rows <= 8 ? launch_t<64, 1, FP8, TC64>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
+                         : launch_t<64, 2, FP8, TC64>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
+    }
     return rows <= 8 ? launch_t<128, 1, FP8, TC>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
                      : launch_t<128, 2, FP8, TC>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
 }
@@ -168,7 +174,7 @@ int attn_ctas_per_sm(int D, int rows) {
 cudaError_t launch_attn(const AttnParams& p, int D, int rows, bool has_prefill, const CUtensorMap& tmQ,
                         const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKn,
                         const CUtensorMap& tmVn, const CUtensorMap& tmQc, cudaStream_t stream, bool fp8) {
-    if (D == 64 && has_prefill) return cudaErrorInvalidValue;   // tensor-core tasks: head_dim 128
+    if (D == 64 && fp8 && has_prefill) return cudaErrorInvalidValue;   // (never planned)
     // plans without tensor-core tasks launch the TC = false code (no prefill body in it)
     if (!fp8)
         return has_prefill ? launch_kv<false, true>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)

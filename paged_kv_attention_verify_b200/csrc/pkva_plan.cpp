@@ -154,8 +154,9 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
                                 "prefix_len of group %ld (%ld) exceeds the committed prefix of sequence %ld", g, P, s);
             }
             if (P == 0) continue;
-            if (a.D != 128)
-                return fail(err, PKVA_EUNSUPPORTED, "shared-prefix groups need head_dim 128 (got %ld)", a.D);
+            if (a.D != 128 && a.kv_elem_bytes != 2)
+                return fail(err, PKVA_EUNSUPPORTED,
+                            "shared-prefix groups over FP8 caches need head_dim 128 (got %ld)", a.D);
             if (p.G > kPrefillTileM)
                 return fail(err, PKVA_EUNSUPPORTED, "shared-prefix groups need at most 128 query heads per KV head");
             for (int s = first[g]; s <= last[g]; ++s) grp_of[s] = g;
@@ -168,7 +169,9 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
 
     // -- prefill tiles: long causal chunks go to the tensor-core prefill kernel ---------
     std::vector<char> on_prefill(a.num_seqs, 0);
-    if (a.use_prefill_kernel && a.D == 128) {
+    // tensor-core tasks: head_dim 128, and 64 over bf16 caches (the FP8 staging copies are 128)
+    const bool tc_ok = a.use_prefill_kernel && (a.D == 128 || a.kv_elem_bytes == 2);
+    if (tc_ok) {
         for (int s = 0; s < a.num_seqs; ++s) {
             const SeqInfo& si = p.seqs[s];
             if (si.mask_kind != PKVA_CAUSAL || si.query_len < kPrefillMinTokens) continue;
@@ -233,7 +236,7 @@ int build_host_plan(const PlanArgs& a, HostPlan* out, std::string* err) {
     //    Qwen2-7B verify class 0.0614 against 0.0655 ms, the unified batch 0.170 against
     //    0.166 ms).
     std::vector<char> on_own(a.num_seqs, 0);
-    if (a.self_cascade && a.use_prefill_kernel && a.D == 128 && a.kv_elem_bytes == 2 && p.G <= kPrefillTileM) {
+    if (a.self_cascade && tc_ok && a.D == 128 && a.kv_elem_bytes == 2 && p.G <= kPrefillTileM) {
         int64_t own_pages = 0, all_pages = 0;
         for (int s = 0; s < a.num_seqs; ++s) {
             if (on_prefill[s]) continue;

@@ -65,6 +65,23 @@ constexpr int kOffBar = kOffV + kNV * kTileBytes;
 constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 2 + 2 + 2 + 1 + 1 + 1;
 constexpr int kOffFlag = kOffBar + kNumBars * 8;         // the task's abort flag
 constexpr int kSmemBytes = kOffFlag + 16;
+
+// The layout above for head_dim D (64 or 128): Q, K and V tiles are 128 rows of D bf16 in
+// D / 64 swizzle halves; S stays 128 x 128 (keys), O is 128 x D.
+template <int D>
+struct Lay {
+    static_assert(D == 64 || D == 128, "tensor-core tasks: head_dim 64 or 128");
+    static constexpr int kHalves = D / 64;
+    static constexpr int kTileBytes = kHalves * kHalfBytes;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + 2 * kTileBytes;
+    static constexpr int kOffV = kOffK + kNK * kTileBytes;
+    static constexpr int kOffBar = kOffV + kNV * kTileBytes;
+    static constexpr int kOffFlag = kOffBar + kNumBars * 8;
+    static constexpr int kSmemBytes = kOffFlag + 16;
+    static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);   // P from TMEM, V MN-major
+};
+static_assert(Lay<128>::kSmemBytes == kSmemBytes, "head_dim 128 layout");
 constexpr int kSmemAlloc = kSmemBytes + 1008;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;
@@ -89,8 +106,9 @@ struct Bars {
     uint64_t* k_fix;         // a K tile the producer patches before releasing it
 };
 
+template <int D>
 __device__ __forceinline__ Bars bars_at(uint8_t* sm) {
-    uint64_t* b = reinterpret_cast<uint64_t*>(sm + kOffBar);
+    uint64_t* b = reinterpret_cast<uint64_t*>(sm + Lay<D>::kOffBar);
     Bars r;
     r.q_full = b;
     r.k_full = b + 1;
@@ -145,12 +163,14 @@ __device__ __forceinline__ void tile_rows(const PrefillParams& p, const int32_t*
     }
 }
 
+template <int D>
 __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, const int rows[8]) {
-    mbar_arrive_expect_tx(bar, kTileBytes);
+    mbar_arrive_expect_tx(bar, Lay<D>::kTileBytes);
 #pragma unroll
     for (int pg = 0; pg < 8; ++pg)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) tma_load_2d(dst + h * kHalfBytes + pg * (kPageSize * 128), map, bar, h * 64, rows[pg]);
+        for (int h = 0; h < Lay<D>::kHalves; ++h)
+            tma_load_2d(dst + h * kHalfBytes + pg * (kPageSize * 128), map, bar, h * 64, rows[pg]);
 }
 
 // One prefill task; every thread of the block (at least kPThreads) calls it; warps past
@@ -171,10 +191,12 @@ __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, 
 // same rows (Q loaded once), tile b takes the KV tiles j with j % 2 == b, so the tensor
 // cores run one half's PV and next QK^T while the other half's softmax runs, and the two
 // halves' (max, sum, output) are combined before the partial is written.
+template <int D>
 __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, const CUtensorMap& tmQ,
                                              const CUtensorMap& tmK, const CUtensorMap& tmV,
                                              const CUtensorMap& tmKn, const CUtensorMap& tmVn,
                                              const CUtensorMap& tmQc, uint32_t tmem, uint8_t* sm) {
+    using L = Lay<D>;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool cascade = task >= p.num_prefill;
     const int ci = task - p.num_prefill;
@@ -189,8 +211,8 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         w = p.work[task];
     }
     const SeqInfo si = p.seqs[w.seq];
-    const Bars B = bars_at(sm);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffFlag);
+    const Bars B = bars_at<D>(sm);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kOffFlag);
     const bool append = p.append != 0 && !cascade;
     const int TOK = p.cascade_tok;                      // cascade: tokens per query tile
     const bool il = cascade && cw.ntok <= TOK;          // one query tile, KV tiles interleaved
@@ -249,22 +271,22 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
                 prefetch_tensormap(&tmQc);
                 prefetch_tensormap(&tmK);
                 const int nq = il ? 1 : 2;                 // interleaved: both halves read Q tile 0
-                mbar_arrive_expect_tx(B.q_full, 2u * (uint32_t)nq * (uint32_t)(p.G * TOK) * 128u);
+                mbar_arrive_expect_tx(B.q_full, (uint32_t)L::kHalves * (uint32_t)nq * (uint32_t)(p.G * TOK) * 128u);
                 for (int b = 0; b < nq; ++b)
 #pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        tma_load_3d(sm + kOffQ + b * kTileBytes + h * kHalfBytes, &tmQc, B.q_full, h * 64,
+                    for (int h = 0; h < L::kHalves; ++h)
+                        tma_load_3d(sm + L::kOffQ + b * L::kTileBytes + h * kHalfBytes, &tmQc, B.q_full, h * 64,
                                     kvh * p.G, cw.tok0 + b * TOK);
             } else if (is_k) {
                 prefetch_tensormap(&tmQ);
                 prefetch_tensormap(&tmK);
                 if (append) prefetch_tensormap(&tmKn);
-                mbar_arrive_expect_tx(B.q_full, 2 * kTileBytes);
+                mbar_arrive_expect_tx(B.q_full, 2 * L::kTileBytes);
 #pragma unroll
                 for (int b = 0; b < 2; ++b)
 #pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        tma_load_3d(sm + kOffQ + b * kTileBytes + h * kHalfBytes, &tmQ, B.q_full, h * 64,
+                    for (int h = 0; h < L::kHalves; ++h)
+                        tma_load_3d(sm + L::kOffQ + b * L::kTileBytes + h * kHalfBytes, &tmQ, B.q_full, h * 64,
                                     b ? w.q_head1 : w.q_head, si.q_start + (b ? w.tok1 : w.tok0));
             } else {
                 prefetch_tensormap(&tmV);
@@ -275,21 +297,21 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         uint64_t* full = is_k ? B.k_full : B.v_full;
         uint64_t* empty = is_k ? B.k_empty : B.v_empty;
         uint64_t* fixbar = is_k ? B.k_fix : B.v_fix;
-        uint8_t* base = sm + (is_k ? kOffK : kOffV);
+        uint8_t* base = sm + (is_k ? L::kOffK : L::kOffV);
         int nfix = 0;                                  // phases of fixbar used
         for (int j = 0; j < nmax; ++j) {
             const int st = j % NSt;
             if (j >= NSt &&
                 !__all_sync(0xffffffffu, wait_or_abort(&empty[st], ((j / NSt) - 1) & 1, p.err, abort_flag)))
                 break;
-            uint8_t* dst = base + st * kTileBytes;
+            uint8_t* dst = base + st * L::kTileBytes;
             if (j >= nc) {
                 // new tokens [128 (j - nc), +128) of the chunk, straight from the input
                 if (lane == 0) {
                     const int row0 = si.q_start + (j - nc) * kPrefillTileN;
-                    mbar_arrive_expect_tx(&full[st], kTileBytes);
+                    mbar_arrive_expect_tx(&full[st], L::kTileBytes);
 #pragma unroll
-                    for (int h = 0; h < 2; ++h)
+                    for (int h = 0; h < L::kHalves; ++h)
                         tma_load_3d(dst + h * kHalfBytes, is_k ? &tmKn : &tmVn, &full[st], h * 64, kvh, row0);
                 }
                 continue;
@@ -302,26 +324,26 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
             const bool patch = own && p.append && kb + kPrefillTileN > prefix && kb < si.seq_len;
             const bool zero = !is_k && j == fix_tile;
             if (!patch && !zero) {
-                if (lane == 0) load_tile(dst, is_k ? &tmK : &tmV, &full[st], rows);
+                if (lane == 0) load_tile<D>(dst, is_k ? &tmK : &tmV, &full[st], rows);
                 continue;
             }
-            if (lane == 0) load_tile(dst, is_k ? &tmK : &tmV, fixbar, rows);
+            if (lane == 0) load_tile<D>(dst, is_k ? &tmK : &tmV, fixbar, rows);
             if (!__all_sync(0xffffffffu, wait_or_abort(fixbar, nfix & 1, p.err, abort_flag))) break;
             ++nfix;
             if (patch) {
                 const int k0 = max(prefix, kb), k1 = min(si.seq_len, kb + kPrefillTileN);
                 const __nv_bfloat16* src = is_k ? p.k_new : p.v_new;
-                for (int idx = lane; idx < (k1 - k0) * 16; idx += 32) {
-                    const int key = k0 + (idx >> 4), c = idx & 15, r = key - kb;   // chunk c: half c / 8
+                for (int idx = lane; idx < (k1 - k0) * (D / 8); idx += 32) {
+                    const int key = k0 + idx / (D / 8), c = idx % (D / 8), r = key - kb;   // chunk c: half c / 8
                     const uint4 v = *reinterpret_cast<const uint4*>(
-                        src + ((int64_t)(si.q_start + key - prefix) * p.Hkv + kvh) * kD + c * 8);
+                        src + ((int64_t)(si.q_start + key - prefix) * p.Hkv + kvh) * D + c * 8);
                     *reinterpret_cast<uint4*>(dst + (c >> 3) * kHalfBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
                 }
             }
             if (zero) {
                 const int pg = (key_limit / kPageSize) % 8, r0 = key_limit % kPageSize;
-                for (int idx = lane; idx < (kPageSize - r0) * 16; idx += 32) {
-                    const int r = r0 + (idx >> 4), c = idx & 15;
+                for (int idx = lane; idx < (kPageSize - r0) * (D / 8); idx += 32) {
+                    const int r = r0 + idx / (D / 8), c = idx % (D / 8);
                     *reinterpret_cast<uint4*>(dst + (c >> 3) * kHalfBytes + (pg * kPageSize + r) * 128 + (c & 7) * 16) =
                         make_uint4(0u, 0u, 0u, 0u);
                 }
@@ -337,18 +359,18 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
     } else if (warp == kWarpMma) {
         // ------------------------------ MMA issuer -------------------------------------------
         if (lane == 0) {
-            const uint32_t q_base = smem_addr(sm + kOffQ);
-            const uint32_t k_base = smem_addr(sm + kOffK);
-            const uint32_t v_base = smem_addr(sm + kOffV);
+            const uint32_t q_base = smem_addr(sm + L::kOffQ);
+            const uint32_t k_base = smem_addr(sm + L::kOffK);
+            const uint32_t v_base = smem_addr(sm + L::kOffV);
             auto issue_qk = [&](int b, int j) {           // S_b = Q_b K_j^T (interleaved: Q_0)
                 const int st = j % kNK;
                 const uint32_t d = tmem + kColS + b * 128;
-                const uint32_t qt = q_base + (il ? 0 : b) * kTileBytes;
+                const uint32_t qt = q_base + (il ? 0 : b) * L::kTileBytes;
 #pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks) {
+                for (int ks = 0; ks < D / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * kHalfBytes + (ks & 3) * 32;
                     const uint64_t ad = smem_desc_sw128(qt + off, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(k_base + st * kTileBytes + off, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(k_base + st * L::kTileBytes + off, 16, 1024);
                     tc_mma_ss(d, ad, bd, kIdescQK, ks > 0);
                 }
                 tc_commit(&B.s_full[b]);
@@ -358,8 +380,8 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
                 const uint32_t pcol = tmem + kColS + b * 128;
 #pragma unroll
                 for (int ks = 0; ks < kPrefillTileN / 16; ++ks) {
-                    const uint64_t bd = smem_desc_sw128(v_base + st * kTileBytes + ks * 2048, kHalfBytes, 1024);
-                    tc_mma_ts(tmem + kColO + b * 128, pcol + ks * 8, bd, kIdescPV, (acc || ks > 0) ? 1u : 0u);
+                    const uint64_t bd = smem_desc_sw128(v_base + st * L::kTileBytes + ks * 2048, kHalfBytes, 1024);
+                    tc_mma_ts(tmem + kColO + b * D, pcol + ks * 8, bd, L::kIdescPV, (acc || ks > 0) ? 1u : 0u);
                 }
             };
             bool ok = wait_or_abort(B.q_full, 0, p.err, abort_flag) &&
@@ -454,7 +476,7 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         const int nb = b ? n1 : n0;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t s_addr = tmem + lane_off + kColS + b * 128;
-        const uint32_t o_addr = tmem + lane_off + kColO + b * 128;
+        const uint32_t o_addr = tmem + lane_off + kColO + b * D;
         const int row_in_task = (il ? 0 : b) * kPrefillTileM + r;   // interleaved: tile 0's rows
         // this tile's query head and tokens (a cascade task's rows come from its row map)
         const int qh = b ? w.q_head1 : w.q_head;
@@ -579,7 +601,7 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
                 // rescale O_b (done with S, so its registers are free). O_b is complete for
                 // tile j-1: S_b of tile j was committed after that PV was issued.
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < D / 32; ++c) {
                     uint32_t ov[32];
                     tmem_ld32(o_addr + c * 32, ov);
                     tmem_wait_ld();
@@ -600,7 +622,7 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
             if (il) {
                 // combine the halves: each warpgroup hands its (max, sum) over through Q tile
                 // 1's shared memory (never loaded in this mode), then writes half the columns
-                float* xch = reinterpret_cast<float*>(sm + kOffQ + kTileBytes);    // [2][128][2]
+                float* xch = reinterpret_cast<float*>(sm + L::kOffQ + L::kTileBytes);    // [2][128][2]
                 const bool mine = nb > 0 && alive;
                 xch[(b * kPrefillTileM + r) * 2] = mine ? m_ref : -INFINITY;
                 xch[(b * kPrefillTileM + r) * 2 + 1] = mine ? l_sum : 0.f;
@@ -615,12 +637,12 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
                                                                 (n1 == 0 || wait_or_abort(&B.o_ready[1], 0, p.err, abort_flag)));
                 if (waited && cw.own != 2) {
                     tc_fence_after();
-                    float* dst = p.part_o + (int64_t)(part_idx < 0 ? 0 : part_idx) * kD;
+                    float* dst = p.part_o + (int64_t)(part_idx < 0 ? 0 : part_idx) * D;
                     const float vsc = p.v_scale ? p.v_scale[kvh] : 1.f;
                     const float f0 = w0 * vsc, f1 = w1 * vsc;
-                    const uint32_t o0 = tmem + lane_off + kColO, o1 = o0 + 128;
+                    const uint32_t o0 = tmem + lane_off + kColO, o1 = o0 + D;
 #pragma unroll
-                    for (int c = 2 * b; c < 2 * b + 2; ++c) {
+                    for (int c = b * (D / 64); c < (b + 1) * (D / 64); ++c) {
                         uint32_t v0[32], v1[32];
                         if (n0 > 0) tmem_ld32(o0 + c * 32, v0);
                         if (n1 > 0) tmem_ld32(o1 + c * 32, v1);
@@ -650,10 +672,10 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
                     const float Lr = l0 * w0 + l1 * w1;
                     const float inv = (Lr > 0.f ? 1.f / Lr : 0.f) * (p.v_scale ? p.v_scale[kvh] : 1.f);
                     const float f0 = w0 * inv, f1 = w1 * inv;
-                    __nv_bfloat16* dst = p.out + ((int64_t)(si.q_start + r / p.G) * p.Hq + kvh * p.G + r % p.G) * kD;
-                    const uint32_t o0 = tmem + lane_off + kColO, o1 = o0 + 128;
+                    __nv_bfloat16* dst = p.out + ((int64_t)(si.q_start + r / p.G) * p.Hq + kvh * p.G + r % p.G) * D;
+                    const uint32_t o0 = tmem + lane_off + kColO, o1 = o0 + D;
 #pragma unroll
-                    for (int c = 2 * b; c < 2 * b + 2; ++c) {
+                    for (int c = b * (D / 64); c < (b + 1) * (D / 64); ++c) {
                         uint32_t v0[32], v1[32];
                         if (n0 > 0) tmem_ld32(o0 + c * 32, v0);
                         if (n1 > 0) tmem_ld32(o1 + c * 32, v1);
@@ -674,11 +696,11 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
                 }
             } else if (nb > 0 && alive && __all_sync(0xffffffffu, wait_or_abort(&B.o_ready[b], 0, p.err, abort_flag))) {
                 tc_fence_after();
-                float* dst = p.part_o + (int64_t)(part_idx < 0 ? 0 : part_idx) * kD;
+                float* dst = p.part_o + (int64_t)(part_idx < 0 ? 0 : part_idx) * D;
                 // FP8 caches: the V scale of this KV head, as on every other partial
                 const float vsc = p.v_scale ? p.v_scale[kvh] : 1.f;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < D / 32; ++c) {
                     uint32_t ov[32];
                     tmem_ld32(o_addr + c * 32, ov);
                     tmem_wait_ld();
@@ -698,7 +720,7 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
             // for their tiles' last PV), so the Q tiles' shared memory is free for the flags.
             __threadfence();
             asm volatile("bar.sync 1, 256;" ::: "memory");
-            int* cnt = reinterpret_cast<int*>(sm + kOffQ);      // [256] rows of each completed unit, else 0
+            int* cnt = reinterpret_cast<int*>(sm + L::kOffQ);      // [256] rows of each completed unit, else 0
             int* uid = cnt + 256;                                // [256]
             int* pref = uid + 256;                               // [256] compacted prefix sums
             int* cuid = pref + 256;                              // [256] compacted unit ids
@@ -727,7 +749,7 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
             __threadfence();
             const int total = totals[0], n_done = totals[1];
             if (n_done > 0)
-                merge_units<kD>(warp, 8, lane, cuid, pref, n_done, total, p.units, p.part_o, p.part_ml, p.seqs,
+                merge_units<D>(warp, 8, lane, cuid, pref, n_done, total, p.units, p.part_o, p.part_ml, p.seqs,
                                 p.out, p.Hq, p.G);
         }
         // ---- epilogue: O / l -> bf16 rows --------------------------------------------------
@@ -736,9 +758,9 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
             const bool real_row = r < ntok_b;
             float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
             if (p.v_scale) inv *= p.v_scale[kvh];
-            __nv_bfloat16* dst = p.out + ((int64_t)(si.q_start + tok) * p.Hq + qh) * kD;
+            __nv_bfloat16* dst = p.out + ((int64_t)(si.q_start + tok) * p.Hq + qh) * D;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < D / 32; ++c) {
                 uint32_t ov[32];
                 tmem_ld32(o_addr + c * 32, ov);
                 tmem_wait_ld();
@@ -761,7 +783,7 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
         // (no other task reads those cache slots: any task whose tiles hold them patches them
         // from the dense input)
         if (jbase + ncas == (si.seq_len + kPrefillTileN - 1) / kPrefillTileN)
-            append_rows<kD>(p.k_new, p.v_new, p.k_cache, p.v_cache, p.block_table, p.bt_stride, p.num_pages,
+            append_rows<D>(p.k_new, p.v_new, p.k_cache, p.v_cache, p.block_table, p.bt_stride, p.num_pages,
                             p.Hkv, p.err, si, w.seq, kvh, 0, si.query_len, lane, 32);
     } else if (append) {
         // ------------------- warp 11: this task's share of the cache writes -------------------
@@ -772,7 +794,7 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
             const int gi = (b ? w.q_head1 : w.q_head) % p.G;
             const int t_begin = t0 + (int)((int64_t)nt * gi / p.G);
             const int t_end = t0 + (int)((int64_t)nt * (gi + 1) / p.G);
-            append_rows<kD>(p.k_new, p.v_new, p.k_cache, p.v_cache, p.block_table, p.bt_stride, p.num_pages,
+            append_rows<D>(p.k_new, p.v_new, p.k_cache, p.v_cache, p.block_table, p.bt_stride, p.num_pages,
                             p.Hkv, p.err, si, w.seq, kvh, t_begin, t_end, lane, 32);
         }
     }
@@ -782,7 +804,7 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
     __syncthreads();
     tc_fence_after();
     if (tid == 0) {
-        uint64_t* b = reinterpret_cast<uint64_t*>(sm + kOffBar);
+        uint64_t* b = reinterpret_cast<uint64_t*>(sm + L::kOffBar);
         for (int i = 0; i < kNumBars; ++i) mbar_inval(&b[i]);
     }
 }

@@ -253,11 +253,16 @@ def test_planner_rejects_bad_groups(groups, lens, code):
     assert ei.value.code == code
 
 
-def test_shared_prefix_needs_head_dim_128():
-    with pytest.raises(pk.PkvaError) as ei:
-        pk.inspect([40, 60], [1, 1], [0, 0], num_q_heads=8, num_kv_heads=2, head_dim=64,
-                   num_pages=12, bt_stride=4, prefix_group=[0, 0], prefix_len=[32])
-    assert ei.value.code == -2
+def test_shared_prefix_and_prefill_tasks_at_head_dim_64():
+    """Over bf16 caches the tensor-core tasks also run at head_dim 64: a shared-prefix group
+    gets cascade tasks and a long causal chunk prefill tasks (FP8 plans keep them at 128,
+    their staging copies being head_dim 128: the GPU tests check that refusal)."""
+    items = pk.inspect([40, 60], [1, 1], [0, 0], num_q_heads=8, num_kv_heads=2, head_dim=64,
+                       num_pages=12, bt_stride=4, prefix_group=[0, 0], prefix_len=[32])
+    assert any(it["kind"] == 2 and it["key_end"] == 32 for it in items)
+    items = pk.inspect([700, 40], [300, 1], [0, 0], num_q_heads=8, num_kv_heads=2, head_dim=64,
+                       num_pages=50, bt_stride=44)
+    assert any(it["kind"] == 1 for it in items)
 
 
 @pytest.mark.parametrize("num_sms, ctas", [(1, 1), (4, 3), (148, 3)])

@@ -59,7 +59,8 @@ def test_append_small_decode_verify(seed, d, max_q):
     run_append_case(b, expect_identical=True)
 
 
-def test_append_prefill_chunks():
+@pytest.mark.parametrize("d", [128, 64])
+def test_append_prefill_chunks(d):
     """Chunks on the tensor-core prefill path: prefix 0, page- and tile-aligned prefixes,
     ragged ones, a chunk that is not a multiple of the tile, mixed with decode rows."""
     seqs = [W.SeqSpec(300, 300, W.CAUSAL, []),          # no prefix
@@ -69,7 +70,7 @@ def test_append_prefill_chunks():
             W.SeqSpec(7 + 100, 100, W.CAUSAL, []),      # prefix inside the first page
             W.SeqSpec(900, 1, W.CAUSAL, []),
             W.SeqSpec(45, 4, W.TREE, [-1, 0, 0, 2])]
-    b = W.build_batch("append_prefill", seqs, 16, 2, 128, seed=21, device=DEV, bt_extra=1)
+    b = W.build_batch("append_prefill", seqs, 16, 2, d, seed=21, device=DEV, bt_extra=1)
     plan = pk.plan_for_batch(b)
     assert plan.info()["num_prefill_items"] > 0
     plan.close()

@@ -253,3 +253,20 @@ def test_fp8_large_verify_trees_all_rows(Hq, Hkv, d):
 def test_fp8_append_with_large_verify_trees(d):
     b = W.build_batch("large_trees_fp8_append", _large_tree_seqs(), 28, 4, d, seed=93, device=DEV)
     _fp8_append_case(b)
+
+
+def test_fp8_head_dim_64_keeps_tensor_core_tasks_off():
+    """Over FP8 caches the tensor-core tasks run at head_dim 128 only (their staging copies are
+    head_dim 128): a head_dim 64 causal chunk runs as decode tasks, and a shared-prefix group
+    at head_dim 64 is refused with PKVA_EUNSUPPORTED."""
+    b = W.build_batch("fp8_d64_chunk", [W.SeqSpec(40 + 300, 300, W.CAUSAL, [])], 16, 4, 64, seed=5, device=DEV)
+    f = W.fp8_kv(b)
+    out, plan = run_fp8(b, f)
+    assert plan.info()["num_prefill_items"] == 0
+    rows, exp = fp8_oracle_rows(b, f)
+    assert_close(out[rows], exp, "fp8 head_dim 64 chunk")
+    plan.close()
+    sb = W.random_shared_small(0, 16, 4, device=DEV, d=64)
+    with pytest.raises(pk.PkvaError) as ei:
+        pk.plan_for_batch(sb, kv_fp8=True)
+    assert ei.value.code == -2

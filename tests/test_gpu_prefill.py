@@ -1,5 +1,5 @@
-"""GPU parity of the tensor-core prefill path (causal chunks of >= 64 new tokens, d = 128)
-against the float64 oracle, including chunk lengths that leave a ragged last tile, cached
+"""GPU parity of the tensor-core prefill path (causal chunks of >= 64 new tokens, d = 128 and
+64) against the float64 oracle, including chunk lengths that leave a ragged last tile, cached
 prefixes that do not align with the 128-key tiles, and GQA groups of several sizes."""
 import pytest
 import torch
@@ -24,10 +24,11 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("d", [128, 64])
 @pytest.mark.parametrize("case", CASES, ids=lambda c: f"p{c[0]}_T{c[1]}_H{c[2]}x{c[3]}")
-def test_prefill_chunk(case):
+def test_prefill_chunk(case, d):
     prefix, T, Hq, Hkv = case
-    b = W.build_batch("pf", [W.SeqSpec(prefix + T, T, W.CAUSAL, [])], Hq, Hkv, 128, seed=prefix + T,
+    b = W.build_batch("pf", [W.SeqSpec(prefix + T, T, W.CAUSAL, [])], Hq, Hkv, d, seed=prefix + T,
                       device=DEV)
     plan = pk.plan_for_batch(b)
     assert plan.info()["num_prefill_items"] > 0
@@ -37,12 +38,13 @@ def test_prefill_chunk(case):
     assert_close(out[rows], exp, f"prefill {case}")
 
 
-def test_prefill_mixed_with_decode_and_verify():
+@pytest.mark.parametrize("d", [128, 64])
+def test_prefill_mixed_with_decode_and_verify(d):
     gen = torch.Generator().manual_seed(8)
     seqs = [W.SeqSpec(300, 100, W.CAUSAL, []), W.SeqSpec(900, 1, W.CAUSAL, []),
             W.SeqSpec(77, 77, W.CAUSAL, []), W.SeqSpec(1500 + 7, 7, W.TREE, W.random_tree(gen, 7)),
             W.SeqSpec(2048, 256, W.CAUSAL, [])]
-    b = W.build_batch("mixed", seqs, 28, 4, 128, seed=5, device=DEV)
+    b = W.build_batch("mixed", seqs, 28, 4, d, seed=5, device=DEV)
     plan = pk.plan_for_batch(b)
     info = plan.info()
     assert info["num_prefill_items"] > 0 and info["num_decode_items"] > 0
@@ -81,8 +83,8 @@ def test_prefill_matches_decode_body_on_same_rows(monkeypatch):
 
 
 def test_chunk_below_the_prefill_threshold_runs_as_decode_tasks():
-    """63 new tokens (threshold 64) and head_dim 64 chunks go to the warp-level body."""
-    for prefix, T, d in ((255, 63, 128), (40, 300, 64)):
+    """63 new tokens (threshold 64) go to the warp-level body, at either head_dim."""
+    for prefix, T, d in ((255, 63, 128), (40, 63, 64)):
         b = W.build_batch("below", [W.SeqSpec(prefix + T, T, W.CAUSAL, [])], 16, 4, d, seed=T + d, device=DEV)
         plan = pk.plan_for_batch(b)
         assert plan.info()["num_prefill_items"] == 0

@@ -21,9 +21,10 @@ def bits(t):
     return t.view(torch.int16)
 
 
+@pytest.mark.parametrize("d", [128, 64])
 @pytest.mark.parametrize("seed, heads", [(0, (16, 4)), (1, (28, 4)), (2, (8, 8)), (3, (64, 2)), (4, (32, 1))])
-def test_shared_prefix_small_all_rows(seed, heads):
-    b = W.random_shared_small(seed, *heads, device=DEV)
+def test_shared_prefix_small_all_rows(seed, heads, d):
+    b = W.random_shared_small(seed, *heads, device=DEV, d=d)
     plan = pk.plan_for_batch(b)
     assert plan.info()["num_cascade_items"] > 0
     out = plan.run(b.q, b.k_cache, b.v_cache)
@@ -64,8 +65,9 @@ def test_shared_prefix_config_full_size():
     plain.close()
 
 
-def test_shared_prefix_with_fused_append():
-    b = W.random_shared_small(5, 16, 4, device=DEV)
+@pytest.mark.parametrize("d", [128, 64])
+def test_shared_prefix_with_fused_append(d):
+    b = W.random_shared_small(5, 16, 4, device=DEV, d=d)
     k_new, v_new = W.new_token_kv(b)
     pg, sl = W.new_token_slots(b)
     kc, vc = b.k_cache.clone(), b.v_cache.clone()

@@ -265,8 +265,8 @@ def build_shared_batch(name: str, seqs: Sequence[SeqSpec], prefix_group: Sequenc
                  prefix_group=list(prefix_group), prefix_len=list(prefix_len))
 
 
-def random_shared_small(seed: int, Hq: int = 16, Hkv: int = 4, device="cpu") -> Batch:
-    """A small shared-prefix batch (head_dim 128): group 0 has six decode / verify members on
+def random_shared_small(seed: int, Hq: int = 16, Hkv: int = 4, device="cpu", d: int = 128) -> Batch:
+    """A small shared-prefix batch (head_dim d): group 0 has six decode / verify members on
     48 shared keys; one sequence belongs to no group; group 1 has three members on 160
     shared keys, one of them a 100-token causal chunk (which runs as a prefill task)."""
     gen = torch.Generator().manual_seed(seed)
@@ -282,7 +282,7 @@ def random_shared_small(seed: int, Hq: int = 16, Hkv: int = 4, device="cpu") -> 
     for T in (3, 100, 1):
         seqs.append(SeqSpec(160 + 20 + T, T, CAUSAL, []))
         group.append(1)
-    return build_shared_batch(f"shared_small_{seed}", seqs, group, [48, 160], Hq, Hkv, 128, seed=seed,
+    return build_shared_batch(f"shared_small_{seed}", seqs, group, [48, 160], Hq, Hkv, d, seed=seed,
                               device=device)
 
 
