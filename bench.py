@@ -173,8 +173,21 @@ class OracleRunner:
 def workload_name(args):
     """The workload as both arms name it (the GPU arm's batch options included)."""
     return f"{args.config}" + (f" (first {args.seqs} sequences)" if args.seqs else "") + \
+        (f" ({args.only_class} sequences alone)" if args.only_class else "") + \
         (f" (seed {args.seed})" if args.seed is not None else "") + \
         (" over FP8 E4M3 caches" if args.kv_fp8 else "")
+
+
+def make_batch(W, args, device):
+    """The named configuration's batch with the options both arms apply (first N sequences,
+    seed, one class of a mixed batch alone over the same caches)."""
+    batch = W.make_config(args.config, device=device, max_seqs=args.seqs, seed=args.seed)
+    if args.only_class:
+        parts = W.class_batches(batch)
+        if args.only_class not in parts:
+            raise SystemExit(f"--only-class {args.only_class}: {args.config} has no such sequences")
+        batch = parts[args.only_class]
+    return batch
 
 
 def parallelism_text(args, ws, num_kv_heads):
@@ -191,7 +204,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     import workloads as W
-    batch = W.make_config(args.config, device="cpu", seed=args.seed)
+    batch = make_batch(W, args, "cpu")
     runner = OracleRunner(batch)
     step_s = args.ref_seconds / (args.warmup + args.steps)
     for _ in range(args.warmup):
@@ -397,7 +410,7 @@ def run_ours(args):
     peaks = load_peaks()
     stream = torch.cuda.current_stream()
 
-    batch = W.make_config(args.config, device=dev, max_seqs=args.seqs, seed=args.seed)
+    batch = make_batch(W, args, dev)
     job_tokens = None
     parallelism = parallelism_text(args, ws, batch.num_kv_heads)
     config = workload_config(args.config, batch, workload_name(args), parallelism)
@@ -537,7 +550,7 @@ def run_ours(args):
 
     # the other benchmark batches, same measurement (one launch per step)
     per_config = {}
-    if ws == 1 and not args.seqs and not args.no_other_configs:
+    if ws == 1 and not args.seqs and not args.only_class and not args.no_other_configs:
         for name in ("llama3_8b_decode", "llama33_70b_prefill", "long_ctx_split"):
             if name == args.config:
                 continue
@@ -627,7 +640,7 @@ def run_ours(args):
     if rank == 0:
         cpu = None
         if ws == 1 and not args.no_cpu_baseline:
-            b = W.make_config(args.config, device=dev, max_seqs=args.seqs, seed=args.seed)
+            b = make_batch(W, args, dev)
             runner = OracleRunner(b)
             tk, sec = runner.run(args.cpu_seconds)
             cpu = {"value": tk / sec, "unit": "tokens/s", "cores": runner.threads, "kind": "oracle",
@@ -684,6 +697,8 @@ def main():
                     help="host time for the oracle baseline line of our arm")
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="total host time the reference arm spreads over warm-up + steps")
+    ap.add_argument("--only-class", choices=["prefill", "decode", "verify"], default=None,
+                    help="time one class of a mixed batch alone over the same caches (profiler captures)")
     ap.add_argument("--seed", type=int, default=None,
                     help="seed of the workload draw (default: the config's index, as the tests use)")
     args = ap.parse_args()
