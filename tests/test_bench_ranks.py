@@ -111,3 +111,26 @@ def test_bench_algorithmic_counts_match_the_oracle_masks():
         pairs += int(m.sum())
     assert bench.batch_attn_flops(b) == pairs * b.num_q_heads * 4 * b.head_dim
     assert bench.batch_kv_bytes(b) == sum(sp.seq_len for sp in b.seqs) * b.num_kv_heads * b.head_dim * 4
+
+
+def test_only_class_keeps_one_class_over_the_same_caches():
+    """``--only-class`` times one class of the mixed batch alone: the batch keeps only that
+    class's sequences (their query rows and block-table rows) over the same page pool, and
+    both arms name the workload with the class."""
+    import argparse
+    import torch
+    import bench
+    import workloads as W
+    full = W.make_config(bench.DEFAULT_CONFIG)
+    for cls in ("prefill", "decode", "verify"):
+        args = argparse.Namespace(config=bench.DEFAULT_CONFIG, seqs=None, seed=None, only_class=cls, kv_fp8=False)
+        b = bench.make_batch(W, args, "cpu")
+        keep = [i for i, sp in enumerate(full.seqs) if W.seq_class(sp) == cls]
+        assert keep and [sp.seq_len for sp in b.seqs] == [full.seqs[i].seq_len for i in keep]
+        assert b.k_cache.shape == full.k_cache.shape
+        assert torch.equal(b.block_table, full.block_table[keep])
+        assert b.q.shape[0] == sum(full.seqs[i].query_len for i in keep)
+        assert f"({cls} sequences alone)" in bench.workload_name(args)
+    args = argparse.Namespace(config="llama3_8b_decode", seqs=None, seed=None, only_class="verify", kv_fp8=False)
+    with pytest.raises(SystemExit):
+        bench.make_batch(W, args, "cpu")
