@@ -163,14 +163,23 @@ __device__ __forceinline__ void tile_rows(const PrefillParams& p, const int32_t*
     }
 }
 
+// The whole warp calls this: lane 0 posts the tile's bytes on `bar`, then lanes 0-7 each
+// load one page (its D / 64 boxes). One thread issuing all of a tile's boxes streams about
+// 20 GB/s; eight lanes about twice that (measured on B200).
 template <int D>
-__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, const int rows[8]) {
-    mbar_arrive_expect_tx(bar, Lay<D>::kTileBytes);
+__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, const int rows[8],
+                                          int lane) {
+    if (lane == 0) mbar_arrive_expect_tx(bar, Lay<D>::kTileBytes);
+    __syncwarp();
+    int row = rows[0];
 #pragma unroll
-    for (int pg = 0; pg < 8; ++pg)
+    for (int pg = 1; pg < 8; ++pg)
+        if (lane == pg) row = rows[pg];
+    if (lane < 8) {
 #pragma unroll
         for (int h = 0; h < Lay<D>::kHalves; ++h)
-            tma_load_2d(dst + h * kHalfBytes + pg * (kPageSize * 128), map, bar, h * 64, rows[pg]);
+            tma_load_2d(dst + h * kHalfBytes + lane * (kPageSize * 128), map, bar, h * 64, row);
+    }
 }
 
 // One prefill task; every thread of the block (at least kPThreads) calls it; warps past
@@ -324,10 +333,10 @@ __device__ __forceinline__ void prefill_task(const PrefillParams& p, int task, c
             const bool patch = own && p.append && kb + kPrefillTileN > prefix && kb < si.seq_len;
             const bool zero = !is_k && j == fix_tile;
             if (!patch && !zero) {
-                if (lane == 0) load_tile<D>(dst, is_k ? &tmK : &tmV, &full[st], rows);
+                load_tile<D>(dst, is_k ? &tmK : &tmV, &full[st], rows, lane);
                 continue;
             }
-            if (lane == 0) load_tile<D>(dst, is_k ? &tmK : &tmV, fixbar, rows);
+            load_tile<D>(dst, is_k ? &tmK : &tmV, fixbar, rows, lane);
             if (!__all_sync(0xffffffffu, wait_or_abort(fixbar, nfix & 1, p.err, abort_flag))) break;
             ++nfix;
             if (patch) {
