@@ -63,11 +63,14 @@ struct AttnSmem {
 
 // FP8: decode/verify tasks read the E4M3 pages; tensor-core tasks read their bf16 staging copies.
 // Tensor-core tasks run at head_dim 128 and, over bf16 caches, 64.
-template <int D, int NT, bool FP8, bool TC>
+// TCM: 0 no tensor-core tasks; 1 tensor-core tasks; 2 tensor-core tasks beside decode blocks,
+// run as prefill_task_rs (the block's registers split between its warpgroups)
+template <int D, int NT, bool FP8, int TCM>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKn,
             const __grid_constant__ CUtensorMap tmVn, const __grid_constant__ CUtensorMap tmQc) {
+    constexpr bool TC = TCM != 0;
     using S = AttnSmem<D, NT, FP8, TC>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -86,7 +89,10 @@ attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const _
             tc_fence_after();
             const uint32_t tmem = *tmem_slot;
             // over FP8 caches the tensor-core tasks read the bf16 staging pages (tmKn / tmVn)
-            pre::prefill_task<D>(p.pre, e, tmQ, FP8 ? tmKn : tmK, FP8 ? tmVn : tmV, tmKn, tmVn, tmQc, tmem, sm);
+            if constexpr (TCM == 2)
+                pre::prefill_task_rs<D>(p.pre, e, tmQ, FP8 ? tmKn : tmK, FP8 ? tmVn : tmV, tmKn, tmVn, tmQc, tmem, sm);
+            else
+                pre::prefill_task<D>(p.pre, e, tmQ, FP8 ? tmKn : tmK, FP8 ? tmVn : tmV, tmKn, tmVn, tmQc, tmem, sm);
             tc_fence_before();
             __syncthreads();
             tc_fence_after();
@@ -120,17 +126,17 @@ attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const _
                                                                     sm + g * S::GROUP_BYTES);
 }
 
-template <int D, int NT, bool FP8, bool TC>
+template <int D, int NT, bool FP8, int TCM>
 cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                      const CUtensorMap& tmKn, const CUtensorMap& tmVn, const CUtensorMap& tmQc,
                      cudaStream_t stream) {
-    using S = AttnSmem<D, NT, FP8, TC>;
+    using S = AttnSmem<D, NT, FP8, TCM != 0>;
     cudaError_t e =
-        cudaFuncSetAttribute(attn_kernel<D, NT, FP8, TC>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::ALLOC);
+        cudaFuncSetAttribute(attn_kernel<D, NT, FP8, TCM>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::ALLOC);
     if (e != cudaSuccess) return e;
     const int grid = p.num_blocks;
     if (grid == 0) return cudaSuccess;
-    attn_kernel<D, NT, FP8, TC><<<grid, kAttnThreads, S::ALLOC, stream>>>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc);
+    attn_kernel<D, NT, FP8, TCM><<<grid, kAttnThreads, S::ALLOC, stream>>>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc);
     return cudaGetLastError();
 }
 
@@ -139,28 +145,28 @@ int ctas_t() {
     constexpr bool TC = true;
     using S = AttnSmem<D, NT, false, TC>;
     int n = 0;
-    if (cudaFuncSetAttribute(attn_kernel<D, NT, false, TC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(attn_kernel<D, NT, false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              S::ALLOC) != cudaSuccess)
         return 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_kernel<D, NT, false, TC>, kAttnThreads, S::ALLOC) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_kernel<D, NT, false, 1>, kAttnThreads, S::ALLOC) !=
         cudaSuccess)
         return 0;
     return n;
 }
 
-template <bool FP8, bool TC>
+template <bool FP8, int TCM>
 cudaError_t launch_kv(const AttnParams& p, int D, int rows, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                       const CUtensorMap& tmV, const CUtensorMap& tmKn, const CUtensorMap& tmVn,
                       const CUtensorMap& tmQc, cudaStream_t stream) {
     if (D == 64) {
         // head_dim 64 tensor-core tasks run over bf16 caches only (the FP8 staging copies are
         // head_dim 128)
-        constexpr bool TC64 = TC && !FP8;
-        return rows <= 8 ? launch_t<64, 1, FP8, TC64>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
-                         : launch_t<64, 2, FP8, TC64>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
+        constexpr int TCM64 = FP8 ? 0 : TCM;
+        return rows <= 8 ? launch_t<64, 1, FP8, TCM64>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
+                         : launch_t<64, 2, FP8, TCM64>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
     }
-    return rows <= 8 ? launch_t<128, 1, FP8, TC>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
-                     : launch_t<128, 2, FP8, TC>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
+    return rows <= 8 ? launch_t<128, 1, FP8, TCM>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
+                     : launch_t<128, 2, FP8, TCM>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
 }
 
 }  // namespace
@@ -175,12 +181,16 @@ cudaError_t launch_attn(const AttnParams& p, int D, int rows, bool has_prefill, 
                         const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKn,
                         const CUtensorMap& tmVn, const CUtensorMap& tmQc, cudaStream_t stream, bool fp8) {
     if (D == 64 && fp8 && has_prefill) return cudaErrorInvalidValue;   // (never planned)
-    // plans without tensor-core tasks launch the TC = false code (no prefill body in it)
+    // plans without tensor-core tasks launch the code without the prefill body; plans with
+    // tensor-core and decode tasks the one whose tensor-core blocks split their registers
+    const bool mixed = has_prefill && p.num_decode > 0;
     if (!fp8)
-        return has_prefill ? launch_kv<false, true>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
-                           : launch_kv<false, false>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
-    return has_prefill ? launch_kv<true, true>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
-                       : launch_kv<true, false>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
+        return mixed ? launch_kv<false, 2>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
+               : has_prefill ? launch_kv<false, 1>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
+                             : launch_kv<false, 0>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
+    return mixed ? launch_kv<true, 2>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
+           : has_prefill ? launch_kv<true, 1>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream)
+                         : launch_kv<true, 0>(p, D, rows, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
 }
 
 }  // namespace pkva
