@@ -34,6 +34,10 @@ constexpr int kAttnThreads = 384;                 // prefill uses 352; decode 3 
 constexpr int kDecWarps = 4;                      // page-streaming warps per decode task
 static_assert(kAttnThreads >= pre::kPThreadsAppend, "block too small for a prefill task");
 static_assert(kAttnThreads == kDecTasksPerBlock * 128, "one 128-thread group per decode task");
+// prefill_task_rs splits a block's registers as 2 x 128 threads x 192 + 128 x 120: exactly the
+// 384 x 168 a block is launched with (a larger split would wait for registers forever)
+constexpr int kSplitLaunchRegs = 168;
+static_assert(2 * 128 * 192 + 128 * 120 == kAttnThreads * kSplitLaunchRegs, "register split");
 
 template <int D, bool FP8 = false>
 struct AttnNS {
@@ -126,10 +130,23 @@ attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmQ, const _
                                                                     sm + g * S::GROUP_BYTES);
 }
 
+// The register split is used only where the compiled kernel is launched with exactly the
+// registers it divides; otherwise the launch falls back to the unsplit task body.
+template <int D, int NT, bool FP8>
+bool split_fits() {
+    static const bool ok = [] {
+        cudaFuncAttributes a{};
+        return cudaFuncGetAttributes(&a, attn_kernel<D, NT, FP8, 2>) == cudaSuccess && a.numRegs == kSplitLaunchRegs;
+    }();
+    return ok;
+}
+
 template <int D, int NT, bool FP8, int TCM>
 cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                      const CUtensorMap& tmKn, const CUtensorMap& tmVn, const CUtensorMap& tmQc,
                      cudaStream_t stream) {
+    if constexpr (TCM == 2)
+        if (!split_fits<D, NT, FP8>()) return launch_t<D, NT, FP8, 1>(p, tmQ, tmK, tmV, tmKn, tmVn, tmQc, stream);
     using S = AttnSmem<D, NT, FP8, TCM != 0>;
     cudaError_t e =
         cudaFuncSetAttribute(attn_kernel<D, NT, FP8, TCM>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::ALLOC);
